@@ -1,0 +1,221 @@
+/*
+ * osdn_ref.c -- fp64 CPU oracle for the Online Scaled DeltaNet (OSDN) forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously correct statement of what
+ * the GPU library computes.  Only the tests, the smoke check and the benchmark's CPU
+ * baseline may load it; the product path never does.  It shares no code, header,
+ * table or helper with the CUDA library.
+ *
+ * Source: the technical summary pages of "OSDN: Improving Delta Rule with Provable Online
+ * Preconditioning in Linear Attention" (Italian and German editions, same sections):
+ *   - section 1 (problem statement): per-token loss f_t(S) = 1/2 ||S k_t - v_t||^2 and
+ *     the delta rule S_t = S_{t-1} + beta_t (v_t - S_{t-1} k_t) k_t^T;
+ *   - section 2.1 (algebraic equivalence): the right-preconditioned gradient step
+ *     S_t = S_{t-1} - beta_t grad f_t(S_{t-1}) D_t equals the delta rule with the write
+ *     key replaced by k~_t = d_t (.) k_t;
+ *   - section 2.2 (decoupled hypergradient feedback): d_t is updated by online gradient
+ *     descent on the surrogate h_t, whose closed form is
+ *     h_t(d) = ((1 - beta_t <d, k_t^2>)^2 - 1) / (2 ||k_t||^2); its gradient is
+ *     grad_d h_t = -beta_t (1 - beta_t <d, k_t^2>) k_t^2 / ||k_t||^2;
+ *   - section 2.3 (APF): a per-token, per-head retention gate r_{t,h} multiplies d only.
+ *
+ * Readings taken where the pages are silent or garbled (each is pinned by a test):
+ *   - The APF equation is printed with "+ eta grad h"; section 2.2 calls the update
+ *     gradient DESCENT on h, and only descent lowers h, so the step here is
+ *     d_{t+1} = r_t d_t - eta grad_d h_t(d_t).  No projection or clipping is applied.
+ *   - Token t writes with d_t, the preconditioner before its own update; d_0 defaults
+ *     to the all-ones vector, S_0 to zero.  The output is o_t = scale * S_t q_t, read
+ *     from the state after token t's write (DeltaNet convention).
+ *   - When ||k_t||^2 == 0 the gradient is taken to be zero.
+ *   - With packed variable-length input (cu_seqlens) every sequence starts from its
+ *     own d_0 / S_0 and returns its own final state.
+ *
+ * Layouts (row-major, fp64):
+ *   q, k, k_tilde : [B, T, H, Dk]        v, o : [B, T, H, Dv]
+ *   beta, r       : [B, T, H]            S0, ST : [N, H, Dv, Dk]   d0, dT : [N, H, Dk]
+ *   Fixed length: N = B and sequence n is rows n*T .. n*T+T-1.
+ *   Packed: B == 1, T = total tokens, N = num_seqs and sequence n is rows
+ *   cu_seqlens[n] .. cu_seqlens[n+1]-1 (cu_seqlens is a HOST array of N+1 entries).
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static void seq_bounds(int32_t n, const int32_t* cu_seqlens, int32_t T, int64_t* first,
+                       int64_t* count) {
+    if (cu_seqlens) {
+        *first = cu_seqlens[n];
+        *count = (int64_t)cu_seqlens[n + 1] - (int64_t)cu_seqlens[n];
+    } else {
+        *first = (int64_t)n * T;
+        *count = T;
+    }
+}
+
+int osdn_ref_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------------------------
+ * Phase 1: the preconditioner scan over the key stream (section 2.2, two-phase split,
+ * step 1).  Emits k~_t = d_t (.) k_t for every token and the final d.
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_precond_scan(const double* k, const double* beta, const double* r, double eta,
+                           const double* d0, double* k_tilde, double* dT,
+                           const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                           int32_t H, int32_t Dk) {
+    const int32_t N = cu_seqlens ? num_seqs : B;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int32_t n = 0; n < N; ++n) {
+        for (int32_t h = 0; h < H; ++h) {
+            double* d = (double*)malloc(sizeof(double) * Dk);
+            for (int32_t i = 0; i < Dk; ++i) d[i] = d0 ? d0[((int64_t)n * H + h) * Dk + i] : 1.0;
+            int64_t first, count;
+            seq_bounds(n, cu_seqlens, T, &first, &count);
+            for (int64_t t = first; t < first + count; ++t) {
+                const int64_t th = t * H + h;
+                const double* kt = k + th * Dk;
+                const double bt = beta[th];
+                const double rt = r ? r[th] : 1.0;
+                double knorm2 = 0.0, s = 0.0; /* ||k_t||^2 and <d_t, k_t^2> */
+                for (int32_t i = 0; i < Dk; ++i) {
+                    knorm2 += kt[i] * kt[i];
+                    s += d[i] * kt[i] * kt[i];
+                }
+                for (int32_t i = 0; i < Dk; ++i) k_tilde[th * Dk + i] = d[i] * kt[i];
+                for (int32_t i = 0; i < Dk; ++i) {
+                    const double grad =
+                        knorm2 > 0.0 ? -bt * (1.0 - bt * s) * kt[i] * kt[i] / knorm2 : 0.0;
+                    d[i] = rt * d[i] - eta * grad;
+                }
+            }
+            if (dT)
+                for (int32_t i = 0; i < Dk; ++i) dT[((int64_t)n * H + h) * Dk + i] = d[i];
+            free(d);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------------
+ * Phase 2: the delta rule with a separate write key (section 2.1), token by token:
+ *   u_t = v_t - S_{t-1} k_t,   S_t = S_{t-1} + beta_t u_t k~_t^T,   o_t = scale S_t q_t.
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_delta_fwd(const double* q, const double* k, const double* k_tilde, const double* v,
+                        const double* beta, double scale, const double* S0, double* o,
+                        double* ST, const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                        int32_t T, int32_t H, int32_t Dk, int32_t Dv) {
+    const int32_t N = cu_seqlens ? num_seqs : B;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int32_t n = 0; n < N; ++n) {
+        for (int32_t h = 0; h < H; ++h) {
+            double* S = (double*)malloc(sizeof(double) * Dv * Dk);
+            double* u = (double*)malloc(sizeof(double) * Dv);
+            const int64_t sbase = ((int64_t)n * H + h) * Dv * Dk;
+            for (int64_t e = 0; e < (int64_t)Dv * Dk; ++e) S[e] = S0 ? S0[sbase + e] : 0.0;
+            int64_t first, count;
+            seq_bounds(n, cu_seqlens, T, &first, &count);
+            for (int64_t t = first; t < first + count; ++t) {
+                const int64_t th = t * H + h;
+                const double* kt = k + th * Dk;
+                const double* kw = k_tilde + th * Dk;
+                const double* qt = q + th * Dk;
+                const double* vt = v + th * Dv;
+                const double bt = beta[th];
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double sk = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) sk += S[(int64_t)j * Dk + i] * kt[i];
+                    u[j] = vt[j] - sk;
+                }
+                for (int32_t j = 0; j < Dv; ++j)
+                    for (int32_t i = 0; i < Dk; ++i) S[(int64_t)j * Dk + i] += bt * u[j] * kw[i];
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double sq = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) sq += S[(int64_t)j * Dk + i] * qt[i];
+                    o[th * Dv + j] = scale * sq;
+                }
+            }
+            if (ST)
+                for (int64_t e = 0; e < (int64_t)Dv * Dk; ++e) ST[sbase + e] = S[e];
+            free(u);
+            free(S);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------------
+ * Both phases in one token loop: the method exactly as stated, with no split.
+ * Per token: k~ = d (.) k;  u = v - S k;  S += beta u k~^T;  o = scale S q;
+ *            d <- r d - eta grad_d h(d).
+ * k_tilde and dT may be NULL.
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_fwd(const double* q, const double* k, const double* v, const double* beta,
+                  const double* r, double eta, const double* d0, const double* S0, double scale,
+                  double* o, double* k_tilde, double* ST, double* dT, const int32_t* cu_seqlens,
+                  int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv) {
+    const int32_t N = cu_seqlens ? num_seqs : B;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int32_t n = 0; n < N; ++n) {
+        for (int32_t h = 0; h < H; ++h) {
+            double* S = (double*)malloc(sizeof(double) * Dv * Dk);
+            double* d = (double*)malloc(sizeof(double) * Dk);
+            double* kw = (double*)malloc(sizeof(double) * Dk);
+            double* u = (double*)malloc(sizeof(double) * Dv);
+            const int64_t sbase = ((int64_t)n * H + h) * Dv * Dk;
+            const int64_t dbase = ((int64_t)n * H + h) * Dk;
+            for (int64_t e = 0; e < (int64_t)Dv * Dk; ++e) S[e] = S0 ? S0[sbase + e] : 0.0;
+            for (int32_t i = 0; i < Dk; ++i) d[i] = d0 ? d0[dbase + i] : 1.0;
+            int64_t first, count;
+            seq_bounds(n, cu_seqlens, T, &first, &count);
+            for (int64_t t = first; t < first + count; ++t) {
+                const int64_t th = t * H + h;
+                const double* kt = k + th * Dk;
+                const double* qt = q + th * Dk;
+                const double* vt = v + th * Dv;
+                const double bt = beta[th];
+                const double rt = r ? r[th] : 1.0;
+                double knorm2 = 0.0, s = 0.0;
+                for (int32_t i = 0; i < Dk; ++i) {
+                    knorm2 += kt[i] * kt[i];
+                    s += d[i] * kt[i] * kt[i];
+                    kw[i] = d[i] * kt[i];
+                }
+                if (k_tilde)
+                    for (int32_t i = 0; i < Dk; ++i) k_tilde[th * Dk + i] = kw[i];
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double sk = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) sk += S[(int64_t)j * Dk + i] * kt[i];
+                    u[j] = vt[j] - sk;
+                }
+                for (int32_t j = 0; j < Dv; ++j)
+                    for (int32_t i = 0; i < Dk; ++i) S[(int64_t)j * Dk + i] += bt * u[j] * kw[i];
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double sq = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) sq += S[(int64_t)j * Dk + i] * qt[i];
+                    o[th * Dv + j] = scale * sq;
+                }
+                for (int32_t i = 0; i < Dk; ++i) {
+                    const double grad =
+                        knorm2 > 0.0 ? -bt * (1.0 - bt * s) * kt[i] * kt[i] / knorm2 : 0.0;
+                    d[i] = rt * d[i] - eta * grad;
+                }
+            }
+            if (ST)
+                for (int64_t e = 0; e < (int64_t)Dv * Dk; ++e) ST[sbase + e] = S[e];
+            if (dT)
+                for (int32_t i = 0; i < Dk; ++i) dT[dbase + i] = d[i];
+            free(u);
+            free(kw);
+            free(d);
+            free(S);
+        }
+    }
+}
