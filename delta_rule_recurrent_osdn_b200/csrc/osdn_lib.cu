@@ -1,0 +1,285 @@
+// osdn_lib.cu -- libosdn: host side of the C ABI declared in include/osdn.h.
+//
+// One translation unit holds every kernel (so the device status word is a single symbol).
+// The host code validates arguments, picks a kernel for the sizes and dtype, and enqueues it
+// on the caller's stream.  It never allocates memory and never synchronizes, except in
+// osdn_get_device_status, whose job is to synchronize.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "osdn.h"
+#include "common.cuh"
+#include "scan_warp.cuh"
+#include "chunk_simt.cuh"
+#include "watchdog.cuh"
+
+namespace osdn {
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+inline size_t io_size(osdn_dtype_t io) { return io == OSDN_BF16 ? 2 : 4; }
+
+struct Dims {
+    int32_t B, T, H, Dk, Dv, N;
+    int64_t rows() const { return (int64_t)B * T; }
+};
+
+osdn_status_t check_common(const int32_t* cu, int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                           int32_t Dk, osdn_dtype_t io, Dims& d) {
+    if (io != OSDN_BF16 && io != OSDN_F32) return OSDN_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H < 1 || num_seqs < 0) return OSDN_ERR_INVALID_ARG;
+    if (cu && B != 1) return OSDN_ERR_INVALID_ARG;
+    if (cu && !aligned16(cu)) return OSDN_ERR_ALIGNMENT;
+    if (Dk != 64 && Dk != 128) return OSDN_ERR_UNSUPPORTED;
+    d.B = B;
+    d.T = T;
+    d.H = H;
+    d.Dk = Dk;
+    d.Dv = Dk;
+    d.N = cu ? num_seqs : B;
+    return OSDN_OK;
+}
+
+inline osdn_status_t launch_status() {
+    return cudaGetLastError() == cudaSuccess ? OSDN_OK : OSDN_ERR_CUDA;
+}
+
+template <typename KernelT>
+inline bool set_smem(KernelT kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)bytes) == cudaSuccess;
+}
+
+// ---------------------------------------------------------------- phase 1 dispatch
+template <typename IO>
+osdn_status_t launch_scan(const void* k, const float* beta, const float* r, float eta,
+                          const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                          const Dims& d, cudaStream_t stream) {
+    const int units = d.N * d.H;
+    if (units == 0) return OSDN_OK;
+    const dim3 block(128), grid((units + 3) / 4);
+    if (d.Dk == 128)
+        precond_scan_warp_kernel<128, IO><<<grid, block, 0, stream>>>(
+            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, cu, d.N,
+            d.T, d.H);
+    else
+        precond_scan_warp_kernel<64, IO><<<grid, block, 0, stream>>>(
+            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, cu, d.N,
+            d.T, d.H);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- phase 2 dispatch
+template <int DK, int DV, int C, typename IO>
+osdn_status_t launch_chunk_simt(const void* q, const void* k, const void* kt, const void* v,
+                                const float* beta, float scale, const float* S0, void* o,
+                                float* ST, const int32_t* cu, const Dims& d,
+                                cudaStream_t stream) {
+    constexpr int BV = 32;
+    const int64_t ctas = (int64_t)d.N * d.H * (DV / BV);
+    if (ctas == 0) return OSDN_OK;
+    if (ctas > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    auto kernel = chunk_fwd_simt_kernel<DK, DV, BV, C, IO>;
+    const size_t smem = SimtSmem<DK, BV, C>::bytes;
+    if (!set_smem(kernel, smem)) return OSDN_ERR_CUDA;
+    kernel<<<dim3((unsigned)ctas), dim3(256), smem, stream>>>(
+        static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(kt),
+        static_cast<const IO*>(v), beta, scale, S0, static_cast<IO*>(o), ST, cu, d.N, d.T, d.H);
+    return launch_status();
+}
+
+template <int DK, int DV, typename IO>
+osdn_status_t launch_chunk_c(int chunk, const void* q, const void* k, const void* kt,
+                             const void* v, const float* beta, float scale, const float* S0,
+                             void* o, float* ST, const int32_t* cu, const Dims& d,
+                             cudaStream_t stream) {
+    switch (chunk) {
+        case 16:
+            return launch_chunk_simt<DK, DV, 16, IO>(q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+                                                     stream);
+        case 32:
+            return launch_chunk_simt<DK, DV, 32, IO>(q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+                                                     stream);
+        case 64:
+            return launch_chunk_simt<DK, DV, 64, IO>(q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+                                                     stream);
+        default:
+            return OSDN_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename IO>
+osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* kt,
+                           const void* v, const float* beta, float scale, const float* S0,
+                           void* o, float* ST, const int32_t* cu, const Dims& d,
+                           cudaStream_t stream) {
+    if (d.Dk == 128 && d.Dv == 128)
+        return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+                                            stream);
+    if (d.Dk == 128 && d.Dv == 64)
+        return launch_chunk_c<128, 64, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+                                           stream);
+    if (d.Dk == 64 && d.Dv == 128)
+        return launch_chunk_c<64, 128, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+                                           stream);
+    return launch_chunk_c<64, 64, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
+}
+
+osdn_status_t validate_scan(const void* k, const float* beta, const float* r, const float* d0,
+                            const void* k_tilde, const float* dT, const Dims& d,
+                            osdn_dtype_t io) {
+    // token tensors may be NULL only when there are no tokens at all
+    if (d.rows() * d.H > 0 && (!k || !beta || !k_tilde)) return OSDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {k, beta, r, d0, k_tilde, dT};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
+    const size_t kbytes = (size_t)d.rows() * d.H * d.Dk * io_size(io);
+    if (overlaps(k, kbytes, k_tilde, kbytes)) return OSDN_ERR_INVALID_ARG;
+    return OSDN_OK;
+}
+
+osdn_status_t validate_chunk(const void* q, const void* k, const void* kt, const void* v,
+                             const float* beta, const float* S0, const void* o, const float* ST,
+                             const Dims& d, int chunk, osdn_dtype_t io) {
+    if (d.rows() * d.H > 0 && (!q || !k || !kt || !v || !beta || !o)) return OSDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, kt, v, beta, S0, o, ST};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
+    if (d.Dv != 64 && d.Dv != 128) return OSDN_ERR_UNSUPPORTED;
+    if (io == OSDN_BF16 ? chunk != 64 : (chunk != 16 && chunk != 32 && chunk != 64))
+        return OSDN_ERR_UNSUPPORTED;
+    const size_t es = io_size(io);
+    const size_t kb = (size_t)d.rows() * d.H * d.Dk * es, vb = (size_t)d.rows() * d.H * d.Dv * es;
+    if (overlaps(o, vb, q, kb) || overlaps(o, vb, k, kb) || overlaps(o, vb, kt, kb) ||
+        overlaps(o, vb, v, vb))
+        return OSDN_ERR_INVALID_ARG;
+    return OSDN_OK;
+}
+
+}  // namespace
+}  // namespace osdn
+
+using namespace osdn;
+
+extern "C" {
+
+int32_t osdn_abi_version(void) { return OSDN_ABI_VERSION; }
+
+const char* osdn_status_string(osdn_status_t s) {
+    switch (s) {
+        case OSDN_OK: return "ok";
+        case OSDN_ERR_INVALID_ARG: return "invalid argument";
+        case OSDN_ERR_UNSUPPORTED: return "unsupported size or mode";
+        case OSDN_ERR_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+        case OSDN_ERR_CUDA: return "CUDA runtime error";
+        case OSDN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case OSDN_ERR_DEVICE_BOUNDS: return "device-side cu_seqlens check failed";
+    }
+    return "unknown status";
+}
+
+osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r, float eta,
+                                const float* d0, void* k_tilde, float* dT,
+                                const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                                int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io,
+                                void* stream) {
+    Dims d;
+    osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
+    if (st != OSDN_OK) return st;
+    st = validate_scan(k, beta, r, d0, k_tilde, dT, d, io);
+    if (st != OSDN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (io == OSDN_BF16)
+        return launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, k_tilde, dT, cu_seqlens, d, s);
+    return launch_scan<float>(k, beta, r, eta, d0, k_tilde, dT, cu_seqlens, d, s);
+}
+
+osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, const void* v,
+                             const float* beta, float scale, const float* S0, void* o, float* ST,
+                             const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                             int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
+                             void* stream) {
+    Dims d;
+    osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
+    if (st != OSDN_OK) return st;
+    d.Dv = Dv;
+    st = validate_chunk(q, k, k_tilde, v, beta, S0, o, ST, d, chunk, io);
+    if (st != OSDN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (io == OSDN_BF16)
+        return launch_chunk<__nv_bfloat16>(chunk, q, k, k_tilde, v, beta, scale, S0, o, ST,
+                                           cu_seqlens, d, s);
+    return launch_chunk<float>(chunk, q, k, k_tilde, v, beta, scale, S0, o, ST, cu_seqlens, d, s);
+}
+
+size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io) {
+    if (B < 0 || T < 0 || H < 1 || (Dk != 64 && Dk != 128) || (io != OSDN_BF16 && io != OSDN_F32))
+        return 0;
+    const size_t raw = (size_t)B * T * H * Dk * io_size(io);
+    return (raw + 255) & ~(size_t)255;
+}
+
+osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* r, float eta, const float* d0, const float* S0, float scale,
+                       void* o, float* ST, float* dT, void* k_tilde_out,
+                       const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                       int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    Dims d;
+    osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
+    if (st != OSDN_OK) return st;
+    d.Dv = Dv;
+    // where the preconditioned keys go: the caller's buffer, else the workspace
+    void* kt = k_tilde_out;
+    const size_t need = osdn_fwd_workspace_bytes(B, T, H, Dk, io);
+    if (!kt && need > 0) {
+        if (!workspace || workspace_bytes < need) return OSDN_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return OSDN_ERR_ALIGNMENT;
+        kt = workspace;
+    }
+    st = validate_scan(k, beta, r, d0, kt, dT, d, io);
+    if (st != OSDN_OK) return st;
+    st = validate_chunk(q, k, kt, v, beta, S0, o, ST, d, chunk, io);
+    if (st != OSDN_OK) return st;
+    const size_t es = io_size(io);
+    const size_t kb = (size_t)d.rows() * d.H * d.Dk * es, vb = (size_t)d.rows() * d.H * d.Dv * es;
+    if (overlaps(kt, kb, q, kb) || overlaps(kt, kb, v, vb)) return OSDN_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (io == OSDN_BF16) {
+        st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, dT, cu_seqlens, d, s);
+        if (st != OSDN_OK) return st;
+        return launch_chunk<__nv_bfloat16>(chunk, q, k, kt, v, beta, scale, S0, o, ST,
+                                           cu_seqlens, d, s);
+    }
+    st = launch_scan<float>(k, beta, r, eta, d0, kt, dT, cu_seqlens, d, s);
+    if (st != OSDN_OK) return st;
+    return launch_chunk<float>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu_seqlens, d, s);
+}
+
+osdn_status_t osdn_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return OSDN_ERR_CUDA;
+    int value = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&value, g_device_status, sizeof(int)) != cudaSuccess)
+        return OSDN_ERR_CUDA;
+    if (value != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+        return OSDN_ERR_CUDA;
+    return static_cast<osdn_status_t>(value);
+}
+
+osdn_status_t osdn_debug_watchdog_selftest(int64_t spin_limit, void* stream) {
+    if (spin_limit < 1 || spin_limit > (int64_t(1) << 30)) return OSDN_ERR_INVALID_ARG;
+    watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(spin_limit);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -190,3 +190,22 @@ def select(inp: OsdnInputs, seqs=None, heads=None) -> OsdnInputs:
     d0 = None if inp.d0 is None else np.ascontiguousarray(inp.d0[seqs][:, heads])
     S0 = None if inp.S0 is None else np.ascontiguousarray(inp.S0[seqs][:, heads])
     return dataclasses.replace(inp, q=q, k=k, v=v, beta=beta, r=r, d0=d0, S0=S0, cu_seqlens=cu)
+
+
+def to_torch(inp: OsdnInputs, device="cuda"):
+    """Device tensors for one batch: io tensors in the io dtype, gates/states float32,
+    cu_seqlens int32.  Returns a dict keyed like the binding's arguments."""
+    import torch
+    dt = torch.bfloat16 if inp.io == "bf16" else torch.float32
+
+    def io(a):
+        return torch.from_numpy(a).to(device=device, dtype=dt).contiguous()
+
+    def f32(a):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+
+    out = dict(q=io(inp.q), k=io(inp.k), v=io(inp.v), beta=f32(inp.beta), r=f32(inp.r),
+               d0=f32(inp.d0), S0=f32(inp.S0), eta=inp.eta, scale=inp.scale, chunk=inp.chunk)
+    out["cu_seqlens"] = None if inp.cu_seqlens is None else \
+        torch.from_numpy(inp.cu_seqlens.astype(np.int32)).to(device)
+    return out

@@ -1,0 +1,234 @@
+"""Python binding of libosdn (the C ABI in include/osdn.h): argument marshalling only.
+
+Every function here takes CUDA tensors, checks their dtype/shape/contiguity, allocates the
+outputs the caller did not pass (``torch.empty`` on the inputs' device), and calls the
+C entry point of the same name on the current CUDA stream.  All arithmetic runs in the
+library's kernels.  There is no fallback: if ``libosdn.so`` is missing, importing this module
+raises, and a non-OK status raises :class:`OsdnError`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libosdn.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "osdn.h")
+
+OSDN_OK = 0
+OSDN_ERR_INVALID_ARG = 1
+OSDN_ERR_UNSUPPORTED = 2
+OSDN_ERR_ALIGNMENT = 3
+OSDN_ERR_CUDA = 4
+OSDN_ERR_DEVICE_TIMEOUT = 5
+OSDN_ERR_DEVICE_BOUNDS = 6
+OSDN_BF16 = 0
+OSDN_F32 = 1
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_f32 = ctypes.c_float
+
+
+class OsdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m delta_rule_recurrent_osdn_b200.build`"
+            " (there is no non-CUDA implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.osdn_abi_version.argtypes = []
+    lib.osdn_abi_version.restype = _i32
+    lib.osdn_status_string.argtypes = [ctypes.c_int]
+    lib.osdn_status_string.restype = ctypes.c_char_p
+    lib.osdn_precond_scan.argtypes = [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                      _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_precond_scan.restype = ctypes.c_int
+    lib.osdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i32, _i32,
+                                   _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_chunk_fwd.restype = ctypes.c_int
+    lib.osdn_fwd_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, ctypes.c_int]
+    lib.osdn_fwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.osdn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _f32, _vp, _vp, _vp, _vp,
+                             _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
+                             ctypes.c_size_t, _vp]
+    lib.osdn_fwd.restype = ctypes.c_int
+    lib.osdn_get_device_status.argtypes = [_vp]
+    lib.osdn_get_device_status.restype = ctypes.c_int
+    lib.osdn_debug_watchdog_selftest.argtypes = [ctypes.c_int64, _vp]
+    lib.osdn_debug_watchdog_selftest.restype = ctypes.c_int
+    return lib
+
+
+LIB = _load()
+
+
+def header_symbols() -> list:
+    """Names of the functions include/osdn.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^OSDN_API\s+[\w\s\*]*?(osdn_\w+)\s*\(", text, re.M)))
+
+
+def status_string(status: int) -> str:
+    return LIB.osdn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != OSDN_OK:
+        raise OsdnError(status, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _io(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return OSDN_BF16
+    if t.dtype == torch.float32:
+        return OSDN_F32
+    raise TypeError(f"io tensors must be bfloat16 or float32, got {t.dtype}")
+
+
+def _req(t, name, dtype=None, shape=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _seqs(cu_seqlens, B):
+    if cu_seqlens is None:
+        return 0, B
+    _req(cu_seqlens, "cu_seqlens", torch.int32)
+    n = cu_seqlens.numel() - 1
+    return n, n
+
+
+def osdn_precond_scan(k, beta, r=None, eta: float = 0.0, d0=None, cu_seqlens=None,
+                      k_tilde=None, dT=None, return_dT: bool = True, stream=None):
+    """Phase 1: returns ``(k_tilde, dT)`` (``dT`` is None when ``return_dT`` is False)."""
+    B, T, H, Dk = k.shape
+    io = _io(k)
+    num_seqs, N = _seqs(cu_seqlens, B)
+    _req(k, "k")
+    _req(beta, "beta", torch.float32, (B, T, H))
+    _req(r, "r", torch.float32, (B, T, H))
+    _req(d0, "d0", torch.float32, (N, H, Dk))
+    if k_tilde is None:
+        k_tilde = torch.empty_like(k)
+    _req(k_tilde, "k_tilde", k.dtype, k.shape)
+    if dT is None and return_dT:
+        dT = torch.empty((N, H, Dk), dtype=torch.float32, device=k.device)
+    _req(dT, "dT", torch.float32, (N, H, Dk))
+    _check(LIB.osdn_precond_scan(_p(k), _p(beta), _p(r), float(eta), _p(d0), _p(k_tilde), _p(dT),
+                                 _p(cu_seqlens), num_seqs, B, T, H, Dk, io, _stream(stream)),
+           "osdn_precond_scan")
+    return k_tilde, dT
+
+
+def osdn_chunk_fwd(q, k, k_tilde, v, beta, scale: float = 1.0, S0=None, chunk: int = 64,
+                   cu_seqlens=None, o=None, ST=None, return_ST: bool = True, stream=None):
+    """Phase 2: returns ``(o, ST)`` (``ST`` is None when ``return_ST`` is False)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    io = _io(q)
+    num_seqs, N = _seqs(cu_seqlens, B)
+    for name, t in (("q", q), ("k", k), ("k_tilde", k_tilde)):
+        _req(t, name, q.dtype, (B, T, H, Dk))
+    _req(v, "v", q.dtype, (B, T, H, Dv))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    _req(S0, "S0", torch.float32, (N, H, Dv, Dk))
+    if o is None:
+        o = torch.empty_like(v)
+    _req(o, "o", q.dtype, (B, T, H, Dv))
+    if ST is None and return_ST:
+        ST = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=q.device)
+    _req(ST, "ST", torch.float32, (N, H, Dv, Dk))
+    _check(LIB.osdn_chunk_fwd(_p(q), _p(k), _p(k_tilde), _p(v), _p(beta), float(scale), _p(S0),
+                              _p(o), _p(ST), _p(cu_seqlens), num_seqs, B, T, H, Dk, Dv,
+                              int(chunk), io, _stream(stream)),
+           "osdn_chunk_fwd")
+    return o, ST
+
+
+def osdn_fwd_workspace_bytes(B: int, T: int, H: int, Dk: int, dtype=torch.bfloat16) -> int:
+    io = OSDN_BF16 if dtype == torch.bfloat16 else OSDN_F32
+    return int(LIB.osdn_fwd_workspace_bytes(B, T, H, Dk, io))
+
+
+def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: float = 1.0,
+             chunk: int = 64, cu_seqlens=None, o=None, ST=None, dT=None, k_tilde=None,
+             workspace=None, return_states: bool = True, stream=None):
+    """Both phases: returns ``(o, ST, dT)`` (states None when ``return_states`` is False).
+
+    When neither ``k_tilde`` nor ``workspace`` is given, a workspace of
+    ``osdn_fwd_workspace_bytes`` bytes is allocated with torch (device memory plumbing).
+    """
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    io = _io(q)
+    num_seqs, N = _seqs(cu_seqlens, B)
+    for name, t in (("q", q), ("k", k)):
+        _req(t, name, q.dtype, (B, T, H, Dk))
+    _req(v, "v", q.dtype, (B, T, H, Dv))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    _req(r, "r", torch.float32, (B, T, H))
+    _req(d0, "d0", torch.float32, (N, H, Dk))
+    _req(S0, "S0", torch.float32, (N, H, Dv, Dk))
+    _req(k_tilde, "k_tilde", q.dtype, (B, T, H, Dk))
+    if o is None:
+        o = torch.empty_like(v)
+    _req(o, "o", q.dtype, (B, T, H, Dv))
+    if return_states:
+        if ST is None:
+            ST = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=q.device)
+        if dT is None:
+            dT = torch.empty((N, H, Dk), dtype=torch.float32, device=q.device)
+    _req(ST, "ST", torch.float32, (N, H, Dv, Dk))
+    _req(dT, "dT", torch.float32, (N, H, Dk))
+    ws_bytes = 0
+    if k_tilde is None:
+        need = int(LIB.osdn_fwd_workspace_bytes(B, T, H, Dk, io))
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if workspace is not None:
+            _req(workspace, "workspace")
+            ws_bytes = workspace.numel() * workspace.element_size()
+    _check(LIB.osdn_fwd(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), _p(d0), _p(S0),
+                        float(scale), _p(o), _p(ST), _p(dT), _p(k_tilde), _p(cu_seqlens),
+                        num_seqs, B, T, H, Dk, Dv, int(chunk), io,
+                        _p(workspace) if k_tilde is None else None, ws_bytes, _stream(stream)),
+           "osdn_fwd")
+    return o, ST, dT
+
+
+def osdn_get_device_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status word."""
+    return int(LIB.osdn_get_device_status(_stream(stream)))
+
+
+def osdn_debug_watchdog_selftest(spin_limit: int, stream=None):
+    _check(LIB.osdn_debug_watchdog_selftest(int(spin_limit), _stream(stream)),
+           "osdn_debug_watchdog_selftest")

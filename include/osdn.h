@@ -1,0 +1,157 @@
+/*
+ * osdn.h -- C ABI of libosdn, the B200 (sm_100a) forward pass of the Online Scaled DeltaNet
+ * (OSDN) token mixer.
+ *
+ * The method is the one of "OSDN: Improving Delta Rule with Provable Online Preconditioning
+ * in Linear Attention" (technical summary pages):
+ *   - section 2.1: the right-preconditioned delta-rule step equals the delta rule with the
+ *     write key k~_t = d_t (.) k_t, so the chunkwise WY pipeline of DeltaNet carries over
+ *     with K~ in place of K in the chunk Gram matrix and the intra-chunk scores;
+ *   - section 2.2: the preconditioner d follows online gradient descent on a surrogate whose
+ *     closed form depends only on k_t, beta_t and d_t, which splits the forward pass into a
+ *     light scan over the keys (phase 1) and the chunked DeltaNet pass (phase 2);
+ *   - section 2.3: APF, a per-token, per-head retention gate r_{t,h} applied to d only.
+ *
+ * Per (sequence n, head h), tokens t = 0..T_n-1, with a_t = k_t (.) k_t:
+ *   phase 1:  k~_t = d_t (.) k_t
+ *             d_{t+1} = r_t d_t + eta * beta_t (1 - beta_t <d_t, a_t>) a_t / ||k_t||^2
+ *             (descent on the surrogate; the step is 0 when ||k_t|| == 0; r == 1 without APF)
+ *   phase 2:  S_t = S_{t-1} + beta_t (v_t - S_{t-1} k_t) k~_t^T,   o_t = scale * S_t q_t
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers to dense row-major tensors owned by the caller, unless a
+ *     parameter says otherwise.  The library never allocates, frees or keeps a pointer.
+ *   - Every tensor pointer must be 16-byte aligned (OSDN_ERR_ALIGNMENT otherwise).
+ *   - Layouts:  q, k, k_tilde : [B, T, H, Dk]      v, o : [B, T, H, Dv]   (io dtype)
+ *               beta, r       : [B, T, H]  float32 in every io mode
+ *               S0, ST        : [N, H, Dv, Dk] float32 (row i of S is value channel i)
+ *               d0, dT        : [N, H, Dk] float32
+ *     Fixed length: cu_seqlens == NULL and N = B; sequence n is rows n*T .. n*T+T-1.
+ *     Packed variable length: cu_seqlens != NULL (DEVICE int32 array of num_seqs+1 offsets,
+ *     cu_seqlens[0] == 0, non-decreasing, cu_seqlens[num_seqs] == T), B == 1 and
+ *     N = num_seqs; sequence n is rows cu_seqlens[n] .. cu_seqlens[n+1]-1.  Chunks restart
+ *     at every sequence start and states are per sequence.  The offsets are checked on the
+ *     device: a sequence whose offsets are out of order or out of range is skipped and the
+ *     device status word records OSDN_ERR_DEVICE_BOUNDS (read it with
+ *     osdn_get_device_status).
+ *   - Supported sizes: Dk, Dv in {64, 128}; chunk 64 for OSDN_BF16, 16, 32 or 64 for
+ *     OSDN_F32; T >= 0, B >= 0, H >= 1.  Anything else returns OSDN_ERR_UNSUPPORTED.
+ *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Every call only
+ *     enqueues work on it and returns; nothing synchronizes.  Calls on different streams
+ *     may run concurrently as long as their output buffers do not overlap.
+ *   - Argument errors are reported before anything is enqueued and leave outputs untouched.
+ *     A failed kernel launch returns OSDN_ERR_CUDA.  No C++ exception crosses this ABI.
+ */
+#ifndef OSDN_H_
+#define OSDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OSDN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define OSDN_API __attribute__((visibility("default")))
+#else
+#define OSDN_API
+#endif
+
+typedef enum osdn_status {
+    OSDN_OK = 0,
+    OSDN_ERR_INVALID_ARG = 1,    /* NULL where a tensor is required, negative size, ...     */
+    OSDN_ERR_UNSUPPORTED = 2,    /* a size or mode this build does not implement            */
+    OSDN_ERR_ALIGNMENT = 3,      /* a tensor pointer that is not 16-byte aligned            */
+    OSDN_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed             */
+    OSDN_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait ran out (kernel returned)    */
+    OSDN_ERR_DEVICE_BOUNDS = 6   /* device-side check of cu_seqlens failed; sequence skipped */
+} osdn_status_t;
+
+typedef enum osdn_dtype {
+    OSDN_BF16 = 0, /* q, k, k_tilde, v, o in bfloat16; gates and states float32 */
+    OSDN_F32 = 1   /* q, k, k_tilde, v, o in float32 (every product in fp32 FMA) */
+} osdn_dtype_t;
+
+/* Version of this ABI (OSDN_ABI_VERSION of the build). */
+OSDN_API int32_t osdn_abi_version(void);
+
+/* Short English text for a status code (static storage; never NULL). */
+OSDN_API const char* osdn_status_string(osdn_status_t status);
+
+/*
+ * Phase 1: the preconditioner scan (section 2.2, first step of the two-phase split, with
+ * the APF gate of section 2.3).
+ *   k       [B,T,H,Dk] io dtype, read.
+ *   beta    [B,T,H] float32, read.
+ *   r       [B,T,H] float32 retention gate, or NULL for r == 1 (plain OSDN, no APF).
+ *   eta     step size of the preconditioner's gradient descent (eta == 0 freezes d).
+ *   d0      [N,H,Dk] initial preconditioner, or NULL for all ones.
+ *   k_tilde [B,T,H,Dk] io dtype, written: k~_t = d_t (.) k_t.  Must not alias k.
+ *   dT      [N,H,Dk] final preconditioner, written; NULL skips it.
+ */
+OSDN_API osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r, float eta,
+                                const float* d0, void* k_tilde, float* dT,
+                                const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                                int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io,
+                                void* stream);
+
+/*
+ * Phase 2: the chunkwise-parallel delta rule with write key K~ (section 2.1: K~ replaces K
+ * in the chunk Gram matrix and in the intra-chunk scores).
+ *   q, k    [B,T,H,Dk] io dtype, read (k is the erase/read key of the residual).
+ *   k_tilde [B,T,H,Dk] io dtype, read (the write key).
+ *   v       [B,T,H,Dv] io dtype, read.   beta [B,T,H] float32, read.
+ *   scale   multiplies o only (1.0 for unit-norm q).
+ *   S0      [N,H,Dv,Dk] initial state, or NULL for zeros.
+ *   o       [B,T,H,Dv] io dtype, written: o_t = scale * S_t q_t (state after token t).
+ *   ST      [N,H,Dv,Dk] final state, written; NULL skips it.
+ *   chunk   tokens per chunk (64 for bf16; 16, 32 or 64 for f32).  The result does not
+ *           depend on it beyond rounding.
+ */
+OSDN_API osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, const void* v,
+                             const float* beta, float scale, const float* S0, void* o, float* ST,
+                             const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                             int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
+                             void* stream);
+
+/* Bytes of device workspace osdn_fwd needs for these sizes (0 when none). */
+OSDN_API size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io);
+
+/*
+ * Both phases (section 2.2's two-phase forward pass) on one stream.  Arguments are those of
+ * osdn_precond_scan and osdn_chunk_fwd; in addition:
+ *   k_tilde_out  [B,T,H,Dk] io dtype, or NULL.  When given, the preconditioned keys are
+ *                written there and the workspace is not used.
+ *   workspace    device scratch of at least osdn_fwd_workspace_bytes(...) bytes, 256-byte
+ *                aligned, used when k_tilde_out is NULL; NULL only if that size is 0.
+ */
+OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* r, float eta, const float* d0, const float* S0, float scale,
+                       void* o, float* ST, float* dT, void* k_tilde_out,
+                       const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                       int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronizes `stream`, then returns and clears the device status word of the current
+ * device: OSDN_OK, OSDN_ERR_DEVICE_TIMEOUT or OSDN_ERR_DEVICE_BOUNDS (the first error any
+ * kernel recorded since the last call; the word is shared by all streams of the device).
+ * Returns OSDN_ERR_CUDA if the synchronization itself fails.
+ */
+OSDN_API osdn_status_t osdn_get_device_status(void* stream);
+
+/*
+ * Diagnostic: launches one block that waits on a shared-memory barrier nobody arrives at,
+ * with at most `spin_limit` polls (1 .. 2^30), so the bounded wait runs out, records
+ * OSDN_ERR_DEVICE_TIMEOUT in the device status word and returns.  Enqueue only.
+ */
+OSDN_API osdn_status_t osdn_debug_watchdog_selftest(int64_t spin_limit, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OSDN_H_ */

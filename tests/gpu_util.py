@@ -1,0 +1,76 @@
+"""Shared helpers for the GPU tests: run the library through its binding, run the oracle on the
+same seeded inputs, and measure max|delta| / rms(reference)."""
+import numpy as np
+import torch
+
+from delta_rule_recurrent_osdn_b200 import inputs as W
+
+TOL = {"bf16": 1e-2, "f32": 1e-4}  # max|gpu - oracle| / rms(oracle), per output
+
+
+def half_ulp(x, io):
+    """Half a unit in the last place of |x| in the output dtype: the error of storing the exact
+    value in that dtype (bf16: 8 significant bits; f32: 24)."""
+    bits = {"bf16": 8, "f32": 24}[io]
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - bits), 0.0)
+
+
+def rel_err(gpu, ref, io=None):
+    """max_i |gpu_i - ref_i| / rms(ref).  With `io` given (the dtype the GPU stored the result
+    in), each element's error first loses half an ulp of ref_i in that dtype: the rounding of
+    the exact result to the output dtype is not an error of the computation."""
+    ref = np.asarray(ref, dtype=np.float64)
+    gpu = np.asarray(gpu, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    if ref.size == 0:
+        return 0.0
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    assert np.all(np.isfinite(gpu)), "non-finite GPU output"
+    err = np.abs(gpu - ref)
+    if io is not None:
+        err = np.maximum(err - half_ulp(ref, io), 0.0)
+    return float(np.max(err)) / max(rms, 1e-30)
+
+
+def host(t):
+    return None if t is None else t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def gpu_fwd(inp, chunk=None, split=False):
+    """Run the library on one batch; returns numpy (o, k_tilde, ST, dT)."""
+    from delta_rule_recurrent_osdn_b200 import osdn
+    d = W.to_torch(inp)
+    chunk = chunk or d["chunk"]
+    if split:
+        kt, dT = osdn.osdn_precond_scan(d["k"], d["beta"], d["r"], d["eta"], d["d0"],
+                                        d["cu_seqlens"])
+        o, ST = osdn.osdn_chunk_fwd(d["q"], d["k"], kt, d["v"], d["beta"], d["scale"], d["S0"],
+                                    chunk, d["cu_seqlens"])
+    else:
+        kt = torch.empty_like(d["k"])
+        o, ST, dT = osdn.osdn_fwd(d["q"], d["k"], d["v"], d["beta"], d["r"], d["eta"], d["d0"],
+                                  d["S0"], d["scale"], chunk, d["cu_seqlens"], k_tilde=kt)
+    torch.cuda.synchronize()
+    assert osdn.osdn_get_device_status() == osdn.OSDN_OK
+    return host(o), host(kt), host(ST), host(dT)
+
+
+def oracle_fwd(ref, inp):
+    return ref.fwd(inp.q, inp.k, inp.v, inp.beta, inp.r, inp.eta, inp.d0, inp.S0, inp.scale,
+                   inp.cu_seqlens)
+
+
+# o and k~ are stored in the io dtype, S_T and d_T in float32
+STORED = {"o": None, "k_tilde": None, "ST": "f32", "dT": "f32"}
+
+
+def check_all(got, want, io, names=("o", "k_tilde", "ST", "dT")):
+    """Parity of every output: max|gpu - oracle| / rms(oracle) <= TOL[io], after removing from
+    each element the half-ulp rounding of the exact value to the dtype it is stored in."""
+    errs = {n: rel_err(g, w, STORED[n] or io) for n, g, w in zip(names, got, want)}
+    raw = {n: rel_err(g, w) for n, g, w in zip(names, got, want)}
+    bad = {n: e for n, e in errs.items() if not e <= TOL[io]}
+    assert not bad, f"parity failed ({io}, tol {TOL[io]}): {errs} (raw {raw})"
+    return {"err": errs, "raw": raw}

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every symbol include/osdn.h declares,
+and rejects bad arguments before anything reaches CUDA (no compute call is made here)."""
+import ctypes
+
+import pytest
+
+osdn = pytest.importorskip("delta_rule_recurrent_osdn_b200.osdn")
+L = osdn.LIB
+A = 0x10000000  # a 16-byte aligned fake address; validation failures never dereference it
+
+
+def fake(i):
+    return ctypes.c_void_p(A + i * 0x1000000)
+
+
+def chunk_call(**kw):
+    args = dict(q=fake(1), k=fake(2), kt=fake(3), v=fake(4), beta=fake(5), scale=1.0, S0=None,
+                o=fake(6), ST=None, cu=None, num_seqs=0, B=1, T=8, H=1, Dk=128, Dv=128, chunk=64,
+                io=osdn.OSDN_BF16)
+    args.update(kw)
+    return L.osdn_chunk_fwd(args["q"], args["k"], args["kt"], args["v"], args["beta"],
+                            args["scale"], args["S0"], args["o"], args["ST"], args["cu"],
+                            args["num_seqs"], args["B"], args["T"], args["H"], args["Dk"],
+                            args["Dv"], args["chunk"], args["io"], None)
+
+
+def scan_call(**kw):
+    args = dict(k=fake(1), beta=fake(2), r=None, eta=0.1, d0=None, kt=fake(3), dT=None, cu=None,
+                num_seqs=0, B=1, T=8, H=1, Dk=128, io=osdn.OSDN_BF16)
+    args.update(kw)
+    return L.osdn_precond_scan(args["k"], args["beta"], args["r"], args["eta"], args["d0"],
+                               args["kt"], args["dT"], args["cu"], args["num_seqs"], args["B"],
+                               args["T"], args["H"], args["Dk"], args["io"], None)
+
+
+def test_exports_every_declared_symbol():
+    names = osdn.header_symbols()
+    assert {"osdn_precond_scan", "osdn_chunk_fwd", "osdn_fwd", "osdn_fwd_workspace_bytes",
+            "osdn_status_string", "osdn_get_device_status"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings():
+    assert L.osdn_abi_version() == 1
+    for s in range(7):
+        assert osdn.status_string(s)
+    assert osdn.status_string(99) == "unknown status"
+
+
+def test_workspace_size():
+    assert L.osdn_fwd_workspace_bytes(4, 4096, 16, 128, osdn.OSDN_BF16) == 4 * 4096 * 16 * 128 * 2
+    assert L.osdn_fwd_workspace_bytes(1, 3, 1, 64, osdn.OSDN_F32) == 768
+    assert L.osdn_fwd_workspace_bytes(1, 1, 1, 96, osdn.OSDN_BF16) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Dk=96), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(Dv=32), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(chunk=32), osdn.OSDN_ERR_UNSUPPORTED),          # bf16 path runs 64-token chunks
+    (dict(chunk=48, io=osdn.OSDN_F32), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(q=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(o=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(B=-1), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(H=0), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(T=-5), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(io=7), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(cu=fake(9), num_seqs=2, B=2), osdn.OSDN_ERR_INVALID_ARG),  # packed needs B == 1
+    (dict(v=ctypes.c_void_p(A + 8)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(S0=ctypes.c_void_p(A + 4)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(o=fake(1)), osdn.OSDN_ERR_INVALID_ARG),          # output aliases q
+])
+def test_chunk_fwd_rejects(kw, status):
+    assert chunk_call(**kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Dk=32), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(k=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(kt=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(kt=fake(1)), osdn.OSDN_ERR_INVALID_ARG),          # in place k~ == k
+    (dict(kt=ctypes.c_void_p(A + 0x1000000 + 256)), osdn.OSDN_ERR_INVALID_ARG),  # overlap
+    (dict(r=ctypes.c_void_p(A + 2)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(cu=ctypes.c_void_p(A + 4), num_seqs=1), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(num_seqs=-1), osdn.OSDN_ERR_INVALID_ARG),
+])
+def test_precond_scan_rejects(kw, status):
+    assert scan_call(**kw) == status
+
+
+def test_fwd_rejects_small_workspace():
+    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
+                    None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16, fake(7), 100,
+                    None)
+    assert st == osdn.OSDN_ERR_INVALID_ARG
+    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
+                    None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16,
+                    ctypes.c_void_p(A + 0x7000010), 1 << 20, None)
+    assert st == osdn.OSDN_ERR_ALIGNMENT  # workspace must be 256-byte aligned
+
+
+def test_parity_metric_allows_exactly_the_output_rounding():
+    """The GPU tests' metric: storing the exact value in bf16 costs nothing; anything beyond
+    half an ulp counts."""
+    import numpy as np
+    from delta_rule_recurrent_osdn_b200.inputs import bf16_round
+    from tests.gpu_util import rel_err
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(100000) * 3).astype(np.float32).astype(np.float64)
+    xb = bf16_round(x.astype(np.float32)).astype(np.float64)
+    assert rel_err(xb, x) > 1e-3           # raw rounding error is visible
+    assert rel_err(xb, x, "bf16") == 0.0   # and is exactly what the allowance removes
+    y = xb.copy()
+    y[7] += 0.05
+    assert 0.04 / 3 < rel_err(y, x, "bf16") < 0.06 / 2.9
