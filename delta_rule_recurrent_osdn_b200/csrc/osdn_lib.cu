@@ -4,6 +4,8 @@
 // The host code validates arguments, picks a kernel for the sizes and dtype, and enqueues it
 // on the caller's stream.  It never allocates memory and never synchronizes, except in
 // osdn_get_device_status, whose job is to synchronize.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -13,6 +15,7 @@
 #include "scan_warp.cuh"
 #include "chunk_simt.cuh"
 #include "watchdog.cuh"
+#include "chunk_tc.cuh"
 
 namespace osdn {
 namespace {
@@ -116,11 +119,73 @@ osdn_status_t launch_chunk_c(int chunk, const void* q, const void* k, const void
     }
 }
 
+// The tensor-core phase-2 kernel is built but not yet dispatched.
+constexpr bool kTensorCoreChunk = false;
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (the library
+// does not link libcuda directly).
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+EncodeTiledFn tensor_map_encoder() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 3-D bf16 view [rows][H][D] of a [B, T, H, D] tensor; boxes of 64 channels x 1 head x 64
+// tokens, 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_tile_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows) {
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (!enc || rows <= 0) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DV>
+osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, const void* v,
+                              const float* beta, float scale, const float* S0, void* o,
+                              float* ST, const int32_t* cu, const Dims& d, cudaStream_t stream) {
+    const int64_t ctas = (int64_t)d.N * d.H * (DV / 64);
+    if (ctas == 0) return OSDN_OK;
+    if (ctas > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mkt, mv;
+    const int64_t rows = d.rows();
+    if (!make_tile_map(&mq, q, 128, d.H, rows) || !make_tile_map(&mk, k, 128, d.H, rows) ||
+        !make_tile_map(&mkt, kt, 128, d.H, rows) || !make_tile_map(&mv, v, DV, d.H, rows))
+        return OSDN_ERR_CUDA;
+    auto kernel = chunk_fwd_tc_kernel<DV>;
+    if (!set_smem(kernel, TcSmem::BYTES)) return OSDN_ERR_CUDA;
+    kernel<<<dim3((unsigned)ctas), dim3(128), TcSmem::BYTES, stream>>>(
+        mq, mk, mkt, mv, beta, scale, S0, static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T, d.H,
+        (long long)kWaitLimitNs);
+    return launch_status();
+}
+
 template <typename IO>
 osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* kt,
                            const void* v, const float* beta, float scale, const float* S0,
                            void* o, float* ST, const int32_t* cu, const Dims& d,
                            cudaStream_t stream) {
+    // bf16 I/O with 128 key channels runs on the tensor cores; fp32 I/O, 64 key channels and
+    // token-free calls (states pass through) run the fp32 SIMT kernel.
+    if constexpr (sizeof(IO) == 2 && kTensorCoreChunk) {
+        if (d.Dk == 128 && chunk == 64 && d.rows() > 0 && d.rows() < (int64_t(1) << 31)) {
+            if (d.Dv == 128)
+                return launch_chunk_tc<128>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
+            return launch_chunk_tc<64>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
+        }
+    }
     if (d.Dk == 128 && d.Dv == 128)
         return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
                                             stream);

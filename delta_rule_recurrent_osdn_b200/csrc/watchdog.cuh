@@ -43,15 +43,30 @@ __device__ __forceinline__ bool mbar_try_parity(uint64_t* bar, uint32_t parity) 
     return done != 0;
 }
 
-// Wait until the phase with the given parity has completed, polling at most `limit` times.
-// Returns false (after recording OSDN_ERR_DEVICE_TIMEOUT) if it never completed.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait until the phase with the given parity has completed, for at most `limit_ns`
+// nanoseconds of wall time.  Returns false (after recording OSDN_ERR_DEVICE_TIMEOUT) if it
+// never completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  int64_t limit) {
-    for (int64_t i = 0; i < limit; ++i)
+                                                  int64_t limit_ns) {
+    if (mbar_try_parity(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
         if (mbar_try_parity(bar, parity)) return true;
+        if (global_ns() - t0 > static_cast<uint64_t>(limit_ns)) break;
+    }
     record_status(OSDN_ERR_DEVICE_TIMEOUT);
     return false;
 }
+
+// Bound on every wait inside the tensor-core kernels: far above any legitimate wait (those
+// last microseconds), short enough that a stuck kernel returns within seconds.
+constexpr int64_t kWaitLimitNs = 2000000000LL;
 
 // Diagnostic kernel: waits on a barrier that nobody arrives at, with a bounded number of
 // non-blocking polls, so that the timeout path runs and the kernel returns.

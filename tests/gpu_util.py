@@ -57,7 +57,28 @@ def gpu_fwd(inp, chunk=None, split=False):
     return host(o), host(kt), host(ST), host(dT)
 
 
+def round_io(x, io):
+    """x rounded to the io dtype (bf16 RNE, or fp32), returned as float64."""
+    x = np.asarray(x, dtype=np.float32)
+    return (W.bf16_round(x) if io == "bf16" else x).astype(np.float64)
+
+
 def oracle_fwd(ref, inp):
+    """Expected (o, k_tilde, ST, dT) for the two-phase forward pass.
+
+    Phase 1 is the oracle's scan.  Phase 2 is the oracle's token loop fed k~ rounded to the io
+    dtype: the two-phase interface hands k~ from the scan to the chunked pass as an io-dtype
+    tensor, so that rounding is part of what the library is asked to compute.  Everything else
+    is fp64.
+    """
+    kt, dT = ref.precond_scan(inp.k, inp.beta, inp.r, inp.eta, inp.d0, inp.cu_seqlens)
+    o, ST = ref.delta_fwd(inp.q, inp.k, round_io(kt, inp.io), inp.v, inp.beta, inp.scale,
+                          inp.S0, inp.cu_seqlens)
+    return o, kt, ST, dT
+
+
+def oracle_fwd_unrounded(ref, inp):
+    """The fp64 oracle with no io rounding of k~ between the phases (for reporting)."""
     return ref.fwd(inp.q, inp.k, inp.v, inp.beta, inp.r, inp.eta, inp.d0, inp.S0, inp.scale,
                    inp.cu_seqlens)
 
