@@ -348,3 +348,65 @@ osdn_status_t osdn_debug_watchdog_selftest(int64_t spin_limit, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// osdn_fwd_noalloc: osdn_fwd for callers that cannot allocate device memory.
+//
+// The preconditioned keys that phase 1 hands to phase 2 normally live in a workspace the
+// caller allocates.  Here they live in this file's fixed device array instead, so the caller
+// passes only its inputs and outputs.  The array is part of the library image: every GPU that
+// loads the library reserves it until the process exits.
+// ------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace osdn {
+namespace {
+
+constexpr size_t kNoallocScratchBytes = OSDN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device.  In host code the array's name is only a
+// host-side stand-in, so the address is looked up once per device (with that device current)
+// and cached.
+osdn_status_t noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OSDN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return OSDN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return OSDN_OK;
+}
+
+}  // namespace
+}  // namespace osdn
+
+extern "C" osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                          const float* beta, const float* r, float eta,
+                                          const float* d0, const float* S0, float scale, void* o,
+                                          float* ST, float* dT, const int32_t* cu_seqlens,
+                                          int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                                          int32_t Dk, int32_t Dv, int32_t chunk,
+                                          osdn_dtype_t io, void* stream) {
+    if (B < 0 || T < 0 || H < 1 || (io != OSDN_BF16 && io != OSDN_F32))
+        return OSDN_ERR_INVALID_ARG;
+    if (Dk != 64 && Dk != 128) return OSDN_ERR_UNSUPPORTED;
+    const size_t need = osdn_fwd_workspace_bytes(B, T, H, Dk, io);
+    if (need > kNoallocScratchBytes) return OSDN_ERR_UNSUPPORTED;  // keys do not fit the array
+    void* scratch = nullptr;
+    if (need > 0) {
+        const osdn_status_t st = noalloc_scratch(&scratch);
+        if (st != OSDN_OK) return st;
+    }
+    return osdn_fwd(q, k, v, beta, r, eta, d0, S0, scale, o, ST, dT, nullptr, cu_seqlens,
+                    num_seqs, B, T, H, Dk, Dv, chunk, io, scratch, need > 0 ? kNoallocScratchBytes : 0,
+                    stream);
+}

@@ -136,6 +136,35 @@ OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, con
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * osdn_fwd without any workspace, for callers that cannot allocate device memory: code that
+ * runs inside a host application or plugin framework which owns every device allocation, or a
+ * latency-critical service that forbids cudaMalloc after start-up (an allocation can
+ * synchronize the device and fragments a fixed memory budget).  The original paper has no
+ * counterpart: this is an interface convenience, not part of the method.
+ *
+ * Arguments are those of osdn_fwd minus k_tilde_out / workspace.  The preconditioned keys that
+ * phase 1 hands to phase 2 go to a fixed device array built into the library,
+ * OSDN_NOALLOC_SCRATCH_BYTES (32 MiB) long, which every GPU that loads the library reserves
+ * until the process exits.
+ *   - Limit: B * T * H * Dk * sizeof(io element) must not exceed OSDN_NOALLOC_SCRATCH_BYTES;
+ *     larger calls return OSDN_ERR_UNSUPPORTED before anything is enqueued.
+ *   - The first call on each device (with that device current) looks up the array's device
+ *     address and caches it; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.  Phase 1 rewrites
+ *     every key before phase 2 reads it, so nothing needs clearing; but calls that overlap on
+ *     the GPU (other streams, other host threads) race on it and must be serialized.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define OSDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                        const float* beta, const float* r, float eta,
+                                        const float* d0, const float* S0, float scale, void* o,
+                                        float* ST, float* dT, const int32_t* cu_seqlens,
+                                        int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                                        int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
+                                        void* stream);
+
+/*
  * Synchronizes `stream`, then returns and clears the device status word of the current
  * device: OSDN_OK, OSDN_ERR_DEVICE_TIMEOUT or OSDN_ERR_DEVICE_BOUNDS (the first error any
  * kernel recorded since the last call; the word is shared by all streams of the device).
