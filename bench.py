@@ -58,7 +58,7 @@ def kernel_source_sha(names):
 
 
 KERNEL_SOURCES = {"scan": ["common.cuh", "scan_warp.cuh"],
-                  "chunk": ["common.cuh", "chunk_simt.cuh"]}
+                  "chunk": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "chunk_tc.cuh"]}
 
 
 def profiled_traffic(kernel):

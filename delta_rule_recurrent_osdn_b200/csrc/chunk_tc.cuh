@@ -37,7 +37,7 @@ struct TcSmem {
     static constexpr uint32_t Z = 2 * STAGE;          // fp32 [T; P], 2 K-blocks of 16K
     static constexpr uint32_t SHI = Z + 32768;        // bf16 S^T hi, 128 rows x 128 B
     static constexpr uint32_t SLO = SHI + 16384;
-    static constexpr uint32_t RW = SLO + 16384;       // fp32 R, then W (2 column blocks of 8K)
+    static constexpr uint32_t RW = SLO + 16384;       // fp32 R^T, then W^T (K-major, 2 blocks of 8K)
     static constexpr uint32_t WHI = RW + 16384;       // bf16 W hi, 64 rows x 128 B
     static constexpr uint32_t WLO = WHI + 8192;
     static constexpr uint32_t SOLVE = RW;             // fp32 L and M scratch (64 x 65 each)
@@ -58,16 +58,17 @@ __device__ __forceinline__ uint32_t z_off(uint32_t r, uint32_t c) {
     return (c >> 5) * 16384u + tc::sw128_off(r, (c & 31u) >> 2) + (c & 3u) * 4u;
 }
 
-// Write one fp32 row of 64 values into an MN-major fp32 tile (two 32-wide column blocks,
-// 8 KB apart): row = K index.
-__device__ __forceinline__ void st_row_f32_mn(uint8_t* tile, uint32_t row, const float* x) {
+// Write token row t (64 fp32 values over the value channels c) as column t of a K-major fp32
+// B operand: rows = N index c (64 rows), K index t in two 32-wide blocks 8 KB apart.  (The MMA
+// accepts 32-bit MN-major operands only in a 32-byte-atom swizzle; the K-major form keeps the
+// standard 128-byte swizzle.)  The 32 lanes of a warp fill one 128-byte row: no bank conflicts.
+__device__ __forceinline__ void st_col_f32_k(uint8_t* tile, uint32_t t, const float* x) {
+    uint8_t* base = tile + (t >> 5) * 8192u + (t & 3u) * 4u;
+    const uint32_t chunk = (t & 31u) >> 2;
 #pragma unroll
-    for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(tile + blk * 8192 + tc::sw128_off(row, j)) =
-                make_float4(x[blk * 32 + 4 * j], x[blk * 32 + 4 * j + 1], x[blk * 32 + 4 * j + 2],
-                            x[blk * 32 + 4 * j + 3]);
+    for (int c = 0; c < 64; ++c)
+        *reinterpret_cast<float*>(base + (uint32_t)c * 128u + ((chunk ^ ((uint32_t)c & 7u)) << 4)) =
+            x[c];
 }
 
 // Split a 64-value fp32 row into bf16 hi + lo and write both rows (128 B each, swizzled).
@@ -261,7 +262,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     };
     constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);   // [K;Q] x K~^T
     constexpr uint32_t ID_1 = tc::idesc(1, 0, 1, 128, 64);   // [K;Q] x S^T
-    constexpr uint32_t ID_TF = tc::idesc(2, 0, 1, 128, 64);  // [T;P] x (R | W), tf32
+    constexpr uint32_t ID_TF = tc::idesc(2, 0, 0, 128, 64);  // [T;P] x (R | W), tf32
     constexpr uint32_t ID_3 = tc::idesc(1, 1, 1, 128, 64);   // K~^T x W
 
 #pragma unroll 1
@@ -344,7 +345,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     r[8 * j + 2 * e + 1] = bt * (vv.y - y[8 * j + 2 * e + 1]);
                 }
             }
-            st_row_f32_mn(RW, tid, r);
+            st_col_f32_k(RW, tid, r);
         }
         tc::fence_async_smem();
         if (sync_failed()) break;
@@ -356,14 +357,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int s = 0; s < 8; ++s)
                 tc::mma_tf32(tmem + TC_COL_D2,
                              tc::sw128_desc(aZ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             tc::sw128_desc(aRW + s * 1024, 8192, 1024), ID_TF, s > 0);
+                             tc::sw128_desc(aRW + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_TF, s > 0);
             commit();
         }
         wait_mma();
         if (tid < 64) {
             float w[64];
             tc::tmem_ld64(t_D2, w);
-            st_row_f32_mn(RW, tid, w);
+            st_col_f32_k(RW, tid, w);
             st_row_split_bf16(WHI, WLO, tid, w);
         }
         tc::fence_async_smem();
@@ -383,7 +384,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int s = 0; s < 8; ++s)
                 tc::mma_tf32(tmem + TC_COL_D1,
                              tc::sw128_desc(aZ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             tc::sw128_desc(aRW + s * 1024, 8192, 1024), ID_TF, 1);
+                             tc::sw128_desc(aRW + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_TF, 1);
             commit();
         }
         wait_mma();

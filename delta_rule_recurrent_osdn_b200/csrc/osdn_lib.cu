@@ -119,9 +119,6 @@ osdn_status_t launch_chunk_c(int chunk, const void* q, const void* k, const void
     }
 }
 
-// The tensor-core phase-2 kernel is built but not yet dispatched.
-constexpr bool kTensorCoreChunk = false;
-
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime (the library
 // does not link libcuda directly).
 using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
@@ -179,7 +176,7 @@ osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* 
                            cudaStream_t stream) {
     // bf16 I/O with 128 key channels runs on the tensor cores; fp32 I/O, 64 key channels and
     // token-free calls (states pass through) run the fp32 SIMT kernel.
-    if constexpr (sizeof(IO) == 2 && kTensorCoreChunk) {
+    if constexpr (sizeof(IO) == 2) {
         if (d.Dk == 128 && chunk == 64 && d.rows() > 0 && d.rows() < (int64_t(1) << 31)) {
             if (d.Dv == 128)
                 return launch_chunk_tc<128>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
