@@ -57,7 +57,7 @@ def kernel_source_sha(names):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"scan": ["common.cuh", "scan_warp.cuh"],
+KERNEL_SOURCES = {"scan": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "scan_chunk.cuh"],
                   "chunk": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "chunk_tc.cuh"]}
 
 

@@ -7,15 +7,16 @@
 //   G = K K~^T,  P = tril(Q K~^T)                 one bf16 MMA, A = [K; Q] (M = 128)
 //   T = (I + strict_tril(diag(beta) G))^-1        fp32 blocked solve in shared memory
 //   R = diag(beta) (V - K S_0^T)                  A = [K; Q], B = S_0^T  (rows 64..127: Q S_0^T)
-//   W = T R                                       A = Z = [T; P], B = R  (tf32)
-//   O = Q S_0^T + P W                             A = Z, B = W, accumulated onto Q S_0^T (tf32)
+//   W = T R                                       A = Z = [T; P], B = R
+//   O = Q S_0^T + P W                             A = Z, B = W, accumulated onto Q S_0^T
 //   S_C^T = S_0^T + K~^T W                        A = K~^T (MN-major view of the K~ tile)
 //
-// Precision.  Products of an exact bf16 input (K, Q, K~) with the state or with W use a
-// two-term bf16 split of the computed operand (x = hi + lo, both bf16; two MMAs), which keeps
-// about 16 significant bits; products of two computed operands (T, P, R, W) run as tf32 MMAs.
-// An all-bf16 variant was measured (CPU emulation) at 1.5-2.5% max/rms error on o and S_T for
-// the 340M and 1.3B workloads, this scheme at 0.13-0.24%.
+// Precision.  Every computed MMA operand x is split into two bf16 terms, x = hi + lo (about 16
+// significant bits).  A product of an exact bf16 input (K, Q, K~) with a computed operand takes
+// two MMAs (hi, lo); a product of two computed operands ([T; P] with R or W) takes three
+// (hi*hi + hi*lo + lo*hi).  In a CPU emulation of this chunk algorithm against the oracle, plain
+// bf16 operands gave 1.5-2.5% max/rms error on o and S_T for the 340M and 1.3B workloads, and
+// single-term tf32 products 0.25-0.46%; the split scheme is at the fp32 rounding level.
 //
 // Layout.  One CTA per (sequence, head, 64 value channels), 128 threads: thread t owns tensor
 // memory lane t.  Accumulators in tensor memory (fp32, 128 lanes): S^T (lanes = key channel),
@@ -34,13 +35,17 @@ namespace osdn {
 struct TcSmem {
     static constexpr uint32_t STAGE = 57344;          // [K;Q] 32K | K~ 16K | V 8K
     static constexpr uint32_t KQ = 0, KT = 32768, V = 49152;
-    static constexpr uint32_t Z = 2 * STAGE;          // fp32 [T; P], 2 K-blocks of 16K
-    static constexpr uint32_t SHI = Z + 32768;        // bf16 S^T hi, 128 rows x 128 B
+    // bf16 [T; P] hi and lo, K-major, 128 rows x 128 B each.  While T is being solved it is
+    // held in fp32 in rows 0..63 of both tiles (the bytes of z_off(r < 64, c)).
+    static constexpr uint32_t ZHI = 2 * STAGE;
+    static constexpr uint32_t ZLO = ZHI + 16384;
+    static constexpr uint32_t SHI = ZLO + 16384;      // bf16 S^T hi, 128 rows x 128 B
     static constexpr uint32_t SLO = SHI + 16384;
-    static constexpr uint32_t RW = SLO + 16384;       // fp32 R^T, then W^T (K-major, 2 blocks of 8K)
-    static constexpr uint32_t WHI = RW + 16384;       // bf16 W hi, 64 rows x 128 B
+    static constexpr uint32_t RHI = SLO + 16384;      // bf16 R hi / lo, 64 rows x 128 B
+    static constexpr uint32_t RLO = RHI + 8192;
+    static constexpr uint32_t WHI = RLO + 8192;       // bf16 W hi / lo, 64 rows x 128 B
     static constexpr uint32_t WLO = WHI + 8192;
-    static constexpr uint32_t SOLVE = RW;             // fp32 L and M scratch (64 x 65 each)
+    static constexpr uint32_t SOLVE = RHI;            // fp32 L and M scratch (64 x 65 each)
     static constexpr uint32_t SOLVE_END = SOLVE + 2 * 64 * 65 * 4;
     static constexpr uint32_t BAR = SOLVE_END;        // 3 mbarriers
     static constexpr uint32_t TMEM_SLOT = BAR + 32;
@@ -53,22 +58,10 @@ static_assert(TcSmem::BYTES <= 232448, "shared memory");
 constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 128, TC_COL_G = 192;
 constexpr uint32_t TC_TMEM_COLS = 256;
 
-// fp32 element (r, c) of the [T; P] tile: K-major, 32 fp32 per 128-byte row, 2 K-blocks.
+// fp32 element (r, c), r < 64, of T while it is being solved: 32 fp32 per 128-byte row, the
+// two 32-column halves in the hi and lo tiles.
 __device__ __forceinline__ uint32_t z_off(uint32_t r, uint32_t c) {
     return (c >> 5) * 16384u + tc::sw128_off(r, (c & 31u) >> 2) + (c & 3u) * 4u;
-}
-
-// Write token row t (64 fp32 values over the value channels c) as column t of a K-major fp32
-// B operand: rows = N index c (64 rows), K index t in two 32-wide blocks 8 KB apart.  (The MMA
-// accepts 32-bit MN-major operands only in a 32-byte-atom swizzle; the K-major form keeps the
-// standard 128-byte swizzle.)  The 32 lanes of a warp fill one 128-byte row: no bank conflicts.
-__device__ __forceinline__ void st_col_f32_k(uint8_t* tile, uint32_t t, const float* x) {
-    uint8_t* base = tile + (t >> 5) * 8192u + (t & 3u) * 4u;
-    const uint32_t chunk = (t & 31u) >> 2;
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-        *reinterpret_cast<float*>(base + (uint32_t)c * 128u + ((chunk ^ ((uint32_t)c & 7u)) << 4)) =
-            x[c];
 }
 
 // Split a 64-value fp32 row into bf16 hi + lo and write both rows (128 B each, swizzled).
@@ -146,6 +139,20 @@ __device__ __forceinline__ void solve_unit_lower_64(const float* sL, float* sM, 
     }
 }
 
+// D (+)= [T; P] X over K = 64 tokens, as hi*hi + hi*lo + lo*hi: A = the K-major [T; P] tiles
+// (z[0] = hi, z[1] = lo), B = the MN-major 64 x 64 tiles of X (x[0] = hi, x[1] = lo).
+__device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, const uint32_t* x,
+                                           uint32_t id, bool accumulate) {
+    const int pairs[3][2] = {{0, 0}, {0, 1}, {1, 0}};
+#pragma unroll
+    for (int p = 0; p < 3; ++p)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            tc::mma_bf16(d_tmem, tc::sw128_desc(z[pairs[p][0]] + s * 32, 16, 1024),
+                         tc::sw128_desc(x[pairs[p][1]] + s * 2048, 8192, 1024), id,
+                         (accumulate || p > 0 || s > 0) ? 1u : 0u);
+}
+
 template <int DV>
 __global__ void __launch_bounds__(128, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -171,10 +178,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* mma_bar = tma_bar + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
-    uint8_t* Z = smem + L::Z;
+    uint8_t* Z = smem + L::ZHI;  // fp32 T during the solve (rows 0..63 of ZHI and ZLO)
+    uint8_t* ZHI = smem + L::ZHI;
+    uint8_t* ZLO = smem + L::ZLO;
     uint8_t* SHI = smem + L::SHI;
     uint8_t* SLO = smem + L::SLO;
-    uint8_t* RW = smem + L::RW;
+    uint8_t* RHI = smem + L::RHI;
+    uint8_t* RLO = smem + L::RLO;
     uint8_t* WHI = smem + L::WHI;
     uint8_t* WLO = smem + L::WLO;
     float* sL = reinterpret_cast<float*>(smem + L::SOLVE);
@@ -262,7 +272,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     };
     constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);   // [K;Q] x K~^T
     constexpr uint32_t ID_1 = tc::idesc(1, 0, 1, 128, 64);   // [K;Q] x S^T
-    constexpr uint32_t ID_TF = tc::idesc(2, 0, 0, 128, 64);  // [T;P] x (R | W), tf32
+    constexpr uint32_t ID_Z = tc::idesc(1, 0, 1, 128, 64);   // [T;P] x (R | W)
     constexpr uint32_t ID_3 = tc::idesc(1, 1, 1, 128, 64);   // K~^T x W
 
 #pragma unroll 1
@@ -270,7 +280,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int stage = ch & 1;
         uint8_t* st = smem + stage * L::STAGE;
         const uint32_t aKQ = smem_u32(st + L::KQ), aKT = smem_u32(st + L::KT);
-        const uint32_t aZ = smem_u32(Z), aRW = smem_u32(RW);
+        const uint32_t aZ[2] = {smem_u32(ZHI), smem_u32(ZLO)};
+        const uint32_t aR[2] = {smem_u32(RHI), smem_u32(RLO)};
+        const uint32_t aW[2] = {smem_u32(WHI), smem_u32(WLO)};
         const int64_t cs = (int64_t)ch * C;
         const int Lc = (count - cs) < C ? (int)(count - cs) : C;
         const float bt = (tid < Lc) ? __ldg(beta + (first + cs + tid) * H + h) : 0.f;
@@ -305,12 +317,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             } else {
                 const int r = tid - 64;
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    *reinterpret_cast<float*>(Z + z_off(tid, j)) = j <= r ? g[j] : 0.f;
+                for (int j = 0; j < 64; ++j) g[j] = j <= r ? g[j] : 0.f;
+                st_row_split_bf16(ZHI, ZLO, tid, g);  // P rows 64..127
             }
         }
         if (sync_failed()) break;
         solve_unit_lower_64(sL, sM, Z, tid);  // ends with __syncthreads
+        {
+            float x[64];
+            if (tid < 64) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) x[j] = *reinterpret_cast<const float*>(Z + z_off(tid, j));
+            }
+            __syncthreads();  // every fp32 row is read before the bf16 rows overwrite it
+            if (tid < 64) st_row_split_bf16(ZHI, ZLO, tid, x);  // T rows 0..63
+        }
         tc::fence_async_smem();
         if (sync_failed()) break;
 
@@ -345,46 +366,36 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     r[8 * j + 2 * e + 1] = bt * (vv.y - y[8 * j + 2 * e + 1]);
                 }
             }
-            st_col_f32_k(RW, tid, r);
+            st_row_split_bf16(RHI, RLO, tid, r);
         }
         tc::fence_async_smem();
         if (sync_failed()) break;
 
-        // ---- D2 = [T; P] R  (tf32; rows 0..63 hold W)
+        // ---- D2 = [T; P] R  (three split terms; rows 0..63 hold W)
         if (tid == 0) {
             tc::fence_after_sync();
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                tc::mma_tf32(tmem + TC_COL_D2,
-                             tc::sw128_desc(aZ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             tc::sw128_desc(aRW + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_TF, s > 0);
+            mma_split3(tmem + TC_COL_D2, aZ, aR, ID_Z, false);
             commit();
         }
         wait_mma();
         if (tid < 64) {
             float w[64];
             tc::tmem_ld64(t_D2, w);
-            st_col_f32_k(RW, tid, w);
             st_row_split_bf16(WHI, WLO, tid, w);
         }
         tc::fence_async_smem();
         if (sync_failed()) break;
 
-        // ---- S^T += K~^T W (two bf16 terms of W);  D1 += [T; P] W (tf32; rows 64..127: O)
+        // ---- S^T += K~^T W (two terms of W);  D1 += [T; P] W (three terms; rows 64..127: O)
         if (tid == 0) {
             tc::fence_after_sync();
-            const uint32_t parts[2] = {smem_u32(WHI), smem_u32(WLO)};
 #pragma unroll
             for (int p = 0; p < 2; ++p)
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     tc::mma_bf16(tmem + TC_COL_S, tc::sw128_desc(aKT + s * 2048, 8192, 1024),
-                                 tc::sw128_desc(parts[p] + s * 2048, 8192, 1024), ID_3, 1);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                tc::mma_tf32(tmem + TC_COL_D1,
-                             tc::sw128_desc(aZ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                             tc::sw128_desc(aRW + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), ID_TF, 1);
+                                 tc::sw128_desc(aW[p] + s * 2048, 8192, 1024), ID_3, 1);
+            mma_split3(tmem + TC_COL_D1, aZ, aW, ID_Z, true);
             commit();
         }
         wait_mma();

@@ -16,6 +16,7 @@
 #include "chunk_simt.cuh"
 #include "watchdog.cuh"
 #include "chunk_tc.cuh"
+#include "scan_chunk.cuh"
 
 namespace osdn {
 namespace {
@@ -63,9 +64,9 @@ inline bool set_smem(KernelT kernel, size_t bytes) {
 
 // ---------------------------------------------------------------- phase 1 dispatch
 template <typename IO>
-osdn_status_t launch_scan(const void* k, const float* beta, const float* r, float eta,
-                          const float* d0, void* k_tilde, float* dT, const int32_t* cu,
-                          const Dims& d, cudaStream_t stream) {
+osdn_status_t launch_scan_warp(const void* k, const float* beta, const float* r, float eta,
+                               const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                               const Dims& d, cudaStream_t stream) {
     const int units = d.N * d.H;
     if (units == 0) return OSDN_OK;
     const dim3 block(128), grid((units + 3) / 4);
@@ -147,6 +148,35 @@ bool make_tile_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows)
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+osdn_status_t launch_scan_chunk(const void* k, const float* beta, const float* r, float eta,
+                                const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                                const Dims& d, cudaStream_t stream) {
+    const int64_t ctas = (int64_t)d.N * d.H;
+    if (ctas == 0) return OSDN_OK;
+    if (ctas > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    CUtensorMap mk;
+    if (!make_tile_map(&mk, k, 128, d.H, d.rows())) return OSDN_ERR_CUDA;
+    auto kernel = precond_scan_chunk_kernel;
+    if (!set_smem(kernel, ScanSmem::BYTES)) return OSDN_ERR_CUDA;
+    kernel<<<dim3((unsigned)ctas), dim3(256), ScanSmem::BYTES, stream>>>(
+        mk, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde), dT, cu, d.N, d.T, d.H,
+        (long long)kWaitLimitNs);
+    return launch_status();
+}
+
+// Phase 1: bf16 keys with 128 channels use the chunk-parallel kernel; fp32 I/O, 64 channels
+// and token-free calls use the warp-per-(sequence, head) scan.
+template <typename IO>
+osdn_status_t launch_scan(const void* k, const float* beta, const float* r, float eta,
+                          const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                          const Dims& d, cudaStream_t stream) {
+    if constexpr (sizeof(IO) == 2) {
+        if (d.Dk == 128 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
+            return launch_scan_chunk(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
+    }
+    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
 }
 
 template <int DV>
