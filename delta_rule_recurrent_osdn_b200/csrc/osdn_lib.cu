@@ -193,7 +193,7 @@ osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, cons
         return OSDN_ERR_CUDA;
     auto kernel = chunk_fwd_tc_kernel<DV>;
     if (!set_smem(kernel, TcSmem::BYTES)) return OSDN_ERR_CUDA;
-    kernel<<<dim3((unsigned)ctas), dim3(128), TcSmem::BYTES, stream>>>(
+    kernel<<<dim3((unsigned)ctas), dim3(TC_THREADS), TcSmem::BYTES, stream>>>(
         mq, mk, mkt, mv, beta, scale, S0, static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T, d.H,
         (long long)kWaitLimitNs);
     return launch_status();
