@@ -46,9 +46,9 @@ struct TcSmem {
     static constexpr uint32_t SLO = SHI + 16384;
     static constexpr uint32_t RHI = SLO + 16384;      // bf16 R then W, hi / lo, 64 x 128 B
     static constexpr uint32_t RLO = RHI + 8192;
-    static constexpr uint32_t SL = RLO + 8192;        // fp32 L, 64 x 65
-    static constexpr uint32_t SMT = SL + 64 * 65 * 4; // fp32 T, 64 x 65
-    static constexpr uint32_t BAR = SMT + 64 * 65 * 4;
+    static constexpr uint32_t SL = RLO + 8192;        // fp32 L, 64 x 64, swizzled (tsw)
+    static constexpr uint32_t SMT = SL + 64 * 64 * 4; // fp32 T, 64 x 64, swizzled (tsw)
+    static constexpr uint32_t BAR = SMT + 64 * 64 * 4;
     static constexpr uint32_t TMEM_SLOT = BAR + 80;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;     // + alignment slack
@@ -101,7 +101,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float* __restrict__ beta, float scale, const float* __restrict__ S0,
                     __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
                     const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
-    constexpr int DK = 128, BV = 64, C = 64, NVT = DV / BV, S = kTrilStride;
+    constexpr int DK = 128, BV = 64, C = 64, NVT = DV / BV;
     using L = TcSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -220,9 +220,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float g[64];
             tc::tmem_ld64(tmem + lane + TC_COL_G, g);
             if (leader) mbar_arrive(&stage_empty[s]);  // the Gram was the prep's last use of the stage
-            if (t < 64) {
+            if (t < 64) {  // row t of L; only j < t is read by the inverse
 #pragma unroll
-                for (int j = 0; j < 64; ++j) sL[t * S + j] = j < t ? bt * g[j] : 0.f;
+                for (int q = 0; q < 16; ++q)
+                    tsw_st4(sL, t, q, make_float4(bt * g[4 * q], bt * g[4 * q + 1], bt * g[4 * q + 2],
+                                                  bt * g[4 * q + 3]));
             } else {
                 const int r = t - 64;
 #pragma unroll
@@ -234,8 +236,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (group_any(2, 128, !mbar_wait_bounded(z_empty, (uint32_t)ch & 1u, limit_ns))) break;
             if (t < 64) {
                 float x[64];
+                tsw_row<16>(sT, t, 0, x);
 #pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = sT[t * S + j];
+                for (int j = 0; j < 64; ++j) x[j] = j <= t ? x[j] : 0.f;  // T is lower triangular
                 st_row_split_bf16(ZHI, ZLO, t, x);  // T rows 0..63
             } else {
                 st_row_split_bf16(ZHI, ZLO, t, g);  // P rows 64..127

@@ -1,105 +1,35 @@
-// tril_inverse.cuh -- (I + L)^-1 for a strictly lower-triangular 64x64 fp32 matrix L, computed by
-// 256 threads in shared memory.
+// tril_inverse.cuh -- T = (I + L)^-1 for a strictly lower-triangular 64x64 fp32 matrix L, computed
+// in shared memory by a group of 128 threads.
 //
-// Both phases of the chunked forward pass need this inverse once per 64-token chunk: phase 2 for
-// the WY factor T = (I + strict_tril(diag(beta) K K~^T))^-1 (the (I + T)^-1 solve the Gated
-// DeltaNet-2 summary names for the same building block), phase 1 for the analogous factor of
-// the preconditioner recurrence.  Blocked algorithm, all in fp32:
-//   1. the four diagonal 16x16 blocks by forward substitution (one column per thread);
-//   2. 16x16 level: T_IJ = -T_II (L_IJ T_JJ) for (I, J) = (1, 0), (3, 2);
-//   3. 32x32 level: T_[10] = -T_[11] (L_[10] T_[00]) on the 2x2 grid of 32x32 blocks.
-// Matrices use row stride 65 (conflict-free row and column walks).
+// The chunked DeltaNet forward pass needs this WY factor once per 64-token chunk, with
+// L = strict_tril(diag(beta) K K~^T) (the UT-transform solve of the chunkwise DeltaNet
+// algorithm).  Blocked algorithm, all in fp32:
+//   A. the four diagonal 16x16 blocks by forward substitution (one column per thread);
+//   B. 16x16 level, (I, J) = (1, 0) and (3, 2):  X = L_IJ T_JJ,  T_IJ = -T_II X;
+//   C. 32x32 level on the 2x2 grid of 32x32 blocks:  X = L_10 T_00,  T_10 = -T_11 X.
+// Each thread keeps one column of the right-hand factor in registers and produces 4 (level B)
+// or 8 (level C) outputs of that column, reading the left factor's rows as broadcast 16-byte
+// loads, so a product step is a few dozen shared loads per thread rather than two per FMA.
+//
+// Matrix layout ("tsw"): row stride 64 floats, the 16-byte group g of row r stored at group
+// position g ^ (r & 15).  A thread that writes its own row as 16 float4 stores, a warp that
+// reads one row (broadcast) and a warp that reads 32 consecutive columns of one row are all
+// free of bank conflicts.
 #pragma once
 
 namespace osdn {
 
-constexpr int kTrilStride = 65;
+// Word offset of element (r, c) of a 64x64 fp32 matrix in the swizzled layout.
+__device__ __forceinline__ int tsw(int r, int c) {
+    return r * 64 + ((((c >> 2) ^ r) & 15) << 2) + (c & 3);
+}
 
-// sL: L (only the strictly lower part is read).  sT: receives T (all 64x64 entries written).
-// sX: 64x65 fp32 scratch.  Must be called by all 256 threads of the block; ends synchronized.
-__device__ __forceinline__ void tril_inverse_64(const float* __restrict__ sL, float* __restrict__ sT,
-                                                float* __restrict__ sX, int tid) {
-    constexpr int S = kTrilStride;
-    // ---- 1. diagonal blocks; other threads clear everything above the block diagonal
-    if (tid < 64) {
-        const int b = tid >> 4, col = tid & 15, o = 16 * b;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
-#pragma unroll
-            for (int m = 0; m < r; ++m)
-                if (m >= col) acc = fmaf(sL[(o + r) * S + o + m], x[m], acc);
-            x[r] = r < col ? 0.f : (r == col ? 1.f : -acc);
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(o + r) * S + o + col] = x[r];
-    } else {
-        for (int idx = tid - 64; idx < 64 * 64; idx += 192) {
-            const int r = idx >> 6, c = idx & 63;
-            if ((c >> 4) > (r >> 4)) sT[r * S + c] = 0.f;
-        }
-    }
-    __syncthreads();
-    // ---- 2. 16x16 level, blocks (1,0) and (3,2): X = L_IJ T_JJ (T_JJ lower: m >= c).  Loops are
-    //      fully unrolled with the triangular bound as a predicate so the loads pipeline.
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int idx = tid + 256 * k;
-        const int I = (idx >> 8) ? 3 : 1, J = I - 1, r = (idx >> 4) & 15, c = idx & 15;
-        const float* lrow = sL + (16 * I + r) * S + 16 * J;
-        const float* tcol = sT + (16 * J) * S + 16 * J + c;
-        float acc = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m)
-            if (m >= c) acc = fmaf(lrow[m], tcol[m * S], acc);
-        sX[(16 * I + r) * S + 16 * J + c] = acc;
-    }
-    __syncthreads();
-    //      T_IJ = -T_II X (T_II lower: m <= r)
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int idx = tid + 256 * k;
-        const int I = (idx >> 8) ? 3 : 1, J = I - 1, r = (idx >> 4) & 15, c = idx & 15;
-        const float* trow = sT + (16 * I + r) * S + 16 * I;
-        const float* xcol = sX + (16 * I) * S + 16 * J + c;
-        float acc = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m)
-            if (m <= r) acc = fmaf(trow[m], xcol[m * S], acc);
-        sT[(16 * I + r) * S + 16 * J + c] = -acc;
-    }
-    __syncthreads();
-    // ---- 3. 32x32 level: X = L[32:64, 0:32] T[0:32, 0:32]  (T lower: m >= c)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int idx = tid + 256 * k, r = idx >> 5, c = idx & 31;
-        const float* lrow = sL + (32 + r) * S;
-        const float* tcol = sT + c;
-        float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; m += 2) {
-            if (m >= c) acc0 = fmaf(lrow[m], tcol[m * S], acc0);
-            if (m + 1 >= c) acc1 = fmaf(lrow[m + 1], tcol[(m + 1) * S], acc1);
-        }
-        sX[(32 + r) * S + c] = acc0 + acc1;
-    }
-    __syncthreads();
-    //      T[32:64, 0:32] = -T[32:64, 32:64] X   (m <= r)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int idx = tid + 256 * k, r = idx >> 5, c = idx & 31;
-        const float* trow = sT + (32 + r) * S + 32;
-        const float* xcol = sX + 32 * S + c;
-        float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; m += 2) {
-            if (m <= r) acc0 = fmaf(trow[m], xcol[m * S], acc0);
-            if (m + 1 <= r) acc1 = fmaf(trow[m + 1], xcol[(m + 1) * S], acc1);
-        }
-        sT[(32 + r) * S + c] = -(acc0 + acc1);
-    }
-    __syncthreads();
+__device__ __forceinline__ float4 tsw_ld4(const float* m, int r, int g) {
+    return *reinterpret_cast<const float4*>(m + r * 64 + (((g ^ r) & 15) << 2));
+}
+
+__device__ __forceinline__ void tsw_st4(float* m, int r, int g, float4 v) {
+    *reinterpret_cast<float4*>(m + r * 64 + (((g ^ r) & 15) << 2)) = v;
 }
 
 __device__ __forceinline__ void group_bar(int id, int nthreads) {
@@ -119,88 +49,129 @@ __device__ __forceinline__ bool group_any(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
-// The same inverse computed by a group of 128 threads (t = 0..127) that synchronizes on named
-// barrier `bar_id`.  It needs no scratch beyond sT: the intermediate products X are kept,
-// transposed, in the part of sT above the block diagonal, which is cleared at the end.
+// Load row r, columns [c0, c0 + 4*NG) of a swizzled matrix into x (c0 a multiple of 4).
+template <int NG>
+__device__ __forceinline__ void tsw_row(const float* m, int r, int c0, float* x) {
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const float4 v = tsw_ld4(m, r, (c0 >> 2) + g);
+        x[4 * g] = v.x;
+        x[4 * g + 1] = v.y;
+        x[4 * g + 2] = v.z;
+        x[4 * g + 3] = v.w;
+    }
+}
+
+// sL: L in the swizzled layout; only its strictly lower triangle is read.  sT (swizzled)
+// receives T on and below the diagonal; the entries above the diagonal are left holding
+// scratch values, so a reader masks them (T is lower triangular with a unit diagonal).
+// Called by all 128 threads t = 0..127 of a group synchronizing on named barrier `bar_id`;
+// returns synchronized.
 __device__ __forceinline__ void tril_inverse_64_g128(const float* __restrict__ sL,
                                                      float* __restrict__ sT, int t, int bar_id) {
-    constexpr int S = kTrilStride, NT = 128;
-    if (t < 64) {  // diagonal 16x16 blocks
-        const int b = t >> 4, col = t & 15, o = 16 * b;
+    constexpr int NT = 128;
+    // ---- A. diagonal blocks: column `col` of block b, x[r] = [r == col] - sum_{m<r} L_rm x[m]
+    if (t < 64) {
+        const int o = 16 * (t >> 4), col = t & 15;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
+            float lr[16];
+#pragma unroll
+            for (int g = 0; 4 * g < r; ++g) {
+                const float4 v = tsw_ld4(sL, o + r, (o >> 2) + g);
+                lr[4 * g] = v.x;
+                lr[4 * g + 1] = v.y;
+                lr[4 * g + 2] = v.z;
+                lr[4 * g + 3] = v.w;
+            }
+            float acc = 0.f;  // x[m] == 0 for m < col, so no per-lane bound is needed
+#pragma unroll
+            for (int m = 0; m < r; ++m) acc = fmaf(-lr[m], x[m], acc);
+            x[r] = r == col ? 1.f : (r < col ? 0.f : acc);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[tsw(o + r, o + col)] = x[r];
+    }
+    group_bar(bar_id, NT);
+    // ---- B. 16x16 level; thread: block pair (t >> 6), column c, rows 4*rq .. 4*rq + 3
+    {
+        const int I = (t >> 6) ? 3 : 1, J = I - 1, c = t & 15, rq = (t >> 4) & 3;
+        float col[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) col[m] = sT[tsw(16 * J + m, 16 * J + c)];  // T_JJ[:, c]
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {  // X = L_IJ T_JJ, kept in the free block (J, I)
+            const int r = 4 * rq + rr;
+            float lr[16];
+            tsw_row<4>(sL, 16 * I + r, 16 * J, lr);
             float acc = 0.f;
 #pragma unroll
-            for (int m = 0; m < r; ++m)
-                if (m >= col) acc = fmaf(sL[(o + r) * S + o + m], x[m], acc);
-            x[r] = r < col ? 0.f : (r == col ? 1.f : -acc);
+            for (int m = 0; m < 16; ++m) acc = fmaf(lr[m], col[m], acc);
+            sT[tsw(16 * J + r, 16 * I + c)] = acc;
+        }
+        group_bar(bar_id, NT);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) col[m] = sT[tsw(16 * J + m, 16 * I + c)];  // X[:, c]
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {  // T_IJ = -T_II X  (T_II[r][m] == 0 for m > r)
+            const int r = 4 * rq + rr;
+            float tr[16];
+            tsw_row<4>(sT, 16 * I + r, 16 * I, tr);
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) acc = fmaf(-tr[m], col[m], acc);
+            sT[tsw(16 * I + r, 16 * J + c)] = acc;
+        }
+    }
+    group_bar(bar_id, NT);
+    // ---- C. 32x32 level; thread: column c, rows 8*rq .. 8*rq + 7 (rq = warp of the group)
+    {
+        const int c = t & 31, rq = t >> 5;
+        float col[32];
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {  // T_00[:, c]; block (0, 1) holds scratch, so mask m < c
+            const float v = sT[tsw(m, c)];
+            col[m] = m >= c ? v : 0.f;
+        }
+        float acc[8];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // X = L_10 T_00, kept in the free block (0, 1) of 32x32
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                float lr[16];
+                tsw_row<4>(sL, 32 + 8 * rq + rr, 16 * h, lr);
+#pragma unroll
+                for (int m = 0; m < 16; ++m) acc[rr] = fmaf(lr[m], col[16 * h + m], acc[rr]);
+            }
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(o + r) * S + o + col] = x[r];
-    }
-    group_bar(bar_id, NT);
-    // 16x16 level, (I, J) = (1, 0) and (3, 2): X = L_IJ T_JJ, stored transposed in block (J, I)
+        for (int rr = 0; rr < 8; ++rr) sT[tsw(8 * rq + rr, 32 + c)] = acc[rr];
+        group_bar(bar_id, NT);
+        // T_10 = -T_11 X.  Rows 32..47 of T_11 are zero past column 47 (and columns 48..63 of
+        // those rows hold level-B scratch), so warps 0-1 take only the first 16 terms.
+        const int mlen = rq < 2 ? 16 : 32;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int idx = t + NT * k;
-        const int I = (idx >> 8) ? 3 : 1, J = I - 1, r = (idx >> 4) & 15, c = idx & 15;
-        const float* lrow = sL + (16 * I + r) * S + 16 * J;
-        const float* tcol = sT + (16 * J) * S + 16 * J + c;
-        float acc = 0.f;
+        for (int m = 0; m < 32; ++m)
+            if (m < mlen) col[m] = sT[tsw(m, 32 + c)];  // X[:, c]
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-            if (m >= c) acc = fmaf(lrow[m], tcol[m * S], acc);
-        sT[(16 * J + c) * S + 16 * I + r] = acc;
-    }
-    group_bar(bar_id, NT);
-    //      T_IJ = -T_II X
+        for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int idx = t + NT * k;
-        const int I = (idx >> 8) ? 3 : 1, J = I - 1, r = (idx >> 4) & 15, c = idx & 15;
-        const float* trow = sT + (16 * I + r) * S + 16 * I;
-        const float* xrow = sT + (16 * J + c) * S + 16 * I;
-        float acc = 0.f;
+        for (int h = 0; h < 2; ++h) {
+            if (h * 16 < mlen) {
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-            if (m <= r) acc = fmaf(trow[m], xrow[m], acc);
-        sT[(16 * I + r) * S + 16 * J + c] = -acc;
-    }
-    group_bar(bar_id, NT);
-    // 32x32 level: X = L[32:64, 0:32] T[0:32, 0:32], stored transposed in rows 0..31, cols 32..63
+                for (int rr = 0; rr < 8; ++rr) {
+                    float tr[16];
+                    tsw_row<4>(sT, 32 + 8 * rq + rr, 32 + 16 * h, tr);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int idx = t + NT * k, r = idx >> 5, c = idx & 31;
-        const float* lrow = sL + (32 + r) * S;
-        const float* tcol = sT + c;
-        float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; m += 2) {
-            if (m >= c) acc0 = fmaf(lrow[m], tcol[m * S], acc0);
-            if (m + 1 >= c) acc1 = fmaf(lrow[m + 1], tcol[(m + 1) * S], acc1);
+                    for (int m = 0; m < 16; ++m) acc[rr] = fmaf(-tr[m], col[16 * h + m], acc[rr]);
+                }
+            }
         }
-        sT[c * S + 32 + r] = acc0 + acc1;
-    }
-    group_bar(bar_id, NT);
-    //      T[32:64, 0:32] = -T[32:64, 32:64] X
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int idx = t + NT * k, r = idx >> 5, c = idx & 31;
-        const float* trow = sT + (32 + r) * S + 32;
-        const float* xrow = sT + c * S + 32;
-        float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 32; m += 2) {
-            if (m <= r) acc0 = fmaf(trow[m], xrow[m], acc0);
-            if (m + 1 <= r) acc1 = fmaf(trow[m + 1], xrow[m + 1], acc1);
-        }
-        sT[(32 + r) * S + c] = -(acc0 + acc1);
-    }
-    group_bar(bar_id, NT);
-    for (int idx = t; idx < 64 * 64; idx += NT) {  // clear everything above the block diagonal
-        const int r = idx >> 6, c = idx & 63;
-        if ((c >> 4) > (r >> 4)) sT[r * S + c] = 0.f;
+        for (int rr = 0; rr < 8; ++rr) sT[tsw(32 + 8 * rq + rr, c)] = acc[rr];
     }
     group_bar(bar_id, NT);
 }
