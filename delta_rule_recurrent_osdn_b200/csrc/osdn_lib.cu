@@ -16,7 +16,7 @@
 #include "chunk_simt.cuh"
 #include "watchdog.cuh"
 #include "chunk_tc.cuh"
-#include "scan_chunk.cuh"
+#include "scan_tc.cuh"
 
 namespace osdn {
 namespace {
@@ -150,18 +150,55 @@ bool make_tile_map(CUtensorMap* m, const void* base, int D, int H, int64_t rows)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-osdn_status_t launch_scan_chunk(const void* k, const float* beta, const float* r, float eta,
-                                const float* d0, void* k_tilde, float* dT, const int32_t* cu,
-                                const Dims& d, cudaStream_t stream) {
-    const int64_t ctas = (int64_t)d.N * d.H;
-    if (ctas == 0) return OSDN_OK;
-    if (ctas > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
-    CUtensorMap mk;
-    if (!make_tile_map(&mk, k, 128, d.H, d.rows())) return OSDN_ERR_CUDA;
-    auto kernel = precond_scan_chunk_kernel;
-    if (!set_smem(kernel, ScanSmem::BYTES)) return OSDN_ERR_CUDA;
-    kernel<<<dim3((unsigned)ctas), dim3(256), ScanSmem::BYTES, stream>>>(
-        mk, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde), dT, cu, d.N, d.T, d.H,
+// 3-D fp32 view [rows][H][64] of a bf16 [B, T, H, 128] buffer (one 256-byte row per token and
+// head); boxes of 64 values x 1 head x 64 tokens, no swizzle: the prep kernel's T_d tiles.
+bool make_td_map(CUtensorMap* m, const void* base, int H, int64_t rows) {
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (!enc || rows <= 0) return false;
+    cuuint64_t dims[3] = {64, (cuuint64_t)H, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {256, (cuuint64_t)H * 256};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+// Phase 1, bf16 with 128 key channels: T_d of every chunk (prep kernel, written into the k~
+// buffer), then the chain across chunks (one CTA per (sequence, head)).
+osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, float eta,
+                             const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                             const Dims& d, cudaStream_t stream) {
+    const int64_t nh = (int64_t)d.N * d.H;
+    if (nh == 0) return OSDN_OK;
+    if (nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    const int64_t rows = d.rows();  // > 0: token-free calls take the warp scan
+    CUtensorMap mk, mtd;
+    if (!make_tile_map(&mk, k, 128, d.H, rows) || !make_td_map(&mtd, k_tilde, d.H, rows))
+        return OSDN_ERR_CUDA;
+    // chunks per (sequence, head): exact for fixed length, about the mean for packed sequences
+    const int64_t per_seq = cu ? rows / d.N / 64 + 1 : ((int64_t)d.T + 63) / 64;
+    int64_t gy = (3 * (int64_t)sm_count() + nh - 1) / nh;
+    gy = gy > per_seq ? per_seq : gy;
+    gy = gy < 1 ? 1 : (gy > 65535 ? 65535 : gy);
+    auto prep = precond_prep_kernel;
+    if (!set_smem(prep, ScanPrepSmem::BYTES)) return OSDN_ERR_CUDA;
+    prep<<<dim3((unsigned)nh, (unsigned)gy), dim3(128), ScanPrepSmem::BYTES, stream>>>(
+        mk, beta, r, eta, static_cast<float*>(k_tilde), cu, d.N, d.T, d.H, (long long)kWaitLimitNs);
+    const osdn_status_t st = launch_status();
+    if (st != OSDN_OK) return st;
+    auto chain = precond_chain_kernel;
+    if (!set_smem(chain, ScanChainSmem::BYTES)) return OSDN_ERR_CUDA;
+    chain<<<dim3((unsigned)nh), dim3(SCAN_CHAIN_THREADS), ScanChainSmem::BYTES, stream>>>(
+        mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde), dT, cu, d.N, d.T, d.H,
         (long long)kWaitLimitNs);
     return launch_status();
 }
@@ -174,7 +211,7 @@ osdn_status_t launch_scan(const void* k, const float* beta, const float* r, floa
                           const Dims& d, cudaStream_t stream) {
     if constexpr (sizeof(IO) == 2) {
         if (d.Dk == 128 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
-            return launch_scan_chunk(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
+            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
     }
     return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
 }
@@ -233,8 +270,13 @@ osdn_status_t validate_scan(const void* k, const float* beta, const float* r, co
     const void* ptrs[] = {k, beta, r, d0, k_tilde, dT};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
+    // the k~ buffer is written before the gates and states are read: no input may lie in it
     const size_t kbytes = (size_t)d.rows() * d.H * d.Dk * io_size(io);
-    if (overlaps(k, kbytes, k_tilde, kbytes)) return OSDN_ERR_INVALID_ARG;
+    const size_t gbytes = (size_t)d.rows() * d.H * 4, sbytes = (size_t)d.N * d.H * d.Dk * 4;
+    if (overlaps(k, kbytes, k_tilde, kbytes) || overlaps(beta, gbytes, k_tilde, kbytes) ||
+        overlaps(r, gbytes, k_tilde, kbytes) || overlaps(d0, sbytes, k_tilde, kbytes) ||
+        overlaps(dT, sbytes, k_tilde, kbytes))
+        return OSDN_ERR_INVALID_ARG;
     return OSDN_OK;
 }
 

@@ -1,0 +1,528 @@
+// scan_tc.cuh -- phase 1 of the OSDN forward pass (bf16 I/O, d_k = 128) as two kernels.
+//
+// The preconditioner recurrence ("OSDN: Improving Delta Rule with Provable Online
+// Preconditioning in Linear Attention", technical summary, sections 2.2 and 2.3; section 2.3
+// notes that the APF update keeps the recurrence affine) is, with a_t = k_t (.) k_t,
+// e_t = eta beta_t / ||k_t||^2 (0 when k_t = 0) and x_t = e_t (1 - beta_t <d_t, a_t>):
+//   d_{t+1} = r_t d_t + x_t a_t,     k~_t = d_t (.) k_t.
+// Within a chunk of C = 64 tokens starting from d_0, with R_t = prod_{i<t} r_i and
+// Gamma_tj = prod_{j<i<t} r_i:
+//   <d_t, a_t> = R_t <d_0, a_t> + sum_{j<t} Gamma_tj <a_j, a_t> x_j, hence
+//   (I + L_d) x = b,  b = e (.) (1 - beta (.) R (.) A d_0),  L_d[t][j] = e_t beta_t Gamma_tj <a_t, a_j>,
+//   d_C = R_C d_0 + A^T (g (.) x),  g_j = Gamma_Cj.
+// L_d and T_d = (I + L_d)^-1 do not depend on d_0, so they are computed for every chunk at once
+// by precond_prep_kernel; what remains sequential across chunks is three matrix-vector products
+// per chunk (p = A d_0, x = T_d b, d_C), done by precond_chain_kernel, whose other warps emit
+// k~ for each chunk by the token recurrence above while the next chunk's products run.
+//
+// Hand-off without extra memory: for d_k = 128 in bf16, one chunk's k~ rows (64 tokens x 256 B)
+// are exactly the size of its fp32 64 x 64 T_d.  The prep kernel writes T_d into the k~ buffer,
+// at the chunk's own rows; the chain kernel loads it (TMA) before it overwrites those rows with
+// k~.  Row t of T_d is stored with the 16-byte groups permuted as in the tsw layout
+// (tril_inverse.cuh), so a straight copy into shared memory is ready for conflict-free reads.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tril_inverse.cuh"
+
+namespace osdn {
+
+constexpr int SCAN_C = 64;
+
+// Gate prefix quantities of one chunk, computed by one warp (lane l: tokens 2l and 2l + 1).
+// r is 1 and beta 0 for tokens past the chunk's end.  Gamma_tj = sg[t] sg1[j] exp(lr[t] - lr1[j]).
+struct GatePrefix {
+    float lr0, lr1_0, lr_1, lr1_1;  // lr and lr1 of tokens 2l, 2l + 1
+    float sg0, sg1_0, sg_1, sg1_1;
+    float lrC, sgC;                 // over the whole chunk
+};
+
+__device__ __forceinline__ GatePrefix gate_prefix(float r0, float r1, int lane) {
+    const float l0 = __logf(fmaxf(fabsf(r0), 1e-30f)), l1 = __logf(fmaxf(fabsf(r1), 1e-30f));
+    const int n0 = r0 < 0.f, n1 = r1 < 0.f;
+    float ps = l0 + l1;
+    int pn = n0 + n1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float ys = __shfl_up_sync(0xffffffffu, ps, off);
+        const int yn = __shfl_up_sync(0xffffffffu, pn, off);
+        if (lane >= off) {
+            ps += ys;
+            pn += yn;
+        }
+    }
+    GatePrefix g;
+    const float ex = ps - (l0 + l1);
+    const int en = pn - (n0 + n1);
+    g.lr0 = ex;
+    g.lr_1 = ex + l0;
+    g.lr1_0 = ex + l0;
+    g.lr1_1 = ex + l0 + l1;
+    g.sg0 = (en & 1) ? -1.f : 1.f;
+    g.sg_1 = ((en + n0) & 1) ? -1.f : 1.f;
+    g.sg1_0 = g.sg_1;
+    g.sg1_1 = ((en + n0 + n1) & 1) ? -1.f : 1.f;
+    g.lrC = __shfl_sync(0xffffffffu, ps, 31);
+    g.sgC = (__shfl_sync(0xffffffffu, pn, 31) & 1) ? -1.f : 1.f;
+    return g;
+}
+
+// ===================================================================== prep: T_d per chunk
+
+struct ScanPrepSmem {
+    static constexpr uint32_t K = 0;              // bf16 k tile: 2 K-blocks x (64 rows x 128 B)
+    static constexpr uint32_t A = 16384;          // bf16 [a_hi; a_lo] per K-block, 2 x 16 KB
+    static constexpr uint32_t SL = A;             // fp32 L_d (tsw), over A once the Gram is done
+    static constexpr uint32_t ST = A + 16384;     // fp32 T_d (tsw), over A
+    static constexpr uint32_t VEC = A + 32768;    // c, lr, lr1, sg, sg1 (5 x 64 floats)
+    static constexpr uint32_t BAR = VEC + 5 * 256;
+    static constexpr uint32_t TMEM_SLOT = BAR + 16;
+    static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
+    static constexpr size_t BYTES = TOTAL + 1024;
+};
+
+// Grid (N * H, gy): CTA (nh, y) handles chunks y, y + gy, ... of its (sequence, head).
+// 128 threads; td_out is the k~ buffer seen as fp32 rows of 64 values.
+__global__ void __launch_bounds__(128, 3)
+precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ beta,
+                    const float* __restrict__ r, float eta, float* __restrict__ td_out,
+                    const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
+    constexpr int C = SCAN_C;
+    using L = ScanPrepSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
+    if (n >= N) return;
+    int64_t first, count;
+    if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the CTA
+    const int nchunks = (int)((count + C - 1) / C);
+    const int gy = gridDim.y;
+    int ch = blockIdx.y;
+    if (ch >= nchunks) return;
+
+    uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
+    uint64_t* mma_bar = tma_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
+    uint8_t* sK = smem + L::K;
+    uint8_t* sA = smem + L::A;
+    float* sL = reinterpret_cast<float*>(smem + L::SL);
+    float* sT = reinterpret_cast<float*>(smem + L::ST);
+    float* vc = reinterpret_cast<float*>(smem + L::VEC);
+    float* vlr = vc + 64;
+    float* vlr1 = vc + 128;
+    float* vsg = vc + 192;
+    float* vsg1 = vc + 256;
+
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 128);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        tc::fence_mbar_init();
+        tc::prefetch_tmap(&tm_k);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tlane = static_cast<uint32_t>(warp * 32) << 16;
+
+    auto issue_load = [&](int c) {
+        const int row = (int)(first + (int64_t)c * C);
+        tc::mbar_expect_tx(tma_bar, 16384);
+        tc::tma_load_3d(sK, &tm_k, 0, h, row, tma_bar);
+        tc::tma_load_3d(sK + 8192, &tm_k, 64, h, row, tma_bar);
+    };
+    if (tid == 0) issue_load(ch);
+    bool tma_pend = tid == 0, mma_pend = false, fail = false;
+    uint32_t tph = 0, mph = 0;
+    constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);
+
+#pragma unroll 1
+    for (; ch < nchunks; ch += gy) {
+        const int64_t cs = (int64_t)ch * C;
+        const int Lc = count - cs < C ? (int)(count - cs) : C;
+        const int64_t row0 = first + cs;
+        const bool got = mbar_wait_bounded(tma_bar, tph, limit_ns);
+        if (__syncthreads_or(!got)) {
+            fail = true;
+            break;
+        }
+        tph ^= 1u;
+        tma_pend = false;
+        // ---- a = k (.) k split into bf16 hi + lo rows; e and c = e beta per token.
+        //      Thread: row t = 16 warp + (lane & 15), K-block = lane >> 4.
+        {
+            const int t = 16 * warp + (lane & 15), blk = lane >> 4;
+            const bool valid = t < Lc;
+            float nk = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t off = blk * 8192u + tc::sw128_off(t, j);
+                const uint4 raw = *reinterpret_cast<const uint4*>(sK + off);
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                    const float a0 = valid ? kk.x * kk.x : 0.f, a1 = valid ? kk.y * kk.y : 0.f;
+                    nk += a0 + a1;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+                    const float2 hf = __bfloat1622float2(h2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+                    hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                    lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+                }
+                const uint32_t aoff = blk * 16384u + tc::sw128_off(t, j);
+                *reinterpret_cast<uint4*>(sA + aoff) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(sA + aoff + 8192u) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            nk += __shfl_xor_sync(0xffffffffu, nk, 16);
+            if (blk == 0) {
+                const float bt = valid ? __ldg(beta + (row0 + t) * H + h) : 0.f;
+                const float e = nk > 0.f ? eta * bt / nk : 0.f;
+                vc[t] = e * bt;
+            }
+        }
+        if (warp == 3) {  // prefix of log|r| over the chunk
+            const int t0 = 2 * lane;
+            const float r0 = (r && t0 < Lc) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
+            const float r1 = (r && t0 + 1 < Lc) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
+            const GatePrefix g = gate_prefix(r0, r1, lane);
+            vlr[t0] = g.lr0;
+            vlr[t0 + 1] = g.lr_1;
+            vlr1[t0] = g.lr1_0;
+            vlr1[t0 + 1] = g.lr1_1;
+            vsg[t0] = g.sg0;
+            vsg[t0 + 1] = g.sg_1;
+            vsg1[t0] = g.sg1_0;
+            vsg1[t0 + 1] = g.sg1_1;
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tc::fence_after_sync();
+            // Gram: cols 0..63 = [a_hi; a_lo] a_hi^T, cols 64..127 = [a_hi; a_lo] a_lo^T
+            const uint32_t aA = smem_u32(sA);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t o = (s >> 2) * 16384u + (s & 3) * 32u;
+                tc::mma_bf16(tmem + 0, tc::sw128_desc(aA + o, 16, 1024), tc::sw128_desc(aA + o, 16, 1024),
+                             ID_G, s > 0);
+                tc::mma_bf16(tmem + 64, tc::sw128_desc(aA + o, 16, 1024),
+                             tc::sw128_desc(aA + o + 8192, 16, 1024), ID_G, s > 0);
+            }
+            tc::mma_commit(mma_bar);
+            mma_pend = true;
+            if (ch + gy < nchunks) {  // the key tile has been read: fetch the next chunk's
+                tc::fence_async_smem();
+                issue_load(ch + gy);
+                tma_pend = true;
+            }
+        }
+        const bool mdone = mbar_wait_bounded(mma_bar, mph, limit_ns);
+        if (__syncthreads_or(!mdone)) {
+            fail = true;
+            break;
+        }
+        mph ^= 1u;
+        mma_pend = false;
+        tc::fence_after_sync();
+        // ---- G = hi hi^T + hi lo^T (lanes 0..63) + lo hi^T (lanes 64..127, added through sT)
+        {
+            float* dst = warp < 2 ? sL : sT;
+            const int row = warp < 2 ? tid : tid - 64;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float g0[16], g1[16];
+                tc::tmem_ld16(tmem + tlane + 16 * q, g0);
+                if (warp < 2) tc::tmem_ld16(tmem + tlane + 64 + 16 * q, g1);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    float4 o;
+                    o.x = g0[4 * v] + (warp < 2 ? g1[4 * v] : 0.f);
+                    o.y = g0[4 * v + 1] + (warp < 2 ? g1[4 * v + 1] : 0.f);
+                    o.z = g0[4 * v + 2] + (warp < 2 ? g1[4 * v + 2] : 0.f);
+                    o.w = g0[4 * v + 3] + (warp < 2 ? g1[4 * v + 3] : 0.f);
+                    tsw_st4(dst, row, 4 * q + v, o);
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- L_d[t][j] = c_t Gamma_tj G_tj for j < t; thread: row t = tid & 63, 32 columns
+        {
+            const int t = tid & 63, g0 = 8 * (tid >> 6);
+            const float ct = vc[t], lrt = vlr[t], sgt = vsg[t];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 a = tsw_ld4(sL, t, g0 + q), b = tsw_ld4(sT, t, g0 + q);
+                const float gs[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
+                float o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * (g0 + q) + e;
+                    o[e] = j < t ? ct * sgt * vsg1[j] * __expf(lrt - vlr1[j]) * gs[e] : 0.f;
+                }
+                tsw_st4(sL, t, g0 + q, make_float4(o[0], o[1], o[2], o[3]));
+            }
+        }
+        __syncthreads();
+        tril_inverse_64_g128(sL, sT, tid, 1);
+        // ---- rows t < Lc of T_d (tsw order kept) to the chunk's rows of the k~ buffer
+        {
+            const int t = tid >> 1, half = tid & 1;
+            if (t < Lc) {
+                const float4* src = reinterpret_cast<const float4*>(sT + t * 64) + 8 * half;
+                float4* dst = reinterpret_cast<float4*>(td_out + ((row0 + t) * H + h) * 64) + 8 * half;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dst[q] = src[q];
+            }
+        }
+        __syncthreads();  // sT and sL lie over the next chunk's a tiles
+    }
+    if (fail && tid == 0) {
+        if (tma_pend) mbar_wait_bounded(tma_bar, tph, limit_ns);
+        if (mma_pend) mbar_wait_bounded(mma_bar, mph, limit_ns);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
+// ===================================================================== chain: d across chunks
+
+struct ScanChainSmem {
+    static constexpr uint32_t KT = 0;                 // 3 x bf16 k tiles (16 KB, SW128)
+    static constexpr uint32_t TD = 3 * 16384;         // 3 x fp32 T_d tiles (16 KB, tsw rows)
+    static constexpr uint32_t VEC = 6 * 16384;        // 3 x {R, g, r, beta [64], R_C}
+    static constexpr uint32_t VECB = 1280;
+    static constexpr uint32_t D = VEC + 3 * VECB;     // 3 x d at chunk start [128]
+    static constexpr uint32_t X = D + 3 * 512;        // 3 x x [64]
+    static constexpr uint32_t GX = X + 3 * 256;       // g (.) x [64]
+    static constexpr uint32_t BV = GX + 256;          // b [64]
+    static constexpr uint32_t BAR = BV + 256;         // 15 mbarriers
+    static constexpr uint32_t TOTAL = BAR + 15 * 8;
+    static constexpr size_t BYTES = TOTAL + 1024;
+};
+constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output, 8 loads and gates
+
+// One CTA per (sequence, head).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
+__global__ void __launch_bounds__(SCAN_CHAIN_THREADS, 1)
+precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_td,
+                     const float* __restrict__ beta, const float* __restrict__ r, float eta,
+                     const float* __restrict__ d0, __nv_bfloat16* __restrict__ k_tilde,
+                     float* __restrict__ dT, const int32_t* __restrict__ cu, int N, int T, int H,
+                     long long limit_ns) {
+    constexpr int C = SCAN_C, DK = 128;
+    using L = ScanChainSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
+    if (n >= N) return;
+    int64_t first, count;
+    if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the CTA
+    const int nchunks = (int)((count + C - 1) / C);
+    const int64_t dbase = ((int64_t)n * H + h) * DK;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
+    uint64_t* full = bars;         // [3] TMA: k tile + T_d tile
+    uint64_t* vready = bars + 3;   // [3] gate vectors (32 arrivals)
+    uint64_t* kempty = bars + 6;   // [3] output warps done with the slot (128)
+    uint64_t* xready = bars + 9;   // [3] x and d of a chunk ready (128)
+    uint64_t* outdone = bars + 12; // [3] output warps done with x / d buffers (128)
+    float* sD = reinterpret_cast<float*>(smem + L::D);
+    float* sX = reinterpret_cast<float*>(smem + L::X);
+    float* sGX = reinterpret_cast<float*>(smem + L::GX);
+    float* sB = reinterpret_cast<float*>(smem + L::BV);
+    auto vecs = [&](int s) { return reinterpret_cast<float*>(smem + L::VEC + s * L::VECB); };
+    auto chunk_len = [&](int c) -> int {
+        const int64_t rem = count - (int64_t)c * C;
+        return rem < C ? (int)rem : C;
+    };
+
+    if (tid == 0) {
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&vready[s], 32);
+            mbar_init(&kempty[s], 128);
+            mbar_init(&xready[s], 128);
+            mbar_init(&outdone[s], 128);
+        }
+        tc::fence_mbar_init();
+    }
+    if (tid < DK) sD[tid] = d0 ? __ldg(d0 + dbase + tid) : 1.0f;
+    __syncthreads();
+
+    if (warp == 8) {
+        // =============================================== loads and gate vectors
+        if (lane == 0) {
+            tc::prefetch_tmap(&tm_k);
+            tc::prefetch_tmap(&tm_td);
+        }
+        int last_issued = -1;
+        bool fail = false;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % 3;
+            if (c >= 3 && !mbar_wait_bounded(&kempty[s], (uint32_t)(c / 3 - 1) & 1u, limit_ns)) {
+                fail = true;
+                break;
+            }
+            const int64_t row0 = first + (int64_t)c * C;
+            if (lane == 0) {
+                uint8_t* kt = smem + L::KT + s * 16384;
+                tc::mbar_expect_tx(&full[s], 32768);
+                tc::tma_load_3d(kt, &tm_k, 0, h, (int)row0, &full[s]);
+                tc::tma_load_3d(kt + 8192, &tm_k, 64, h, (int)row0, &full[s]);
+                tc::tma_load_3d(smem + L::TD + s * 16384, &tm_td, 0, h, (int)row0, &full[s]);
+            }
+            last_issued = c;
+            const int Lc = chunk_len(c), t0 = 2 * lane;
+            const bool v0 = t0 < Lc, v1 = t0 + 1 < Lc;
+            const float r0 = (r && v0) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
+            const float r1 = (r && v1) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
+            const GatePrefix g = gate_prefix(r0, r1, lane);
+            float* vv = vecs(s);  // R | g | r | beta | R_C
+            vv[t0] = g.sg0 * __expf(g.lr0);
+            vv[t0 + 1] = g.sg_1 * __expf(g.lr_1);
+            vv[64 + t0] = g.sgC * g.sg1_0 * __expf(g.lrC - g.lr1_0);
+            vv[64 + t0 + 1] = g.sgC * g.sg1_1 * __expf(g.lrC - g.lr1_1);
+            vv[128 + t0] = r0;
+            vv[128 + t0 + 1] = r1;
+            vv[192 + t0] = v0 ? __ldg(beta + (row0 + t0) * H + h) : 0.f;
+            vv[192 + t0 + 1] = v1 ? __ldg(beta + (row0 + t0 + 1) * H + h) : 0.f;
+            if (lane == 0) vv[256] = g.sgC * __expf(g.lrC);
+            mbar_arrive(&vready[s]);
+        }
+        if (fail && lane == 0 && last_issued >= 0) {  // let the loads in flight land
+            for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
+                mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
+        }
+    } else if (warp < 4) {
+        // =============================================== p = A d, x = T_d b, next d
+        const int u = tid;
+        const int t = 16 * warp + (lane & 15), half = lane >> 4;  // step 1/2 roles
+        const int ci = u, cblk = ci >> 6, cj = (ci & 63) >> 3, ce = ci & 7;  // step 3 role
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % 3;
+            const uint32_t ph = (uint32_t)(c / 3) & 1u;
+            bool got = mbar_wait_bounded(&full[s], ph, limit_ns) &&
+                       mbar_wait_bounded(&vready[s], ph, limit_ns);
+            if (got && c >= 2)
+                got = mbar_wait_bounded(&outdone[(c - 2) % 3], (uint32_t)((c - 2) / 3) & 1u, limit_ns);
+            if (group_any(1, 128, !got)) {
+                ok = false;
+                break;
+            }
+            const int Lc = chunk_len(c);
+            const uint8_t* kt = smem + L::KT + s * 16384;
+            const float* td = reinterpret_cast<const float*>(smem + L::TD + s * 16384);
+            const float* vv = vecs(s);
+            const float* d = sD + (c % 3) * 128;
+            // ---- step 1: p_t = <a_t, d>, ||k_t||^2, b_t
+            {
+                float p = 0.f, nk = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 raw = *reinterpret_cast<const uint4*>(kt + half * 8192u + tc::sw128_off(t, j));
+                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                    const float4 da = *reinterpret_cast<const float4*>(d + 64 * half + 8 * j);
+                    const float4 db = *reinterpret_cast<const float4*>(d + 64 * half + 8 * j + 4);
+                    const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                        const float a0 = kk.x * kk.x, a1 = kk.y * kk.y;
+                        nk += a0 + a1;
+                        p = fmaf(a0, dv[2 * e], p);
+                        p = fmaf(a1, dv[2 * e + 1], p);
+                    }
+                }
+                p += __shfl_xor_sync(0xffffffffu, p, 16);
+                nk += __shfl_xor_sync(0xffffffffu, nk, 16);
+                if (half == 0) {
+                    const float bt = vv[192 + t];
+                    const float e = (t < Lc && nk > 0.f) ? eta * bt / nk : 0.f;
+                    sB[t] = e * (1.f - bt * vv[t] * p);
+                }
+            }
+            group_bar(1, 128);
+            // ---- step 2: x_t = sum_{j <= t} T_d[t][j] b_j
+            {
+                float acc = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int g = 8 * half + q;
+                    const float4 tv = tsw_ld4(td, t, g);
+                    const float4 bv = *reinterpret_cast<const float4*>(sB + 4 * g);
+                    const int j = 4 * g;
+                    acc = fmaf(j <= t ? tv.x : 0.f, bv.x, acc);
+                    acc = fmaf(j + 1 <= t ? tv.y : 0.f, bv.y, acc);
+                    acc = fmaf(j + 2 <= t ? tv.z : 0.f, bv.z, acc);
+                    acc = fmaf(j + 3 <= t ? tv.w : 0.f, bv.w, acc);
+                }
+                acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+                if (half == 0) {
+                    const float x = t < Lc ? acc : 0.f;
+                    sX[(c % 3) * 64 + t] = x;
+                    sGX[t] = vv[64 + t] * x;
+                }
+            }
+            group_bar(1, 128);
+            // ---- step 3: d_C[i] = R_C d[i] + sum_j g_j x_j a_j[i]
+            {
+                float acc = vv[256] * d[ci];
+                const uint8_t* col = kt + cblk * 8192u + ce * 2;
+#pragma unroll 16
+                for (int j = 0; j < C; ++j) {
+                    const float kv = __bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16*>(col + tc::sw128_off(j, cj)));
+                    acc = fmaf(sGX[j], kv * kv, acc);
+                }
+                sD[((c + 1) % 3) * 128 + ci] = acc;
+            }
+            mbar_arrive(&xready[c % 3]);
+            group_bar(1, 128);
+        }
+        if (ok && dT) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
+    } else {
+        // =============================================== k~ = d (.) k, token by token
+        const int i = tid - 128, blk = i >> 6, cj = (i & 63) >> 3, ce = i & 7;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % 3;
+            if (group_any(2, 128, !mbar_wait_bounded(&xready[c % 3], (uint32_t)(c / 3) & 1u, limit_ns)))
+                break;
+            const int Lc = chunk_len(c);
+            const uint8_t* col = smem + L::KT + s * 16384 + blk * 8192u + ce * 2;
+            const float* xv = sX + (c % 3) * 64;
+            const float* rv = vecs(s) + 128;
+            float dd = sD[(c % 3) * 128 + i];
+            __nv_bfloat16* out = k_tilde + ((first + (int64_t)c * C) * H + h) * DK + i;
+            const int64_t rs = (int64_t)H * DK;
+#pragma unroll 8
+            for (int t = 0; t < Lc; ++t) {
+                const float kv = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16*>(col + tc::sw128_off(t, cj)));
+                out[t * rs] = __float2bfloat16_rn(dd * kv);
+                dd = fmaf(rv[t], dd, xv[t] * kv * kv);
+            }
+            mbar_arrive(&kempty[s]);
+            mbar_arrive(&outdone[c % 3]);
+        }
+    }
+    __syncthreads();
+}
+
+}  // namespace osdn

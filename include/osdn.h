@@ -89,7 +89,9 @@ OSDN_API const char* osdn_status_string(osdn_status_t status);
  *   r       [B,T,H] float32 retention gate, or NULL for r == 1 (plain OSDN, no APF).
  *   eta     step size of the preconditioner's gradient descent (eta == 0 freezes d).
  *   d0      [N,H,Dk] initial preconditioner, or NULL for all ones.
- *   k_tilde [B,T,H,Dk] io dtype, written: k~_t = d_t (.) k_t.  Must not alias k.
+ *   k_tilde [B,T,H,Dk] io dtype, written: k~_t = d_t (.) k_t.  Must not overlap k, beta, r,
+ *           d0 or dT (OSDN_ERR_INVALID_ARG): for bf16 with Dk = 128 the call first uses this
+ *           buffer as scratch for per-chunk factors, then overwrites it with k~.
  *   dT      [N,H,Dk] final preconditioner, written; NULL skips it.
  */
 OSDN_API osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r, float eta,

@@ -80,6 +80,10 @@ def test_chunk_fwd_rejects(kw, status):
     (dict(kt=None), osdn.OSDN_ERR_INVALID_ARG),
     (dict(kt=fake(1)), osdn.OSDN_ERR_INVALID_ARG),          # in place k~ == k
     (dict(kt=ctypes.c_void_p(A + 0x1000000 + 256)), osdn.OSDN_ERR_INVALID_ARG),  # overlap
+    (dict(beta=ctypes.c_void_p(A + 3 * 0x1000000 + 64)), osdn.OSDN_ERR_INVALID_ARG),  # in k~
+    (dict(r=ctypes.c_void_p(A + 3 * 0x1000000 + 512)), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(d0=ctypes.c_void_p(A + 3 * 0x1000000)), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(dT=ctypes.c_void_p(A + 3 * 0x1000000 + 1024)), osdn.OSDN_ERR_INVALID_ARG),
     (dict(r=ctypes.c_void_p(A + 2)), osdn.OSDN_ERR_ALIGNMENT),
     (dict(cu=ctypes.c_void_p(A + 4), num_seqs=1), osdn.OSDN_ERR_ALIGNMENT),
     (dict(num_seqs=-1), osdn.OSDN_ERR_INVALID_ARG),
