@@ -104,8 +104,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     constexpr int DK = 128, BV = 64, C = 64, NVT = DV / BV;
     using L = TcSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = smem_align1024(smem_raw);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int vt = blockIdx.x % NVT, nh = blockIdx.x / NVT;

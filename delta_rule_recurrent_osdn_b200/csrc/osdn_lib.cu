@@ -184,15 +184,15 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     CUtensorMap mk, mtd;
     if (!make_tile_map(&mk, k, 128, d.H, rows) || !make_td_map(&mtd, k_tilde, d.H, rows))
         return OSDN_ERR_CUDA;
-    // chunks per (sequence, head): exact for fixed length, about the mean for packed sequences
-    const int64_t per_seq = cu ? rows / d.N / 64 + 1 : ((int64_t)d.T + 63) / 64;
-    int64_t gy = (3 * (int64_t)sm_count() + nh - 1) / nh;
-    gy = gy > per_seq ? per_seq : gy;
-    gy = gy < 1 ? 1 : (gy > 65535 ? 65535 : gy);
+    // persistent prep grid over (64-row window, head) items
+    const int64_t items = ((rows + 63) / 64) * d.H;
+    int64_t grid = (int64_t)SCAN_PREP_CTAS_PER_SM * sm_count();
+    grid = grid < items ? grid : items;
     auto prep = precond_prep_kernel;
     if (!set_smem(prep, ScanPrepSmem::BYTES)) return OSDN_ERR_CUDA;
-    prep<<<dim3((unsigned)nh, (unsigned)gy), dim3(128), ScanPrepSmem::BYTES, stream>>>(
-        mk, beta, r, eta, static_cast<float*>(k_tilde), cu, d.N, d.T, d.H, (long long)kWaitLimitNs);
+    prep<<<dim3((unsigned)grid), dim3(128), ScanPrepSmem::BYTES, stream>>>(
+        mk, beta, r, eta, static_cast<float*>(k_tilde), cu, d.N, d.T, d.H, rows,
+        (long long)kWaitLimitNs);
     const osdn_status_t st = launch_status();
     if (st != OSDN_OK) return st;
     auto chain = precond_chain_kernel;

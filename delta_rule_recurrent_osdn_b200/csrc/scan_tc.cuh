@@ -72,6 +72,73 @@ __device__ __forceinline__ GatePrefix gate_prefix(float r0, float r1, int lane) 
 
 // ===================================================================== prep: T_d per chunk
 
+// Walks the chunks of the whole batch for a persistent CTA.  Work item w = (64-row window of
+// the token rows, head); a window holds the start of at most one chunk of each sequence that
+// overlaps it (chunk starts are 64 rows apart), so items are near-uniform in size whatever the
+// sequence lengths.  Items w = blockIdx.x, blockIdx.x + gridDim.x, ...
+struct ChunkWalk {
+    const int32_t* cu;
+    int N, T, H;
+    int64_t rows, W, w;
+    int n;          // next sequence to examine in the current window
+    bool fresh;     // the current window's first sequence is not located yet
+    // output of next(): the chunk
+    int64_t row0;
+    int Lc, h;
+
+    __device__ void init(const int32_t* cu_, int N_, int T_, int H_, int64_t rows_) {
+        cu = cu_;
+        N = N_;
+        T = T_;
+        H = H_;
+        rows = rows_;
+        W = ((rows + SCAN_C - 1) / SCAN_C) * H;
+        w = blockIdx.x;
+        fresh = true;
+    }
+    // Last sequence whose first row is <= row (sequences are contiguous and ordered).
+    __device__ int seq_at(int64_t row) const {
+        if (!cu) {
+            const int64_t q = row / T;
+            return q < N - 1 ? (int)q : N - 1;
+        }
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((int64_t)__ldg(cu + mid) <= row) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    }
+    // Advance to the next chunk; false when the CTA's items are exhausted.
+    __device__ bool next() {
+        while (w < W) {
+            const int64_t lo = (w / H) * SCAN_C;
+            const int64_t hi = lo + SCAN_C < rows ? lo + SCAN_C : rows;
+            if (fresh) {
+                n = seq_at(lo);
+                fresh = false;
+            }
+            while (n < N) {
+                int64_t first, count;
+                if (!seq_range(cu, n, N, T, first, count)) return false;
+                if (first >= hi) break;
+                ++n;
+                const int64_t end = first + count;
+                const int64_t s = first >= lo ? first : first + ((lo - first + SCAN_C - 1) / SCAN_C) * SCAN_C;
+                if (s < hi && s < end) {
+                    row0 = s;
+                    Lc = end - s < SCAN_C ? (int)(end - s) : SCAN_C;
+                    h = (int)(w % H);
+                    return true;
+                }
+            }
+            w += gridDim.x;
+            fresh = true;
+        }
+        return false;
+    }
+};
+
 struct ScanPrepSmem {
     static constexpr uint32_t K = 0;              // bf16 k tile: 2 K-blocks x (64 rows x 128 B)
     static constexpr uint32_t A = 16384;          // bf16 [a_hi; a_lo] per K-block, 2 x 16 KB
@@ -83,27 +150,22 @@ struct ScanPrepSmem {
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
+constexpr int SCAN_PREP_CTAS_PER_SM = 3;
 
-// Grid (N * H, gy): CTA (nh, y) handles chunks y, y + gy, ... of its (sequence, head).
-// 128 threads; td_out is the k~ buffer seen as fp32 rows of 64 values.
-__global__ void __launch_bounds__(128, 3)
+// Persistent grid (one to three CTAs per SM) of 128 threads walking the batch's chunks with
+// ChunkWalk.  td_out is the k~ buffer seen as fp32 rows of 64 values.
+__global__ void __launch_bounds__(128, SCAN_PREP_CTAS_PER_SM)
 precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ beta,
                     const float* __restrict__ r, float eta, float* __restrict__ td_out,
-                    const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
-    constexpr int C = SCAN_C;
+                    const int32_t* __restrict__ cu, int N, int T, int H, int64_t rows,
+                    long long limit_ns) {
     using L = ScanPrepSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = smem_align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
-    if (n >= N) return;
-    int64_t first, count;
-    if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the CTA
-    const int nchunks = (int)((count + C - 1) / C);
-    const int gy = gridDim.y;
-    int ch = blockIdx.y;
-    if (ch >= nchunks) return;
+    ChunkWalk walk;
+    walk.init(cu, N, T, H, rows);
+    if (!walk.next()) return;  // uniform over the CTA
 
     uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* mma_bar = tma_bar + 1;
@@ -134,22 +196,20 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
     const uint32_t tmem = *tmem_slot;
     const uint32_t tlane = static_cast<uint32_t>(warp * 32) << 16;
 
-    auto issue_load = [&](int c) {
-        const int row = (int)(first + (int64_t)c * C);
+    auto issue_load = [&](int64_t row, int hh) {
         tc::mbar_expect_tx(tma_bar, 16384);
-        tc::tma_load_3d(sK, &tm_k, 0, h, row, tma_bar);
-        tc::tma_load_3d(sK + 8192, &tm_k, 64, h, row, tma_bar);
+        tc::tma_load_3d(sK, &tm_k, 0, hh, (int)row, tma_bar);
+        tc::tma_load_3d(sK + 8192, &tm_k, 64, hh, (int)row, tma_bar);
     };
-    if (tid == 0) issue_load(ch);
-    bool tma_pend = tid == 0, mma_pend = false, fail = false;
+    if (tid == 0) issue_load(walk.row0, walk.h);
+    bool tma_pend = tid == 0, mma_pend = false, fail = false, more = true;
     uint32_t tph = 0, mph = 0;
     constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);
 
 #pragma unroll 1
-    for (; ch < nchunks; ch += gy) {
-        const int64_t cs = (int64_t)ch * C;
-        const int Lc = count - cs < C ? (int)(count - cs) : C;
-        const int64_t row0 = first + cs;
+    while (more) {
+        const int64_t row0 = walk.row0;
+        const int Lc = walk.Lc, h = walk.h;
         const bool got = mbar_wait_bounded(tma_bar, tph, limit_ns);
         if (__syncthreads_or(!got)) {
             fail = true;
@@ -222,11 +282,12 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
             }
             tc::mma_commit(mma_bar);
             mma_pend = true;
-            if (ch + gy < nchunks) {  // the key tile has been read: fetch the next chunk's
-                tc::fence_async_smem();
-                issue_load(ch + gy);
-                tma_pend = true;
-            }
+        }
+        more = walk.next();  // uniform: every thread walks the same items
+        if (tid == 0 && more) {  // the key tile has been read: fetch the next chunk's
+            tc::fence_async_smem();
+            issue_load(walk.row0, walk.h);
+            tma_pend = true;
         }
         const bool mdone = mbar_wait_bounded(mma_bar, mph, limit_ns);
         if (__syncthreads_or(!mdone)) {
@@ -326,8 +387,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     constexpr int C = SCAN_C, DK = 128;
     using L = ScanChainSmem;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = smem_align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x / H, h = blockIdx.x - n * H;
     if (n >= N) return;
@@ -373,6 +433,18 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         }
         int last_issued = -1;
         bool fail = false;
+        // gates of the next chunk are fetched one iteration early to hide their load latency
+        float nr0 = 1.f, nr1 = 1.f, nb0 = 0.f, nb1 = 0.f;
+        auto fetch_gates = [&](int c) {
+            const int64_t row0 = first + (int64_t)c * C;
+            const int Lc = chunk_len(c), t0 = 2 * lane;
+            const bool v0 = t0 < Lc, v1 = t0 + 1 < Lc;
+            nr0 = (r && v0) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
+            nr1 = (r && v1) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
+            nb0 = v0 ? __ldg(beta + (row0 + t0) * H + h) : 0.f;
+            nb1 = v1 ? __ldg(beta + (row0 + t0 + 1) * H + h) : 0.f;
+        };
+        if (nchunks > 0) fetch_gates(0);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % 3;
             if (c >= 3 && !mbar_wait_bounded(&kempty[s], (uint32_t)(c / 3 - 1) & 1u, limit_ns)) {
@@ -388,10 +460,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 tc::tma_load_3d(smem + L::TD + s * 16384, &tm_td, 0, h, (int)row0, &full[s]);
             }
             last_issued = c;
-            const int Lc = chunk_len(c), t0 = 2 * lane;
-            const bool v0 = t0 < Lc, v1 = t0 + 1 < Lc;
-            const float r0 = (r && v0) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
-            const float r1 = (r && v1) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
+            const int t0 = 2 * lane;
+            const float r0 = nr0, r1 = nr1, b0 = nb0, b1 = nb1;
+            if (c + 1 < nchunks) fetch_gates(c + 1);
             const GatePrefix g = gate_prefix(r0, r1, lane);
             float* vv = vecs(s);  // R | g | r | beta | R_C
             vv[t0] = g.sg0 * __expf(g.lr0);
@@ -400,8 +471,8 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             vv[64 + t0 + 1] = g.sgC * g.sg1_1 * __expf(g.lrC - g.lr1_1);
             vv[128 + t0] = r0;
             vv[128 + t0 + 1] = r1;
-            vv[192 + t0] = v0 ? __ldg(beta + (row0 + t0) * H + h) : 0.f;
-            vv[192 + t0 + 1] = v1 ? __ldg(beta + (row0 + t0 + 1) * H + h) : 0.f;
+            vv[192 + t0] = b0;
+            vv[192 + t0 + 1] = b1;
             if (lane == 0) vv[256] = g.sgC * __expf(g.lrC);
             mbar_arrive(&vready[s]);
         }
@@ -413,7 +484,8 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         // =============================================== p = A d, x = T_d b, next d
         const int u = tid;
         const int t = 16 * warp + (lane & 15), half = lane >> 4;  // step 1/2 roles
-        const int ci = u, cblk = ci >> 6, cj = (ci & 63) >> 3, ce = ci & 7;  // step 3 role
+        const int cp = u >> 1, par = u & 1;  // step 3 role: channel pair, token half
+        const int cblk = cp >> 5, cj = (cp & 31) >> 2, cpe = 2 * (cp & 3);
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % 3;
@@ -481,17 +553,29 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 }
             }
             group_bar(1, 128);
-            // ---- step 3: d_C[i] = R_C d[i] + sum_j g_j x_j a_j[i]
+            // ---- step 3: d_C[i] = R_C d[i] + sum_j g_j x_j a_j[i]; thread: channels 2cp, 2cp + 1
+            //      over the tokens with bit 2 clear (par 0) or set (par 1) -- rows whose swizzle
+            //      phases differ, so the lane pair reads disjoint banks -- summed by a shuffle
             {
-                float acc = vv[256] * d[ci];
-                const uint8_t* col = kt + cblk * 8192u + ce * 2;
-#pragma unroll 16
-                for (int j = 0; j < C; ++j) {
-                    const float kv = __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16*>(col + tc::sw128_off(j, cj)));
-                    acc = fmaf(sGX[j], kv * kv, acc);
+                float acc0 = 0.f, acc1 = 0.f;
+                const uint8_t* col = kt + cblk * 8192u + cpe * 2;
+#pragma unroll 8
+                for (int jj = 0; jj < C / 2; ++jj) {
+                    const int j = (jj & 3) + ((jj >> 2) << 3) + 4 * par;
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(col + tc::sw128_off(j, cj));
+                    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+                    const float gx = sGX[j];
+                    acc0 = fmaf(gx, kv.x * kv.x, acc0);
+                    acc1 = fmaf(gx, kv.y * kv.y, acc1);
                 }
-                sD[((c + 1) % 3) * 128 + ci] = acc;
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+                if (par == 0) {
+                    const float rc = vv[256];
+                    const float2 dv = *reinterpret_cast<const float2*>(d + 2 * cp);
+                    *reinterpret_cast<float2*>(sD + ((c + 1) % 3) * 128 + 2 * cp) =
+                        make_float2(fmaf(rc, dv.x, acc0), fmaf(rc, dv.y, acc1));
+                }
             }
             mbar_arrive(&xready[c % 3]);
             group_bar(1, 128);
@@ -509,14 +593,40 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             const float* xv = sX + (c % 3) * 64;
             const float* rv = vecs(s) + 128;
             float dd = sD[(c % 3) * 128 + i];
-            __nv_bfloat16* out = k_tilde + ((first + (int64_t)c * C) * H + h) * DK + i;
-            const int64_t rs = (int64_t)H * DK;
-#pragma unroll 8
-            for (int t = 0; t < Lc; ++t) {
-                const float kv = __bfloat162float(
-                    *reinterpret_cast<const __nv_bfloat16*>(col + tc::sw128_off(t, cj)));
-                out[t * rs] = __float2bfloat16_rn(dd * kv);
-                dd = fmaf(rv[t], dd, xv[t] * kv * kv);
+            // k~ goes to the chunk's T_d slot (consumed by step 2 before x was published) in the
+            // key tile's swizzled layout, then to global memory as whole 16-byte row pieces:
+            // scattered 2-byte stores would cost about three times the whole token pass
+            uint8_t* stage = smem + L::TD + s * 16384;
+            uint8_t* ocol = stage + blk * 8192u + ce * 2;
+#pragma unroll 1
+            for (int t0 = 0; t0 < Lc; t0 += 16) {
+                float kv[16], xt[16], rt[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    kv[u] = __bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16*>(col + tc::sw128_off(t0 + u, cj)));
+                    xt[u] = xv[t0 + u];
+                    rt[u] = rv[t0 + u];
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    *reinterpret_cast<__nv_bfloat16*>(ocol + tc::sw128_off(t0 + u, cj)) =
+                        __float2bfloat16_rn(dd * kv[u]);
+                    dd = fmaf(rt[u], dd, xt[u] * kv[u] * kv[u]);
+                }
+            }
+            group_bar(2, 128);
+            {
+                const int piece = i & 15, blk16 = piece >> 3, j16 = piece & 7;
+                __nv_bfloat16* orow = k_tilde + ((first + (int64_t)c * C) * H + h) * DK + 8 * piece;
+                const int64_t rs = (int64_t)H * DK;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int row = (i >> 4) + 8 * q;
+                    if (row < Lc)
+                        *reinterpret_cast<uint4*>(orow + row * rs) = *reinterpret_cast<const uint4*>(
+                            stage + blk16 * 8192u + tc::sw128_off(row, j16));
+                }
             }
             mbar_arrive(&kempty[s]);
             mbar_arrive(&outdone[c % 3]);
