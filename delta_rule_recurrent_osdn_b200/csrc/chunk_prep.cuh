@@ -1,0 +1,190 @@
+// chunk_prep.cuh -- the WY factor of every phase-2 chunk, computed for all chunks at once.
+//
+// The chunkwise delta rule with write key K~ ("OSDN: Improving Delta Rule with Provable Online
+// Preconditioning in Linear Attention", technical summary, section 2.1) needs, per chunk of 64
+// tokens with rows K, K~ and gates beta,
+//   T = (I + strict_tril(diag(beta) K K~^T))^-1,
+// which does not depend on the state.  wy_prep_kernel computes it for every chunk in parallel:
+// K K~^T by one bf16 MMA (both operands are exact bf16, so the fp32 accumulation is the only
+// rounding), the inverse by tril_inverse_64_g128.  The sequential kernel (chunk_tc.cuh) then
+// only reads T.
+//
+// Hand-off through the output buffer o, which the sequential kernel writes only after reading
+// T: the strictly lower triangle of T (its diagonal is 1), row-major and packed -- entry (t, j),
+// j < t, at index t (t - 1) / 2 + j; 2016 floats for a full chunk -- is written into each
+// 64-channel value tile's slice of the chunk's o rows (64 rows x 128 bytes), one copy per tile,
+// so every sequential CTA reads the copy in its own slice before overwriting that slice with
+// its outputs.  A chunk of Lc < 64 tokens needs Lc (Lc - 1) / 2 floats, which fit in its Lc rows.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tril_inverse.cuh"
+#include "chunk_walk.cuh"
+
+namespace osdn {
+
+struct WyPrepSmem {
+    static constexpr uint32_t K = 0;            // bf16 K tile: 2 K-blocks x (64 rows x 128 B)
+    static constexpr uint32_t KT = 16384;       // bf16 K~ tile, same layout
+    static constexpr uint32_t SL = 32768;       // fp32 L (tsw)
+    static constexpr uint32_t ST = 49152;       // fp32 T (tsw)
+    static constexpr uint32_t BETA = 65536;     // 64 floats
+    static constexpr uint32_t BAR = BETA + 256;
+    static constexpr uint32_t TMEM_SLOT = BAR + 16;
+    static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
+    static constexpr size_t BYTES = TOTAL + 1024;
+};
+constexpr int WY_PREP_CTAS_PER_SM = 3;
+
+// Packed index t (t - 1) / 2 + j  ->  row t (the j follows).
+__device__ __forceinline__ int packed_row(int f) {
+    int t = (int)((1.f + sqrtf(8.f * (float)f + 1.f)) * 0.5f);
+    while (t * (t - 1) / 2 > f) --t;
+    while ((t + 1) * t / 2 <= f) ++t;
+    return t;
+}
+
+// Persistent grid of 128-thread CTAs walking the batch's chunks (ChunkWalk).  o_f32 is the
+// output buffer [rows, H, Dv] (bf16) seen as floats; Dv = 64 * (number of value tiles).
+__global__ void __launch_bounds__(128, WY_PREP_CTAS_PER_SM)
+wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kt,
+               const float* __restrict__ beta, float* __restrict__ o_f32, int Dv,
+               const int32_t* __restrict__ cu, int N, int T, int H, int64_t rows,
+               long long limit_ns) {
+    using L = WyPrepSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align1024(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    ChunkWalk walk;
+    walk.init(cu, N, T, H, rows);
+    if (!walk.next()) return;  // uniform over the CTA
+
+    uint64_t* tma_bar = reinterpret_cast<uint64_t*>(smem + L::BAR);
+    uint64_t* mma_bar = tma_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
+    uint8_t* sK = smem + L::K;
+    uint8_t* sKT = smem + L::KT;
+    float* sL = reinterpret_cast<float*>(smem + L::SL);
+    float* sT = reinterpret_cast<float*>(smem + L::ST);
+    float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
+
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 64);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        tc::fence_mbar_init();
+        tc::prefetch_tmap(&tm_k);
+        tc::prefetch_tmap(&tm_kt);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tlane = static_cast<uint32_t>(warp * 32) << 16;
+
+    auto issue_load = [&](int64_t row, int hh) {
+        tc::mbar_expect_tx(tma_bar, 32768);
+        tc::tma_load_3d(sK, &tm_k, 0, hh, (int)row, tma_bar);
+        tc::tma_load_3d(sK + 8192, &tm_k, 64, hh, (int)row, tma_bar);
+        tc::tma_load_3d(sKT, &tm_kt, 0, hh, (int)row, tma_bar);
+        tc::tma_load_3d(sKT + 8192, &tm_kt, 64, hh, (int)row, tma_bar);
+    };
+    auto load_beta = [&](int64_t row, int Lc, int hh) {
+        return tid < Lc ? __ldg(beta + (row + tid) * H + hh) : 0.f;
+    };
+    if (tid == 0) issue_load(walk.row0, walk.h);
+    float bnext = tid < 64 ? load_beta(walk.row0, walk.Lc, walk.h) : 0.f;
+    bool tma_pend = tid == 0, mma_pend = false, fail = false, more = true;
+    uint32_t tph = 0, mph = 0;
+    // M = 128 over the K tile: rows 64..127 of the operand view are the next 64 rows of shared
+    // memory (finite data), whose products land in TMEM lanes 64..127 and are never read
+    constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);
+    const int nvt = Dv / 64, half_f = Dv / 2;
+
+#pragma unroll 1
+    while (more) {
+        const int64_t row0 = walk.row0;
+        const int Lc = walk.Lc, h = walk.h;
+        if (tid < 64) sBeta[tid] = bnext;
+        const bool got = mbar_wait_bounded(tma_bar, tph, limit_ns);
+        if (__syncthreads_or(!got)) {
+            fail = true;
+            break;
+        }
+        tph ^= 1u;
+        tma_pend = false;
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t aK = smem_u32(sK), aKT = smem_u32(sKT);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t o = (s >> 2) * 8192u + (s & 3) * 32u;
+                tc::mma_bf16(tmem, tc::sw128_desc(aK + o, 16, 1024), tc::sw128_desc(aKT + o, 16, 1024),
+                             ID_G, s > 0);
+            }
+            tc::mma_commit(mma_bar);
+            mma_pend = true;
+        }
+        more = walk.next();  // uniform: every thread walks the same items
+        if (more && tid < 64) bnext = load_beta(walk.row0, walk.Lc, walk.h);
+        const bool mdone = mbar_wait_bounded(mma_bar, mph, limit_ns);
+        if (__syncthreads_or(!mdone)) {
+            fail = true;
+            break;
+        }
+        mph ^= 1u;
+        mma_pend = false;
+        tc::fence_after_sync();
+        if (tid == 0 && more) {  // the tiles have been consumed by the MMA: fetch the next chunk's
+            issue_load(walk.row0, walk.h);
+            tma_pend = true;
+        }
+        // ---- L[t][j] = beta_t (K K~^T)[t][j] for j < t (lanes 0..63 = rows)
+        if (warp < 2) {
+            const float bt = sBeta[tid];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float g[16];
+                tc::tmem_ld16(tmem + tlane + 16 * q, g);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int j = 16 * q + 4 * v;
+                    tsw_st4(sL, tid, 4 * q + v,
+                            make_float4(j < tid ? bt * g[4 * v] : 0.f, j + 1 < tid ? bt * g[4 * v + 1] : 0.f,
+                                        j + 2 < tid ? bt * g[4 * v + 2] : 0.f,
+                                        j + 3 < tid ? bt * g[4 * v + 3] : 0.f));
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        tril_inverse_64_g128(sL, sT, tid, 1);
+        // ---- packed strictly-lower T, one copy per value tile
+        {
+            const int npk = Lc * (Lc - 1) / 2;
+            for (int f = tid; f < npk; f += 128) {
+                const int t = packed_row(f), j = f - t * (t - 1) / 2;
+                const float val = sT[tsw(t, j)];
+                float* dst = o_f32 + ((row0 + (f >> 5)) * H + h) * half_f + (f & 31);
+                for (int vt = 0; vt < nvt; ++vt) dst[32 * vt] = val;
+            }
+        }
+        __syncthreads();  // sL / sT are rewritten by the next chunk
+    }
+    if (fail && tid == 0) {
+        if (tma_pend) mbar_wait_bounded(tma_bar, tph, limit_ns);
+        if (mma_pend) mbar_wait_bounded(mma_bar, mph, limit_ns);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 64);
+}
+
+}  // namespace osdn

@@ -4,8 +4,9 @@
 // Preconditioning in Linear Attention", technical summary, section 2.1: K~ replaces K in the
 // chunk Gram matrix and in the intra-chunk scores).  Per chunk of C = 64 tokens, state S_0
 // (value rows), this CTA's 64 value channels:
-//   G = K K~^T,  P = tril(Q K~^T)                 one bf16 MMA, A = [K; Q] (M = 128)
-//   T = (I + strict_tril(diag(beta) G))^-1        fp32 blocked inverse in shared memory
+//   P = tril(Q K~^T)                              one bf16 MMA, A = [K; Q] (M = 128)
+//   T = (I + strict_tril(diag(beta) K K~^T))^-1   computed for all chunks beforehand by
+//                                                 wy_prep_kernel (chunk_prep.cuh), read here
 //   R = diag(beta) (V - K S_0^T)                  A = [K; Q], B = S_0^T  (rows 64..127: Q S_0^T)
 //   W = T R                                       A = Z = [T; P], B = R
 //   O = Q S_0^T + P W                             A = Z, B = W, accumulated onto Q S_0^T
@@ -21,7 +22,8 @@
 // Warp roles (one CTA per (sequence, head, 64 value channels), 288 threads):
 //   chain    warps 0-3: the state-dependent MMA chain of chunk c and its epilogues (thread t owns
 //            tensor-memory lane t);
-//   prep     warps 4-7: chunk c+1's Gram MMA, L, P, the inverse T and the [T; P] operand tiles,
+//   prep     warps 4-7: chunk c+1's [T; P] operand tiles (T unpacked from the copy the
+//            pre-kernel left in this CTA's slice of the chunk's o rows, P from a Gram MMA),
 //            overlapping chunk c's chain;
 //   producer warp 8: TMA loads of the chunk tiles into a 2-stage ring (no multicast).
 // Handshakes are mbarriers: z_full / z_empty for the [T; P] tiles, stage_empty for the ring.
@@ -38,17 +40,15 @@
 namespace osdn {
 
 struct TcSmem {
-    static constexpr uint32_t STAGE = 57344;          // [K;Q] 32K | K~ 16K | V 8K
-    static constexpr uint32_t KQ = 0, KT = 32768, V = 49152;
+    static constexpr uint32_t STAGE = 65536;          // [K;Q] 32K | K~ 16K | V 8K | packed T 8K
+    static constexpr uint32_t KQ = 0, KT = 32768, V = 49152, TP = 57344;
     static constexpr uint32_t ZHI = 2 * STAGE;        // bf16 [T; P] hi / lo, K-major, 128 x 128 B
     static constexpr uint32_t ZLO = ZHI + 16384;
     static constexpr uint32_t SHI = ZLO + 16384;      // bf16 S^T hi / lo, MN-major, 128 x 128 B
     static constexpr uint32_t SLO = SHI + 16384;
     static constexpr uint32_t RHI = SLO + 16384;      // bf16 R then W, hi / lo, 64 x 128 B
     static constexpr uint32_t RLO = RHI + 8192;
-    static constexpr uint32_t SL = RLO + 8192;        // fp32 L, 64 x 64, swizzled (tsw)
-    static constexpr uint32_t SMT = SL + 64 * 64 * 4; // fp32 T, 64 x 64, swizzled (tsw)
-    static constexpr uint32_t BAR = SMT + 64 * 64 * 4;
+    static constexpr uint32_t BAR = RLO + 8192;
     static constexpr uint32_t TMEM_SLOT = BAR + 80;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;     // + alignment slack
@@ -98,6 +98,7 @@ template <int DV>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_tp,
                     const float* __restrict__ beta, float scale, const float* __restrict__ S0,
                     __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
                     const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
@@ -130,8 +131,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint8_t* SLO = smem + L::SLO;
     uint8_t* RHI = smem + L::RHI;
     uint8_t* RLO = smem + L::RLO;
-    float* sL = reinterpret_cast<float*>(smem + L::SL);
-    float* sT = reinterpret_cast<float*>(smem + L::SMT);
 
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, TC_TMEM_COLS);
@@ -166,6 +165,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_kt);
             tc::prefetch_tmap(&tm_v);
+            tc::prefetch_tmap(&tm_tp);
             int pend[2] = {-1, -1};
             for (int ch = 0; ch < nchunks; ++ch) {
                 const int s = ch & 1;
@@ -181,6 +181,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tma_load_3d(st + L::KT + 0, &tm_kt, 0, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::KT + 8192, &tm_kt, 64, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::V, &tm_v, c0, h, row, &tma_full[s]);
+                tc::tma_load_3d(st + L::TP, &tm_tp, 32 * vt, h, row, &tma_full[s]);
                 pend[s] = (ch >> 1) & 1;
             }
             // let this CTA's own copies land before the block can leave
@@ -194,12 +195,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);
         bool pend = false;
         uint32_t mphase = 0;
-        float bnext = (t < 64 && nchunks > 0 && t < chunk_len(0)) ? __ldg(beta + (first + t) * H + h) : 0.f;
         for (int ch = 0; ch < nchunks; ++ch) {
             const int s = ch & 1;
-            const float bt = bnext;
-            if (t < 64 && ch + 1 < nchunks)
-                bnext = t < chunk_len(ch + 1) ? __ldg(beta + (first + (int64_t)(ch + 1) * C + t) * H + h) : 0.f;
             if (group_any(2, 128, !mbar_wait_bounded(&tma_full[s], (uint32_t)(ch >> 1) & 1u, limit_ns))) break;
             uint8_t* st = smem + s * L::STAGE;
             if (leader) {
@@ -212,36 +209,29 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::mma_commit(mma_p);
                 pend = true;
             }
+            // row t of T from the packed strictly-lower copy (unit diagonal; identity rows past
+            // the chunk's end), while the Gram runs
+            float x[64];
+            if (t < 64) {
+                const float* tp = reinterpret_cast<const float*>(st + L::TP);
+                const int base = t * (t - 1) / 2;
+                const bool in = t < chunk_len(ch);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) x[j] = (in && j < t) ? tp[base + j] : (j == t ? 1.f : 0.f);
+            }
             if (group_any(2, 128, !mbar_wait_bounded(mma_p, mphase, limit_ns))) break;
             mphase ^= 1u;
             pend = false;
             tc::fence_after_sync();
-            float g[64];
-            tc::tmem_ld64(tmem + lane + TC_COL_G, g);
-            if (leader) mbar_arrive(&stage_empty[s]);  // the Gram was the prep's last use of the stage
-            if (t < 64) {  // row t of L; only j < t is read by the inverse
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    tsw_st4(sL, t, q, make_float4(bt * g[4 * q], bt * g[4 * q + 1], bt * g[4 * q + 2],
-                                                  bt * g[4 * q + 3]));
-            } else {
+            if (leader) mbar_arrive(&stage_empty[s]);  // the prep's last use of the stage
+            if (t >= 64) {  // P row t - 64 = tril(Q K~^T)
+                tc::tmem_ld64(tmem + lane + TC_COL_G, x);
                 const int r = t - 64;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) g[j] = j <= r ? g[j] : 0.f;  // P row, kept in registers
+                for (int j = 0; j < 64; ++j) x[j] = j <= r ? x[j] : 0.f;
             }
-            tc::fence_before_sync();
-            group_bar(2, 128);
-            tril_inverse_64_g128(sL, sT, t, 2);
             if (group_any(2, 128, !mbar_wait_bounded(z_empty, (uint32_t)ch & 1u, limit_ns))) break;
-            if (t < 64) {
-                float x[64];
-                tsw_row<16>(sT, t, 0, x);
-#pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = j <= t ? x[j] : 0.f;  // T is lower triangular
-                st_row_split_bf16(ZHI, ZLO, t, x);  // T rows 0..63
-            } else {
-                st_row_split_bf16(ZHI, ZLO, t, g);  // P rows 64..127
-            }
+            st_row_split_bf16(ZHI, ZLO, t, x);  // rows 0..63: T, rows 64..127: P
             tc::fence_async_smem();
             group_bar(2, 128);
             if (leader) mbar_arrive(z_full);

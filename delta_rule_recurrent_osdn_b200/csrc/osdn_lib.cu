@@ -16,6 +16,7 @@
 #include "chunk_simt.cuh"
 #include "watchdog.cuh"
 #include "chunk_tc.cuh"
+#include "chunk_prep.cuh"
 #include "scan_tc.cuh"
 
 namespace osdn {
@@ -216,6 +217,22 @@ osdn_status_t launch_scan(const void* k, const float* beta, const float* r, floa
     return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
 }
 
+// 3-D fp32 view [rows][H][Dv / 2] of the bf16 output buffer; boxes of 32 values (one 64-channel
+// value tile's 128-byte slice of a row) x 1 head x 64 tokens: the packed WY factors.
+bool make_tp_map(CUtensorMap* m, const void* o, int Dv, int H, int64_t rows) {
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (!enc || rows <= 0) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)Dv / 2, (cuuint64_t)H, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)Dv * 2, (cuuint64_t)H * Dv * 2};
+    cuuint32_t box[3] = {32, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(o), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Phase 2, bf16 with d_k = 128: the WY factors of all chunks (persistent pre-kernel, written
+// into o), then one CTA per (sequence, head, 64 value channels) for the state chain.
 template <int DV>
 osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, const void* v,
                               const float* beta, float scale, const float* S0, void* o,
@@ -223,16 +240,26 @@ osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, cons
     const int64_t ctas = (int64_t)d.N * d.H * (DV / 64);
     if (ctas == 0) return OSDN_OK;
     if (ctas > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
-    CUtensorMap mq, mk, mkt, mv;
-    const int64_t rows = d.rows();
+    CUtensorMap mq, mk, mkt, mv, mtp;
+    const int64_t rows = d.rows();  // > 0 on this path
     if (!make_tile_map(&mq, q, 128, d.H, rows) || !make_tile_map(&mk, k, 128, d.H, rows) ||
-        !make_tile_map(&mkt, kt, 128, d.H, rows) || !make_tile_map(&mv, v, DV, d.H, rows))
+        !make_tile_map(&mkt, kt, 128, d.H, rows) || !make_tile_map(&mv, v, DV, d.H, rows) ||
+        !make_tp_map(&mtp, o, DV, d.H, rows))
         return OSDN_ERR_CUDA;
+    const int64_t items = ((rows + 63) / 64) * d.H;
+    int64_t grid = (int64_t)WY_PREP_CTAS_PER_SM * sm_count();
+    grid = grid < items ? grid : items;
+    auto prep = wy_prep_kernel;
+    if (!set_smem(prep, WyPrepSmem::BYTES)) return OSDN_ERR_CUDA;
+    prep<<<dim3((unsigned)grid), dim3(128), WyPrepSmem::BYTES, stream>>>(
+        mk, mkt, beta, static_cast<float*>(o), DV, cu, d.N, d.T, d.H, rows, (long long)kWaitLimitNs);
+    const osdn_status_t st = launch_status();
+    if (st != OSDN_OK) return st;
     auto kernel = chunk_fwd_tc_kernel<DV>;
     if (!set_smem(kernel, TcSmem::BYTES)) return OSDN_ERR_CUDA;
     kernel<<<dim3((unsigned)ctas), dim3(TC_THREADS), TcSmem::BYTES, stream>>>(
-        mq, mk, mkt, mv, beta, scale, S0, static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T, d.H,
-        (long long)kWaitLimitNs);
+        mq, mk, mkt, mv, mtp, beta, scale, S0, static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T,
+        d.H, (long long)kWaitLimitNs);
     return launch_status();
 }
 
@@ -292,8 +319,12 @@ osdn_status_t validate_chunk(const void* q, const void* k, const void* kt, const
         return OSDN_ERR_UNSUPPORTED;
     const size_t es = io_size(io);
     const size_t kb = (size_t)d.rows() * d.H * d.Dk * es, vb = (size_t)d.rows() * d.H * d.Dv * es;
+    // o is also scratch for per-chunk factors before it receives the outputs: nothing that is
+    // read may lie in it
+    const size_t gb = (size_t)d.rows() * d.H * 4, sb = (size_t)d.N * d.H * d.Dv * d.Dk * 4;
     if (overlaps(o, vb, q, kb) || overlaps(o, vb, k, kb) || overlaps(o, vb, kt, kb) ||
-        overlaps(o, vb, v, vb))
+        overlaps(o, vb, v, vb) || overlaps(o, vb, beta, gb) || overlaps(o, vb, S0, sb) ||
+        overlaps(o, vb, ST, sb))
         return OSDN_ERR_INVALID_ARG;
     return OSDN_OK;
 }
@@ -385,7 +416,9 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
     if (st != OSDN_OK) return st;
     const size_t es = io_size(io);
     const size_t kb = (size_t)d.rows() * d.H * d.Dk * es, vb = (size_t)d.rows() * d.H * d.Dv * es;
-    if (overlaps(kt, kb, q, kb) || overlaps(kt, kb, v, vb)) return OSDN_ERR_INVALID_ARG;
+    const size_t db = (size_t)d.N * d.H * d.Dk * 4;
+    if (overlaps(kt, kb, q, kb) || overlaps(kt, kb, v, vb) || overlaps(o, vb, dT, db))
+        return OSDN_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16) {
         st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, dT, cu_seqlens, d, s);

@@ -27,10 +27,11 @@
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "tril_inverse.cuh"
+#include "chunk_walk.cuh"
 
 namespace osdn {
 
-constexpr int SCAN_C = 64;
+constexpr int SCAN_C = kChunk;
 
 // Gate prefix quantities of one chunk, computed by one warp (lane l: tokens 2l and 2l + 1).
 // r is 1 and beta 0 for tokens past the chunk's end.  Gamma_tj = sg[t] sg1[j] exp(lr[t] - lr1[j]).
@@ -71,73 +72,6 @@ __device__ __forceinline__ GatePrefix gate_prefix(float r0, float r1, int lane) 
 }
 
 // ===================================================================== prep: T_d per chunk
-
-// Walks the chunks of the whole batch for a persistent CTA.  Work item w = (64-row window of
-// the token rows, head); a window holds the start of at most one chunk of each sequence that
-// overlaps it (chunk starts are 64 rows apart), so items are near-uniform in size whatever the
-// sequence lengths.  Items w = blockIdx.x, blockIdx.x + gridDim.x, ...
-struct ChunkWalk {
-    const int32_t* cu;
-    int N, T, H;
-    int64_t rows, W, w;
-    int n;          // next sequence to examine in the current window
-    bool fresh;     // the current window's first sequence is not located yet
-    // output of next(): the chunk
-    int64_t row0;
-    int Lc, h;
-
-    __device__ void init(const int32_t* cu_, int N_, int T_, int H_, int64_t rows_) {
-        cu = cu_;
-        N = N_;
-        T = T_;
-        H = H_;
-        rows = rows_;
-        W = ((rows + SCAN_C - 1) / SCAN_C) * H;
-        w = blockIdx.x;
-        fresh = true;
-    }
-    // Last sequence whose first row is <= row (sequences are contiguous and ordered).
-    __device__ int seq_at(int64_t row) const {
-        if (!cu) {
-            const int64_t q = row / T;
-            return q < N - 1 ? (int)q : N - 1;
-        }
-        int lo = 0, hi = N - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if ((int64_t)__ldg(cu + mid) <= row) lo = mid; else hi = mid - 1;
-        }
-        return lo;
-    }
-    // Advance to the next chunk; false when the CTA's items are exhausted.
-    __device__ bool next() {
-        while (w < W) {
-            const int64_t lo = (w / H) * SCAN_C;
-            const int64_t hi = lo + SCAN_C < rows ? lo + SCAN_C : rows;
-            if (fresh) {
-                n = seq_at(lo);
-                fresh = false;
-            }
-            while (n < N) {
-                int64_t first, count;
-                if (!seq_range(cu, n, N, T, first, count)) return false;
-                if (first >= hi) break;
-                ++n;
-                const int64_t end = first + count;
-                const int64_t s = first >= lo ? first : first + ((lo - first + SCAN_C - 1) / SCAN_C) * SCAN_C;
-                if (s < hi && s < end) {
-                    row0 = s;
-                    Lc = end - s < SCAN_C ? (int)(end - s) : SCAN_C;
-                    h = (int)(w % H);
-                    return true;
-                }
-            }
-            w += gridDim.x;
-            fresh = true;
-        }
-        return false;
-    }
-};
 
 struct ScanPrepSmem {
     static constexpr uint32_t K = 0;              // bf16 k tile: 2 K-blocks x (64 rows x 128 B)

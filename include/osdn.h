@@ -108,7 +108,9 @@ OSDN_API osdn_status_t osdn_precond_scan(const void* k, const float* beta, const
  *   v       [B,T,H,Dv] io dtype, read.   beta [B,T,H] float32, read.
  *   scale   multiplies o only (1.0 for unit-norm q).
  *   S0      [N,H,Dv,Dk] initial state, or NULL for zeros.
- *   o       [B,T,H,Dv] io dtype, written: o_t = scale * S_t q_t (state after token t).
+ *   o       [B,T,H,Dv] io dtype, written: o_t = scale * S_t q_t (state after token t).  Must
+ *           not overlap q, k, k_tilde, v, beta, S0 or ST (OSDN_ERR_INVALID_ARG): for bf16 with
+ *           Dk = 128 the call first uses it as scratch for per-chunk factors.
  *   ST      [N,H,Dv,Dk] final state, written; NULL skips it.
  *   chunk   tokens per chunk (64 for bf16; 16, 32 or 64 for f32).  The result does not
  *           depend on it beyond rounding.
@@ -129,6 +131,7 @@ OSDN_API size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_
  *                written there and the workspace is not used.
  *   workspace    device scratch of at least osdn_fwd_workspace_bytes(...) bytes, 256-byte
  *                aligned, used when k_tilde_out is NULL; NULL only if that size is 0.
+ * The buffer rules of both phases apply; o must not overlap dT either.
  */
 OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
                        const float* r, float eta, const float* d0, const float* S0, float scale,

@@ -69,6 +69,9 @@ def test_workspace_size():
     (dict(v=ctypes.c_void_p(A + 8)), osdn.OSDN_ERR_ALIGNMENT),
     (dict(S0=ctypes.c_void_p(A + 4)), osdn.OSDN_ERR_ALIGNMENT),
     (dict(o=fake(1)), osdn.OSDN_ERR_INVALID_ARG),          # output aliases q
+    (dict(beta=ctypes.c_void_p(A + 6 * 0x1000000 + 256)), osdn.OSDN_ERR_INVALID_ARG),  # in o
+    (dict(S0=ctypes.c_void_p(A + 6 * 0x1000000)), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(ST=ctypes.c_void_p(A + 6 * 0x1000000 + 1024)), osdn.OSDN_ERR_INVALID_ARG),
 ])
 def test_chunk_fwd_rejects(kw, status):
     assert chunk_call(**kw) == status
