@@ -39,9 +39,11 @@ struct WyPrepSmem {
 };
 constexpr int WY_PREP_CTAS_PER_SM = 3;
 
-// Packed index t (t - 1) / 2 + j  ->  row t (the j follows).
+// Packed index t (t - 1) / 2 + j  ->  row t (the j follows): a reciprocal-square-root estimate,
+// then exact integer corrections.
 __device__ __forceinline__ int packed_row(int f) {
-    int t = (int)((1.f + sqrtf(8.f * (float)f + 1.f)) * 0.5f);
+    const float y = 8.f * (float)f + 1.f;
+    int t = (int)((1.f + y * rsqrtf(y)) * 0.5f);
     while (t * (t - 1) / 2 > f) --t;
     while ((t + 1) * t / 2 <= f) ++t;
     return t;
@@ -168,11 +170,12 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tril_inverse_64_g128(sL, sT, tid, 1);
         // ---- packed strictly-lower T, one copy per value tile
         {
-            const int npk = Lc * (Lc - 1) / 2;
+            const int npk = Lc * (Lc - 1) / 2, rstride = H * half_f;
+            float* dst0 = o_f32 + (row0 * H + h) * half_f;
             for (int f = tid; f < npk; f += 128) {
                 const int t = packed_row(f), j = f - t * (t - 1) / 2;
                 const float val = sT[tsw(t, j)];
-                float* dst = o_f32 + ((row0 + (f >> 5)) * H + h) * half_f + (f & 31);
+                float* dst = dst0 + (f >> 5) * rstride + (f & 31);
                 for (int vt = 0; vt < nvt; ++vt) dst[32 * vt] = val;
             }
         }

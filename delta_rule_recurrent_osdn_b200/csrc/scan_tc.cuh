@@ -78,8 +78,8 @@ struct ScanPrepSmem {
     static constexpr uint32_t A = 16384;          // bf16 [a_hi; a_lo] per K-block, 2 x 16 KB
     static constexpr uint32_t SL = A;             // fp32 L_d (tsw), over A once the Gram is done
     static constexpr uint32_t ST = A + 16384;     // fp32 T_d (tsw), over A
-    static constexpr uint32_t VEC = A + 32768;    // c, lr, lr1, sg, sg1 (5 x 64 floats)
-    static constexpr uint32_t BAR = VEC + 5 * 256;
+    static constexpr uint32_t VEC = A + 32768;    // c, lr, lr1, sg, sg1, R, Rinv (7 x 64) + flag
+    static constexpr uint32_t BAR = VEC + 7 * 256 + 16;
     static constexpr uint32_t TMEM_SLOT = BAR + 16;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
@@ -113,6 +113,9 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
     float* vlr1 = vc + 128;
     float* vsg = vc + 192;
     float* vsg1 = vc + 256;
+    float* vR = vc + 320;     // sg e^lr
+    float* vRi = vc + 384;    // sg1 e^-lr1
+    int* vsafe = reinterpret_cast<int*>(vc + 448);
 
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, 128);
@@ -198,6 +201,15 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
             vsg[t0 + 1] = g.sg_1;
             vsg1[t0] = g.sg1_0;
             vsg1[t0 + 1] = g.sg1_1;
+            // Gamma_tj = (sg_t e^lr_t) (sg1_j e^-lr1_j) when every prefix is within +-80 (both
+            // factors then stay inside the fp32 range); otherwise one exponential per entry
+            const float mx = fmaxf(fmaxf(fabsf(g.lr0), fabsf(g.lr_1)), fmaxf(fabsf(g.lr1_0), fabsf(g.lr1_1)));
+            const bool safe = __all_sync(0xffffffffu, mx < 80.f);
+            vR[t0] = g.sg0 * __expf(g.lr0);
+            vR[t0 + 1] = g.sg_1 * __expf(g.lr_1);
+            vRi[t0] = g.sg1_0 * __expf(-g.lr1_0);
+            vRi[t0 + 1] = g.sg1_1 * __expf(-g.lr1_1);
+            if (lane == 0) *vsafe = safe ? 1 : 0;
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
@@ -258,15 +270,25 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
         {
             const int t = tid & 63, g0 = 8 * (tid >> 6);
             const float ct = vc[t], lrt = vlr[t], sgt = vsg[t];
+            const bool safe = *vsafe != 0;  // uniform over the CTA
+            const float cr = ct * vR[t];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const float4 a = tsw_ld4(sL, t, g0 + q), b = tsw_ld4(sT, t, g0 + q);
                 const float gs[4] = {a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w};
                 float o[4];
+                if (safe) {
+                    const float4 ri = *reinterpret_cast<const float4*>(vRi + 4 * (g0 + q));
+                    const float rv[4] = {ri.x, ri.y, ri.z, ri.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 4 * (g0 + q) + e;
-                    o[e] = j < t ? ct * sgt * vsg1[j] * __expf(lrt - vlr1[j]) * gs[e] : 0.f;
+                    for (int e = 0; e < 4; ++e)
+                        o[e] = 4 * (g0 + q) + e < t ? cr * rv[e] * gs[e] : 0.f;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * (g0 + q) + e;
+                        o[e] = j < t ? ct * sgt * vsg1[j] * __expf(lrt - vlr1[j]) * gs[e] : 0.f;
+                    }
                 }
                 tsw_st4(sL, t, g0 + q, make_float4(o[0], o[1], o[2], o[3]));
             }

@@ -150,23 +150,24 @@ __device__ __forceinline__ void tril_inverse_64_g128(const float* __restrict__ s
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) sT[tsw(8 * rq + rr, 32 + c)] = acc[rr];
         group_bar(bar_id, NT);
-        // T_10 = -T_11 X.  Rows 32..47 of T_11 are zero past column 47 (and columns 48..63 of
-        // those rows hold level-B scratch), so warps 0-1 take only the first 16 terms.
-        const int mlen = rq < 2 ? 16 : 32;
+        // T_10 = -T_11 X.  T_11 is lower triangular, so warp rq (rows 8 rq .. 8 rq + 7 of T_11)
+        // needs only its first 8 (rq + 1) terms (which also keeps warps 0-1 away from the
+        // level-B scratch in columns 48..63 of rows 32..47).
+        const int mlen = 8 * (rq + 1);
 #pragma unroll
         for (int m = 0; m < 32; ++m)
             if (m < mlen) col[m] = sT[tsw(m, 32 + c)];  // X[:, c]
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            if (h * 16 < mlen) {
+        for (int q = 0; q < 4; ++q) {  // 8-term slices, taken while below the warp's bound
+            if (8 * q < mlen) {
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
-                    float tr[16];
-                    tsw_row<4>(sT, 32 + 8 * rq + rr, 32 + 16 * h, tr);
+                    float tr[8];
+                    tsw_row<2>(sT, 32 + 8 * rq + rr, 32 + 8 * q, tr);
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) acc[rr] = fmaf(-tr[m], col[16 * h + m], acc[rr]);
+                    for (int m = 0; m < 8; ++m) acc[rr] = fmaf(-tr[m], col[8 * q + m], acc[rr]);
                 }
             }
         }

@@ -54,6 +54,16 @@ def test_packed_with_empty_and_tiny_sequences(ref, io):
         np.testing.assert_array_equal(got[3][n], inp.d0[n])
 
 
+def test_packed_many_short_sequences(ref):
+    """Dozens of sequences shorter than a chunk: one 64-row window of the packed batch holds the
+    starts of many chunks, which the persistent per-chunk kernels must all visit."""
+    rng = np.random.default_rng(11)
+    lengths = [int(x) for x in rng.integers(0, 9, size=40)] + [3, 70, 1]
+    inp = W.make_inputs(dict(lengths=lengths, H=3, Dk=128, Dv=128, io="bf16", apf=True, eta=0.1,
+                             seed=12, init_state=True))
+    check_all(gpu_fwd(inp), oracle_fwd(ref, inp), "bf16")
+
+
 def test_packed_equals_separate_calls(ref):
     """Packing is bookkeeping only: bit-identical to one call per sequence."""
     lengths = [70, 1, 129, 64]
