@@ -57,8 +57,10 @@ def kernel_source_sha(names):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"scan": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh", "scan_tc.cuh"],
-                  "chunk": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh", "chunk_tc.cuh"]}
+KERNEL_SOURCES = {"scan": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
+                           "chunk_walk.cuh", "scan_tc.cuh"],
+                  "chunk": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
+                            "chunk_walk.cuh", "chunk_prep.cuh", "chunk_tc.cuh"]}
 
 
 def profiled_traffic(kernel):
@@ -256,7 +258,7 @@ def bench_ours(args):
     ST = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
     dT = torch.empty((N, H, Dk), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    launches_per_step = 3  # phase-1 prep + chain, phase 2
+    launches_per_step = 4  # per phase: a per-chunk pre-kernel and the sequential chain
 
     def step(ev=None):
         if ev:
