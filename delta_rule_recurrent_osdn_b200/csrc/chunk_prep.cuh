@@ -29,15 +29,14 @@ namespace osdn {
 struct WyPrepSmem {
     static constexpr uint32_t K = 0;            // bf16 K tile: 2 K-blocks x (64 rows x 128 B)
     static constexpr uint32_t KT = 16384;       // bf16 K~ tile, same layout
-    static constexpr uint32_t SL = 32768;       // fp32 L (tsw)
-    static constexpr uint32_t ST = 49152;       // fp32 T (tsw)
-    static constexpr uint32_t BETA = 65536;     // 64 floats
+    static constexpr uint32_t SL = 32768;       // fp32 L, then T in place (tsw)
+    static constexpr uint32_t BETA = 49152;     // 64 floats
     static constexpr uint32_t BAR = BETA + 256;
     static constexpr uint32_t TMEM_SLOT = BAR + 16;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
-constexpr int WY_PREP_CTAS_PER_SM = 3;
+constexpr int WY_PREP_CTAS_PER_SM = 4;
 
 // Packed index t (t - 1) / 2 + j  ->  row t (the j follows): a reciprocal-square-root estimate,
 // then exact integer corrections.
@@ -70,7 +69,6 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     uint8_t* sK = smem + L::K;
     uint8_t* sKT = smem + L::KT;
     float* sL = reinterpret_cast<float*>(smem + L::SL);
-    float* sT = reinterpret_cast<float*>(smem + L::ST);
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
 
     if (warp == 0) {
@@ -167,19 +165,19 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         }
         tc::fence_before_sync();
         __syncthreads();
-        tril_inverse_64_g128(sL, sT, tid, 1);
+        tril_inverse_64_g128(sL, tid, 1);  // T over L
         // ---- packed strictly-lower T, one copy per value tile
         {
             const int npk = Lc * (Lc - 1) / 2, rstride = H * half_f;
             float* dst0 = o_f32 + (row0 * H + h) * half_f;
             for (int f = tid; f < npk; f += 128) {
                 const int t = packed_row(f), j = f - t * (t - 1) / 2;
-                const float val = sT[tsw(t, j)];
+                const float val = sL[tsw(t, j)];
                 float* dst = dst0 + (f >> 5) * rstride + (f & 31);
                 for (int vt = 0; vt < nvt; ++vt) dst[32 * vt] = val;
             }
         }
-        __syncthreads();  // sL / sT are rewritten by the next chunk
+        __syncthreads();  // sL is rewritten by the next chunk
     }
     if (fail && tid == 0) {
         if (tma_pend) mbar_wait_bounded(tma_bar, tph, limit_ns);

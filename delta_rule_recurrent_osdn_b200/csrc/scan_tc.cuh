@@ -76,15 +76,15 @@ __device__ __forceinline__ GatePrefix gate_prefix(float r0, float r1, int lane) 
 struct ScanPrepSmem {
     static constexpr uint32_t K = 0;              // bf16 k tile: 2 K-blocks x (64 rows x 128 B)
     static constexpr uint32_t A = 16384;          // bf16 [a_hi; a_lo] per K-block, 2 x 16 KB
-    static constexpr uint32_t SL = A;             // fp32 L_d (tsw), over A once the Gram is done
-    static constexpr uint32_t ST = A + 16384;     // fp32 T_d (tsw), over A
+    static constexpr uint32_t SL = A;             // fp32 L_d, then T_d (tsw), over A after the Gram
+    static constexpr uint32_t ST = A + 16384;     // fp32 scratch (tsw), over A
     static constexpr uint32_t VEC = A + 32768;    // c, lr, lr1, sg, sg1, R, Rinv (7 x 64) + flag
     static constexpr uint32_t BAR = VEC + 7 * 256 + 16;
     static constexpr uint32_t TMEM_SLOT = BAR + 16;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
-constexpr int SCAN_PREP_CTAS_PER_SM = 3;
+constexpr int SCAN_PREP_CTAS_PER_SM = 4;
 
 // Persistent grid (one to three CTAs per SM) of 128 threads walking the batch's chunks with
 // ChunkWalk.  td_out is the k~ buffer seen as fp32 rows of 64 values.
@@ -294,12 +294,12 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
             }
         }
         __syncthreads();
-        tril_inverse_64_g128(sL, sT, tid, 1);
+        tril_inverse_64_g128(sL, tid, 1);  // T_d over L_d
         // ---- rows t < Lc of T_d (tsw order kept) to the chunk's rows of the k~ buffer
         {
             const int t = tid >> 1, half = tid & 1;
             if (t < Lc) {
-                const float4* src = reinterpret_cast<const float4*>(sT + t * 64) + 8 * half;
+                const float4* src = reinterpret_cast<const float4*>(sL + t * 64) + 8 * half;
                 float4* dst = reinterpret_cast<float4*>(td_out + ((row0 + t) * H + h) * 64) + 8 * half;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) dst[q] = src[q];

@@ -62,36 +62,44 @@ __device__ __forceinline__ void tsw_row(const float* m, int r, int c0, float* x)
     }
 }
 
-// sL: L in the swizzled layout; only its strictly lower triangle is read.  sT (swizzled)
-// receives T on and below the diagonal; the entries above the diagonal are left holding
-// scratch values, so a reader masks them (T is lower triangular with a unit diagonal).
+// In place.  On entry M holds L in the swizzled layout (only its strictly lower triangle is
+// read); on return it holds T on and below the diagonal, and the entries above the diagonal hold
+// scratch values, so a reader masks them (T is lower triangular with a unit diagonal).  Every
+// block of L is read before the block of T that replaces it is written: the diagonal blocks
+// through registers and a barrier, the off-diagonal blocks one level later.
 // Called by all 128 threads t = 0..127 of a group synchronizing on named barrier `bar_id`;
 // returns synchronized.
-__device__ __forceinline__ void tril_inverse_64_g128(const float* __restrict__ sL,
-                                                     float* __restrict__ sT, int t, int bar_id) {
+__device__ __forceinline__ void tril_inverse_64_g128(float* __restrict__ M, int t, int bar_id) {
     constexpr int NT = 128;
+    const float* sL = M;
+    float* sT = M;
     // ---- A. diagonal blocks: column `col` of block b, x[r] = [r == col] - sum_{m<r} L_rm x[m]
-    if (t < 64) {
-        const int o = 16 * (t >> 4), col = t & 15;
+    {
+        const int o = 16 * ((t & 63) >> 4), col = t & 15;
         float x[16];
+        if (t < 64) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float lr[16];
+            for (int r = 0; r < 16; ++r) {
+                float lr[16];
 #pragma unroll
-            for (int g = 0; 4 * g < r; ++g) {
-                const float4 v = tsw_ld4(sL, o + r, (o >> 2) + g);
-                lr[4 * g] = v.x;
-                lr[4 * g + 1] = v.y;
-                lr[4 * g + 2] = v.z;
-                lr[4 * g + 3] = v.w;
+                for (int g = 0; 4 * g < r; ++g) {
+                    const float4 v = tsw_ld4(sL, o + r, (o >> 2) + g);
+                    lr[4 * g] = v.x;
+                    lr[4 * g + 1] = v.y;
+                    lr[4 * g + 2] = v.z;
+                    lr[4 * g + 3] = v.w;
+                }
+                float acc = 0.f;  // x[m] == 0 for m < col, so no per-lane bound is needed
+#pragma unroll
+                for (int m = 0; m < r; ++m) acc = fmaf(-lr[m], x[m], acc);
+                x[r] = r == col ? 1.f : (r < col ? 0.f : acc);
             }
-            float acc = 0.f;  // x[m] == 0 for m < col, so no per-lane bound is needed
-#pragma unroll
-            for (int m = 0; m < r; ++m) acc = fmaf(-lr[m], x[m], acc);
-            x[r] = r == col ? 1.f : (r < col ? 0.f : acc);
         }
+        group_bar(bar_id, NT);  // the diagonal blocks of L are read
+        if (t < 64) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[tsw(o + r, o + col)] = x[r];
+            for (int r = 0; r < 16; ++r) sT[tsw(o + r, o + col)] = x[r];
+        }
     }
     group_bar(bar_id, NT);
     // ---- B. 16x16 level; thread: block pair (t >> 6), column c, rows 4*rq .. 4*rq + 3
