@@ -26,7 +26,10 @@
 //            pre-kernel left in this CTA's slice of the chunk's o rows, P from a Gram MMA),
 //            overlapping chunk c's chain;
 //   producer warp 8: TMA loads of the chunk tiles into a 2-stage ring (no multicast).
-// Handshakes are mbarriers: z_full / z_empty for the [T; P] tiles, stage_empty for the ring.
+// Handshakes are mbarriers: zt_* / zp_* for the T and P halves of the [T; P] tiles (W = T R
+// uses only the T rows, the outputs only the P rows, so each half is refilled as soon as its
+// last reader is done; the other half's rows only reach accumulator lanes nobody reads),
+// stage_empty for the ring.
 // Every wait is bounded and followed by a group-wide vote, so a role that gives up (recording
 // OSDN_ERR_DEVICE_TIMEOUT) leaves its loop as a whole group and no named barrier is left waiting.
 #pragma once
@@ -49,14 +52,16 @@ struct TcSmem {
     static constexpr uint32_t RHI = SLO + 16384;      // bf16 R then W, hi / lo, 64 x 128 B
     static constexpr uint32_t RLO = RHI + 8192;
     static constexpr uint32_t BAR = RLO + 8192;
-    static constexpr uint32_t TMEM_SLOT = BAR + 80;
+    static constexpr uint32_t TMEM_SLOT = BAR + 128;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;     // + alignment slack
 };
 static_assert(TcSmem::BYTES <= 232448, "shared memory");
 
-constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 128, TC_COL_G = 192;
-constexpr uint32_t TC_TMEM_COLS = 256;
+// Tensor-memory columns: S, D1 (double-buffered: a chunk's outputs are read during the next
+// chunk), D2, the prep's Gram.
+constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 192, TC_COL_G = 256;
+constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr int TC_THREADS = 288;
 
 // Split a 64-value fp32 row into bf16 hi + lo and write both rows (128 B each, swizzled).
@@ -120,10 +125,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* tma_full = bars + 0;     // [2]
     uint64_t* stage_empty = bars + 2;  // [2], two arrivals: chain and prep
-    uint64_t* z_full = bars + 4;
-    uint64_t* z_empty = bars + 5;
-    uint64_t* mma_c = bars + 6;
-    uint64_t* mma_p = bars + 7;
+    uint64_t* zt_full = bars + 4;      // T rows of [T; P] written
+    uint64_t* zt_empty = bars + 5;     // T rows free (W computed)
+    uint64_t* zp_full = bars + 9;      // P rows written
+    uint64_t* zp_empty = bars + 10;    // P rows free (outputs computed)
+    uint64_t* w_ready = bars + 11;     // W of the chunk written (the output MMAs may start)
+    uint64_t* mma_c = bars + 6;        // chain MMAs on the state's path
+    uint64_t* mma_p = bars + 7;        // prep MMAs
+    uint64_t* mma_o = bars + 8;        // chain MMAs of the outputs
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
     uint8_t* ZHI = smem + L::ZHI;
     uint8_t* ZLO = smem + L::ZLO;
@@ -141,16 +150,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(&tma_full[1], 1);
         mbar_init(&stage_empty[0], 2);
         mbar_init(&stage_empty[1], 2);
-        mbar_init(z_full, 1);
-        mbar_init(z_empty, 1);
+        mbar_init(zt_full, 1);
+        mbar_init(zt_empty, 1);
+        mbar_init(zp_full, 1);
+        mbar_init(zp_empty, 1);
+        mbar_init(w_ready, 1);
         mbar_init(mma_c, 1);
         mbar_init(mma_p, 1);
+        mbar_init(mma_o, 1);
         tc::fence_mbar_init();
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (tid == 0) mbar_arrive(z_empty);  // the [T; P] tiles start out free
+    if (tid == 0) {  // the [T; P] tiles start out free
+        mbar_arrive(zt_empty);
+        mbar_arrive(zp_empty);
+    }
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     auto chunk_len = [&](int ch) -> int {
@@ -160,17 +176,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (warp == 8) {
         // =========================================================== producer
+        // Lane 0 loads the chunk tiles into the 2-stage ring and issues each chunk's output
+        // MMAs (D1 += [T; P] W) once the chain has published W, so that the chain warps go
+        // straight on to the state split.
         if ((tid & 31) == 0) {
             tc::prefetch_tmap(&tm_q);
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_kt);
             tc::prefetch_tmap(&tm_v);
             tc::prefetch_tmap(&tm_tp);
+            constexpr uint32_t ID_O = tc::idesc(1, 0, 1, 128, 64);
+            const uint32_t aZ[2] = {smem_u32(ZHI), smem_u32(ZLO)};
+            const uint32_t aR[2] = {smem_u32(RHI), smem_u32(RLO)};
             int pend[2] = {-1, -1};
-            for (int ch = 0; ch < nchunks; ++ch) {
+            int o_issued = 0;
+            auto load = [&](int ch) {
                 const int s = ch & 1;
-                if (ch >= 2 && !mbar_wait_bounded(&stage_empty[s], (uint32_t)((ch - 2) >> 1) & 1u, limit_ns))
-                    break;
                 uint8_t* st = smem + s * L::STAGE;
                 const int row = (int)(first + (int64_t)ch * C);
                 tc::mbar_expect_tx(&tma_full[s], L::STAGE);
@@ -183,10 +204,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tma_load_3d(st + L::V, &tm_v, c0, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::TP, &tm_tp, 32 * vt, h, row, &tma_full[s]);
                 pend[s] = (ch >> 1) & 1;
+            };
+            for (int ch = 0; ch < nchunks && ch < 2; ++ch) load(ch);
+            for (int ch = 0; ch < nchunks; ++ch) {
+                if (!mbar_wait_bounded(w_ready, (uint32_t)ch & 1u, limit_ns)) break;
+                tc::fence_after_sync();
+                mma_split3(tmem + TC_COL_D1 + 64 * (ch & 1), aZ, aR, ID_O, true);
+                tc::mma_commit(mma_o);
+                ++o_issued;
+                if (ch + 2 < nchunks) {  // chunk ch's stage, once both roles released it
+                    if (!mbar_wait_bounded(&stage_empty[ch & 1], (uint32_t)(ch >> 1) & 1u, limit_ns)) break;
+                    load(ch + 2);
+                }
             }
-            // let this CTA's own copies land before the block can leave
+            // let this CTA's own copies and MMAs land before the block can leave
             for (int s = 0; s < 2; ++s)
                 if (pend[s] >= 0) mbar_wait_bounded(&tma_full[s], (uint32_t)pend[s], limit_ns);
+            if (o_issued > 0) mbar_wait_bounded(mma_o, (uint32_t)(o_issued - 1) & 1u, limit_ns);
         }
     } else if (warp >= 4) {
         // =========================================================== prep
@@ -230,26 +264,36 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int j = 0; j < 64; ++j) x[j] = j <= r ? x[j] : 0.f;
             }
-            if (group_any(2, 128, !mbar_wait_bounded(z_empty, (uint32_t)ch & 1u, limit_ns))) break;
-            st_row_split_bf16(ZHI, ZLO, t, x);  // rows 0..63: T, rows 64..127: P
-            tc::fence_async_smem();
-            group_bar(2, 128);
-            if (leader) mbar_arrive(z_full);
+            // rows 0..63 (T) by warps 4-5 and rows 64..127 (P) by warps 6-7, each half as soon
+            // as the chain is done with its previous contents
+            const int half = t >> 6, hbar = 3 + half;
+            bool bad = group_any(hbar, 64, !mbar_wait_bounded(half ? zp_empty : zt_empty,
+                                                              (uint32_t)ch & 1u, limit_ns));
+            if (!bad) {
+                st_row_split_bf16(ZHI, ZLO, t, x);
+                tc::fence_async_smem();
+            }
+            group_bar(hbar, 64);
+            if (!bad && (t & 63) == 0) mbar_arrive(half ? zp_full : zt_full);
+            if (group_any(2, 128, bad)) break;
         }
         if (leader && pend) mbar_wait_bounded(mma_p, mphase, limit_ns);
     } else {
         // =========================================================== chain
+        // Per chunk c: D1[c&1] = [K;Q] S^T -> R -> W -> S^T += K~^T W (the state's path), and
+        // D1[c&1] += [T;P] W for the outputs, committed apart so the state split does not wait for
+        // them; chunk c's output rows are read and stored by warps 2-3 during chunk c+1's R step,
+        // when only warps 0-1 have work.
         const int t = tid;  // 0..127 = tensor-memory lane
         const bool leader = t == 0;
-        const uint32_t t_S = tmem + lane + TC_COL_S, t_D1 = tmem + lane + TC_COL_D1;
-        const uint32_t t_D2 = tmem + lane + TC_COL_D2;
+        const uint32_t t_S = tmem + lane + TC_COL_S, t_D2 = tmem + lane + TC_COL_D2;
         constexpr uint32_t ID_1 = tc::idesc(1, 0, 1, 128, 64);  // [K;Q] x S^T and [T;P] x (R | W)
         constexpr uint32_t ID_3 = tc::idesc(1, 1, 1, 128, 64);  // K~^T x W
         const uint32_t aZ[2] = {smem_u32(ZHI), smem_u32(ZLO)};
         const uint32_t aR[2] = {smem_u32(RHI), smem_u32(RLO)};
         const uint32_t aS[2] = {smem_u32(SHI), smem_u32(SLO)};
         bool pend = false;
-        uint32_t mphase = 0;
+        uint32_t mphase = 0, ophase = 0;
         bool ok = true;
         auto mma_wait = [&]() -> bool {
             if (group_any(1, 128, !mbar_wait_bounded(mma_c, mphase, limit_ns))) return false;
@@ -258,15 +302,35 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::fence_after_sync();
             return true;
         };
+        // o rows of chunk pc from D1[pc & 1] (warps 2-3: lanes 64..127 = the chunk's tokens)
+        auto store_o = [&](int pc) {
+            const int r = t - 64;
+            float x[64];
+            tc::tmem_ld64(tmem + lane + TC_COL_D1 + 64 * (pc & 1), x);
+            if (r < chunk_len(pc)) {
+                __nv_bfloat16* orow = o + ((first + (int64_t)pc * C + r) * H + h) * DV + c0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale * x[8 * j + 2 * e],
+                                                                        scale * x[8 * j + 2 * e + 1]);
+                        pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+                    *reinterpret_cast<uint4*>(orow + 8 * j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        };
         // initial state: S^T lane i = key channel i, columns = this CTA's value channels
         {
-            float s[64];
+            float s0[64];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] = S0 ? __ldg(S0 + sbase + (int64_t)c * DK + t) : 0.f;
+            for (int c = 0; c < 64; ++c) s0[c] = S0 ? __ldg(S0 + sbase + (int64_t)c * DK + t) : 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) tc::tmem_st16(t_S + 16 * q, s + 16 * q);
+            for (int q = 0; q < 4; ++q) tc::tmem_st16(t_S + 16 * q, s0 + 16 * q);
             tc::tmem_st_wait();
-            st_row_split_bf16(SHI, SLO, t, s);
+            st_row_split_bf16(SHI, SLO, t, s0);
             tc::fence_async_smem();
             tc::fence_before_sync();
             group_bar(1, 128);
@@ -274,16 +338,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         float bnext = (t < 64 && nchunks > 0 && t < chunk_len(0)) ? __ldg(beta + (first + t) * H + h) : 0.f;
         for (int ch = 0; ch < nchunks && ok; ++ch) {
             const int s = ch & 1;
-            const int Lc = chunk_len(ch);
             const int64_t cs = (int64_t)ch * C;
+            const uint32_t t_D1 = tmem + lane + TC_COL_D1 + 64 * s;
             const float bt = bnext;
             if (t < 64 && ch + 1 < nchunks)
                 bnext = t < chunk_len(ch + 1) ? __ldg(beta + (first + cs + C + t) * H + h) : 0.f;
             uint8_t* st = smem + s * L::STAGE;
             const uint32_t aKQ = smem_u32(st + L::KQ), aKT = smem_u32(st + L::KT);
-            const bool got = mbar_wait_bounded(&tma_full[s], (uint32_t)(ch >> 1) & 1u, limit_ns) &&
-                             mbar_wait_bounded(z_full, (uint32_t)ch & 1u, limit_ns);
-            if (group_any(1, 128, !got)) {
+            if (group_any(1, 128, !mbar_wait_bounded(&tma_full[s], (uint32_t)(ch >> 1) & 1u, limit_ns))) {
                 ok = false;
                 break;
             }
@@ -294,7 +356,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int p = 0; p < 2; ++p)
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        tc::mma_bf16(tmem + TC_COL_D1, tc::sw128_desc(aKQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                        tc::mma_bf16(tmem + TC_COL_D1 + 64 * s,
+                                     tc::sw128_desc(aKQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
                                      tc::sw128_desc(aS[p] + k * 2048, 8192, 1024), ID_1, (p | k) != 0);
                 tc::mma_commit(mma_c);
                 pend = true;
@@ -319,7 +382,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            group_bar(1, 128);
+            if (group_any(1, 128, !mbar_wait_bounded(zt_full, (uint32_t)ch & 1u, limit_ns))) {
+                ok = false;
+                break;
+            }
             // ---- D2 = [T; P] R  (rows 0..63: W)
             if (leader) {
                 tc::fence_after_sync();
@@ -328,15 +394,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 pend = true;
             }
             if (!mma_wait()) { ok = false; break; }
+            if (leader) mbar_arrive(zt_empty);  // the T rows have been used
             if (t < 64) {
                 float w[64];
                 tc::tmem_ld64(t_D2, w);
                 st_row_split_bf16(RHI, RLO, t, w);  // R is consumed: W takes its tiles
+            } else if (ch > 0) {
+                store_o(ch - 1);  // its output MMAs completed before this chunk's R
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            group_bar(1, 128);
-            // ---- S^T += K~^T W (two terms of W);  D1 += [T; P] W (three terms; rows 64..127: O)
+            if (group_any(1, 128, !mbar_wait_bounded(zp_full, (uint32_t)ch & 1u, limit_ns))) {
+                ok = false;
+                break;
+            }
+            if (leader) mbar_arrive(w_ready);  // the producer warp issues the output MMAs
+            // ---- S^T += K~^T W (two terms of W); the outputs' D1 += [T; P] W is issued by the
+            //      producer warp and completes on the output barrier
             if (leader) {
                 tc::fence_after_sync();
 #pragma unroll
@@ -345,48 +419,37 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int k = 0; k < 4; ++k)
                         tc::mma_bf16(tmem + TC_COL_S, tc::sw128_desc(aKT + k * 2048, 8192, 1024),
                                      tc::sw128_desc(aR[p] + k * 2048, 8192, 1024), ID_3, 1);
-                mma_split3(tmem + TC_COL_D1, aZ, aR, ID_1, true);
                 tc::mma_commit(mma_c);
                 pend = true;
             }
             if (!mma_wait()) { ok = false; break; }
-            if (leader) {
-                mbar_arrive(z_empty);          // [T; P] no longer read
-                mbar_arrive(&stage_empty[s]);  // nor this chunk's tiles
-            }
-            if (t >= 64) {  // o rows of this chunk
-                float x[64];
-                tc::tmem_ld64(t_D1, x);
-                const int r = t - 64;
-                if (r < Lc) {
-                    __nv_bfloat16* orow = o + ((first + cs + r) * H + h) * DV + c0;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale * x[8 * j + 2 * e],
-                                                                            scale * x[8 * j + 2 * e + 1]);
-                            pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        *reinterpret_cast<uint4*>(orow + 8 * j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
-                }
-            }
             {
                 float x[64];
                 tc::tmem_ld64(t_S, x);
                 st_row_split_bf16(SHI, SLO, t, x);
             }
+            // the output MMAs read the P rows, this chunk's tiles and W: wait for them before
+            // releasing those, and before the next chunk's R overwrites W
+            if (group_any(1, 128, !mbar_wait_bounded(mma_o, ophase, limit_ns))) {
+                ok = false;
+                break;
+            }
+            ophase ^= 1u;
+            tc::fence_after_sync();
+            if (leader) {
+                mbar_arrive(zp_empty);         // the P rows have been used
+                mbar_arrive(&stage_empty[s]);  // and this chunk's tiles
+            }
             tc::fence_async_smem();
             tc::fence_before_sync();
             group_bar(1, 128);
         }
+        if (ok && nchunks > 0 && t >= 64) store_o(nchunks - 1);
         if (ok && ST) {
-            float s[64];
-            tc::tmem_ld64(t_S, s);
+            float s1[64];
+            tc::tmem_ld64(t_S, s1);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) ST[sbase + (int64_t)c * DK + t] = s[c];
+            for (int c = 0; c < 64; ++c) ST[sbase + (int64_t)c * DK + t] = s1[c];
         }
         if (leader && pend) mbar_wait_bounded(mma_c, mphase, limit_ns);
     }
