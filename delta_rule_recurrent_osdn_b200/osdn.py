@@ -62,6 +62,9 @@ def _load() -> ctypes.CDLL:
                              _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
                              ctypes.c_size_t, _vp]
     lib.osdn_fwd.restype = ctypes.c_int
+    lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp, _vp, _i32, _i32,
+                              _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_step.restype = ctypes.c_int
     lib.osdn_get_device_status.argtypes = [_vp]
     lib.osdn_get_device_status.restype = ctypes.c_int
     lib.osdn_debug_watchdog_selftest.argtypes = [ctypes.c_int64, _vp]
@@ -222,6 +225,31 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
                         _p(workspace) if k_tilde is None else None, ws_bytes, _stream(stream)),
            "osdn_fwd")
     return o, ST, dT
+
+
+def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0, o=None,
+              k_tilde=None, stream=None):
+    """One recurrent step per (sequence, head) (the decode path).  q, k: [N, H, Dk]; v: [N, H, Dv];
+    beta, r: [N, H] float32; S: [N, H, Dv, Dk] and d: [N, H, Dk] float32, updated in place.
+    Returns o [N, H, Dv] (and writes k_tilde [N, H, Dk] when given)."""
+    N, H, Dk = q.shape
+    Dv = v.shape[-1]
+    io = _io(q)
+    _req(q, "q")
+    _req(k, "k", q.dtype, (N, H, Dk))
+    _req(v, "v", q.dtype, (N, H, Dv))
+    _req(beta, "beta", torch.float32, (N, H))
+    _req(r, "r", torch.float32, (N, H))
+    _req(S, "S", torch.float32, (N, H, Dv, Dk))
+    _req(d, "d", torch.float32, (N, H, Dk))
+    if o is None:
+        o = torch.empty_like(v)
+    _req(o, "o", q.dtype, (N, H, Dv))
+    _req(k_tilde, "k_tilde", q.dtype, (N, H, Dk))
+    _check(LIB.osdn_step(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), float(scale), _p(S),
+                         _p(d), _p(o), _p(k_tilde), N, H, Dk, Dv, io, _stream(stream)),
+           "osdn_step")
+    return o
 
 
 def osdn_get_device_status(stream=None) -> int:

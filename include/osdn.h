@@ -175,6 +175,26 @@ OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void
  * kernel recorded since the last call; the word is shared by all streams of the device).
  * Returns OSDN_ERR_CUDA if the synchronization itself fails.
  */
+/*
+ * One recurrent step per (sequence, head) -- the decode path (sections 2.1-2.3 applied to a
+ * single token, the state carried in memory).  For each of the N*H (sequence, head) pairs, with
+ * a = k (.) k, nk = ||k||^2 and s = <d, a>:
+ *   k~ = d (.) k;  u = v - S k;  S <- S + beta u k~^T;  o = scale * S q;
+ *   d <- r d + eta * beta * (1 - beta s) * a / nk   (0 when nk = 0).
+ *   q, k     [N,H,Dk] io dtype, read.        v [N,H,Dv] io dtype, read.
+ *   beta     [N,H] float32, read.            r [N,H] float32, or NULL for r == 1.
+ *   S        [N,H,Dv,Dk] float32, read and written in place (row = value channel).
+ *   d        [N,H,Dk] float32, read and written in place.
+ *   o        [N,H,Dv] io dtype, written.     k_tilde [N,H,Dk] io dtype, written, or NULL.
+ * Dk, Dv in {64, 128}.  Pointers 16-byte aligned.  S, d, o and k_tilde must not overlap one
+ * another or the inputs (OSDN_ERR_INVALID_ARG).  N == 0 is a no-op.  A sequence of steps
+ * equals osdn_fwd over the same tokens (up to fp32 summation order).
+ */
+OSDN_API osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
+                        const float* r, float eta, float scale, float* S, float* d, void* o,
+                        void* k_tilde, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
+                        osdn_dtype_t io, void* stream);
+
 OSDN_API osdn_status_t osdn_get_device_status(void* stream);
 
 /*

@@ -120,3 +120,31 @@ def test_parity_metric_allows_exactly_the_output_rounding():
     y = xb.copy()
     y[7] += 0.05
     assert 0.04 / 3 < rel_err(y, x, "bf16") < 0.06 / 2.9
+
+
+def step_call(**kw):
+    args = dict(q=fake(1), k=fake(2), v=fake(3), beta=fake(4), r=None, eta=0.1, scale=1.0,
+                S=fake(5), d=fake(6), o=fake(7), kt=None, N=4, H=2, Dk=128, Dv=128,
+                io=osdn.OSDN_BF16)
+    args.update(kw)
+    return L.osdn_step(args["q"], args["k"], args["v"], args["beta"], args["r"], args["eta"],
+                       args["scale"], args["S"], args["d"], args["o"], args["kt"], args["N"],
+                       args["H"], args["Dk"], args["Dv"], args["io"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Dk=96), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(Dv=32), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(io=5), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(H=0), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(N=-1), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(S=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(o=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(S=ctypes.c_void_p(A + 5 * 0x1000000 + 8)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(o=fake(1)), osdn.OSDN_ERR_INVALID_ARG),                                 # o aliases q
+    (dict(d=ctypes.c_void_p(A + 5 * 0x1000000 + 4096)), osdn.OSDN_ERR_INVALID_ARG),  # d in S
+    (dict(kt=fake(2)), osdn.OSDN_ERR_INVALID_ARG),                                # k~ aliases k
+    (dict(N=0), osdn.OSDN_OK),                                                    # nothing to do
+])
+def test_step_rejects(kw, status):
+    assert step_call(**kw) == status
