@@ -60,13 +60,14 @@ def kernel_source_sha(names):
 KERNEL_SOURCES = {"scan": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
                            "chunk_walk.cuh", "scan_tc.cuh"],
                   "chunk": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
-                            "chunk_walk.cuh", "chunk_prep.cuh", "chunk_tc.cuh"]}
+                            "chunk_walk.cuh", "chunk_prep.cuh", "chunk_tc.cuh"],
+                  "step": ["common.cuh", "step.cuh"]}
 
 
-def profiled_traffic(kernel):
+def profiled_traffic(kernel, workload=WORKLOAD):
     """DRAM bytes per launch from the committed ncu summary of this kernel, if it was taken on
     the current source (its recorded source hash matches); else None."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{WORKLOAD}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -359,6 +360,140 @@ def bench_ours(args):
     return 0
 
 
+DECODE_METRIC = ("OSDN decode tokens/s (one recurrent step per sequence, 256 sequences x 16 heads, "
+                 "d_k=d_v=128); % of HBM roofline")
+DECODE = dict(B=256, T=8, H=16, Dk=128, Dv=128, io="bf16", apf=True, eta=0.05, chunk=64, seed=7,
+              init_state=True)
+
+
+def decode_bytes_per_step(N, H, Dk, Dv, es=2):
+    """HBM bytes of one decode step: the fp32 state read and written, d read and written,
+    q, k, v in and o out in the io dtype, beta and r."""
+    return N * H * (2 * Dv * Dk * 4 + 2 * Dk * 4 + (2 * Dk + 2 * Dv) * es + 8)
+
+
+def bench_decode(args):
+    """The decode path: ``osdn_step`` over a batch of sequences, one token each per step, the
+    state carried in HBM (updated in place).  Tokens cycle through 8 seeded draws."""
+    import torch
+    from delta_rule_recurrent_osdn_b200 import inputs as W
+    from delta_rule_recurrent_osdn_b200 import osdn
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = dict(DECODE)
+    if rank:
+        cfg["seed"] = 1000 + rank
+    inp = W.make_inputs(cfg)
+    d = W.to_torch(inp, dev)
+    N, H, Dk, Dv, T = inp.N, inp.H, inp.Dk, inp.Dv, inp.T
+    tok = [{k_: d[k_][:, t].contiguous() for k_ in ("q", "k", "v", "beta", "r")} for t in range(T)]
+    S = d["S0"].clone()
+    dd = d["d0"].clone()
+    o = torch.empty_like(tok[0]["v"])
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        x = tok[i % T]
+        osdn.osdn_step(x["q"], x["k"], x["v"], x["beta"], S, dd, x["r"], inp.eta, inp.scale, o=o)
+
+    for i in range(args.warmup):
+        flush.fill_(1)
+        step(i)
+    torch.cuda.synchronize(dev)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            events[i][0].record(stream)
+            step(i)
+            events[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    if osdn.osdn_get_device_status() != osdn.OSDN_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    step_ms = [e[0].elapsed_time(e[1]) for e in events]
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    value = world * N * args.steps / (total_ms / 1e3)
+
+    # ---- end to end: the step's token data from pinned host memory, o back, copies timed
+    host = [{k_: t.cpu().pin_memory() for k_, t in x.items()} for x in tok]
+    dev_in = {k_: torch.empty_like(t) for k_, t in tok[0].items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step(i):
+        for k_, t in host[i % T].items():
+            dev_in[k_].copy_(t, non_blocking=True)
+        osdn.osdn_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], S, dd, dev_in["r"],
+                       inp.eta, inp.scale, o=o)
+        o_host.copy_(o, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        flush.fill_(3)
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = world * N * args.steps / (e2e_ms / 1e3)
+
+    if rank == 0:
+        hbm, tc, kind = read_peaks()
+        avg = statistics.mean(step_ms)
+        byts = decode_bytes_per_step(N, H, Dk, Dv)
+        achieved = byts / (avg / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": "step", "achieved": achieved, "peak": hbm,
+                "peak_kind": f"{kind} hbm_gbs", "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": profiled_traffic("step", "decode"),
+                "algorithmic_bytes_per_launch": byts, "kernel_ms": {"step": avg}}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            from oracle import osdn_ref as R
+            t0 = time.perf_counter()
+            reps = 0
+            while True:
+                R.fwd(inp.q[:, :1], inp.k[:, :1], inp.v[:, :1], inp.beta[:, :1], inp.r[:, :1],
+                      inp.eta, inp.d0, inp.S0, inp.scale)
+                reps += 1
+                if time.perf_counter() - t0 > min(args.cpu_seconds, 5.0):
+                    break
+            dt = (time.perf_counter() - t0) / reps
+            cpu = {"value": N / dt, "unit": "tokens/s", "cores": R.set_threads(0),
+                   "kind": "oracle",
+                   "sample": f"one step of all {N} sequences x {H} heads (fp64), {reps} run(s)"}
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"OSDN decode step, {N} sequences x {H} heads, d_k=d_v={Dk}, "
+                                   "bf16 I/O, fp32 state, APF",
+                       "N": N, "H": H, "d_k": Dk, "d_v": Dv, "io": "bf16", "apf": True,
+                       "eta": inp.eta, "l2": "flushed between timed steps (256 MiB write)"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps, "clocks": clk.summary(),
+            "gpu": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -367,11 +502,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["forward", "decode"], default="forward",
+                    help="forward: the 1.3B-layer forward pass (default); decode: osdn_step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return bench_reference(args)
+    if args.workload == "decode":
+        return bench_decode(args)
     return bench_ours(args)
 
 
