@@ -344,7 +344,7 @@ osdn_status_t launch_step_io(const void* q, const void* k, const void* v, const 
     const IO *q_ = static_cast<const IO*>(q), *k_ = static_cast<const IO*>(k),
              *v_ = static_cast<const IO*>(v);
     IO *o_ = static_cast<IO*>(o), *kt_ = static_cast<IO*>(kt);
-    const dim3 grid((unsigned)nh), block(STEP_THREADS);
+    const dim3 grid((unsigned)nh), block(step_threads(Dv));
     if (Dk == 128 && Dv == 128)
         osdn_step_kernel<128, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, (int)nh);
     else if (Dk == 128 && Dv == 64)

@@ -8,9 +8,9 @@
 // The step reads and writes the fp32 state once (Dv x Dk x 4 bytes each way) and a few hundred
 // bytes of token data: it is bound by HBM bandwidth.
 //
-// One CTA of 256 threads per (sequence, head).  Warp w owns state rows (value channels)
-// w, w + 8, ...; lane l holds key channels [4l, 4l + 4) (Dk = 128) or [2l, 2l + 2) (Dk = 64).
-// Every row load is issued before the first use, so each warp keeps Dv / 8 row loads in flight.
+// One CTA of Dv / 8 warps per (sequence, head).  Warp w owns the 8 state rows (value channels)
+// w, w + Dv/8, ...; lane l holds key channels [4l, 4l + 4) (Dk = 128) or [2l, 2l + 2) (Dk = 64).
+// Every row load is issued before the first use, so each warp keeps 8 row loads in flight.
 // Plain cached accesses: a decode batch's states (64 KB per head) can stay in L2 between steps.
 #pragma once
 
@@ -18,7 +18,8 @@
 
 namespace osdn {
 
-constexpr int STEP_THREADS = 256;
+// Threads per CTA for a value dimension DV: one warp per 8 state rows.
+constexpr int step_threads(int DV) { return DV * 4; }
 
 template <int N> struct vecf;
 template <> struct vecf<4> {
@@ -49,13 +50,14 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <int DK, int DV, typename IO>
-__global__ void __launch_bounds__(STEP_THREADS)
+__global__ void __launch_bounds__(DV * 4)
 osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                  const float* __restrict__ beta, const float* __restrict__ r, float eta,
                  float scale, float* __restrict__ S, float* __restrict__ d, IO* __restrict__ o,
                  IO* __restrict__ k_tilde, int NH) {
     constexpr int PL = DK / 32;             // key channels per lane
-    constexpr int ROWS = DV / 8;            // state rows per warp
+    constexpr int NW = DV / 8;              // warps
+    constexpr int ROWS = 8;                 // state rows per warp
     using tr = io_traits<IO>;
     const int nh = blockIdx.x;
     if (nh >= NH) return;
@@ -64,7 +66,7 @@ osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
     // state rows first: the bulk of the traffic, in flight while the token data arrives
     float srow[ROWS][PL];
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) vecf<PL>::load(Sh + (int64_t)(warp + 8 * i) * DK + PL * lane, srow[i]);
+    for (int i = 0; i < ROWS; ++i) vecf<PL>::load(Sh + (int64_t)(warp + NW * i) * DK + PL * lane, srow[i]);
     float kk[PL], qq[PL], dd[PL];
 #pragma unroll
     for (int j = 0; j < PL; ++j) {
@@ -81,14 +83,14 @@ osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         nk += a;
         sa = fmaf(dd[j], a, sa);
     }
-    // u_i = v_i - S_i k, S_i += beta u_i k~, o_i = scale S_i q  (row i = warp + 8 i)
+    // u_i = v_i - S_i k, S_i += beta u_i k~, o_i = scale S_i q  (row i = warp + NW i)
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) {
         float sk = 0.f;
 #pragma unroll
         for (int j = 0; j < PL; ++j) sk = fmaf(srow[i][j], kk[j], sk);
         sk = warp_sum(sk);
-        const int row = warp + 8 * i;
+        const int row = warp + NW * i;
         const float u = bt * (tr::to_f32(v[(int64_t)nh * DV + row]) - sk);
         float sq = 0.f;
 #pragma unroll
