@@ -70,7 +70,7 @@ int osdn_ref_set_threads(int n) {
  * step 1).  Emits k~_t = d_t (.) k_t for every token and the final d.
  * ------------------------------------------------------------------------------- */
 void osdn_ref_precond_scan(const double* k, const double* beta, const double* r, double eta,
-                           const double* d0, double* k_tilde, double* dT,
+                           const double* d0, double* k_tilde, double* dT, double* rho,
                            const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                            int32_t H, int32_t Dk) {
     const int32_t N = cu_seqlens ? num_seqs : B;
@@ -92,6 +92,8 @@ void osdn_ref_precond_scan(const double* k, const double* beta, const double* r,
                     s += d[i] * kt[i] * kt[i];
                 }
                 for (int32_t i = 0; i < Dk; ++i) k_tilde[th * Dk + i] = d[i] * kt[i];
+                /* residual-contraction ratio of the write (section 3): (1 - beta_t s_t)^2 */
+                if (rho) rho[th] = (1.0 - bt * s) * (1.0 - bt * s);
                 for (int32_t i = 0; i < Dk; ++i) {
                     const double grad =
                         knorm2 > 0.0 ? -bt * (1.0 - bt * s) * kt[i] * kt[i] / knorm2 : 0.0;

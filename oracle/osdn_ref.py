@@ -87,7 +87,7 @@ class Oracle:
         lib.osdn_ref_set_threads.argtypes = [ctypes.c_int]
         lib.osdn_ref_set_threads.restype = ctypes.c_int
         lib.osdn_ref_precond_scan.argtypes = [
-            _D, _D, _D, ctypes.c_double, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32]
+            _D, _D, _D, ctypes.c_double, _D, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32]
         lib.osdn_ref_precond_scan.restype = None
         lib.osdn_ref_delta_fwd.argtypes = [
             _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32,
@@ -103,8 +103,10 @@ class Oracle:
         """Set the OpenMP thread count (n <= 0 keeps it); returns the count in effect."""
         return int(self.lib.osdn_ref_set_threads(int(n)))
 
-    def precond_scan(self, k, beta, r=None, eta=0.0, d0=None, cu_seqlens=None):
-        """Phase 1 (section 2.2, step 1 of the two-phase split): returns (k_tilde, dT)."""
+    def precond_scan(self, k, beta, r=None, eta=0.0, d0=None, cu_seqlens=None, with_rho=False):
+        """Phase 1 (section 2.2, step 1 of the two-phase split): returns (k_tilde, dT), or
+        (k_tilde, dT, rho) with the per-token residual-contraction ratio
+        rho_t = (1 - beta_t <d_t, k_t^2>)^2 of section 3 when with_rho is set."""
         k, beta, r, d0 = _f64(k), _f64(beta), _f64(r), _f64(d0)
         cu, cup = _cu(cu_seqlens)
         B, T, H, Dk, N = _dims(k, cu)
@@ -112,9 +114,10 @@ class Oracle:
         assert d0 is None or d0.shape == (N, H, Dk)
         k_tilde = np.zeros_like(k)
         dT = np.zeros((N, H, Dk))
+        rho = np.zeros((B, T, H)) if with_rho else None
         self.lib.osdn_ref_precond_scan(_ptr(k), _ptr(beta), _ptr(r), float(eta), _ptr(d0),
-                                       _ptr(k_tilde), _ptr(dT), cup, N, B, T, H, Dk)
-        return k_tilde, dT
+                                       _ptr(k_tilde), _ptr(dT), _ptr(rho), cup, N, B, T, H, Dk)
+        return (k_tilde, dT, rho) if with_rho else (k_tilde, dT)
 
     def delta_fwd(self, q, k, k_tilde, v, beta, scale=1.0, S0=None, cu_seqlens=None):
         """Phase 2 (section 2.1): delta rule with write key k_tilde. Returns (o, ST)."""

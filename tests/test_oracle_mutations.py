@@ -32,6 +32,8 @@ MUTATIONS = {
     "residual_drops_state": ("u[j] = vt[j] - sk;", "u[j] = vt[j];"),
     # <d, k^2> taken as <1, k^2>
     "s_ignores_d": ("s += d[i] * kt[i] * kt[i];", "s += kt[i] * kt[i];"),
+    # residual-contraction ratio without its square
+    "rho_not_squared": ("rho[th] = (1.0 - bt * s) * (1.0 - bt * s);", "rho[th] = (1.0 - bt * s);"),
 }
 
 
@@ -43,6 +45,7 @@ def _pin_suite(ref):
     yield lambda: pins.test_hand_worked_example(ref, "apf_half")
     yield lambda: pins.test_gated_newton_closed_form(ref, 0.9, 0.7, 0.2, 1.0)
     yield lambda: pins.test_residual_ratio_closed_form(ref)
+    yield lambda: pins.test_rho_output_is_the_residual_ratio(ref)
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))

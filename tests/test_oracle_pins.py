@@ -254,6 +254,24 @@ def test_residual_ratio_closed_form(ref):
         S_prev, d_prev = St[0, 0], dt1[0, 0]
 
 
+def test_rho_output_is_the_residual_ratio(ref):
+    """The scan's rho output equals f_t(S_t) / f_t(S_{t-1}) built from the oracle's explicit
+    states and the section-1 loss, token by token, with APF and several heads."""
+    rng = np.random.default_rng(27)
+    q, k, v, beta = rand_case(rng, T=9, H=2, Dk=5, Dv=3)
+    r = rng.uniform(0.7, 1.0, beta.shape)
+    _, _, rho = ref.precond_scan(k, beta, r, 0.3, with_rho=True)
+    for h in range(2):
+        S_prev = np.zeros((3, 5))
+        for t in range(9):
+            _, _, St, _ = ref.fwd(q[:, :t + 1], k[:, :t + 1], v[:, :t + 1], beta[:, :t + 1],
+                                  r[:, :t + 1], 0.3)
+            kk, vv = k[0, t, h], v[0, t, h]
+            ratio = loss(St[0, h], kk, vv) / loss(S_prev, kk, vv)
+            assert abs(rho[0, t, h] - ratio) < 1e-10
+            S_prev = St[0, h]
+
+
 # ------------------------------------------------------------------------------------ P8
 def test_phase1_independent_of_q_v_state(ref):
     """P8 (section 2.2): the surrogate depends only on k, beta (and d), so k~ and d_T do not
