@@ -67,18 +67,18 @@ inline bool set_smem(KernelT kernel, size_t bytes) {
 // ---------------------------------------------------------------- phase 1 dispatch
 template <typename IO>
 osdn_status_t launch_scan_warp(const void* k, const float* beta, const float* r, float eta,
-                               const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                               const float* d0, void* k_tilde, float* dT, float* rho, const int32_t* cu,
                                const Dims& d, cudaStream_t stream) {
     const int units = d.N * d.H;
     if (units == 0) return OSDN_OK;
     const dim3 block(128), grid((units + 3) / 4);
     if (d.Dk == 128)
         precond_scan_warp_kernel<128, IO><<<grid, block, 0, stream>>>(
-            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, cu, d.N,
+            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, rho, cu, d.N,
             d.T, d.H);
     else
         precond_scan_warp_kernel<64, IO><<<grid, block, 0, stream>>>(
-            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, cu, d.N,
+            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, rho, cu, d.N,
             d.T, d.H);
     return launch_status();
 }
@@ -177,7 +177,7 @@ int sm_count() {
 // Phase 1, bf16 with 128 key channels: T_d of every chunk (prep kernel, written into the k~
 // buffer), then the chain across chunks (one CTA per (sequence, head)).
 osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, float eta,
-                             const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                             const float* d0, void* k_tilde, float* dT, float* rho, const int32_t* cu,
                              const Dims& d, cudaStream_t stream) {
     const int64_t nh = (int64_t)d.N * d.H;
     if (nh == 0) return OSDN_OK;
@@ -200,7 +200,7 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     auto chain = precond_chain_kernel;
     if (!set_smem(chain, ScanChainSmem::BYTES)) return OSDN_ERR_CUDA;
     chain<<<dim3((unsigned)nh), dim3(SCAN_CHAIN_THREADS), ScanChainSmem::BYTES, stream>>>(
-        mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde), dT, cu, d.N, d.T, d.H,
+        mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde), dT, rho, cu, d.N, d.T, d.H,
         (long long)kWaitLimitNs);
     return launch_status();
 }
@@ -209,13 +209,13 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
 // and token-free calls use the warp-per-(sequence, head) scan.
 template <typename IO>
 osdn_status_t launch_scan(const void* k, const float* beta, const float* r, float eta,
-                          const float* d0, void* k_tilde, float* dT, const int32_t* cu,
+                          const float* d0, void* k_tilde, float* dT, float* rho, const int32_t* cu,
                           const Dims& d, cudaStream_t stream) {
     if constexpr (sizeof(IO) == 2) {
         if (d.Dk == 128 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
-            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
+            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, dT, rho, cu, d, stream);
     }
-    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, cu, d, stream);
+    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, rho, cu, d, stream);
 }
 
 // 3-D fp32 view [rows][H][Dv / 2] of the bf16 output buffer; boxes of 32 values (one 64-channel
@@ -291,11 +291,11 @@ osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* 
 }
 
 osdn_status_t validate_scan(const void* k, const float* beta, const float* r, const float* d0,
-                            const void* k_tilde, const float* dT, const Dims& d,
+                            const void* k_tilde, const float* dT, const float* rho, const Dims& d,
                             osdn_dtype_t io) {
     // token tensors may be NULL only when there are no tokens at all
     if (d.rows() * d.H > 0 && (!k || !beta || !k_tilde)) return OSDN_ERR_INVALID_ARG;
-    const void* ptrs[] = {k, beta, r, d0, k_tilde, dT};
+    const void* ptrs[] = {k, beta, r, d0, k_tilde, dT, rho};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
     // the k~ buffer is written before the gates and states are read: no input may lie in it
@@ -303,7 +303,10 @@ osdn_status_t validate_scan(const void* k, const float* beta, const float* r, co
     const size_t gbytes = (size_t)d.rows() * d.H * 4, sbytes = (size_t)d.N * d.H * d.Dk * 4;
     if (overlaps(k, kbytes, k_tilde, kbytes) || overlaps(beta, gbytes, k_tilde, kbytes) ||
         overlaps(r, gbytes, k_tilde, kbytes) || overlaps(d0, sbytes, k_tilde, kbytes) ||
-        overlaps(dT, sbytes, k_tilde, kbytes))
+        overlaps(dT, sbytes, k_tilde, kbytes) || overlaps(rho, gbytes, k_tilde, kbytes) ||
+        overlaps(rho, gbytes, k, kbytes) || overlaps(rho, gbytes, beta, gbytes) ||
+        overlaps(rho, gbytes, r, gbytes) || overlaps(rho, gbytes, d0, sbytes) ||
+        overlaps(rho, gbytes, dT, sbytes))
         return OSDN_ERR_INVALID_ARG;
     return OSDN_OK;
 }
@@ -340,19 +343,19 @@ namespace {
 template <typename IO>
 osdn_status_t launch_step_io(const void* q, const void* k, const void* v, const float* beta,
                              const float* r, float eta, float scale, float* S, float* d, void* o,
-                             void* kt, int64_t nh, int Dk, int Dv, cudaStream_t stream) {
+                             void* kt, float* rho, int64_t nh, int Dk, int Dv, cudaStream_t stream) {
     const IO *q_ = static_cast<const IO*>(q), *k_ = static_cast<const IO*>(k),
              *v_ = static_cast<const IO*>(v);
     IO *o_ = static_cast<IO*>(o), *kt_ = static_cast<IO*>(kt);
     const dim3 grid((unsigned)nh), block(step_threads(Dv));
     if (Dk == 128 && Dv == 128)
-        osdn_step_kernel<128, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, (int)nh);
+        osdn_step_kernel<128, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
     else if (Dk == 128 && Dv == 64)
-        osdn_step_kernel<128, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, (int)nh);
+        osdn_step_kernel<128, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
     else if (Dk == 64 && Dv == 128)
-        osdn_step_kernel<64, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, (int)nh);
+        osdn_step_kernel<64, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
     else
-        osdn_step_kernel<64, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, (int)nh);
+        osdn_step_kernel<64, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
     return launch_status();
 }
 }  // namespace
@@ -377,19 +380,19 @@ const char* osdn_status_string(osdn_status_t s) {
 }
 
 osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r, float eta,
-                                const float* d0, void* k_tilde, float* dT,
+                                const float* d0, void* k_tilde, float* dT, float* rho,
                                 const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
                                 int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io,
                                 void* stream) {
     Dims d;
     osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
     if (st != OSDN_OK) return st;
-    st = validate_scan(k, beta, r, d0, k_tilde, dT, d, io);
+    st = validate_scan(k, beta, r, d0, k_tilde, dT, rho, d, io);
     if (st != OSDN_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16)
-        return launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, k_tilde, dT, cu_seqlens, d, s);
-    return launch_scan<float>(k, beta, r, eta, d0, k_tilde, dT, cu_seqlens, d, s);
+        return launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, k_tilde, dT, rho, cu_seqlens, d, s);
+    return launch_scan<float>(k, beta, r, eta, d0, k_tilde, dT, rho, cu_seqlens, d, s);
 }
 
 osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, const void* v,
@@ -419,7 +422,7 @@ size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osd
 
 osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
                        const float* r, float eta, const float* d0, const float* S0, float scale,
-                       void* o, float* ST, float* dT, void* k_tilde_out,
+                       void* o, float* ST, float* dT, float* rho, void* k_tilde_out,
                        const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                        int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                        void* workspace, size_t workspace_bytes, void* stream) {
@@ -435,30 +438,34 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return OSDN_ERR_ALIGNMENT;
         kt = workspace;
     }
-    st = validate_scan(k, beta, r, d0, kt, dT, d, io);
+    st = validate_scan(k, beta, r, d0, kt, dT, rho, d, io);
     if (st != OSDN_OK) return st;
     st = validate_chunk(q, k, kt, v, beta, S0, o, ST, d, chunk, io);
     if (st != OSDN_OK) return st;
     const size_t es = io_size(io);
     const size_t kb = (size_t)d.rows() * d.H * d.Dk * es, vb = (size_t)d.rows() * d.H * d.Dv * es;
     const size_t db = (size_t)d.N * d.H * d.Dk * 4;
-    if (overlaps(kt, kb, q, kb) || overlaps(kt, kb, v, vb) || overlaps(o, vb, dT, db))
+    const size_t gb = (size_t)d.rows() * d.H * 4;
+    if (overlaps(kt, kb, q, kb) || overlaps(kt, kb, v, vb) || overlaps(o, vb, dT, db) ||
+        overlaps(o, vb, rho, gb) || overlaps(rho, gb, q, kb) || overlaps(rho, gb, v, vb) ||
+        overlaps(rho, gb, S0, (size_t)d.N * d.H * d.Dv * d.Dk * 4) ||
+        overlaps(rho, gb, ST, (size_t)d.N * d.H * d.Dv * d.Dk * 4))
         return OSDN_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16) {
-        st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, dT, cu_seqlens, d, s);
+        st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, dT, rho, cu_seqlens, d, s);
         if (st != OSDN_OK) return st;
         return launch_chunk<__nv_bfloat16>(chunk, q, k, kt, v, beta, scale, S0, o, ST,
                                            cu_seqlens, d, s);
     }
-    st = launch_scan<float>(k, beta, r, eta, d0, kt, dT, cu_seqlens, d, s);
+    st = launch_scan<float>(k, beta, r, eta, d0, kt, dT, rho, cu_seqlens, d, s);
     if (st != OSDN_OK) return st;
     return launch_chunk<float>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu_seqlens, d, s);
 }
 
 osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
                         const float* r, float eta, float scale, float* S, float* d, void* o,
-                        void* k_tilde, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
+                        void* k_tilde, float* rho, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
                         osdn_dtype_t io, void* stream) {
     if (io != OSDN_BF16 && io != OSDN_F32) return OSDN_ERR_INVALID_ARG;
     if (N < 0 || H < 1) return OSDN_ERR_INVALID_ARG;
@@ -467,22 +474,22 @@ osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float
     if (nh == 0) return OSDN_OK;
     if (nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
     if (!q || !k || !v || !beta || !S || !d || !o) return OSDN_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, beta, r, S, d, o, k_tilde};
+    const void* ptrs[] = {q, k, v, beta, r, S, d, o, k_tilde, rho};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
     const size_t es = io_size(io);
     const size_t qb = nh * Dk * es, vb = nh * Dv * es, gb = nh * 4, sb = nh * Dv * Dk * 4,
                  db = nh * Dk * 4;
-    // every written buffer (S, d, o, k_tilde: slots 5..8) against every other buffer
-    const void* all[] = {q, k, v, beta, r, S, d, o, k_tilde};
-    const size_t allb[] = {qb, qb, vb, gb, gb, sb, db, vb, qb};
-    for (int a = 5; a < 9; ++a)
-        for (int b = 0; b < 9; ++b)
+    // every written buffer (S, d, o, k_tilde, rho: slots 5..9) against every other buffer
+    const void* all[] = {q, k, v, beta, r, S, d, o, k_tilde, rho};
+    const size_t allb[] = {qb, qb, vb, gb, gb, sb, db, vb, qb, gb};
+    for (int a = 5; a < 10; ++a)
+        for (int b = 0; b < 10; ++b)
             if (b != a && overlaps(all[a], allb[a], all[b], allb[b])) return OSDN_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16)
-        return osdn::launch_step_io<__nv_bfloat16>(q, k, v, beta, r, eta, scale, S, d, o, k_tilde, nh, Dk, Dv, s);
-    return osdn::launch_step_io<float>(q, k, v, beta, r, eta, scale, S, d, o, k_tilde, nh, Dk, Dv, s);
+        return osdn::launch_step_io<__nv_bfloat16>(q, k, v, beta, r, eta, scale, S, d, o, k_tilde, rho, nh, Dk, Dv, s);
+    return osdn::launch_step_io<float>(q, k, v, beta, r, eta, scale, S, d, o, k_tilde, rho, nh, Dk, Dv, s);
 }
 
 osdn_status_t osdn_get_device_status(void* stream) {
@@ -548,7 +555,8 @@ osdn_status_t noalloc_scratch(void** out) {
 extern "C" osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void* v,
                                           const float* beta, const float* r, float eta,
                                           const float* d0, const float* S0, float scale, void* o,
-                                          float* ST, float* dT, const int32_t* cu_seqlens,
+                                          float* ST, float* dT, float* rho,
+                                          const int32_t* cu_seqlens,
                                           int32_t num_seqs, int32_t B, int32_t T, int32_t H,
                                           int32_t Dk, int32_t Dv, int32_t chunk,
                                           osdn_dtype_t io, void* stream) {
@@ -562,7 +570,7 @@ extern "C" osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const vo
         const osdn_status_t st = noalloc_scratch(&scratch);
         if (st != OSDN_OK) return st;
     }
-    return osdn_fwd(q, k, v, beta, r, eta, d0, S0, scale, o, ST, dT, nullptr, cu_seqlens,
+    return osdn_fwd(q, k, v, beta, r, eta, d0, S0, scale, o, ST, dT, rho, nullptr, cu_seqlens,
                     num_seqs, B, T, H, Dk, Dv, chunk, io, scratch, need > 0 ? kNoallocScratchBytes : 0,
                     stream);
 }

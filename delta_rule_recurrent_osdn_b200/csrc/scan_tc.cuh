@@ -338,8 +338,8 @@ __global__ void __launch_bounds__(SCAN_CHAIN_THREADS, 1)
 precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_td,
                      const float* __restrict__ beta, const float* __restrict__ r, float eta,
                      const float* __restrict__ d0, __nv_bfloat16* __restrict__ k_tilde,
-                     float* __restrict__ dT, const int32_t* __restrict__ cu, int N, int T, int H,
-                     long long limit_ns) {
+                     float* __restrict__ dT, float* __restrict__ rho,
+                     const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
     constexpr int C = SCAN_C, DK = 128;
     using L = ScanChainSmem;
     extern __shared__ uint8_t smem_raw[];
@@ -460,6 +460,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             const float* vv = vecs(s);
             const float* d = sD + (c % 3) * 128;
             // ---- step 1: p_t = <a_t, d>, ||k_t||^2, b_t
+            float e_t = 0.f, bRp = 0.f;  // kept for the residual ratio of step 2
             {
                 float p = 0.f, nk = 0.f;
 #pragma unroll
@@ -482,8 +483,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 nk += __shfl_xor_sync(0xffffffffu, nk, 16);
                 if (half == 0) {
                     const float bt = vv[192 + t];
-                    const float e = (t < Lc && nk > 0.f) ? eta * bt / nk : 0.f;
-                    sB[t] = e * (1.f - bt * vv[t] * p);
+                    e_t = (t < Lc && nk > 0.f) ? eta * bt / nk : 0.f;
+                    sB[t] = e_t * (1.f - bt * vv[t] * p);
+                    bRp = bt * vv[t] * p;
                 }
             }
             group_bar(1, 128);
@@ -506,6 +508,12 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     const float x = t < Lc ? acc : 0.f;
                     sX[(c % 3) * 64 + t] = x;
                     sGX[t] = vv[64 + t] * x;
+                    // residual-contraction ratio (1 - beta s)^2: x = e (1 - beta s) when e != 0;
+                    // else d_t = R_t d_0 on this token's row, so beta s = beta R p
+                    if (rho && t < Lc) {
+                        const float g = e_t != 0.f ? x / e_t : 1.f - bRp;
+                        rho[(first + (int64_t)c * C + t) * H + h] = g * g;
+                    }
                 }
             }
             group_bar(1, 128);

@@ -21,7 +21,7 @@ template <int DK, typename IO>
 __global__ void __launch_bounds__(128)
 precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
                          const float* __restrict__ r, float eta, const float* __restrict__ d0,
-                         IO* __restrict__ k_tilde, float* __restrict__ dT,
+                         IO* __restrict__ k_tilde, float* __restrict__ dT, float* __restrict__ rho,
                          const int32_t* __restrict__ cu, int N, int T, int H) {
     static_assert(DK == 64 || DK == 128, "DK");
     constexpr int E = DK / 32;  // consecutive channels per lane
@@ -89,6 +89,7 @@ precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ bet
                     store4<IO>(ktp + t * rs, make_float4(kt[0], kt[1], kt[2], kt[3]));
                 else
                     store2<IO>(ktp + t * rs, make_float2(kt[0], kt[1]));
+                if (rho && lane == 0) rho[(first + t) * H + h] = (1.f - bt * s) * (1.f - bt * s);
                 const float coef = nk > 0.f ? eta * bt * (1.0f - bt * s) / nk : 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) d[e] = fmaf(rt, d[e], coef * a[e]);

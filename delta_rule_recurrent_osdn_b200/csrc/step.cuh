@@ -4,7 +4,8 @@
 // technical summary, sections 2.1-2.3, applied to a single token with the state carried in
 // HBM.  With a = k (.) k, nk = ||k||^2, s = <d, a>:
 //   k~ = d (.) k,   u = v - S k,   S <- S + beta u k~^T,   o = scale * S q,
-//   d  <- r d + eta beta (1 - beta s) a / nk   (0 when nk = 0).
+//   d  <- r d + eta beta (1 - beta s) a / nk   (0 when nk = 0),
+// and optionally the residual-contraction ratio (1 - beta s)^2 of the write (section 3).
 // The step reads and writes the fp32 state once (Dv x Dk x 4 bytes each way) and a few hundred
 // bytes of token data: it is bound by HBM bandwidth.
 //
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(DV * 4)
 osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                  const float* __restrict__ beta, const float* __restrict__ r, float eta,
                  float scale, float* __restrict__ S, float* __restrict__ d, IO* __restrict__ o,
-                 IO* __restrict__ k_tilde, int NH) {
+                 IO* __restrict__ k_tilde, float* __restrict__ rho, int NH) {
     constexpr int PL = DK / 32;             // key channels per lane
     constexpr int NW = DV / 8;              // warps
     constexpr int ROWS = 8;                 // state rows per warp
@@ -108,6 +109,7 @@ osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         sa = warp_sum(sa);
         const float rt = r ? r[nh] : 1.f;
         const float g = nk > 0.f ? eta * bt * (1.f - bt * sa) / nk : 0.f;
+        if (rho && lane == 0) rho[nh] = (1.f - bt * sa) * (1.f - bt * sa);
 #pragma unroll
         for (int j = 0; j < PL; ++j) {
             if (k_tilde) k_tilde[(int64_t)nh * DK + PL * lane + j] = tr::from_f32(kt[j]);

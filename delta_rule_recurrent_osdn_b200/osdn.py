@@ -50,8 +50,8 @@ def _load() -> ctypes.CDLL:
     lib.osdn_abi_version.restype = _i32
     lib.osdn_status_string.argtypes = [ctypes.c_int]
     lib.osdn_status_string.restype = ctypes.c_char_p
-    lib.osdn_precond_scan.argtypes = [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
-                                      _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_precond_scan.argtypes = [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                      _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_precond_scan.restype = ctypes.c_int
     lib.osdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i32, _i32,
                                    _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
@@ -59,11 +59,11 @@ def _load() -> ctypes.CDLL:
     lib.osdn_fwd_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, ctypes.c_int]
     lib.osdn_fwd_workspace_bytes.restype = ctypes.c_size_t
     lib.osdn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _f32, _vp, _vp, _vp, _vp,
-                             _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
+                             _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
                              ctypes.c_size_t, _vp]
     lib.osdn_fwd.restype = ctypes.c_int
-    lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp, _vp, _i32, _i32,
-                              _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _i32,
+                              _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_step.restype = ctypes.c_int
     lib.osdn_get_device_status.argtypes = [_vp]
     lib.osdn_get_device_status.restype = ctypes.c_int
@@ -130,8 +130,10 @@ def _seqs(cu_seqlens, B):
 
 
 def osdn_precond_scan(k, beta, r=None, eta: float = 0.0, d0=None, cu_seqlens=None,
-                      k_tilde=None, dT=None, return_dT: bool = True, stream=None):
-    """Phase 1: returns ``(k_tilde, dT)`` (``dT`` is None when ``return_dT`` is False)."""
+                      k_tilde=None, dT=None, return_dT: bool = True, rho=None, stream=None):
+    """Phase 1: returns ``(k_tilde, dT)`` (``dT`` is None when ``return_dT`` is False).  Given a
+    float32 tensor ``rho`` of shape [B, T, H], also writes the per-token residual-contraction
+    ratio (1 - beta_t <d_t, k_t^2>)^2 there."""
     B, T, H, Dk = k.shape
     io = _io(k)
     num_seqs, N = _seqs(cu_seqlens, B)
@@ -145,8 +147,10 @@ def osdn_precond_scan(k, beta, r=None, eta: float = 0.0, d0=None, cu_seqlens=Non
     if dT is None and return_dT:
         dT = torch.empty((N, H, Dk), dtype=torch.float32, device=k.device)
     _req(dT, "dT", torch.float32, (N, H, Dk))
+    _req(rho, "rho", torch.float32, (B, T, H))
     _check(LIB.osdn_precond_scan(_p(k), _p(beta), _p(r), float(eta), _p(d0), _p(k_tilde), _p(dT),
-                                 _p(cu_seqlens), num_seqs, B, T, H, Dk, io, _stream(stream)),
+                                 _p(rho), _p(cu_seqlens), num_seqs, B, T, H, Dk, io,
+                                 _stream(stream)),
            "osdn_precond_scan")
     return k_tilde, dT
 
@@ -183,7 +187,7 @@ def osdn_fwd_workspace_bytes(B: int, T: int, H: int, Dk: int, dtype=torch.bfloat
 
 def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: float = 1.0,
              chunk: int = 64, cu_seqlens=None, o=None, ST=None, dT=None, k_tilde=None,
-             workspace=None, return_states: bool = True, stream=None):
+             workspace=None, return_states: bool = True, rho=None, stream=None):
     """Both phases: returns ``(o, ST, dT)`` (states None when ``return_states`` is False).
 
     When neither ``k_tilde`` nor ``workspace`` is given, a workspace of
@@ -211,6 +215,7 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
             dT = torch.empty((N, H, Dk), dtype=torch.float32, device=q.device)
     _req(ST, "ST", torch.float32, (N, H, Dv, Dk))
     _req(dT, "dT", torch.float32, (N, H, Dk))
+    _req(rho, "rho", torch.float32, (B, T, H))
     ws_bytes = 0
     if k_tilde is None:
         need = int(LIB.osdn_fwd_workspace_bytes(B, T, H, Dk, io))
@@ -220,7 +225,7 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
             _req(workspace, "workspace")
             ws_bytes = workspace.numel() * workspace.element_size()
     _check(LIB.osdn_fwd(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), _p(d0), _p(S0),
-                        float(scale), _p(o), _p(ST), _p(dT), _p(k_tilde), _p(cu_seqlens),
+                        float(scale), _p(o), _p(ST), _p(dT), _p(rho), _p(k_tilde), _p(cu_seqlens),
                         num_seqs, B, T, H, Dk, Dv, int(chunk), io,
                         _p(workspace) if k_tilde is None else None, ws_bytes, _stream(stream)),
            "osdn_fwd")
@@ -228,7 +233,7 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
 
 
 def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0, o=None,
-              k_tilde=None, stream=None):
+              k_tilde=None, rho=None, stream=None):
     """One recurrent step per (sequence, head) (the decode path).  q, k: [N, H, Dk]; v: [N, H, Dv];
     beta, r: [N, H] float32; S: [N, H, Dv, Dk] and d: [N, H, Dk] float32, updated in place.
     Returns o [N, H, Dv] (and writes k_tilde [N, H, Dk] when given)."""
@@ -246,8 +251,9 @@ def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0,
         o = torch.empty_like(v)
     _req(o, "o", q.dtype, (N, H, Dv))
     _req(k_tilde, "k_tilde", q.dtype, (N, H, Dk))
+    _req(rho, "rho", torch.float32, (N, H))
     _check(LIB.osdn_step(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), float(scale), _p(S),
-                         _p(d), _p(o), _p(k_tilde), N, H, Dk, Dv, io, _stream(stream)),
+                         _p(d), _p(o), _p(k_tilde), _p(rho), N, H, Dk, Dv, io, _stream(stream)),
            "osdn_step")
     return o
 

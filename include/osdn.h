@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define OSDN_ABI_VERSION 1
+#define OSDN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define OSDN_API __attribute__((visibility("default")))
@@ -93,9 +93,12 @@ OSDN_API const char* osdn_status_string(osdn_status_t status);
  *           d0 or dT (OSDN_ERR_INVALID_ARG): for bf16 with Dk = 128 the call first uses this
  *           buffer as scratch for per-chunk factors, then overwrites it with k~.
  *   dT      [N,H,Dk] final preconditioner, written; NULL skips it.
+ *   rho     [B,T,H] float32, written: the residual-contraction ratio of each write,
+ *           rho_t = (1 - beta_t <d_t, k_t (.) k_t>)^2 (section 3: f_t(S_t) = rho_t f_t(S_{t-1}));
+ *           NULL skips it.  Must not overlap any other buffer.
  */
 OSDN_API osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r, float eta,
-                                const float* d0, void* k_tilde, float* dT,
+                                const float* d0, void* k_tilde, float* dT, float* rho,
                                 const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
                                 int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io,
                                 void* stream);
@@ -135,7 +138,7 @@ OSDN_API size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_
  */
 OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
                        const float* r, float eta, const float* d0, const float* S0, float scale,
-                       void* o, float* ST, float* dT, void* k_tilde_out,
+                       void* o, float* ST, float* dT, float* rho, void* k_tilde_out,
                        const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                        int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                        void* workspace, size_t workspace_bytes, void* stream);
@@ -164,7 +167,7 @@ OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, con
 OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void* v,
                                         const float* beta, const float* r, float eta,
                                         const float* d0, const float* S0, float scale, void* o,
-                                        float* ST, float* dT, const int32_t* cu_seqlens,
+                                        float* ST, float* dT, float* rho, const int32_t* cu_seqlens,
                                         int32_t num_seqs, int32_t B, int32_t T, int32_t H,
                                         int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                                         void* stream);
@@ -186,13 +189,14 @@ OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void
  *   S        [N,H,Dv,Dk] float32, read and written in place (row = value channel).
  *   d        [N,H,Dk] float32, read and written in place.
  *   o        [N,H,Dv] io dtype, written.     k_tilde [N,H,Dk] io dtype, written, or NULL.
+ *   rho      [N,H] float32, written: (1 - beta s)^2, as for osdn_precond_scan; or NULL.
  * Dk, Dv in {64, 128}.  Pointers 16-byte aligned.  S, d, o and k_tilde must not overlap one
  * another or the inputs (OSDN_ERR_INVALID_ARG).  N == 0 is a no-op.  A sequence of steps
  * equals osdn_fwd over the same tokens (up to fp32 summation order).
  */
 OSDN_API osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
                         const float* r, float eta, float scale, float* S, float* d, void* o,
-                        void* k_tilde, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
+                        void* k_tilde, float* rho, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
                         osdn_dtype_t io, void* stream);
 
 OSDN_API osdn_status_t osdn_get_device_status(void* stream);

@@ -25,11 +25,13 @@ def chunk_call(**kw):
 
 
 def scan_call(**kw):
-    args = dict(k=fake(1), beta=fake(2), r=None, eta=0.1, d0=None, kt=fake(3), dT=None, cu=None,
+    args = dict(k=fake(1), beta=fake(2), r=None, eta=0.1, d0=None, kt=fake(3), dT=None, rho=None,
+                cu=None,
                 num_seqs=0, B=1, T=8, H=1, Dk=128, io=osdn.OSDN_BF16)
     args.update(kw)
     return L.osdn_precond_scan(args["k"], args["beta"], args["r"], args["eta"], args["d0"],
-                               args["kt"], args["dT"], args["cu"], args["num_seqs"], args["B"],
+                               args["kt"], args["dT"], args["rho"], args["cu"], args["num_seqs"],
+                               args["B"],
                                args["T"], args["H"], args["Dk"], args["io"], None)
 
 
@@ -42,7 +44,7 @@ def test_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert L.osdn_abi_version() == 1
+    assert L.osdn_abi_version() == 2
     for s in range(7):
         assert osdn.status_string(s)
     assert osdn.status_string(99) == "unknown status"
@@ -87,6 +89,9 @@ def test_chunk_fwd_rejects(kw, status):
     (dict(r=ctypes.c_void_p(A + 3 * 0x1000000 + 512)), osdn.OSDN_ERR_INVALID_ARG),
     (dict(d0=ctypes.c_void_p(A + 3 * 0x1000000)), osdn.OSDN_ERR_INVALID_ARG),
     (dict(dT=ctypes.c_void_p(A + 3 * 0x1000000 + 1024)), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(rho=ctypes.c_void_p(A + 3 * 0x1000000 + 1536)), osdn.OSDN_ERR_INVALID_ARG),  # rho in k~
+    (dict(rho=ctypes.c_void_p(A + 2 * 0x1000000)), osdn.OSDN_ERR_INVALID_ARG),        # rho = beta
+    (dict(rho=ctypes.c_void_p(A + 9 * 0x1000000 + 4)), osdn.OSDN_ERR_ALIGNMENT),
     (dict(r=ctypes.c_void_p(A + 2)), osdn.OSDN_ERR_ALIGNMENT),
     (dict(cu=ctypes.c_void_p(A + 4), num_seqs=1), osdn.OSDN_ERR_ALIGNMENT),
     (dict(num_seqs=-1), osdn.OSDN_ERR_INVALID_ARG),
@@ -97,11 +102,11 @@ def test_precond_scan_rejects(kw, status):
 
 def test_fwd_rejects_small_workspace():
     st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
-                    None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16, fake(7), 100,
+                    None, None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16, fake(7), 100,
                     None)
     assert st == osdn.OSDN_ERR_INVALID_ARG
     st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
-                    None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16,
+                    None, None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16,
                     ctypes.c_void_p(A + 0x7000010), 1 << 20, None)
     assert st == osdn.OSDN_ERR_ALIGNMENT  # workspace must be 256-byte aligned
 
@@ -124,11 +129,12 @@ def test_parity_metric_allows_exactly_the_output_rounding():
 
 def step_call(**kw):
     args = dict(q=fake(1), k=fake(2), v=fake(3), beta=fake(4), r=None, eta=0.1, scale=1.0,
-                S=fake(5), d=fake(6), o=fake(7), kt=None, N=4, H=2, Dk=128, Dv=128,
+                S=fake(5), d=fake(6), o=fake(7), kt=None, rho=None, N=4, H=2, Dk=128, Dv=128,
                 io=osdn.OSDN_BF16)
     args.update(kw)
     return L.osdn_step(args["q"], args["k"], args["v"], args["beta"], args["r"], args["eta"],
-                       args["scale"], args["S"], args["d"], args["o"], args["kt"], args["N"],
+                       args["scale"], args["S"], args["d"], args["o"], args["kt"], args["rho"],
+                       args["N"],
                        args["H"], args["Dk"], args["Dv"], args["io"], None)
 
 
@@ -144,6 +150,7 @@ def step_call(**kw):
     (dict(o=fake(1)), osdn.OSDN_ERR_INVALID_ARG),                                 # o aliases q
     (dict(d=ctypes.c_void_p(A + 5 * 0x1000000 + 4096)), osdn.OSDN_ERR_INVALID_ARG),  # d in S
     (dict(kt=fake(2)), osdn.OSDN_ERR_INVALID_ARG),                                # k~ aliases k
+    (dict(rho=fake(4)), osdn.OSDN_ERR_INVALID_ARG),                               # rho = beta
     (dict(N=0), osdn.OSDN_OK),                                                    # nothing to do
 ])
 def test_step_rejects(kw, status):
