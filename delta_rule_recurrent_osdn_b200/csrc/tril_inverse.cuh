@@ -62,6 +62,20 @@ __device__ __forceinline__ void tsw_row(const float* m, int r, int c0, float* x)
     }
 }
 
+// Packed dot product: acc += m[r][c0 .. c0 + 4 NG) . col2[0 .. 2 NG), with col2[i] holding the
+// column entries c0 + 2i and c0 + 2i + 1, as two-wide fp32 FMAs (two partial sums).
+template <int NG>
+__device__ __forceinline__ float2 tsw_dot2(const float* m, int r, int c0, const float2* col2,
+                                           float2 acc) {
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const float4 v = tsw_ld4(m, r, (c0 >> 2) + g);
+        acc = __ffma2_rn(make_float2(v.x, v.y), col2[2 * g], acc);
+        acc = __ffma2_rn(make_float2(v.z, v.w), col2[2 * g + 1], acc);
+    }
+    return acc;
+}
+
 // In place.  On entry M holds L in the swizzled layout (only its strictly lower triangle is
 // read); on return it holds T on and below the diagonal, and the entries above the diagonal hold
 // scratch values, so a reader masks them (T is lower triangular with a unit diagonal).  Every
@@ -76,111 +90,101 @@ __device__ __forceinline__ void tril_inverse_64_g128(float* __restrict__ M, int 
     // ---- A. diagonal blocks: column `col` of block b, x[r] = [r == col] - sum_{m<r} L_rm x[m]
     {
         const int o = 16 * ((t & 63) >> 4), col = t & 15;
-        float x[16];
+        float2 xp[8];  // x[2i], x[2i + 1]; zero until computed (their L factor is zeroed too,
+                       // but 0 * an uninitialized NaN would still be NaN)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xp[i] = make_float2(0.f, 0.f);
         if (t < 64) {
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float lr[16];
+                float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int g = 0; 4 * g < r; ++g) {
                     const float4 v = tsw_ld4(sL, o + r, (o >> 2) + g);
-                    lr[4 * g] = v.x;
-                    lr[4 * g + 1] = v.y;
-                    lr[4 * g + 2] = v.z;
-                    lr[4 * g + 3] = v.w;
+                    // x[m] == 0 for m < col, so no per-lane bound is needed; terms m >= r are
+                    // excluded by zeroing their L factor
+                    const int m = 4 * g;
+                    const float2 l0 = make_float2(m < r ? v.x : 0.f, m + 1 < r ? v.y : 0.f);
+                    const float2 l1 = make_float2(m + 2 < r ? v.z : 0.f, m + 3 < r ? v.w : 0.f);
+                    acc2 = __ffma2_rn(l0, xp[2 * g], acc2);
+                    acc2 = __ffma2_rn(l1, xp[2 * g + 1], acc2);
                 }
-                float acc = 0.f;  // x[m] == 0 for m < col, so no per-lane bound is needed
-#pragma unroll
-                for (int m = 0; m < r; ++m) acc = fmaf(-lr[m], x[m], acc);
-                x[r] = r == col ? 1.f : (r < col ? 0.f : acc);
+                const float xr = r == col ? 1.f : (r < col ? 0.f : -(acc2.x + acc2.y));
+                if (r & 1) xp[r >> 1].y = xr; else xp[r >> 1] = make_float2(xr, 0.f);
             }
         }
         group_bar(bar_id, NT);  // the diagonal blocks of L are read
         if (t < 64) {
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sT[tsw(o + r, o + col)] = x[r];
+            for (int r = 0; r < 16; ++r) sT[tsw(o + r, o + col)] = (r & 1) ? xp[r >> 1].y : xp[r >> 1].x;
         }
     }
     group_bar(bar_id, NT);
     // ---- B. 16x16 level; thread: block pair (t >> 6), column c, rows 4*rq .. 4*rq + 3
     {
         const int I = (t >> 6) ? 3 : 1, J = I - 1, c = t & 15, rq = (t >> 4) & 3;
-        float col[16];
+        float2 col2[8];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) col[m] = sT[tsw(16 * J + m, 16 * J + c)];  // T_JJ[:, c]
+        for (int m = 0; m < 8; ++m)  // T_JJ[:, c]
+            col2[m] = make_float2(sT[tsw(16 * J + 2 * m, 16 * J + c)], sT[tsw(16 * J + 2 * m + 1, 16 * J + c)]);
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {  // X = L_IJ T_JJ, kept in the free block (J, I)
             const int r = 4 * rq + rr;
-            float lr[16];
-            tsw_row<4>(sL, 16 * I + r, 16 * J, lr);
-            float acc = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) acc = fmaf(lr[m], col[m], acc);
-            sT[tsw(16 * J + r, 16 * I + c)] = acc;
+            const float2 acc = tsw_dot2<4>(sL, 16 * I + r, 16 * J, col2, make_float2(0.f, 0.f));
+            sT[tsw(16 * J + r, 16 * I + c)] = acc.x + acc.y;
         }
         group_bar(bar_id, NT);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) col[m] = sT[tsw(16 * J + m, 16 * I + c)];  // X[:, c]
+        for (int m = 0; m < 8; ++m)  // X[:, c]
+            col2[m] = make_float2(sT[tsw(16 * J + 2 * m, 16 * I + c)], sT[tsw(16 * J + 2 * m + 1, 16 * I + c)]);
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {  // T_IJ = -T_II X  (T_II[r][m] == 0 for m > r)
             const int r = 4 * rq + rr;
-            float tr[16];
-            tsw_row<4>(sT, 16 * I + r, 16 * I, tr);
-            float acc = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) acc = fmaf(-tr[m], col[m], acc);
-            sT[tsw(16 * I + r, 16 * J + c)] = acc;
+            const float2 acc = tsw_dot2<4>(sT, 16 * I + r, 16 * I, col2, make_float2(0.f, 0.f));
+            sT[tsw(16 * I + r, 16 * J + c)] = -(acc.x + acc.y);
         }
     }
     group_bar(bar_id, NT);
     // ---- C. 32x32 level; thread: column c, rows 8*rq .. 8*rq + 7 (rq = warp of the group)
     {
         const int c = t & 31, rq = t >> 5;
-        float col[32];
+        float2 col2[16];
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {  // T_00[:, c]; block (0, 1) holds scratch, so mask m < c
-            const float v = sT[tsw(m, c)];
-            col[m] = m >= c ? v : 0.f;
+        for (int m = 0; m < 16; ++m) {  // T_00[:, c]; block (0, 1) holds scratch, so mask m < c
+            const float v0 = sT[tsw(2 * m, c)], v1 = sT[tsw(2 * m + 1, c)];
+            col2[m] = make_float2(2 * m >= c ? v0 : 0.f, 2 * m + 1 >= c ? v1 : 0.f);
         }
-        float acc[8];
+        float2 acc[8];
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
+        for (int rr = 0; rr < 8; ++rr) acc[rr] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // X = L_10 T_00, kept in the free block (0, 1) of 32x32
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                float lr[16];
-                tsw_row<4>(sL, 32 + 8 * rq + rr, 16 * h, lr);
-#pragma unroll
-                for (int m = 0; m < 16; ++m) acc[rr] = fmaf(lr[m], col[16 * h + m], acc[rr]);
-            }
+            for (int rr = 0; rr < 8; ++rr)
+                acc[rr] = tsw_dot2<4>(sL, 32 + 8 * rq + rr, 16 * h, col2 + 8 * h, acc[rr]);
         }
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) sT[tsw(8 * rq + rr, 32 + c)] = acc[rr];
+        for (int rr = 0; rr < 8; ++rr) sT[tsw(8 * rq + rr, 32 + c)] = acc[rr].x + acc[rr].y;
         group_bar(bar_id, NT);
         // T_10 = -T_11 X.  T_11 is lower triangular, so warp rq (rows 8 rq .. 8 rq + 7 of T_11)
         // needs only its first 8 (rq + 1) terms (which also keeps warps 0-1 away from the
         // level-B scratch in columns 48..63 of rows 32..47).
         const int mlen = 8 * (rq + 1);
 #pragma unroll
-        for (int m = 0; m < 32; ++m)
-            if (m < mlen) col[m] = sT[tsw(m, 32 + c)];  // X[:, c]
+        for (int m = 0; m < 16; ++m)
+            if (2 * m < mlen) col2[m] = make_float2(sT[tsw(2 * m, 32 + c)], sT[tsw(2 * m + 1, 32 + c)]);
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) acc[rr] = 0.f;
+        for (int rr = 0; rr < 8; ++rr) acc[rr] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // 8-term slices, taken while below the warp's bound
             if (8 * q < mlen) {
 #pragma unroll
-                for (int rr = 0; rr < 8; ++rr) {
-                    float tr[8];
-                    tsw_row<2>(sT, 32 + 8 * rq + rr, 32 + 8 * q, tr);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) acc[rr] = fmaf(-tr[m], col[8 * q + m], acc[rr]);
-                }
+                for (int rr = 0; rr < 8; ++rr)
+                    acc[rr] = tsw_dot2<2>(sT, 32 + 8 * rq + rr, 32 + 8 * q, col2 + 4 * q, acc[rr]);
             }
         }
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) sT[tsw(32 + 8 * rq + rr, c)] = acc[rr];
+        for (int rr = 0; rr < 8; ++rr) sT[tsw(32 + 8 * rq + rr, c)] = -(acc[rr].x + acc[rr].y);
     }
     group_bar(bar_id, NT);
 }
