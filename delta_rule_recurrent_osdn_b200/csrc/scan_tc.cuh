@@ -462,23 +462,24 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             // ---- step 1: p_t = <a_t, d>, ||k_t||^2, b_t
             float e_t = 0.f, bRp = 0.f;  // kept for the residual ratio of step 2
             {
-                float p = 0.f, nk = 0.f;
+                float2 p2 = make_float2(0.f, 0.f), nk2 = make_float2(0.f, 0.f);  // channel pairs
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint4 raw = *reinterpret_cast<const uint4*>(kt + half * 8192u + tc::sw128_off(t, j));
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
                     const float4 da = *reinterpret_cast<const float4*>(d + 64 * half + 8 * j);
                     const float4 db = *reinterpret_cast<const float4*>(d + 64 * half + 8 * j + 4);
-                    const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+                    const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w),
+                                          make_float2(db.x, db.y), make_float2(db.z, db.w)};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-                        const float a0 = kk.x * kk.x, a1 = kk.y * kk.y;
-                        nk += a0 + a1;
-                        p = fmaf(a0, dv[2 * e], p);
-                        p = fmaf(a1, dv[2 * e + 1], p);
+                        const float2 a = __fmul2_rn(kk, kk);
+                        nk2 = __fadd2_rn(nk2, a);
+                        p2 = __ffma2_rn(a, dv[e], p2);
                     }
                 }
+                float p = p2.x + p2.y, nk = nk2.x + nk2.y;
                 p += __shfl_xor_sync(0xffffffffu, p, 16);
                 nk += __shfl_xor_sync(0xffffffffu, nk, 16);
                 if (half == 0) {
@@ -521,7 +522,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             //      over the tokens with bit 2 clear (par 0) or set (par 1) -- rows whose swizzle
             //      phases differ, so the lane pair reads disjoint banks -- summed by a shuffle
             {
-                float acc0 = 0.f, acc1 = 0.f;
+                float2 acc = make_float2(0.f, 0.f);  // the two channels of the pair
                 const uint8_t* col = kt + cblk * 8192u + cpe * 2;
 #pragma unroll 8
                 for (int jj = 0; jj < C / 2; ++jj) {
@@ -529,9 +530,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     const uint32_t w = *reinterpret_cast<const uint32_t*>(col + tc::sw128_off(j, cj));
                     const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
                     const float gx = sGX[j];
-                    acc0 = fmaf(gx, kv.x * kv.x, acc0);
-                    acc1 = fmaf(gx, kv.y * kv.y, acc1);
+                    acc = __ffma2_rn(make_float2(gx, gx), __fmul2_rn(kv, kv), acc);
                 }
+                float acc0 = acc.x, acc1 = acc.y;
                 acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
                 acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
                 if (par == 0) {
