@@ -10,11 +10,12 @@
 // only reads T.
 //
 // Hand-off through the output buffer o, which the sequential kernel writes only after reading
-// T: the strictly lower triangle of T (its diagonal is 1), row-major and packed -- entry (t, j),
-// j < t, at index t (t - 1) / 2 + j; 2016 floats for a full chunk -- is written into each
-// 64-channel value tile's slice of the chunk's o rows (64 rows x 128 bytes), one copy per tile,
-// so every sequential CTA reads the copy in its own slice before overwriting that slice with
-// its outputs.  A chunk of Lc < 64 tokens needs Lc (Lc - 1) / 2 floats, which fit in its Lc rows.
+// T: each 128-value (256-byte) row of o for a head holds two 128-byte slices, and row t of a
+// chunk's slices receives row t of T split into bf16 terms, T = hi + lo -- hi in slice 0, lo in
+// slice 1 -- already laid out as a 128-byte-swizzled K-major MMA operand (16-byte group g of
+// row t at group position g ^ (t mod 8)).  The sequential kernel loads both slices with TMA
+// straight into its operand tiles.  A chunk of Lc < 64 tokens has Lc rows of o, so only rows
+// t < Lc are written; the reader completes the tile with identity rows.
 #pragma once
 
 #include <cuda.h>
@@ -38,18 +39,8 @@ struct WyPrepSmem {
 };
 constexpr int WY_PREP_CTAS_PER_SM = 4;
 
-// Packed index t (t - 1) / 2 + j  ->  row t (the j follows): a reciprocal-square-root estimate,
-// then exact integer corrections.
-__device__ __forceinline__ int packed_row(int f) {
-    const float y = 8.f * (float)f + 1.f;
-    int t = (int)((1.f + y * rsqrtf(y)) * 0.5f);
-    while (t * (t - 1) / 2 > f) --t;
-    while ((t + 1) * t / 2 <= f) ++t;
-    return t;
-}
-
 // Persistent grid of 128-thread CTAs walking the batch's chunks (ChunkWalk).  o_f32 is the
-// output buffer [rows, H, Dv] (bf16) seen as floats; Dv = 64 * (number of value tiles).
+// output buffer [rows, H, Dv] (bf16) seen as floats; Dv = 128.
 __global__ void __launch_bounds__(128, WY_PREP_CTAS_PER_SM)
 wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kt,
                const float* __restrict__ beta, float* __restrict__ o_f32, int Dv,
@@ -105,7 +96,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     // M = 128 over the K tile: rows 64..127 of the operand view are the next 64 rows of shared
     // memory (finite data), whose products land in TMEM lanes 64..127 and are never read
     constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);
-    const int nvt = Dv / 64, half_f = Dv / 2;
+    const int half_f = Dv / 2;
 
 #pragma unroll 1
     while (more) {
@@ -166,15 +157,30 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc::fence_before_sync();
         __syncthreads();
         tril_inverse_64_g128(sL, tid, 1);  // T over L
-        // ---- packed strictly-lower T, one copy per value tile
+        // ---- T rows t < Lc as bf16 hi / lo operand rows (thread: row tid mod 64, half tid / 64 of
+        //      its 16-byte groups), into the chunk's o rows
         {
-            const int npk = Lc * (Lc - 1) / 2, rstride = H * half_f;
-            float* dst0 = o_f32 + (row0 * H + h) * half_f;
-            for (int f = tid; f < npk; f += 128) {
-                const int t = packed_row(f), j = f - t * (t - 1) / 2;
-                const float val = sL[tsw(t, j)];
-                float* dst = dst0 + (f >> 5) * rstride + (f & 31);
-                for (int vt = 0; vt < nvt; ++vt) dst[32 * vt] = val;
+            const int r = tid & 63, g0 = 4 * (tid >> 6);
+            if (r < Lc) {
+                uint8_t* orow = reinterpret_cast<uint8_t*>(o_f32 + ((row0 + r) * H + h) * half_f);
+#pragma unroll
+                for (int g = g0; g < g0 + 4; ++g) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 8 * g + 2 * e;
+                        const float a = c < r ? sL[tsw(r, c)] : (c == r ? 1.f : 0.f);
+                        const float b = c + 1 < r ? sL[tsw(r, c + 1)] : (c + 1 == r ? 1.f : 0.f);
+                        const __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+                        const float2 hf = __bfloat1622float2(hb);
+                        const __nv_bfloat162 lb = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+                        hw[e] = *reinterpret_cast<const uint32_t*>(&hb);
+                        lw[e] = *reinterpret_cast<const uint32_t*>(&lb);
+                    }
+                    const int pos = (g ^ (r & 7)) << 4;
+                    *reinterpret_cast<uint4*>(orow + pos) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(orow + 128 + pos) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
             }
         }
         __syncthreads();  // sL is rewritten by the next chunk

@@ -2,36 +2,49 @@
 //
 // The chunkwise delta rule with write key K~ ("OSDN: Improving Delta Rule with Provable Online
 // Preconditioning in Linear Attention", technical summary, section 2.1: K~ replaces K in the
-// chunk Gram matrix and in the intra-chunk scores).  Per chunk of C = 64 tokens, state S_0
-// (value rows), this CTA's 64 value channels:
-//   P = tril(Q K~^T)                              one bf16 MMA, A = [K; Q] (M = 128)
-//   T = (I + strict_tril(diag(beta) K K~^T))^-1   computed for all chunks beforehand by
-//                                                 wy_prep_kernel (chunk_prep.cuh), read here
-//   R = diag(beta) (V - K S_0^T)                  A = [K; Q], B = S_0^T  (rows 64..127: Q S_0^T)
-//   W = T R                                       A = Z = [T; P], B = R
-//   O = Q S_0^T + P W                             A = Z, B = W, accumulated onto Q S_0^T
-//   S_C^T = S_0^T + K~^T W                        A = K~^T (MN-major view of the K~ tile)
+// chunk Gram matrix and in the intra-chunk scores).  Per chunk c of C = 64 tokens with state S_c
+// at its start (value rows), for this CTA's 64 value channels:
+//   T_c = (I + strict_tril(diag(beta) K_c K~_c^T))^-1   computed for all chunks beforehand by
+//                                                       wy_prep_kernel (chunk_prep.cuh), read here
+//   R_c = diag(beta) (V_c - K_c S_c^T)
+//   W_c = T_c R_c
+//   O_c = Q_c S_c^T + P_c W_c,  P_c = tril(Q_c K~_c^T)
+//   S_{c+1}^T = S_c^T + K~_c^T W_c
+//
+// Lookahead form.  Because K_{c+1} S_{c+1}^T = K_{c+1} S_c^T + (K_{c+1} K~_c^T) W_c, the product
+// that starts chunk c+1 is assembled from the state one chunk earlier and from W_c:
+//   D1_{c+1}  = [K_{c+1}; Q_c] S_c^T        A = the ring stage's [K; Q] tile (M = 128)
+//   D1_{c+1} += [X_{c+1}; P_c] W_c          X_{c+1} = K_{c+1} K~_c^T
+// after which rows 0..63 of D1_{c+1} are K_{c+1} S_{c+1}^T and rows 64..127 are O_c.  One Gram
+// MMA, A = [K_{c+1}; Q_c] and B = K~_c, gives X_{c+1} and (masked) P_c together.  The chain's
+// critical path per chunk is R split -> W = T R -> W split -> D1 += [X; P] W: two operand splits
+// and two MMA groups.  The state update S += K~^T W, the state's split and the next
+// [K; Q] S^T product run beside it, one chunk ahead of their use.  (A thread that issues MMAs
+// stalls while the tensor pipe accepts them, so who issues what is part of the schedule.)
 //
 // Precision.  Every computed MMA operand x is split into two bf16 terms, x = hi + lo (about 16
 // significant bits).  A product of an exact bf16 input (K, Q, K~) with a computed operand takes
-// two MMAs (hi, lo); a product of two computed operands ([T; P] with R or W) takes three
-// (hi*hi + hi*lo + lo*hi).  In a CPU emulation of this chunk algorithm against the oracle, plain
-// bf16 operands gave 1.5-2.5% max/rms error on o and S_T for the 340M and 1.3B workloads, and
-// single-term tf32 products 0.25-0.46%; the split scheme is at the fp32 rounding level.
+// two MMAs (hi, lo); a product of two computed operands ([T; .] or [X; P] with R or W) takes
+// three (hi*hi + hi*lo + lo*hi).  In a CPU emulation of this chunk algorithm against the oracle,
+// plain bf16 operands gave 1.5-2.5% max/rms error on o and S_T for the 340M and 1.3B workloads,
+// and single-term tf32 products 0.25-0.46%; the split scheme is at the fp32 rounding level.
 //
 // Warp roles (one CTA per (sequence, head, 64 value channels), 288 threads):
-//   chain    warps 0-3: the state-dependent MMA chain of chunk c and its epilogues (thread t owns
-//            tensor-memory lane t);
-//   prep     warps 4-7: chunk c+1's [T; P] operand tiles (T unpacked from the copy the
-//            pre-kernel left in this CTA's slice of the chunk's o rows, P from a Gram MMA),
-//            overlapping chunk c's chain;
-//   producer warp 8: TMA loads of the chunk tiles into a 2-stage ring (no multicast).
-// Handshakes are mbarriers: zt_* / zp_* for the T and P halves of the [T; P] tiles (W = T R
-// uses only the T rows, the outputs only the P rows, so each half is refilled as soon as its
-// last reader is done; the other half's rows only reach accumulator lanes nobody reads),
-// stage_empty for the ring.
-// Every wait is bounded and followed by a group-wide vote, so a role that gives up (recording
-// OSDN_ERR_DEVICE_TIMEOUT) leaves its loop as a whole group and no named barrier is left waiting.
+//   chain    warps 0-3: R, W = T R, the [X; P] W product and the output rows (thread t owns
+//            tensor-memory lane t); its leader issues only the two MMA groups the chain waits on;
+//   prep     warps 4-7: the state's split, the [X; P] tiles from the Gram, identity rows in the
+//            T tiles of a short last chunk (the pre-kernel leaves T split into bf16 hi / lo operand
+//            rows in the chunk's o rows; they reach the ring stage by TMA);
+//   producer warp 8: TMA loads into a 2-stage ring (no multicast) and the MMAs off the critical
+//            path (Gram, S += K~^T W, the next [K; Q] S^T).  Ring stage i holds [K_i; Q_{i-1}],
+//            K~_{i-1}, V_i and the T_i tiles, for i = 0 .. n (n chunks).
+// The head's two value-tile CTAs run as a 2-CTA cluster: each loads T hi and lo from both
+// 128-byte slices of the o rows, and each overwrites its own slice with outputs, so a CTA stores
+// O_c only after its sibling has loaded stage c (a counter in its shared memory that the
+// sibling's producer raises through distributed shared memory).
+// Handshakes are mbarriers; every wait is bounded and followed by a group-wide vote, so a role
+// that gives up (recording OSDN_ERR_DEVICE_TIMEOUT) leaves its loop as a whole group and no named
+// barrier is left waiting.
 #pragma once
 
 #include <cuda.h>
@@ -43,13 +56,17 @@
 namespace osdn {
 
 struct TcSmem {
-    static constexpr uint32_t STAGE = 65536;          // [K;Q] 32K | K~ 16K | V 8K | packed T 8K
-    static constexpr uint32_t KQ = 0, KT = 32768, V = 49152, TP = 57344;
-    static constexpr uint32_t ZHI = 2 * STAGE;        // bf16 [T; P] hi / lo, K-major, 128 x 128 B
-    static constexpr uint32_t ZLO = ZHI + 16384;
-    static constexpr uint32_t SHI = ZLO + 16384;      // bf16 S^T hi / lo, MN-major, 128 x 128 B
+    // ring stage: [K;Q] 32K | K~ 16K | V 8K | T hi 8K | T lo 8K.  W = T R reads A as the 64 rows
+    // before each T tile followed by the tile ([V; T hi] and [T hi; T lo]), so W lands in
+    // accumulator lanes 64..127 and the rows in front, which stay unchanged while that MMA runs,
+    // reach only lanes 0..63, which nobody reads
+    static constexpr uint32_t STAGE = 73728;
+    static constexpr uint32_t KQ = 0, KT = 32768, V = 49152, THI = 57344, TLO = 65536;
+    static constexpr uint32_t XHI = 2 * STAGE;        // bf16 [X; P] hi / lo, K-major, 128 x 128 B
+    static constexpr uint32_t XLO = XHI + 16384;
+    static constexpr uint32_t SHI = XLO + 16384;      // bf16 S^T hi / lo, MN-major, 128 x 128 B
     static constexpr uint32_t SLO = SHI + 16384;
-    static constexpr uint32_t RHI = SLO + 16384;      // bf16 R then W, hi / lo, 64 x 128 B
+    static constexpr uint32_t RHI = SLO + 16384;      // bf16 R (then W) hi / lo, 64 x 128 B
     static constexpr uint32_t RLO = RHI + 8192;
     static constexpr uint32_t BAR = RLO + 8192;
     static constexpr uint32_t TMEM_SLOT = BAR + 128;
@@ -58,8 +75,8 @@ struct TcSmem {
 };
 static_assert(TcSmem::BYTES <= 232448, "shared memory");
 
-// Tensor-memory columns: S, D1 (double-buffered: a chunk's outputs are read during the next
-// chunk), D2, the prep's Gram.
+// Tensor-memory columns: S, D1 (double-buffered: chunk c+1's product is assembled while chunk c
+// is read), D2, the prep's Gram.
 constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 192, TC_COL_G = 256;
 constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr int TC_THREADS = 288;
@@ -85,7 +102,7 @@ __device__ __forceinline__ void st_row_split_bf16(uint8_t* hi, uint8_t* lo, uint
     }
 }
 
-// D (+)= [T; P] X over K = 64 tokens, as hi*hi + hi*lo + lo*hi: A = the K-major [T; P] tiles
+// D (+)= Z X over K = 64 tokens, as hi*hi + hi*lo + lo*hi: A = the K-major 128-row tiles of Z
 // (z[0] = hi, z[1] = lo), B = the MN-major 64 x 64 tiles of X (x[0] = hi, x[1] = lo).
 __device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, const uint32_t* x,
                                            uint32_t id, bool accumulate) {
@@ -99,6 +116,18 @@ __device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, c
                          (accumulate || p > 0 || s > 0) ? 1u : 0u);
 }
 
+// D = A S^T over K = 128 key channels with the two terms of S^T: A = a ring stage's K-major
+// [K; Q] tile (two 64-channel blocks 16 KB apart), B = the MN-major S^T tiles.
+__device__ __forceinline__ void mma_kq_state(uint32_t d_tmem, uint32_t a_kq, const uint32_t* s,
+                                             uint32_t id) {
+#pragma unroll
+    for (int p = 0; p < 2; ++p)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            tc::mma_bf16(d_tmem, tc::sw128_desc(a_kq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                         tc::sw128_desc(s[p] + k * 2048, 8192, 1024), id, (p | k) != 0);
+}
+
 template <int DV>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -108,6 +137,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
                     const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
     constexpr int DK = 128, BV = 64, C = 64, NVT = DV / BV;
+    static_assert(DV == 128, "the T hand-off uses the two 128-byte slices of a 256-byte o row");
     using L = TcSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
@@ -123,23 +153,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int nchunks = (int)((count + C - 1) / C);
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
-    uint64_t* tma_full = bars + 0;     // [2]
-    uint64_t* stage_empty = bars + 2;  // [2], two arrivals: chain and prep
-    uint64_t* zt_full = bars + 4;      // T rows of [T; P] written
-    uint64_t* zt_empty = bars + 5;     // T rows free (W computed)
-    uint64_t* zp_full = bars + 9;      // P rows written
-    uint64_t* zp_empty = bars + 10;    // P rows free (outputs computed)
-    uint64_t* w_ready = bars + 11;     // W of the chunk written (the output MMAs may start)
-    uint64_t* mma_c = bars + 6;        // chain MMAs on the state's path
-    uint64_t* mma_p = bars + 7;        // prep MMAs
-    uint64_t* mma_o = bars + 8;        // chain MMAs of the outputs
+    uint64_t* tma_full = bars + 0;     // [2] ring stage landed
+    uint64_t* stage_empty = bars + 2;  // [2] two arrivals: chain (W = T R done) and prep (Gram done)
+    uint64_t* zt_full = bars + 4;      // [2] the stage's T tiles complete (identity rows past the
+                                       // end); one per ring slot, so the prep cannot run a phase
+                                       // ahead of a stage the chain has not released
+    uint64_t* mma_c = bars + 6;        // W = T R
+    uint64_t* mma_p = bars + 7;        // the prep's Gram
+    uint64_t* mma_crit = bars + 8;     // D1 += [X; P] W (and everything the chain issued before)
+    uint64_t* mma_s = bars + 9;        // S^T += K~^T W
+    uint64_t* zxp_full = bars + 10;    // [X; P] tiles written
+    uint64_t* d1a_done = bars + 11;    // D1 = [K; Q] S^T of the next chunk
+    uint64_t* s_ready = bars + 12;     // the state's split written
+    uint64_t* w_done = bars + 13;      // W split written
+    uint64_t* o_free = bars + 14;      // a chunk's output rows read out of D1
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
-    uint8_t* ZHI = smem + L::ZHI;
-    uint8_t* ZLO = smem + L::ZLO;
-    uint8_t* SHI = smem + L::SHI;
-    uint8_t* SLO = smem + L::SLO;
-    uint8_t* RHI = smem + L::RHI;
-    uint8_t* RLO = smem + L::RLO;
+    // ring stages the sibling CTA (the head's other value tile) has loaded, written by the sibling
+    uint32_t* peer_loaded = tmem_slot + 2;
 
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, TC_TMEM_COLS);
@@ -150,177 +180,224 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(&tma_full[1], 1);
         mbar_init(&stage_empty[0], 2);
         mbar_init(&stage_empty[1], 2);
-        mbar_init(zt_full, 1);
-        mbar_init(zt_empty, 1);
-        mbar_init(zp_full, 1);
-        mbar_init(zp_empty, 1);
-        mbar_init(w_ready, 1);
+        mbar_init(&zt_full[0], 1);
+        mbar_init(&zt_full[1], 1);
         mbar_init(mma_c, 1);
         mbar_init(mma_p, 1);
-        mbar_init(mma_o, 1);
+        mbar_init(mma_crit, 1);
+        mbar_init(mma_s, 1);
+        mbar_init(zxp_full, 1);
+        mbar_init(d1a_done, 1);
+        mbar_init(s_ready, 1);
+        mbar_init(w_done, 1);
+        mbar_init(o_free, 1);
+        *peer_loaded = 0;
         tc::fence_mbar_init();
     }
     tc::fence_before_sync();
-    __syncthreads();
+    tc::cluster_sync();  // both CTAs of the pair initialised before either writes to the other
     tc::fence_after_sync();
-    if (tid == 0) {  // the [T; P] tiles start out free
-        mbar_arrive(zt_empty);
-        mbar_arrive(zp_empty);
-    }
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     auto chunk_len = [&](int ch) -> int {
         const int64_t rem = count - (int64_t)ch * C;
         return rem < C ? (int)rem : C;
     };
+    auto stage = [&](int i) { return smem + (i & 1) * L::STAGE; };
+    constexpr uint32_t ID_1 = tc::idesc(1, 0, 1, 128, 64);  // K-major A x MN-major B
+    constexpr uint32_t ID_3 = tc::idesc(1, 1, 1, 128, 64);  // K~^T x W
+    constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);  // [K; Q] x K~^T
+    const uint32_t aS[2] = {smem_u32(smem + L::SHI), smem_u32(smem + L::SLO)};
+    const uint32_t aR[2] = {smem_u32(smem + L::RHI), smem_u32(smem + L::RLO)};
 
     if (warp == 8) {
         // =========================================================== producer
-        // Lane 0 loads the chunk tiles into the 2-stage ring and issues each chunk's output
-        // MMAs (D1 += [T; P] W) once the chain has published W, so that the chain warps go
-        // straight on to the state split.
-        if ((tid & 31) == 0) {
+        // Lane 0 runs the ring's TMA loads and issues every MMA off the chain's critical path,
+        // each once its inputs are ready (a thread that issues MMAs stalls while the tensor pipe
+        // takes them, so the chain's own threads issue only the two groups they wait for):
+        //   S^T += K~_{j-1}^T W_{j-1}       after D1_j += [X_j; P_{j-1}] W_{j-1} completed
+        //   Gram [K_{j+1}; Q_j] K~_j^T      when stage j+1 has landed
+        //   D1_{j+1} = [K_{j+1}; Q_j] S_j^T once the prep has split S_j
+        if ((tid & 31) == 0 && nchunks > 0) {
             tc::prefetch_tmap(&tm_q);
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_kt);
             tc::prefetch_tmap(&tm_v);
             tc::prefetch_tmap(&tm_tp);
-            constexpr uint32_t ID_O = tc::idesc(1, 0, 1, 128, 64);
-            const uint32_t aZ[2] = {smem_u32(ZHI), smem_u32(ZLO)};
-            const uint32_t aR[2] = {smem_u32(RHI), smem_u32(RLO)};
             int pend[2] = {-1, -1};
-            int o_issued = 0;
-            auto load = [&](int ch) {
-                const int s = ch & 1;
-                uint8_t* st = smem + s * L::STAGE;
-                const int row = (int)(first + (int64_t)ch * C);
+            uint64_t* last_bar = nullptr;  // this thread's most recent MMA commit
+            uint32_t last_par = 0;
+            // stage i: K_i, V_i and the T_i tiles from the chunk's rows; Q_{i-1} and K~_{i-1} from
+            // the 64 rows before (a negative row reads the fill value; rows past the end are unused)
+            auto load = [&](int i) {
+                const int s = i & 1;
+                uint8_t* st = stage(i);
+                const int row = (int)(first + (int64_t)i * C), prow = row - C;
                 tc::mbar_expect_tx(&tma_full[s], L::STAGE);
                 tc::tma_load_3d(st + L::KQ + 0, &tm_k, 0, h, row, &tma_full[s]);
-                tc::tma_load_3d(st + L::KQ + 8192, &tm_q, 0, h, row, &tma_full[s]);
+                tc::tma_load_3d(st + L::KQ + 8192, &tm_q, 0, h, prow, &tma_full[s]);
                 tc::tma_load_3d(st + L::KQ + 16384, &tm_k, 64, h, row, &tma_full[s]);
-                tc::tma_load_3d(st + L::KQ + 24576, &tm_q, 64, h, row, &tma_full[s]);
-                tc::tma_load_3d(st + L::KT + 0, &tm_kt, 0, h, row, &tma_full[s]);
-                tc::tma_load_3d(st + L::KT + 8192, &tm_kt, 64, h, row, &tma_full[s]);
+                tc::tma_load_3d(st + L::KQ + 24576, &tm_q, 64, h, prow, &tma_full[s]);
+                tc::tma_load_3d(st + L::KT + 0, &tm_kt, 0, h, prow, &tma_full[s]);
+                tc::tma_load_3d(st + L::KT + 8192, &tm_kt, 64, h, prow, &tma_full[s]);
                 tc::tma_load_3d(st + L::V, &tm_v, c0, h, row, &tma_full[s]);
-                tc::tma_load_3d(st + L::TP, &tm_tp, 32 * vt, h, row, &tma_full[s]);
-                pend[s] = (ch >> 1) & 1;
+                tc::tma_load_3d(st + L::THI, &tm_tp, 0, h, row, &tma_full[s]);
+                tc::tma_load_3d(st + L::TLO, &tm_tp, 32, h, row, &tma_full[s]);
+                pend[s] = (i >> 1) & 1;
             };
-            for (int ch = 0; ch < nchunks && ch < 2; ++ch) load(ch);
-            for (int ch = 0; ch < nchunks; ++ch) {
-                if (!mbar_wait_bounded(w_ready, (uint32_t)ch & 1u, limit_ns)) break;
-                tc::fence_after_sync();
-                mma_split3(tmem + TC_COL_D1 + 64 * (ch & 1), aZ, aR, ID_O, true);
-                tc::mma_commit(mma_o);
-                ++o_issued;
-                if (ch + 2 < nchunks) {  // chunk ch's stage, once both roles released it
-                    if (!mbar_wait_bounded(&stage_empty[ch & 1], (uint32_t)(ch >> 1) & 1u, limit_ns)) break;
-                    load(ch + 2);
+            auto state_update = [&](int jj) {  // S^T += K~_jj^T W_jj (K~_jj sits in stage jj+1)
+                const uint32_t aKT = smem_u32(stage(jj + 1) + L::KT);
+#pragma unroll
+                for (int p = 0; p < 2; ++p)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(tmem + TC_COL_S, tc::sw128_desc(aKT + k * 2048, 8192, 1024),
+                                     tc::sw128_desc(aR[p] + k * 2048, 8192, 1024), ID_3, 1);
+                tc::mma_commit(mma_s);
+                last_bar = mma_s;
+                last_par = (uint32_t)jj & 1u;
+            };
+            // stage i loaded (its T tiles read from both CTAs' output slices): tell the sibling
+            const uint32_t peer_ctr = tc::cluster_map(smem_u32(peer_loaded), tc::cluster_rank() ^ 1u);
+            load(0);
+            load(1);
+            bool ok = mbar_wait_bounded(&tma_full[0], 0u, limit_ns);
+            if (ok) tc::st_cluster_release(peer_ctr, 1u);
+            for (int j = 0; j < nchunks && ok; ++j) {
+                const int i = j + 1;
+                if (j > 0) {
+                    if (!(ok = mbar_wait_bounded(mma_crit, (uint32_t)(j - 1) & 1u, limit_ns))) break;
+                    tc::fence_after_sync();
+                    state_update(j - 1);
                 }
+                if (!(ok = mbar_wait_bounded(&tma_full[i & 1], (uint32_t)(i >> 1) & 1u, limit_ns))) break;
+                tc::st_cluster_release(peer_ctr, (uint32_t)i + 1u);
+                {
+                    const uint32_t aKQ = smem_u32(stage(i) + L::KQ), aKT = smem_u32(stage(i) + L::KT);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        tc::mma_bf16(tmem + TC_COL_G, tc::sw128_desc(aKQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                                     tc::sw128_desc(aKT + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_G, k > 0);
+                    tc::mma_commit(mma_p);
+                    last_bar = mma_p;
+                    last_par = (uint32_t)j & 1u;
+                }
+                if (j > 0) {  // (the chain issued D1_0 and D1_1); the buffer's O_{j-1} has been read
+                    if (!(ok = mbar_wait_bounded(s_ready, (uint32_t)(j - 1) & 1u, limit_ns) &&
+                               mbar_wait_bounded(o_free, (uint32_t)(j - 1) & 1u, limit_ns)))
+                        break;
+                    tc::fence_after_sync();
+                    mma_kq_state(tmem + TC_COL_D1 + 64 * (i & 1), smem_u32(stage(i) + L::KQ), aS, ID_1);
+                    tc::mma_commit(d1a_done);
+                    last_bar = d1a_done;
+                    last_par = (uint32_t)j & 1u;
+                }
+                if (j + 2 <= nchunks) {  // stage j+2 once both roles are done with stage j
+                    if (!(ok = mbar_wait_bounded(&stage_empty[j & 1], (uint32_t)(j >> 1) & 1u, limit_ns))) break;
+                    load(j + 2);
+                }
+            }
+            if (ok && mbar_wait_bounded(mma_crit, (uint32_t)(nchunks - 1) & 1u, limit_ns)) {
+                tc::fence_after_sync();
+                state_update(nchunks - 1);
             }
             // let this CTA's own copies and MMAs land before the block can leave
             for (int s = 0; s < 2; ++s)
                 if (pend[s] >= 0) mbar_wait_bounded(&tma_full[s], (uint32_t)pend[s], limit_ns);
-            if (o_issued > 0) mbar_wait_bounded(mma_o, (uint32_t)(o_issued - 1) & 1u, limit_ns);
+            if (last_bar) mbar_wait_bounded(last_bar, last_par, limit_ns);
         }
     } else if (warp >= 4) {
         // =========================================================== prep
+        // Iteration j: the split of S_j once S^T += K~_{j-1}^T W_{j-1} has landed; [X_{j+1}; P_j]
+        // from the Gram; the T tiles of stage j+1 completed for a short chunk.
         const int t = tid - 128;  // 0..127 = tensor-memory lane
         const bool leader = t == 0;
-        constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);
-        bool pend = false;
-        uint32_t mphase = 0;
-        for (int ch = 0; ch < nchunks; ++ch) {
-            const int s = ch & 1;
-            if (group_any(2, 128, !mbar_wait_bounded(&tma_full[s], (uint32_t)(ch >> 1) & 1u, limit_ns))) break;
-            uint8_t* st = smem + s * L::STAGE;
-            if (leader) {
-                const uint32_t aKQ = smem_u32(st + L::KQ), aKT = smem_u32(st + L::KT);
-                tc::fence_after_sync();
+        bool bad = false;
+        auto finish_T = [&](int i) {  // rows past a short chunk's end: identity (hi), zero (lo)
+            const int len = chunk_len(i);
+            if (len < C && t >= len && t < C) {
+                uint8_t* st = stage(i);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    tc::mma_bf16(tmem + TC_COL_G, tc::sw128_desc(aKQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                                 tc::sw128_desc(aKT + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_G, k > 0);
-                tc::mma_commit(mma_p);
-                pend = true;
-            }
-            // row t of T from the packed strictly-lower copy (unit diagonal; identity rows past
-            // the chunk's end), while the Gram runs
-            float x[64];
-            if (t < 64) {
-                const float* tp = reinterpret_cast<const float*>(st + L::TP);
-                const int base = t * (t - 1) / 2;
-                const bool in = t < chunk_len(ch);
-#pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = (in && j < t) ? tp[base + j] : (j == t ? 1.f : 0.f);
-            }
-            if (group_any(2, 128, !mbar_wait_bounded(mma_p, mphase, limit_ns))) break;
-            mphase ^= 1u;
-            pend = false;
-            tc::fence_after_sync();
-            if (leader) mbar_arrive(&stage_empty[s]);  // the prep's last use of the stage
-            if (t >= 64) {  // P row t - 64 = tril(Q K~^T)
-                tc::tmem_ld64(tmem + lane + TC_COL_G, x);
-                const int r = t - 64;
-#pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = j <= r ? x[j] : 0.f;
-            }
-            // rows 0..63 (T) by warps 4-5 and rows 64..127 (P) by warps 6-7, each half as soon
-            // as the chain is done with its previous contents
-            const int half = t >> 6, hbar = 3 + half;
-            bool bad = group_any(hbar, 64, !mbar_wait_bounded(half ? zp_empty : zt_empty,
-                                                              (uint32_t)ch & 1u, limit_ns));
-            if (!bad) {
-                st_row_split_bf16(ZHI, ZLO, t, x);
+                for (int g = 0; g < 8; ++g) {
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    if ((t >> 3) == g) w[(t & 7) >> 1] = (t & 1) ? 0x3f800000u : 0x00003f80u;  // bf16 1.0
+                    const uint32_t off = tc::sw128_off((uint32_t)t, (uint32_t)g);
+                    *reinterpret_cast<uint4*>(st + L::THI + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(st + L::TLO + off) = make_uint4(0u, 0u, 0u, 0u);
+                }
                 tc::fence_async_smem();
             }
-            group_bar(hbar, 64);
-            if (!bad && (t & 63) == 0) mbar_arrive(half ? zp_full : zt_full);
-            if (group_any(2, 128, bad)) break;
+            group_bar(2, 128);
+            if (leader) {
+                mbar_arrive(&zt_full[i & 1]);
+                mbar_arrive(&stage_empty[i & 1]);  // the prep's last use of stage i
+            }
+        };
+        if (nchunks > 0) {
+            bad = group_any(2, 128, !mbar_wait_bounded(&tma_full[0], 0u, limit_ns));
+            if (!bad) finish_T(0);
         }
-        if (leader && pend) mbar_wait_bounded(mma_p, mphase, limit_ns);
+        for (int j = 0; j < nchunks && !bad; ++j) {
+            const int i = j + 1;
+            if (j > 0) {  // split S_j (its previous split was last read by D1_j, already complete)
+                if (group_any(2, 128, !mbar_wait_bounded(mma_s, (uint32_t)(j - 1) & 1u, limit_ns))) {
+                    bad = true;
+                    break;
+                }
+                tc::fence_after_sync();
+                float x[64];
+                tc::tmem_ld64(tmem + lane + TC_COL_S, x);
+                st_row_split_bf16(smem + L::SHI, smem + L::SLO, t, x);
+                tc::fence_async_smem();
+                tc::fence_before_sync();
+                group_bar(2, 128);
+                if (leader) mbar_arrive(s_ready);
+            }
+            // [X_{j+1}; P_j]: its tiles' previous contents were last read by D1_j += [X_j; P_{j-1}]
+            // W_{j-1}, which the state update waited for
+            if (group_any(2, 128, !mbar_wait_bounded(mma_p, (uint32_t)j & 1u, limit_ns))) {
+                bad = true;
+                break;
+            }
+            tc::fence_after_sync();
+            {  // lanes 0..63: X_{j+1} = K_{j+1} K~_j^T; lanes 64..127: P_j = tril(Q_j K~_j^T)
+                float x[64];
+                tc::tmem_ld64(tmem + lane + TC_COL_G, x);
+                if (t >= 64) {
+                    const int r = t - 64;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) x[c] = c <= r ? x[c] : 0.f;
+                }
+                st_row_split_bf16(smem + L::XHI, smem + L::XLO, t, x);
+                tc::fence_async_smem();
+            }
+            tc::fence_before_sync();
+            group_bar(2, 128);
+            if (leader) mbar_arrive(zxp_full);
+            if (i < nchunks) {  // once stage i's copies have landed
+                if (group_any(2, 128, !mbar_wait_bounded(&tma_full[i & 1], (uint32_t)(i >> 1) & 1u, limit_ns))) {
+                    bad = true;
+                    break;
+                }
+                finish_T(i);
+            }
+        }
     } else {
         // =========================================================== chain
-        // Per chunk c: D1[c&1] = [K;Q] S^T -> R -> W -> S^T += K~^T W (the state's path), and
-        // D1[c&1] += [T;P] W for the outputs, committed apart so the state split does not wait for
-        // them; chunk c's output rows are read and stored by warps 2-3 during chunk c+1's R step,
-        // when only warps 0-1 have work.
+        // Warps 0-1 (lanes 0..63, the chunk's token rows of D1): per chunk j, R_j from D1_j, the
+        // MMA W_j = T_j R_j, then D1_{j+1} += [X_{j+1}; P_j] W_j once warps 2-3 have split W_j.
+        // Warps 2-3 (lanes 64..127): the split of W_j (lanes 64..127 of D2) and the output rows
+        // O_j (lanes 64..127 of D1_{j+1}).  The two halves meet only through mbarriers.
         const int t = tid;  // 0..127 = tensor-memory lane
-        const bool leader = t == 0;
+        const bool lower = t < 64, leader = t == 0 || t == 64;
+        const int gbar = lower ? 1 : 3;  // each half's own named barrier
         const uint32_t t_S = tmem + lane + TC_COL_S, t_D2 = tmem + lane + TC_COL_D2;
-        constexpr uint32_t ID_1 = tc::idesc(1, 0, 1, 128, 64);  // [K;Q] x S^T and [T;P] x (R | W)
-        constexpr uint32_t ID_3 = tc::idesc(1, 1, 1, 128, 64);  // K~^T x W
-        const uint32_t aZ[2] = {smem_u32(ZHI), smem_u32(ZLO)};
-        const uint32_t aR[2] = {smem_u32(RHI), smem_u32(RLO)};
-        const uint32_t aS[2] = {smem_u32(SHI), smem_u32(SLO)};
-        bool pend = false;
-        uint32_t mphase = 0, ophase = 0;
+        const uint32_t aXP[2] = {smem_u32(smem + L::XHI), smem_u32(smem + L::XLO)};
         bool ok = true;
-        auto mma_wait = [&]() -> bool {
-            if (group_any(1, 128, !mbar_wait_bounded(mma_c, mphase, limit_ns))) return false;
-            mphase ^= 1u;
-            pend = false;
-            tc::fence_after_sync();
-            return true;
-        };
-        // o rows of chunk pc from D1[pc & 1] (warps 2-3: lanes 64..127 = the chunk's tokens)
-        auto store_o = [&](int pc) {
-            const int r = t - 64;
-            float x[64];
-            tc::tmem_ld64(tmem + lane + TC_COL_D1 + 64 * (pc & 1), x);
-            if (r < chunk_len(pc)) {
-                __nv_bfloat16* orow = o + ((first + (int64_t)pc * C + r) * H + h) * DV + c0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale * x[8 * j + 2 * e],
-                                                                        scale * x[8 * j + 2 * e + 1]);
-                        pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                    }
-                    *reinterpret_cast<uint4*>(orow + 8 * j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
+        uint64_t* last_bar = nullptr;  // the lower leader's most recent commit
+        uint32_t last_par = 0;
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return !group_any(gbar, 64, !mbar_wait_bounded(bar, parity, limit_ns));
         };
         // initial state: S^T lane i = key channel i, columns = this CTA's value channels
         {
@@ -330,131 +407,146 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
             for (int q = 0; q < 4; ++q) tc::tmem_st16(t_S + 16 * q, s0 + 16 * q);
             tc::tmem_st_wait();
-            st_row_split_bf16(SHI, SLO, t, s0);
+            st_row_split_bf16(smem + L::SHI, smem + L::SLO, t, s0);
             tc::fence_async_smem();
             tc::fence_before_sync();
-            group_bar(1, 128);
         }
-        float bnext = (t < 64 && nchunks > 0 && t < chunk_len(0)) ? __ldg(beta + (first + t) * H + h) : 0.f;
-        for (int ch = 0; ch < nchunks && ok; ++ch) {
-            const int s = ch & 1;
-            const int64_t cs = (int64_t)ch * C;
-            const uint32_t t_D1 = tmem + lane + TC_COL_D1 + 64 * s;
-            const float bt = bnext;
-            if (t < 64 && ch + 1 < nchunks)
-                bnext = t < chunk_len(ch + 1) ? __ldg(beta + (first + cs + C + t) * H + h) : 0.f;
-            uint8_t* st = smem + s * L::STAGE;
-            const uint32_t aKQ = smem_u32(st + L::KQ), aKT = smem_u32(st + L::KT);
-            if (group_any(1, 128, !mbar_wait_bounded(&tma_full[s], (uint32_t)(ch >> 1) & 1u, limit_ns))) {
-                ok = false;
-                break;
+        group_bar(1, 128);  // both halves' rows of the state split are written
+        if (lower) {
+            if (nchunks > 0) {  // D1_0 = [K_0; .] S_0^T and D1_1 = [K_1; Q_0] S_0^T
+                ok = wait_all(&tma_full[0], 0u) && wait_all(&tma_full[1], 0u);
+                if (ok && leader) {
+                    tc::fence_after_sync();
+                    mma_kq_state(tmem + TC_COL_D1, smem_u32(stage(0) + L::KQ), aS, ID_1);
+                    mma_kq_state(tmem + TC_COL_D1 + 64, smem_u32(stage(1) + L::KQ), aS, ID_1);
+                    tc::mma_commit(d1a_done);
+                    last_bar = d1a_done;
+                    last_par = 0;
+                }
             }
-            // ---- D1 = [K; Q] S^T  (two terms of S^T)
-            if (leader) {
+            float bnext = (nchunks > 0 && t < chunk_len(0)) ? __ldg(beta + (first + t) * H + h) : 0.f;
+            for (int j = 0; j < nchunks && ok; ++j) {
+                const int s = j & 1;
+                const float bt = bnext;
+                if (j + 1 < nchunks)
+                    bnext = t < chunk_len(j + 1) ? __ldg(beta + (first + (int64_t)(j + 1) * C + t) * H + h) : 0.f;
+                // D1_j complete (D1_0 alone, else [X_j; P_{j-1}] W_{j-1} on top of it), V_j landed
+                if (!(j == 0 ? wait_all(d1a_done, 0u) : wait_all(mma_crit, (uint32_t)(j - 1) & 1u)) ||
+                    !wait_all(&tma_full[s], (uint32_t)(j >> 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
                 tc::fence_after_sync();
+                float y[64];  // R = beta (V - K S^T), token row t
+                tc::tmem_ld64(tmem + lane + TC_COL_D1 + 64 * s, y);
+                const uint8_t* vtile = stage(j) + L::V;
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        tc::mma_bf16(tmem + TC_COL_D1 + 64 * s,
-                                     tc::sw128_desc(aKQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                                     tc::sw128_desc(aS[p] + k * 2048, 8192, 1024), ID_1, (p | k) != 0);
-                tc::mma_commit(mma_c);
-                pend = true;
-            }
-            if (!mma_wait()) { ok = false; break; }
-            if (t < 64) {  // R = beta (V - K S^T), token rows 0..63
-                float y[64];
-                tc::tmem_ld64(t_D1, y);
-                const uint8_t* vtile = st + L::V;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(vtile + tc::sw128_off(t, j));
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 raw = *reinterpret_cast<const uint4*>(vtile + tc::sw128_off(t, q));
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-                        y[8 * j + 2 * e] = bt * (vv.x - y[8 * j + 2 * e]);
-                        y[8 * j + 2 * e + 1] = bt * (vv.y - y[8 * j + 2 * e + 1]);
+                        y[8 * q + 2 * e] = bt * (vv.x - y[8 * q + 2 * e]);
+                        y[8 * q + 2 * e + 1] = bt * (vv.y - y[8 * q + 2 * e + 1]);
                     }
                 }
-                st_row_split_bf16(RHI, RLO, t, y);
+                // W_{j-1} (the R tiles' previous contents) has been read by the state update
+                if (j > 0 && !wait_all(mma_s, (uint32_t)(j - 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                st_row_split_bf16(smem + L::RHI, smem + L::RLO, t, y);
+                tc::fence_async_smem();
+                tc::fence_before_sync();
+                if (!wait_all(&zt_full[s], (uint32_t)(j >> 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                if (leader) {
+                    // [V; T hi] and [T hi; T lo]: the stage's T tiles preceded by 64 stable rows
+                    const uint32_t aT[2] = {smem_u32(stage(j) + L::THI) - 8192u, smem_u32(stage(j) + L::TLO) - 8192u};
+                    tc::fence_after_sync();
+                    mma_split3(tmem + TC_COL_D2, aT, aR, ID_1, false);  // lanes 64..127: W
+                    tc::mma_commit(mma_c);
+                    last_bar = mma_c;
+                    last_par = (uint32_t)j & 1u;
+                }
+                // W_j split by warps 2-3, [X_{j+1}; P_j] written, D1_{j+1} = [K_{j+1}; Q_j] S_j^T complete
+                if (!(wait_all(w_done, (uint32_t)j & 1u) && wait_all(zxp_full, (uint32_t)j & 1u) &&
+                      wait_all(d1a_done, (uint32_t)j & 1u))) {
+                    ok = false;
+                    break;
+                }
+                if (leader) {
+                    tc::fence_after_sync();
+                    mma_split3(tmem + TC_COL_D1 + 64 * ((j + 1) & 1), aXP, aR, ID_1, true);
+                    tc::mma_commit(mma_crit);
+                    last_bar = mma_crit;
+                    last_par = (uint32_t)j & 1u;
+                }
             }
-            tc::fence_async_smem();
-            tc::fence_before_sync();
-            if (group_any(1, 128, !mbar_wait_bounded(zt_full, (uint32_t)ch & 1u, limit_ns))) {
-                ok = false;
-                break;
-            }
-            // ---- D2 = [T; P] R  (rows 0..63: W)
-            if (leader) {
+        } else {
+            const int r = t - 64;  // row of W and of the output
+            for (int j = 0; j < nchunks && ok; ++j) {
+                // ---- W_j = lanes 64..127 of D2, into the R tiles (R_j has been consumed)
+                if (!wait_all(mma_c, (uint32_t)j & 1u)) {
+                    ok = false;
+                    break;
+                }
                 tc::fence_after_sync();
-                mma_split3(tmem + TC_COL_D2, aZ, aR, ID_1, false);
-                tc::mma_commit(mma_c);
-                pend = true;
-            }
-            if (!mma_wait()) { ok = false; break; }
-            if (leader) mbar_arrive(zt_empty);  // the T rows have been used
-            if (t < 64) {
-                float w[64];
-                tc::tmem_ld64(t_D2, w);
-                st_row_split_bf16(RHI, RLO, t, w);  // R is consumed: W takes its tiles
-            } else if (ch > 0) {
-                store_o(ch - 1);  // its output MMAs completed before this chunk's R
-            }
-            tc::fence_async_smem();
-            tc::fence_before_sync();
-            if (group_any(1, 128, !mbar_wait_bounded(zp_full, (uint32_t)ch & 1u, limit_ns))) {
-                ok = false;
-                break;
-            }
-            if (leader) mbar_arrive(w_ready);  // the producer warp issues the output MMAs
-            // ---- S^T += K~^T W (two terms of W); the outputs' D1 += [T; P] W is issued by the
-            //      producer warp and completes on the output barrier
-            if (leader) {
+                if (leader) mbar_arrive(&stage_empty[j & 1]);  // the chain's last use of stage j
+                {
+                    float w[64];
+                    tc::tmem_ld64(t_D2, w);
+                    st_row_split_bf16(smem + L::RHI, smem + L::RLO, r, w);
+                    tc::fence_async_smem();
+                }
+                tc::fence_before_sync();
+                group_bar(3, 64);
+                if (leader) mbar_arrive(w_done);
+                // ---- O_j = lanes 64..127 of D1_{j+1} once D1_{j+1} += [X_{j+1}; P_j] W_j landed and
+                //      the sibling CTA has loaded stage j (it reads T_j from this CTA's slice of o)
+                if (!wait_all(mma_crit, (uint32_t)j & 1u) ||
+                    group_any(3, 64, leader && !tc::wait_counter(smem_u32(peer_loaded), (uint32_t)j + 1u, limit_ns))) {
+                    ok = false;
+                    break;
+                }
                 tc::fence_after_sync();
-#pragma unroll
-                for (int p = 0; p < 2; ++p)
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(tmem + TC_COL_S, tc::sw128_desc(aKT + k * 2048, 8192, 1024),
-                                     tc::sw128_desc(aR[p] + k * 2048, 8192, 1024), ID_3, 1);
-                tc::mma_commit(mma_c);
-                pend = true;
-            }
-            if (!mma_wait()) { ok = false; break; }
-            {
                 float x[64];
-                tc::tmem_ld64(t_S, x);
-                st_row_split_bf16(SHI, SLO, t, x);
+                tc::tmem_ld64(tmem + lane + TC_COL_D1 + 64 * ((j + 1) & 1), x);
+                if (r < chunk_len(j)) {
+                    __nv_bfloat16* orow = o + ((first + (int64_t)j * C + r) * H + h) * DV + c0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale * x[8 * q + 2 * e],
+                                                                            scale * x[8 * q + 2 * e + 1]);
+                            pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                        *reinterpret_cast<uint4*>(orow + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+                tc::fence_before_sync();
+                group_bar(3, 64);
+                if (leader) mbar_arrive(o_free);  // D1_{j+1}'s output rows have been read
             }
-            // the output MMAs read the P rows, this chunk's tiles and W: wait for them before
-            // releasing those, and before the next chunk's R overwrites W
-            if (group_any(1, 128, !mbar_wait_bounded(mma_o, ophase, limit_ns))) {
-                ok = false;
-                break;
-            }
-            ophase ^= 1u;
-            tc::fence_after_sync();
-            if (leader) {
-                mbar_arrive(zp_empty);         // the P rows have been used
-                mbar_arrive(&stage_empty[s]);  // and this chunk's tiles
-            }
-            tc::fence_async_smem();
-            tc::fence_before_sync();
-            group_bar(1, 128);
         }
-        if (ok && nchunks > 0 && t >= 64) store_o(nchunks - 1);
+        // final state: both halves once the last state update has landed
+        if (ok && nchunks > 0) ok = wait_all(mma_s, (uint32_t)(nchunks - 1) & 1u);
         if (ok && ST) {
+            tc::fence_after_sync();
             float s1[64];
             tc::tmem_ld64(t_S, s1);
 #pragma unroll
             for (int c = 0; c < 64; ++c) ST[sbase + (int64_t)c * DK + t] = s1[c];
         }
-        if (leader && pend) mbar_wait_bounded(mma_c, mphase, limit_ns);
+        if (!ok && lower && leader && last_bar) mbar_wait_bounded(last_bar, last_par, limit_ns);
     }
     tc::fence_before_sync();
-    __syncthreads();
+    tc::cluster_sync();  // neither CTA leaves while the other may still write its counter
     if (warp == 0) tc::tmem_dealloc(tmem, TC_TMEM_COLS);
 }
 

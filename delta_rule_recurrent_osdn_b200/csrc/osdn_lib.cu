@@ -218,8 +218,8 @@ osdn_status_t launch_scan(const void* k, const float* beta, const float* r, floa
     return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, rho, cu, d, stream);
 }
 
-// 3-D fp32 view [rows][H][Dv / 2] of the bf16 output buffer; boxes of 32 values (one 64-channel
-// value tile's 128-byte slice of a row) x 1 head x 64 tokens: the packed WY factors.
+// 3-D fp32 view [rows][H][Dv / 2] of the bf16 output buffer; boxes of 32 values (one 128-byte
+// slice of a row) x 1 head x 64 tokens: the WY factor's bf16 hi / lo operand tiles.
 bool make_tp_map(CUtensorMap* m, const void* o, int Dv, int H, int64_t rows) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc || rows <= 0) return false;
@@ -258,9 +258,23 @@ osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, cons
     if (st != OSDN_OK) return st;
     auto kernel = chunk_fwd_tc_kernel<DV>;
     if (!set_smem(kernel, TcSmem::BYTES)) return OSDN_ERR_CUDA;
-    kernel<<<dim3((unsigned)ctas), dim3(TC_THREADS), TcSmem::BYTES, stream>>>(
-        mq, mk, mkt, mv, mtp, beta, scale, S0, static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T,
-        d.H, (long long)kWaitLimitNs);
+    // the head's two value-tile CTAs form a cluster (they share the WY hand-off in o)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = TcSmem::BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = DV / 64;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, mq, mk, mkt, mv, mtp, beta, scale, S0,
+                           static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T, d.H,
+                           (long long)kWaitLimitNs) != cudaSuccess)
+        return OSDN_ERR_CUDA;
     return launch_status();
 }
 
@@ -269,14 +283,11 @@ osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* 
                            const void* v, const float* beta, float scale, const float* S0,
                            void* o, float* ST, const int32_t* cu, const Dims& d,
                            cudaStream_t stream) {
-    // bf16 I/O with 128 key channels runs on the tensor cores; fp32 I/O, 64 key channels and
-    // token-free calls (states pass through) run the fp32 SIMT kernel.
+    // bf16 I/O with 128 key and 128 value channels runs on the tensor cores; fp32 I/O, 64-channel
+    // heads and token-free calls (states pass through) run the fp32 SIMT kernel.
     if constexpr (sizeof(IO) == 2) {
-        if (d.Dk == 128 && chunk == 64 && d.rows() > 0 && d.rows() < (int64_t(1) << 31)) {
-            if (d.Dv == 128)
-                return launch_chunk_tc<128>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
-            return launch_chunk_tc<64>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
-        }
+        if (d.Dk == 128 && d.Dv == 128 && chunk == 64 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
+            return launch_chunk_tc<128>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
     }
     if (d.Dk == 128 && d.Dv == 128)
         return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,

@@ -1,6 +1,7 @@
 // tc_ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the tensor-core path uses:
 // tensor memory (tcgen05.alloc/ld/st), tcgen05.mma issued from shared-memory descriptors,
-// tcgen05.commit to an mbarrier, and TMA tile loads (cp.async.bulk.tensor, no multicast).
+// tcgen05.commit to an mbarrier, thread-block cluster barriers and distributed-shared-memory
+// counters, and TMA tile loads (cp.async.bulk.tensor, no multicast).
 #pragma once
 
 #include <cuda.h>
@@ -118,6 +119,45 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
+}
+
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every CTA of the cluster; orders the CTAs' earlier shared-memory writes
+// before the later reads of all of them.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_release(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_cluster_acquire(uint32_t local) {
+    uint32_t v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(local) : "memory");
+    return v;
+}
+// Wait until the counter at `local` (written by another CTA of the cluster) reaches `target`,
+// for at most `limit_ns`; records OSDN_ERR_DEVICE_TIMEOUT and returns false otherwise.
+__device__ __forceinline__ bool wait_counter(uint32_t local, uint32_t target, int64_t limit_ns) {
+    if (ld_cluster_acquire(local) >= target) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (ld_cluster_acquire(local) >= target) return true;
+        if (global_ns() - t0 > static_cast<uint64_t>(limit_ns)) break;
+        __nanosleep(64);
+    }
+    record_status(OSDN_ERR_DEVICE_TIMEOUT);
+    return false;
 }
 
 // ---------------------------------------------------------------- TMA

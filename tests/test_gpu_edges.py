@@ -109,10 +109,22 @@ def test_chunk_size_invariance_fp32(ref):
         assert rel_err(a, b) <= 1e-5
 
 
+def _bf16_step(x):
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    ax = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 7)
+
+
 @pytest.mark.parametrize("io", ["bf16", "f32"])
 def test_state_chaining(io):
     """Two calls over the halves, the second starting from the first's S_T and d_T, equal one
-    call over the whole sequence."""
+    call over the whole sequence.
+
+    The fp32 path restarts bit-for-bit up to summation order.  The tensor-core path forms a
+    chunk's K S^T from the previous chunk's state and W when it continues a sequence, and
+    directly from S_0 when it starts one: the two agree to the split operands' precision (about
+    2^-16 of the state, bound 1e-4 of rms here), and each bf16 output may then round one step
+    apart."""
     inp = small(io, 256, B=1)
     full = gpu_fwd(inp)
     first = W.select(inp)
@@ -124,10 +136,17 @@ def test_state_chaining(io):
     second.beta, second.r = inp.beta[:, 128:], inp.r[:, 128:]
     second.S0, second.d0 = a[2].astype(np.float32), a[3].astype(np.float32)
     b = gpu_fwd(second)
-    tol = 2e-6 if io == "f32" else 0.0
-    assert rel_err(np.concatenate([a[0], b[0]], axis=1), full[0]) <= max(tol, 1e-6)
-    assert rel_err(b[2], full[2]) <= max(tol, 1e-6)
-    assert rel_err(b[3], full[3]) <= max(tol, 1e-6)
+    o2 = np.concatenate([a[0], b[0]], axis=1).astype(np.float64)
+    o1 = np.asarray(full[0], dtype=np.float64)
+    if io == "f32":
+        assert rel_err(o2, o1) <= 2e-6
+        assert rel_err(b[2], full[2]) <= 2e-6
+    else:
+        rms = np.sqrt(np.mean(o1 ** 2))
+        excess = np.abs(o2 - o1) - _bf16_step(np.maximum(np.abs(o1), np.abs(o2)))
+        assert excess.max() / rms <= 1e-4
+        assert rel_err(b[2], full[2]) <= 1e-4
+    assert rel_err(b[3], full[3]) <= 2e-6  # phase 1 restarts exactly up to summation order
 
 
 def test_no_apf_equals_unit_retention():
