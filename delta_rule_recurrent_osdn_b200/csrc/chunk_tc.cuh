@@ -75,9 +75,10 @@ struct TcSmem {
 };
 static_assert(TcSmem::BYTES <= 232448, "shared memory");
 
-// Tensor-memory columns: S, D1 (double-buffered: chunk c+1's product is assembled while chunk c
-// is read), D2, the prep's Gram.
-constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 192, TC_COL_G = 256;
+// Tensor-memory columns: S; D1 (two buffers: chunk c+1's product is assembled while chunk c is
+// read), D2 and the prep's Gram.  D1 and D2 are 128 columns wide: their MMAs take the hi and lo
+// terms of the right-hand operand side by side (N = 128), and a reader sums the two halves.
+constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 320, TC_COL_G = 448;
 constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr int TC_THREADS = 288;
 
@@ -102,30 +103,48 @@ __device__ __forceinline__ void st_row_split_bf16(uint8_t* hi, uint8_t* lo, uint
     }
 }
 
-// D (+)= Z X over K = 64 tokens, as hi*hi + hi*lo + lo*hi: A = the K-major 128-row tiles of Z
-// (z[0] = hi, z[1] = lo), B = the MN-major 64 x 64 tiles of X (x[0] = hi, x[1] = lo).
-__device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, const uint32_t* x,
-                                           uint32_t id, bool accumulate) {
-    const int pairs[3][2] = {{0, 0}, {0, 1}, {1, 0}};
+// D (+)= Z X over K = 64 tokens as Z_hi [X_hi | X_lo] (N = 128, columns 0..127 of D) + Z_lo X_hi
+// (columns 0..63): A = the K-major 128-row tiles of Z (z[0] = hi, z[1] = lo), B = the MN-major
+// 64 x 64 tiles of X with X_lo 8 KB after X_hi.  The two column halves of D sum to the product.
+__device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, uint32_t x_hi,
+                                           bool accumulate) {
+    constexpr uint32_t ID_W = tc::idesc(1, 0, 1, 128, 128), ID_N = tc::idesc(1, 0, 1, 128, 64);
 #pragma unroll
-    for (int p = 0; p < 3; ++p)
+    for (int s = 0; s < 4; ++s)
+        tc::mma_bf16(d_tmem, tc::sw128_desc(z[0] + s * 32, 16, 1024),
+                     tc::sw128_desc(x_hi + s * 2048, 8192, 1024), ID_W, (accumulate || s > 0) ? 1u : 0u);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            tc::mma_bf16(d_tmem, tc::sw128_desc(z[pairs[p][0]] + s * 32, 16, 1024),
-                         tc::sw128_desc(x[pairs[p][1]] + s * 2048, 8192, 1024), id,
-                         (accumulate || p > 0 || s > 0) ? 1u : 0u);
+    for (int s = 0; s < 4; ++s)
+        tc::mma_bf16(d_tmem, tc::sw128_desc(z[1] + s * 32, 16, 1024),
+                     tc::sw128_desc(x_hi + s * 2048, 8192, 1024), ID_N, 1u);
 }
 
-// D = A S^T over K = 128 key channels with the two terms of S^T: A = a ring stage's K-major
-// [K; Q] tile (two 64-channel blocks 16 KB apart), B = the MN-major S^T tiles.
-__device__ __forceinline__ void mma_kq_state(uint32_t d_tmem, uint32_t a_kq, const uint32_t* s,
-                                             uint32_t id) {
+// D = A [S_hi | S_lo]^T over K = 128 key channels (N = 128, the halves of D sum to A S^T): A = a
+// ring stage's K-major [K; Q] tile (two 64-channel blocks 16 KB apart), B = the MN-major S^T
+// tiles with the lo term 16 KB after the hi term.
+__device__ __forceinline__ void mma_kq_state(uint32_t d_tmem, uint32_t a_kq, uint32_t s_hi) {
+    constexpr uint32_t ID_W = tc::idesc(1, 0, 1, 128, 128);
 #pragma unroll
-    for (int p = 0; p < 2; ++p)
+    for (int k = 0; k < 8; ++k)
+        tc::mma_bf16(d_tmem, tc::sw128_desc(a_kq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                     tc::sw128_desc(s_hi + k * 2048, 16384, 1024), ID_W, k != 0);
+}
+
+// x[c] = D[c] + D[64 + c], c < 64: this thread's lane of a 128-column accumulator.
+__device__ __forceinline__ void tmem_ld64_sum(uint32_t taddr, float* x) {
+    tc::tmem_ld16(taddr + 0, x + 0);
+    tc::tmem_ld16(taddr + 16, x + 16);
+    tc::tmem_ld16(taddr + 32, x + 32);
+    tc::tmem_ld16(taddr + 48, x + 48);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            tc::mma_bf16(d_tmem, tc::sw128_desc(a_kq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                         tc::sw128_desc(s[p] + k * 2048, 8192, 1024), id, (p | k) != 0);
+    for (int h = 0; h < 2; ++h) {
+        float t[32];
+        tc::tmem_ld16(taddr + 64 + 32 * h, t);
+        tc::tmem_ld16(taddr + 80 + 32 * h, t + 16);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[32 * h + c] += t[c];
+    }
 }
 
 template <int DV>
@@ -204,7 +223,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         return rem < C ? (int)rem : C;
     };
     auto stage = [&](int i) { return smem + (i & 1) * L::STAGE; };
-    constexpr uint32_t ID_1 = tc::idesc(1, 0, 1, 128, 64);  // K-major A x MN-major B
     constexpr uint32_t ID_3 = tc::idesc(1, 1, 1, 128, 64);  // K~^T x W
     constexpr uint32_t ID_G = tc::idesc(1, 0, 0, 128, 64);  // [K; Q] x K~^T
     const uint32_t aS[2] = {smem_u32(smem + L::SHI), smem_u32(smem + L::SLO)};
@@ -287,7 +305,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                mbar_wait_bounded(o_free, (uint32_t)(j - 1) & 1u, limit_ns)))
                         break;
                     tc::fence_after_sync();
-                    mma_kq_state(tmem + TC_COL_D1 + 64 * (i & 1), smem_u32(stage(i) + L::KQ), aS, ID_1);
+                    mma_kq_state(tmem + TC_COL_D1 + 128 * (i & 1), smem_u32(stage(i) + L::KQ), aS[0]);
                     tc::mma_commit(d1a_done);
                     last_bar = d1a_done;
                     last_par = (uint32_t)j & 1u;
@@ -417,8 +435,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok = wait_all(&tma_full[0], 0u) && wait_all(&tma_full[1], 0u);
                 if (ok && leader) {
                     tc::fence_after_sync();
-                    mma_kq_state(tmem + TC_COL_D1, smem_u32(stage(0) + L::KQ), aS, ID_1);
-                    mma_kq_state(tmem + TC_COL_D1 + 64, smem_u32(stage(1) + L::KQ), aS, ID_1);
+                    mma_kq_state(tmem + TC_COL_D1, smem_u32(stage(0) + L::KQ), aS[0]);
+                    mma_kq_state(tmem + TC_COL_D1 + 128, smem_u32(stage(1) + L::KQ), aS[0]);
                     tc::mma_commit(d1a_done);
                     last_bar = d1a_done;
                     last_par = 0;
@@ -438,7 +456,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 tc::fence_after_sync();
                 float y[64];  // R = beta (V - K S^T), token row t
-                tc::tmem_ld64(tmem + lane + TC_COL_D1 + 64 * s, y);
+                tmem_ld64_sum(tmem + lane + TC_COL_D1 + 128 * s, y);
                 const uint8_t* vtile = stage(j) + L::V;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -467,7 +485,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     // [V; T hi] and [T hi; T lo]: the stage's T tiles preceded by 64 stable rows
                     const uint32_t aT[2] = {smem_u32(stage(j) + L::THI) - 8192u, smem_u32(stage(j) + L::TLO) - 8192u};
                     tc::fence_after_sync();
-                    mma_split3(tmem + TC_COL_D2, aT, aR, ID_1, false);  // lanes 64..127: W
+                    mma_split3(tmem + TC_COL_D2, aT, aR[0], false);  // lanes 64..127: W
                     tc::mma_commit(mma_c);
                     last_bar = mma_c;
                     last_par = (uint32_t)j & 1u;
@@ -480,7 +498,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (leader) {
                     tc::fence_after_sync();
-                    mma_split3(tmem + TC_COL_D1 + 64 * ((j + 1) & 1), aXP, aR, ID_1, true);
+                    mma_split3(tmem + TC_COL_D1 + 128 * ((j + 1) & 1), aXP, aR[0], true);
                     tc::mma_commit(mma_crit);
                     last_bar = mma_crit;
                     last_par = (uint32_t)j & 1u;
@@ -498,7 +516,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (leader) mbar_arrive(&stage_empty[j & 1]);  // the chain's last use of stage j
                 {
                     float w[64];
-                    tc::tmem_ld64(t_D2, w);
+                    tmem_ld64_sum(t_D2, w);
                     st_row_split_bf16(smem + L::RHI, smem + L::RLO, r, w);
                     tc::fence_async_smem();
                 }
@@ -514,7 +532,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 tc::fence_after_sync();
                 float x[64];
-                tc::tmem_ld64(tmem + lane + TC_COL_D1 + 64 * ((j + 1) & 1), x);
+                tmem_ld64_sum(tmem + lane + TC_COL_D1 + 128 * ((j + 1) & 1), x);
                 if (r < chunk_len(j)) {
                     __nv_bfloat16* orow = o + ((first + (int64_t)j * C + r) * H + h) * DV + c0;
 #pragma unroll
