@@ -22,12 +22,12 @@
 // [K; Q] S^T product run beside it, one chunk ahead of their use.  (A thread that issues MMAs
 // stalls while the tensor pipe accepts them, so who issues what is part of the schedule.)
 //
-// Precision.  Every computed MMA operand x is split into two bf16 terms, x = hi + lo (about 16
-// significant bits).  A product of an exact bf16 input (K, Q, K~) with a computed operand takes
+// Precision.  Every computed MMA operand x is split into two bf16 terms, x = hi + lo with
+// |x - hi - lo| <= 2^-16 |x| (split2_bf16: Veltkamp head, truncated residual).  A product of an exact bf16 input (K, Q, K~) with a computed operand takes
 // two MMAs (hi, lo); a product of two computed operands ([T; .] or [X; P] with R or W) takes
 // three (hi*hi + hi*lo + lo*hi).  In a CPU emulation of this chunk algorithm against the oracle,
 // plain bf16 operands gave 1.5-2.5% max/rms error on o and S_T for the 340M and 1.3B workloads,
-// and single-term tf32 products 0.25-0.46%; the split scheme is at the fp32 rounding level.
+// and single-term tf32 products 0.25-0.46%; the split scheme is within 1e-4 of the oracle.
 //
 // Warp roles (one CTA per (sequence, head, 64 value channels), 288 threads):
 //   chain    warps 0-3: R, W = T R, the [X; P] W product and the output rows (thread t owns
@@ -82,21 +82,15 @@ constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 320, TC_COL_G = 448
 constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr int TC_THREADS = 288;
 
-// Split a 64-value fp32 row into bf16 hi + lo and write both rows (128 B each, swizzled).
+// Split a 64-value fp32 row into bf16 hi + lo (split2_bf16) and write both rows (128 B each,
+// swizzled).
 __device__ __forceinline__ void st_row_split_bf16(uint8_t* hi, uint8_t* lo, uint32_t row,
                                                   const float* x) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         uint32_t h[4], l[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float a = x[8 * j + 2 * e], b = x[8 * j + 2 * e + 1];
-            const __nv_bfloat162 ha = __floats2bfloat162_rn(a, b);
-            const float2 hf = __bfloat1622float2(ha);
-            const __nv_bfloat162 la = __floats2bfloat162_rn(a - hf.x, b - hf.y);
-            h[e] = *reinterpret_cast<const uint32_t*>(&ha);
-            l[e] = *reinterpret_cast<const uint32_t*>(&la);
-        }
+        for (int e = 0; e < 4; ++e) split2_bf16(x[8 * j + 2 * e], x[8 * j + 2 * e + 1], h[e], l[e]);
         const uint32_t off = tc::sw128_off(row, j);
         *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
         *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
@@ -109,14 +103,14 @@ __device__ __forceinline__ void st_row_split_bf16(uint8_t* hi, uint8_t* lo, uint
 __device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, uint32_t x_hi,
                                            bool accumulate) {
     constexpr uint32_t ID_W = tc::idesc(1, 0, 1, 128, 128), ID_N = tc::idesc(1, 0, 1, 128, 64);
-#pragma unroll
-    for (int s = 0; s < 4; ++s)
-        tc::mma_bf16(d_tmem, tc::sw128_desc(z[0] + s * 32, 16, 1024),
-                     tc::sw128_desc(x_hi + s * 2048, 8192, 1024), ID_W, (accumulate || s > 0) ? 1u : 0u);
-#pragma unroll
-    for (int s = 0; s < 4; ++s)
-        tc::mma_bf16(d_tmem, tc::sw128_desc(z[1] + s * 32, 16, 1024),
-                     tc::sw128_desc(x_hi + s * 2048, 8192, 1024), ID_N, 1u);
+    // rolled: issue is paced by the tensor pipe, and the roles share the instruction cache
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+        const int s = i & 3, lo = i >> 2;
+        tc::mma_bf16(d_tmem, tc::sw128_desc(z[lo] + s * 32, 16, 1024),
+                     tc::sw128_desc(x_hi + s * 2048, 8192, 1024), lo ? ID_N : ID_W,
+                     (accumulate || i > 0) ? 1u : 0u);
+    }
 }
 
 // D = A [S_hi | S_lo]^T over K = 128 key channels (N = 128, the halves of D sum to A S^T): A = a
@@ -124,7 +118,7 @@ __device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, u
 // tiles with the lo term 16 KB after the hi term.
 __device__ __forceinline__ void mma_kq_state(uint32_t d_tmem, uint32_t a_kq, uint32_t s_hi) {
     constexpr uint32_t ID_W = tc::idesc(1, 0, 1, 128, 128);
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < 8; ++k)
         tc::mma_bf16(d_tmem, tc::sw128_desc(a_kq + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
                      tc::sw128_desc(s_hi + k * 2048, 16384, 1024), ID_W, k != 0);
@@ -357,41 +351,33 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         for (int j = 0; j < nchunks && !bad; ++j) {
             const int i = j + 1;
-            if (j > 0) {  // split S_j (its previous split was last read by D1_j, already complete)
-                if (group_any(2, 128, !mbar_wait_bounded(mma_s, (uint32_t)(j - 1) & 1u, limit_ns))) {
+            // job 0 (j > 0): split S_j once S^T += K~_{j-1}^T W_{j-1} has landed (its previous split
+            // was last read by D1_j, already complete); job 1: [X_{j+1}; P_j] from the Gram (lanes
+            // 0..63: X_{j+1} = K_{j+1} K~_j^T; lanes 64..127: P_j = tril(Q_j K~_j^T)), whose tiles'
+            // previous contents were last read by D1_j += [X_j; P_{j-1}] W_{j-1}, which the state
+            // update waited for.  One code body for both (the roles share the instruction cache).
+#pragma unroll 1
+            for (int job = j > 0 ? 0 : 1; job < 2; ++job) {
+                uint64_t* bar = job ? mma_p : mma_s;
+                if (group_any(2, 128, !mbar_wait_bounded(bar, (uint32_t)(job ? j : j - 1) & 1u, limit_ns))) {
                     bad = true;
                     break;
                 }
                 tc::fence_after_sync();
                 float x[64];
-                tc::tmem_ld64(tmem + lane + TC_COL_S, x);
-                st_row_split_bf16(smem + L::SHI, smem + L::SLO, t, x);
-                tc::fence_async_smem();
-                tc::fence_before_sync();
-                group_bar(2, 128);
-                if (leader) mbar_arrive(s_ready);
-            }
-            // [X_{j+1}; P_j]: its tiles' previous contents were last read by D1_j += [X_j; P_{j-1}]
-            // W_{j-1}, which the state update waited for
-            if (group_any(2, 128, !mbar_wait_bounded(mma_p, (uint32_t)j & 1u, limit_ns))) {
-                bad = true;
-                break;
-            }
-            tc::fence_after_sync();
-            {  // lanes 0..63: X_{j+1} = K_{j+1} K~_j^T; lanes 64..127: P_j = tril(Q_j K~_j^T)
-                float x[64];
-                tc::tmem_ld64(tmem + lane + TC_COL_G, x);
-                if (t >= 64) {
+                tc::tmem_ld64(tmem + lane + (job ? TC_COL_G : TC_COL_S), x);
+                if (job && t >= 64) {
                     const int r = t - 64;
 #pragma unroll
                     for (int c = 0; c < 64; ++c) x[c] = c <= r ? x[c] : 0.f;
                 }
-                st_row_split_bf16(smem + L::XHI, smem + L::XLO, t, x);
+                st_row_split_bf16(smem + (job ? L::XHI : L::SHI), smem + (job ? L::XLO : L::SLO), t, x);
                 tc::fence_async_smem();
+                tc::fence_before_sync();
+                group_bar(2, 128);
+                if (leader) mbar_arrive(job ? zxp_full : s_ready);
             }
-            tc::fence_before_sync();
-            group_bar(2, 128);
-            if (leader) mbar_arrive(zxp_full);
+            if (bad) break;
             if (i < nchunks) {  // once stage i's copies have landed
                 if (group_any(2, 128, !mbar_wait_bounded(&tma_full[i & 1], (uint32_t)(i >> 1) & 1u, limit_ns))) {
                     bad = true;
@@ -416,6 +402,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint32_t last_par = 0;
         auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
             return !group_any(gbar, 64, !mbar_wait_bounded(bar, parity, limit_ns));
+        };
+        // two barriers, one vote
+        auto wait_all2 = [&](uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1) -> bool {
+            const bool got = mbar_wait_bounded(b0, p0, limit_ns) && mbar_wait_bounded(b1, p1, limit_ns);
+            return !group_any(gbar, 64, !got);
         };
         // initial state: S^T lane i = key channel i, columns = this CTA's value channels
         {
@@ -449,8 +440,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (j + 1 < nchunks)
                     bnext = t < chunk_len(j + 1) ? __ldg(beta + (first + (int64_t)(j + 1) * C + t) * H + h) : 0.f;
                 // D1_j complete (D1_0 alone, else [X_j; P_{j-1}] W_{j-1} on top of it), V_j landed
-                if (!(j == 0 ? wait_all(d1a_done, 0u) : wait_all(mma_crit, (uint32_t)(j - 1) & 1u)) ||
-                    !wait_all(&tma_full[s], (uint32_t)(j >> 1) & 1u)) {
+                if (!wait_all2(j == 0 ? d1a_done : mma_crit, (uint32_t)(j == 0 ? 0 : j - 1) & 1u,
+                               &tma_full[s], (uint32_t)(j >> 1) & 1u)) {
                     ok = false;
                     break;
                 }
@@ -491,8 +482,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     last_par = (uint32_t)j & 1u;
                 }
                 // W_j split by warps 2-3, [X_{j+1}; P_j] written, D1_{j+1} = [K_{j+1}; Q_j] S_j^T complete
-                if (!(wait_all(w_done, (uint32_t)j & 1u) && wait_all(zxp_full, (uint32_t)j & 1u) &&
-                      wait_all(d1a_done, (uint32_t)j & 1u))) {
+                const bool got = mbar_wait_bounded(w_done, (uint32_t)j & 1u, limit_ns) &&
+                                 mbar_wait_bounded(zxp_full, (uint32_t)j & 1u, limit_ns) &&
+                                 mbar_wait_bounded(d1a_done, (uint32_t)j & 1u, limit_ns);
+                if (group_any(gbar, 64, !got)) {
                     ok = false;
                     break;
                 }
