@@ -23,11 +23,12 @@
 // stalls while the tensor pipe accepts them, so who issues what is part of the schedule.)
 //
 // Precision.  Every computed MMA operand x is split into two bf16 terms, x = hi + lo with
-// |x - hi - lo| <= 2^-16 |x| (split2_bf16: Veltkamp head, truncated residual).  A product of an exact bf16 input (K, Q, K~) with a computed operand takes
-// two MMAs (hi, lo); a product of two computed operands ([T; .] or [X; P] with R or W) takes
-// three (hi*hi + hi*lo + lo*hi).  In a CPU emulation of this chunk algorithm against the oracle,
-// plain bf16 operands gave 1.5-2.5% max/rms error on o and S_T for the 340M and 1.3B workloads,
-// and single-term tf32 products 0.25-0.46%; the split scheme is within 1e-4 of the oracle.
+// |x - hi - lo| <= 2^-16 |x| (split2_bf16: Veltkamp head, truncated residual).  A product of an
+// exact bf16 input (K, Q, K~) with a computed operand takes two MMAs (hi, lo); a product of two
+// computed operands ([T; .] or [X; P] with R or W) takes three (hi*hi + hi*lo + lo*hi).  In a
+// CPU emulation of this chunk algorithm against the oracle, plain bf16 operands gave 1.5-2.5%
+// max/rms error on o and S_T for the 340M and 1.3B workloads, and single-term tf32 products
+// 0.25-0.46%; the split scheme is within 1e-4 of the oracle.
 //
 // Warp roles (one CTA per (sequence, head, 64 value channels), 288 threads):
 //   chain    warps 0-3: R, W = T R, the [X; P] W product and the output rows (thread t owns
