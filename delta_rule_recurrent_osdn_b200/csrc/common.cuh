@@ -37,21 +37,6 @@ __device__ __forceinline__ bool seq_range(const int32_t* __restrict__ cu, int n,
     return true;
 }
 
-// Two fp32 values as bf16 MMA operand terms, x = hi + lo with about 16 significant bits: hi is
-// the 8-significant-bit head of x by Veltkamp's splitting (t = (2^16 + 1) x, hi = t - (t - x),
-// exactly representable in bf16, so its bf16 bits are the upper half of its fp32 bits); lo =
-// x - hi is exact in fp32 and keeps its upper half, so |x - hi - lo| <= 2^-16 |x|.  Two-wide fp32
-// arithmetic and byte permutes only.  Returns the packed bf16x2 words (a in the low half).
-__device__ __forceinline__ void split2_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const float2 sig = make_float2(65537.f, 65537.f), m1 = make_float2(-1.f, -1.f);
-    const float2 xv = make_float2(a, b);
-    const float2 tv = __fmul2_rn(sig, xv);
-    const float2 hv = __ffma2_rn(__ffma2_rn(xv, m1, tv), m1, tv);
-    const float2 lv = __ffma2_rn(hv, m1, xv);
-    hi = __byte_perm(__float_as_uint(hv.x), __float_as_uint(hv.y), 0x7632);
-    lo = __byte_perm(__float_as_uint(lv.x), __float_as_uint(lv.y), 0x7632);
-}
-
 // ---- io dtype traits --------------------------------------------------------------------
 template <typename IO> struct io_traits;
 
