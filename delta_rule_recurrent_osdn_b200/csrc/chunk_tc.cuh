@@ -28,7 +28,8 @@
 // computed operands ([T; .] or [X; P] with R or W) takes three (hi*hi + hi*lo + lo*hi).  In a
 // CPU emulation of this chunk algorithm against the oracle, plain bf16 operands gave 1.5-2.5%
 // max/rms error on o and S_T for the 340M and 1.3B workloads, and single-term tf32 products
-// 0.25-0.46%; the split scheme is within 1e-4 of the oracle.
+// 0.25-0.46%; the split scheme's own error, at the 2^-16 level per operand, lies far below the
+// bf16 rounding of the inputs and outputs.
 //
 // Warp roles (one CTA per (sequence, head, 64 value channels), 288 threads):
 //   chain    warps 0-3: R, W = T R, the [X; P] W product and the output rows (thread t owns
