@@ -1,5 +1,6 @@
 /*
- * osdn_ref.c -- fp64 CPU oracle for the Online Scaled DeltaNet (OSDN) forward pass.
+ * osdn_ref.c -- fp64 CPU oracle for the Online Scaled DeltaNet (OSDN) forward pass and, by
+ * reverse-mode differentiation of the same token loop, its gradient (osdn_ref_bwd).
  *
  * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously correct statement of what
  * the GPU library computes.  Only the tests, the smoke check and the benchmark's CPU
@@ -220,4 +221,176 @@ void osdn_ref_fwd(const double* q, const double* k, const double* v, const doubl
             free(S);
         }
     }
+}
+
+/* ---------------------------------------------------------------------------------
+ * Gradient of the forward pass: reverse-mode differentiation of the token loop of
+ * osdn_ref_fwd, step by step in reverse order (the pages give no backward pass; this is
+ * the chain rule applied to the forward steps above, nothing else).  For
+ *   L = <dO, o> + <dST, S_T> + <ddT, d_T>
+ * it returns dL/dq, dL/dk, dL/dv, dL/dbeta, dL/dr (when r is non-NULL), dL/deta (one
+ * scalar over the whole batch), dL/dS0 and dL/dd0.  dST and ddT may be NULL (zero).
+ * Every token's state is kept for the reverse sweep, so this is for small problems.
+ * Per token, with S, d the state before the token and a = k (.) k, n = ||k||^2:
+ *   s = <d, a>, w = d (.) k, u = v - S k, S' = S + beta u w^T, o = scale S' q,
+ *   g = eta beta (1 - beta s) / n (0 when n == 0), d' = r d + g a.
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_bwd(const double* q, const double* k, const double* v, const double* beta,
+                  const double* r, double eta, const double* d0, const double* S0, double scale,
+                  const double* dO, const double* dST, const double* ddT, double* dq, double* dk,
+                  double* dv, double* dbeta, double* dr, double* deta, double* dS0, double* dd0,
+                  const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                  int32_t Dk, int32_t Dv) {
+    const int32_t N = cu_seqlens ? num_seqs : B;
+    const int64_t SZ = (int64_t)Dv * Dk;
+    double eta_total = 0.0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(+ : eta_total)
+    for (int32_t n = 0; n < N; ++n) {
+        for (int32_t h = 0; h < H; ++h) {
+            int64_t first, count;
+            seq_bounds(n, cu_seqlens, T, &first, &count);
+            const int64_t sbase = ((int64_t)n * H + h) * SZ;
+            const int64_t dbase = ((int64_t)n * H + h) * Dk;
+            /* states before each token: Sall[c], dall[c]; after the last token: index count */
+            double* Sall = (double*)malloc(sizeof(double) * (count + 1) * SZ);
+            double* dall = (double*)malloc(sizeof(double) * (count + 1) * Dk);
+            double* w = (double*)malloc(sizeof(double) * Dk);
+            double* u = (double*)malloc(sizeof(double) * Dv);
+            double* gS = (double*)malloc(sizeof(double) * SZ);
+            double* gd = (double*)malloc(sizeof(double) * Dk);
+            double* gdp = (double*)malloc(sizeof(double) * Dk);
+            double* ga = (double*)malloc(sizeof(double) * Dk);
+            double* gk = (double*)malloc(sizeof(double) * Dk);
+            double* gw = (double*)malloc(sizeof(double) * Dk);
+            double* gu = (double*)malloc(sizeof(double) * Dv);
+            for (int64_t e = 0; e < SZ; ++e) Sall[e] = S0 ? S0[sbase + e] : 0.0;
+            for (int32_t i = 0; i < Dk; ++i) dall[i] = d0 ? d0[dbase + i] : 1.0;
+            /* forward sweep (the same steps as osdn_ref_fwd) */
+            for (int64_t c = 0; c < count; ++c) {
+                const int64_t th = (first + c) * H + h;
+                const double* kt = k + th * Dk;
+                const double* vt = v + th * Dv;
+                const double bt = beta[th], rt = r ? r[th] : 1.0;
+                const double* S = Sall + c * SZ;
+                const double* d = dall + c * Dk;
+                double* Sn = Sall + (c + 1) * SZ;
+                double* dn = dall + (c + 1) * Dk;
+                double knorm2 = 0.0, s = 0.0;
+                for (int32_t i = 0; i < Dk; ++i) {
+                    knorm2 += kt[i] * kt[i];
+                    s += d[i] * kt[i] * kt[i];
+                    w[i] = d[i] * kt[i];
+                }
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double sk = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) sk += S[(int64_t)j * Dk + i] * kt[i];
+                    u[j] = vt[j] - sk;
+                }
+                for (int32_t j = 0; j < Dv; ++j)
+                    for (int32_t i = 0; i < Dk; ++i)
+                        Sn[(int64_t)j * Dk + i] = S[(int64_t)j * Dk + i] + bt * u[j] * w[i];
+                const double g = knorm2 > 0.0 ? eta * bt * (1.0 - bt * s) / knorm2 : 0.0;
+                for (int32_t i = 0; i < Dk; ++i) dn[i] = rt * d[i] + g * kt[i] * kt[i];
+            }
+            /* reverse sweep: gS, gd are the adjoints of the state after token c */
+            for (int64_t e = 0; e < SZ; ++e) gS[e] = dST ? dST[sbase + e] : 0.0;
+            for (int32_t i = 0; i < Dk; ++i) gd[i] = ddT ? ddT[dbase + i] : 0.0;
+            for (int64_t c = count - 1; c >= 0; --c) {
+                const int64_t th = (first + c) * H + h;
+                const double* kt = k + th * Dk;
+                const double* qt = q + th * Dk;
+                const double* vt = v + th * Dv;
+                const double* gOt = dO + th * Dv;
+                const double bt = beta[th], rt = r ? r[th] : 1.0;
+                const double* S = Sall + c * SZ;
+                const double* d = dall + c * Dk;
+                const double* Sn = Sall + (c + 1) * SZ;
+                double knorm2 = 0.0, s = 0.0;
+                for (int32_t i = 0; i < Dk; ++i) {
+                    knorm2 += kt[i] * kt[i];
+                    s += d[i] * kt[i] * kt[i];
+                    w[i] = d[i] * kt[i];
+                }
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double sk = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) sk += S[(int64_t)j * Dk + i] * kt[i];
+                    u[j] = vt[j] - sk;
+                }
+                const double g = knorm2 > 0.0 ? eta * bt * (1.0 - bt * s) / knorm2 : 0.0;
+                double gbeta = 0.0;
+                /* o = scale S' q */
+                for (int32_t i = 0; i < Dk; ++i) {
+                    double acc = 0.0;
+                    for (int32_t j = 0; j < Dv; ++j) acc += Sn[(int64_t)j * Dk + i] * gOt[j];
+                    dq[th * Dk + i] = scale * acc;
+                }
+                for (int32_t j = 0; j < Dv; ++j)
+                    for (int32_t i = 0; i < Dk; ++i) gS[(int64_t)j * Dk + i] += scale * gOt[j] * qt[i];
+                /* d' = r d + g a */
+                double gr = 0.0, gg = 0.0;
+                for (int32_t i = 0; i < Dk; ++i) {
+                    gr += gd[i] * d[i];
+                    gg += gd[i] * kt[i] * kt[i];
+                    ga[i] = g * gd[i];
+                    gdp[i] = rt * gd[i];
+                }
+                if (dr) dr[th] = gr;
+                if (knorm2 > 0.0) {  /* g = eta beta (1 - beta s) / n */
+                    eta_total += gg * bt * (1.0 - bt * s) / knorm2;
+                    gbeta += gg * eta * (1.0 - 2.0 * bt * s) / knorm2;
+                    const double gs = gg * (-eta * bt * bt / knorm2);
+                    const double gn = gg * (-g / knorm2);
+                    for (int32_t i = 0; i < Dk; ++i) {
+                        gdp[i] += gs * kt[i] * kt[i];  /* s = <d, a> */
+                        ga[i] += gs * d[i] + gn;       /* s and n = sum of a */
+                    }
+                }
+                /* S' = S + beta u w^T */
+                for (int32_t j = 0; j < Dv; ++j) {
+                    double acc = 0.0;
+                    for (int32_t i = 0; i < Dk; ++i) {
+                        gbeta += gS[(int64_t)j * Dk + i] * u[j] * w[i];
+                        acc += gS[(int64_t)j * Dk + i] * w[i];
+                    }
+                    gu[j] = bt * acc;
+                }
+                for (int32_t i = 0; i < Dk; ++i) {
+                    double acc = 0.0;
+                    for (int32_t j = 0; j < Dv; ++j) acc += gS[(int64_t)j * Dk + i] * u[j];
+                    gw[i] = bt * acc;
+                }
+                /* u = v - S k */
+                for (int32_t j = 0; j < Dv; ++j) dv[th * Dv + j] = gu[j];
+                for (int32_t i = 0; i < Dk; ++i) {
+                    double acc = 0.0;
+                    for (int32_t j = 0; j < Dv; ++j) acc += gu[j] * S[(int64_t)j * Dk + i];
+                    gk[i] = -acc;
+                }
+                for (int32_t j = 0; j < Dv; ++j)
+                    for (int32_t i = 0; i < Dk; ++i) gS[(int64_t)j * Dk + i] -= gu[j] * kt[i];
+                /* w = d (.) k and a = k (.) k */
+                for (int32_t i = 0; i < Dk; ++i) {
+                    gdp[i] += gw[i] * kt[i];
+                    gk[i] += gw[i] * d[i] + 2.0 * kt[i] * ga[i];
+                    dk[th * Dk + i] = gk[i];
+                    gd[i] = gdp[i];
+                }
+                dbeta[th] = gbeta;
+            }
+            for (int64_t e = 0; e < SZ; ++e) dS0[sbase + e] = gS[e];
+            for (int32_t i = 0; i < Dk; ++i) dd0[dbase + i] = gd[i];
+            free(gu);
+            free(gw);
+            free(gk);
+            free(ga);
+            free(gdp);
+            free(gd);
+            free(gS);
+            free(u);
+            free(w);
+            free(dall);
+            free(Sall);
+        }
+    }
+    if (deta) *deta = eta_total;
 }

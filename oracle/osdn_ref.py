@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for the OSDN forward pass -- TEST INFRASTRUCTURE ONLY.
+"""fp64 CPU oracle for the OSDN forward pass and its gradient -- TEST INFRASTRUCTURE ONLY.
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
 import this module.  The product path (the CUDA library and its Python binding) never
@@ -97,6 +97,10 @@ class Oracle:
             _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _D, _D, _D, _I,
             _i32, _i32, _i32, _i32, _i32, _i32]
         lib.osdn_ref_fwd.restype = None
+        lib.osdn_ref_bwd.argtypes = [
+            _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _D, _D, _D, _D, _D,
+            _D, _D, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32, _i32]
+        lib.osdn_ref_bwd.restype = None
         self.lib = lib
 
     def set_threads(self, n: int = 0) -> int:
@@ -154,6 +158,33 @@ class Oracle:
         return o, k_tilde, ST, dT
 
 
+    def bwd(self, q, k, v, beta, dO, r=None, eta=0.0, d0=None, S0=None, scale=1.0, dST=None,
+            ddT=None, cu_seqlens=None):
+        """Gradient of L = <dO, o> + <dST, S_T> + <ddT, d_T> for the forward pass ``fwd`` with
+        the same arguments, by reverse-mode differentiation of its token loop.  Returns a dict
+        with dq, dk, dv, dbeta, dr (None without r), deta (float), dS0, dd0."""
+        q, k, v, beta, r, d0, S0, dO, dST, ddT = map(_f64, (q, k, v, beta, r, d0, S0, dO, dST, ddT))
+        cu, cup = _cu(cu_seqlens)
+        B, T, H, Dk, N = _dims(k, cu)
+        Dv = v.shape[-1]
+        assert q.shape == k.shape and v.shape == (B, T, H, Dv) and beta.shape == (B, T, H)
+        assert dO.shape == v.shape and (r is None or r.shape == (B, T, H))
+        assert d0 is None or d0.shape == (N, H, Dk)
+        assert S0 is None or S0.shape == (N, H, Dv, Dk)
+        assert dST is None or dST.shape == (N, H, Dv, Dk)
+        assert ddT is None or ddT.shape == (N, H, Dk)
+        g = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
+             "dbeta": np.zeros_like(beta), "dr": None if r is None else np.zeros_like(r),
+             "dS0": np.zeros((N, H, Dv, Dk)), "dd0": np.zeros((N, H, Dk))}
+        deta = np.zeros(1)
+        self.lib.osdn_ref_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), float(eta), _ptr(d0),
+                              _ptr(S0), float(scale), _ptr(dO), _ptr(dST), _ptr(ddT), _ptr(g["dq"]),
+                              _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]), _ptr(g["dr"]),
+                              _ptr(deta), _ptr(g["dS0"]), _ptr(g["dd0"]), cup, N, B, T, H, Dk, Dv)
+        g["deta"] = float(deta[0])
+        return g
+
+
 _default = None
 
 
@@ -178,3 +209,7 @@ def delta_fwd(*args, **kwargs):
 
 def fwd(*args, **kwargs):
     return _oracle().fwd(*args, **kwargs)
+
+
+def bwd(*args, **kwargs):
+    return _oracle().bwd(*args, **kwargs)
