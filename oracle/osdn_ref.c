@@ -154,16 +154,12 @@ void osdn_ref_delta_fwd(const double* q, const double* k, const double* k_tilde,
     }
 }
 
-/* ---------------------------------------------------------------------------------
- * Both phases in one token loop: the method exactly as stated, with no split.
- * Per token: k~ = d (.) k;  u = v - S k;  S += beta u k~^T;  o = scale S q;
- *            d <- r d - eta grad_d h(d).
- * k_tilde and dT may be NULL.
- * ------------------------------------------------------------------------------- */
-void osdn_ref_fwd(const double* q, const double* k, const double* v, const double* beta,
-                  const double* r, double eta, const double* d0, const double* S0, double scale,
-                  double* o, double* k_tilde, double* ST, double* dT, const int32_t* cu_seqlens,
-                  int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv) {
+/* The token loop of both phases; alpha (NULL: no decay) as in osdn_ref_fwd_gated below. */
+static void fwd_impl(const double* q, const double* k, const double* v, const double* beta,
+                     const double* r, double eta, const double* d0, const double* S0, double scale,
+                     const double* alpha, int32_t alpha_per_channel, double* o, double* k_tilde,
+                     double* ST, double* dT, const int32_t* cu_seqlens, int32_t num_seqs, int32_t B,
+                     int32_t T, int32_t H, int32_t Dk, int32_t Dv) {
     const int32_t N = cu_seqlens ? num_seqs : B;
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int32_t n = 0; n < N; ++n) {
@@ -185,6 +181,10 @@ void osdn_ref_fwd(const double* q, const double* k, const double* v, const doubl
                 const double* vt = v + th * Dv;
                 const double bt = beta[th];
                 const double rt = r ? r[th] : 1.0;
+                if (alpha)  /* the backbone's decay of the key channels, before the write */
+                    for (int32_t j = 0; j < Dv; ++j)
+                        for (int32_t i = 0; i < Dk; ++i)
+                            S[(int64_t)j * Dk + i] *= alpha_per_channel ? alpha[th * Dk + i] : alpha[th];
                 double knorm2 = 0.0, s = 0.0;
                 for (int32_t i = 0; i < Dk; ++i) {
                     knorm2 += kt[i] * kt[i];
@@ -221,6 +221,43 @@ void osdn_ref_fwd(const double* q, const double* k, const double* v, const doubl
             free(S);
         }
     }
+}
+
+/* ---------------------------------------------------------------------------------
+ * Both phases in one token loop: the method exactly as stated, with no split.
+ * Per token: k~ = d (.) k;  u = v - S k;  S += beta u k~^T;  o = scale S q;
+ *            d <- r d - eta grad_d h(d).
+ * k_tilde and dT may be NULL.
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_fwd(const double* q, const double* k, const double* v, const double* beta,
+                  const double* r, double eta, const double* d0, const double* S0, double scale,
+                  double* o, double* k_tilde, double* ST, double* dT, const int32_t* cu_seqlens,
+                  int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv) {
+    fwd_impl(q, k, v, beta, r, eta, d0, S0, scale, NULL, 0, o, k_tilde, ST, dT, cu_seqlens, num_seqs,
+             B, T, H, Dk, Dv);
+}
+
+/* ---------------------------------------------------------------------------------
+ * Both phases on a gated backbone (OSDN on Gated DeltaNet or Kimi Delta Attention).
+ * The pages train OSDN on GDN and KDA backbones without printing the combined update; the
+ * Gated DeltaNet-2 page (section 1) gives the gated delta rule, key-major,
+ * S_t = (I - beta k k^T) D_t S_{t-1} + beta k v^T with D_t = Diag(alpha_t) for KDA and
+ * alpha_t I for GDN.  Reading taken here: the state decays first, then OSDN's write key
+ * replaces the written key,
+ *   Sbar = S_{t-1} Diag(alpha_t)  (value-major S: the key channels decay),
+ *   S_t = Sbar + beta (v - Sbar k) k~^T,   k~ = d (.) k,
+ * and the preconditioner recurrence is unchanged (its surrogate is f_t around Sbar, the same
+ * function of k, beta and d).  alpha is [B,T,H] (GDN) when alpha_per_channel == 0, or
+ * [B,T,H,Dk] (KDA) when it is 1; all other arguments as osdn_ref_fwd.
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_fwd_gated(const double* q, const double* k, const double* v, const double* beta,
+                        const double* r, double eta, const double* d0, const double* S0,
+                        double scale, const double* alpha, int32_t alpha_per_channel, double* o,
+                        double* k_tilde, double* ST, double* dT, const int32_t* cu_seqlens,
+                        int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk,
+                        int32_t Dv) {
+    fwd_impl(q, k, v, beta, r, eta, d0, S0, scale, alpha, alpha_per_channel, o, k_tilde, ST, dT,
+             cu_seqlens, num_seqs, B, T, H, Dk, Dv);
 }
 
 /* ---------------------------------------------------------------------------------

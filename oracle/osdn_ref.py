@@ -97,6 +97,10 @@ class Oracle:
             _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _D, _D, _D, _I,
             _i32, _i32, _i32, _i32, _i32, _i32]
         lib.osdn_ref_fwd.restype = None
+        lib.osdn_ref_fwd_gated.argtypes = [
+            _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _i32, _D, _D, _D, _D,
+            _I, _i32, _i32, _i32, _i32, _i32, _i32]
+        lib.osdn_ref_fwd_gated.restype = None
         lib.osdn_ref_bwd.argtypes = [
             _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _D, _D, _D, _D, _D,
             _D, _D, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32, _i32]
@@ -158,6 +162,27 @@ class Oracle:
         return o, k_tilde, ST, dT
 
 
+    def fwd_gated(self, q, k, v, beta, alpha, r=None, eta=0.0, d0=None, S0=None, scale=1.0,
+                  cu_seqlens=None):
+        """Both phases on a gated backbone: the state's key channels decay by alpha before each
+        token's write (alpha [B,T,H]: Gated DeltaNet; [B,T,H,Dk]: Kimi Delta Attention).
+        Returns (o, k_tilde, ST, dT) like ``fwd``."""
+        q, k, v, beta, alpha, r, d0, S0 = map(_f64, (q, k, v, beta, alpha, r, d0, S0))
+        cu, cup = _cu(cu_seqlens)
+        B, T, H, Dk, N = _dims(k, cu)
+        Dv = v.shape[-1]
+        assert alpha.shape in ((B, T, H), (B, T, H, Dk))
+        per_channel = 1 if alpha.shape == (B, T, H, Dk) else 0
+        o = np.zeros((B, T, H, Dv))
+        k_tilde = np.zeros_like(k)
+        ST = np.zeros((N, H, Dv, Dk))
+        dT = np.zeros((N, H, Dk))
+        self.lib.osdn_ref_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), float(eta),
+                                    _ptr(d0), _ptr(S0), float(scale), _ptr(alpha), per_channel,
+                                    _ptr(o), _ptr(k_tilde), _ptr(ST), _ptr(dT), cup, N, B, T, H, Dk,
+                                    Dv)
+        return o, k_tilde, ST, dT
+
     def bwd(self, q, k, v, beta, dO, r=None, eta=0.0, d0=None, S0=None, scale=1.0, dST=None,
             ddT=None, cu_seqlens=None):
         """Gradient of L = <dO, o> + <dST, S_T> + <ddT, d_T> for the forward pass ``fwd`` with
@@ -213,3 +238,7 @@ def fwd(*args, **kwargs):
 
 def bwd(*args, **kwargs):
     return _oracle().bwd(*args, **kwargs)
+
+
+def fwd_gated(*args, **kwargs):
+    return _oracle().fwd_gated(*args, **kwargs)
