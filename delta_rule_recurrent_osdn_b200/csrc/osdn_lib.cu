@@ -353,20 +353,21 @@ namespace osdn {
 namespace {
 template <typename IO>
 osdn_status_t launch_step_io(const void* q, const void* k, const void* v, const float* beta,
-                             const float* r, float eta, float scale, float* S, float* d, void* o,
-                             void* kt, float* rho, int64_t nh, int Dk, int Dv, cudaStream_t stream) {
+                             const float* r, const float* alpha, int apc, float eta, float scale,
+                             float* S, float* d, void* o, void* kt, float* rho, int64_t nh, int Dk,
+                             int Dv, cudaStream_t stream) {
     const IO *q_ = static_cast<const IO*>(q), *k_ = static_cast<const IO*>(k),
              *v_ = static_cast<const IO*>(v);
     IO *o_ = static_cast<IO*>(o), *kt_ = static_cast<IO*>(kt);
     const dim3 grid((unsigned)nh), block(step_threads(Dv));
     if (Dk == 128 && Dv == 128)
-        osdn_step_kernel<128, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
+        osdn_step_kernel<128, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, alpha, apc, (int)nh);
     else if (Dk == 128 && Dv == 64)
-        osdn_step_kernel<128, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
+        osdn_step_kernel<128, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, alpha, apc, (int)nh);
     else if (Dk == 64 && Dv == 128)
-        osdn_step_kernel<64, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
+        osdn_step_kernel<64, 128, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, alpha, apc, (int)nh);
     else
-        osdn_step_kernel<64, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, (int)nh);
+        osdn_step_kernel<64, 64, IO><<<grid, block, 0, stream>>>(q_, k_, v_, beta, r, eta, scale, S, d, o_, kt_, rho, alpha, apc, (int)nh);
     return launch_status();
 }
 }  // namespace
@@ -475,32 +476,36 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
 }
 
 osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
-                        const float* r, float eta, float scale, float* S, float* d, void* o,
-                        void* k_tilde, float* rho, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
-                        osdn_dtype_t io, void* stream) {
+                        const float* r, const float* alpha, int32_t alpha_per_channel, float eta,
+                        float scale, float* S, float* d, void* o, void* k_tilde, float* rho,
+                        int32_t N, int32_t H, int32_t Dk, int32_t Dv, osdn_dtype_t io,
+                        void* stream) {
     if (io != OSDN_BF16 && io != OSDN_F32) return OSDN_ERR_INVALID_ARG;
+    if (alpha_per_channel != 0 && alpha_per_channel != 1) return OSDN_ERR_INVALID_ARG;
     if (N < 0 || H < 1) return OSDN_ERR_INVALID_ARG;
     if ((Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128)) return OSDN_ERR_UNSUPPORTED;
     const int64_t nh = (int64_t)N * H;
     if (nh == 0) return OSDN_OK;
     if (nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
     if (!q || !k || !v || !beta || !S || !d || !o) return OSDN_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, beta, r, S, d, o, k_tilde, rho};
+    const void* ptrs[] = {q, k, v, beta, r, alpha, S, d, o, k_tilde, rho};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
     const size_t es = io_size(io);
     const size_t qb = nh * Dk * es, vb = nh * Dv * es, gb = nh * 4, sb = nh * Dv * Dk * 4,
-                 db = nh * Dk * 4;
-    // every written buffer (S, d, o, k_tilde, rho: slots 5..9) against every other buffer
-    const void* all[] = {q, k, v, beta, r, S, d, o, k_tilde, rho};
-    const size_t allb[] = {qb, qb, vb, gb, gb, sb, db, vb, qb, gb};
-    for (int a = 5; a < 10; ++a)
-        for (int b = 0; b < 10; ++b)
+                 db = nh * Dk * 4, ab = alpha_per_channel ? db : gb;
+    // every written buffer (S, d, o, k_tilde, rho: slots 6..10) against every other buffer
+    const void* all[] = {q, k, v, beta, r, alpha, S, d, o, k_tilde, rho};
+    const size_t allb[] = {qb, qb, vb, gb, gb, ab, sb, db, vb, qb, gb};
+    for (int a = 6; a < 11; ++a)
+        for (int b = 0; b < 11; ++b)
             if (b != a && overlaps(all[a], allb[a], all[b], allb[b])) return OSDN_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16)
-        return osdn::launch_step_io<__nv_bfloat16>(q, k, v, beta, r, eta, scale, S, d, o, k_tilde, rho, nh, Dk, Dv, s);
-    return osdn::launch_step_io<float>(q, k, v, beta, r, eta, scale, S, d, o, k_tilde, rho, nh, Dk, Dv, s);
+        return osdn::launch_step_io<__nv_bfloat16>(q, k, v, beta, r, alpha, alpha_per_channel, eta,
+                                                   scale, S, d, o, k_tilde, rho, nh, Dk, Dv, s);
+    return osdn::launch_step_io<float>(q, k, v, beta, r, alpha, alpha_per_channel, eta, scale, S, d,
+                                       o, k_tilde, rho, nh, Dk, Dv, s);
 }
 
 osdn_status_t osdn_get_device_status(void* stream) {

@@ -6,6 +6,10 @@
 //   k~ = d (.) k,   u = v - S k,   S <- S + beta u k~^T,   o = scale * S q,
 //   d  <- r d + eta beta (1 - beta s) a / nk   (0 when nk = 0),
 // and optionally the residual-contraction ratio (1 - beta s)^2 of the write (section 3).
+// On a gated backbone (Gated DeltaNet: one decay factor per token and head; Kimi Delta
+// Attention: one per key channel) the state's key channels first decay, S <- S Diag(alpha), and
+// the step above runs on the decayed state: the gated delta rule of the Gated DeltaNet-2 page
+// (section 1) with OSDN's write key; the preconditioner is unchanged.
 // The step reads and writes the fp32 state once (Dv x Dk x 4 bytes each way) and a few hundred
 // bytes of token data: it is bound by HBM bandwidth.
 //
@@ -55,7 +59,8 @@ __global__ void __launch_bounds__(DV * 4)
 osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* __restrict__ v,
                  const float* __restrict__ beta, const float* __restrict__ r, float eta,
                  float scale, float* __restrict__ S, float* __restrict__ d, IO* __restrict__ o,
-                 IO* __restrict__ k_tilde, float* __restrict__ rho, int NH) {
+                 IO* __restrict__ k_tilde, float* __restrict__ rho, const float* __restrict__ alpha,
+                 int alpha_per_channel, int NH) {
     constexpr int PL = DK / 32;             // key channels per lane
     constexpr int NW = DV / 8;              // warps
     constexpr int ROWS = 8;                 // state rows per warp
@@ -76,6 +81,16 @@ osdn_step_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         dd[j] = d[(int64_t)nh * DK + PL * lane + j];
     }
     const float bt = beta[nh];
+    if (alpha) {  // decay of the key channels, before the write
+        float av[PL];
+#pragma unroll
+        for (int j = 0; j < PL; ++j)
+            av[j] = alpha_per_channel ? alpha[(int64_t)nh * DK + PL * lane + j] : alpha[nh];
+#pragma unroll
+        for (int i = 0; i < ROWS; ++i)
+#pragma unroll
+            for (int j = 0; j < PL; ++j) srow[i][j] *= av[j];
+    }
     float kt[PL], nk = 0.f, sa = 0.f;
 #pragma unroll
     for (int j = 0; j < PL; ++j) {

@@ -62,8 +62,8 @@ def _load() -> ctypes.CDLL:
                              _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
                              ctypes.c_size_t, _vp]
     lib.osdn_fwd.restype = ctypes.c_int
-    lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp, _vp, _vp, _i32,
-                              _i32, _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _vp, _vp, _vp,
+                              _vp, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_step.restype = ctypes.c_int
     lib.osdn_get_device_status.argtypes = [_vp]
     lib.osdn_get_device_status.restype = ctypes.c_int
@@ -233,10 +233,11 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
 
 
 def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0, o=None,
-              k_tilde=None, rho=None, stream=None):
+              k_tilde=None, rho=None, stream=None, alpha=None):
     """One recurrent step per (sequence, head) (the decode path).  q, k: [N, H, Dk]; v: [N, H, Dv];
-    beta, r: [N, H] float32; S: [N, H, Dv, Dk] and d: [N, H, Dk] float32, updated in place.
-    Returns o [N, H, Dv] (and writes k_tilde [N, H, Dk] when given)."""
+    beta, r: [N, H] float32; S: [N, H, Dv, Dk] and d: [N, H, Dk] float32, updated in place;
+    alpha: the decay of a gated backbone, [N, H] (Gated DeltaNet) or [N, H, Dk] (Kimi Delta
+    Attention) float32, or None.  Returns o [N, H, Dv] (and writes k_tilde [N, H, Dk] when given)."""
     N, H, Dk = q.shape
     Dv = v.shape[-1]
     io = _io(q)
@@ -252,8 +253,11 @@ def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0,
     _req(o, "o", q.dtype, (N, H, Dv))
     _req(k_tilde, "k_tilde", q.dtype, (N, H, Dk))
     _req(rho, "rho", torch.float32, (N, H))
-    _check(LIB.osdn_step(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), float(scale), _p(S),
-                         _p(d), _p(o), _p(k_tilde), _p(rho), N, H, Dk, Dv, io, _stream(stream)),
+    per_channel = alpha is not None and alpha.dim() == 3
+    _req(alpha, "alpha", torch.float32, (N, H, Dk) if per_channel else (N, H))
+    _check(LIB.osdn_step(_p(q), _p(k), _p(v), _p(beta), _p(r), _p(alpha), int(per_channel),
+                         float(eta), float(scale), _p(S), _p(d), _p(o), _p(k_tilde), _p(rho), N, H,
+                         Dk, Dv, io, _stream(stream)),
            "osdn_step")
     return o
 

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define OSDN_ABI_VERSION 2
+#define OSDN_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define OSDN_API __attribute__((visibility("default")))
@@ -190,14 +190,21 @@ OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void
  *   d        [N,H,Dk] float32, read and written in place.
  *   o        [N,H,Dv] io dtype, written.     k_tilde [N,H,Dk] io dtype, written, or NULL.
  *   rho      [N,H] float32, written: (1 - beta s)^2, as for osdn_precond_scan; or NULL.
+ *   alpha    decay of a gated backbone, or NULL for none: [N,H] float32 (Gated DeltaNet, one
+ *            factor per token and head; alpha_per_channel = 0) or [N,H,Dk] float32 (Kimi Delta
+ *            Attention, one per key channel; alpha_per_channel = 1).  The state's key channels
+ *            decay first, S <- S Diag(alpha), then the step above runs on the decayed state (the
+ *            gated delta rule of the Gated DeltaNet-2 page, section 1, with OSDN's write key; d
+ *            is unchanged by the decay).  alpha_per_channel must be 0 or 1.
  * Dk, Dv in {64, 128}.  Pointers 16-byte aligned.  S, d, o and k_tilde must not overlap one
  * another or the inputs (OSDN_ERR_INVALID_ARG).  N == 0 is a no-op.  A sequence of steps
  * equals osdn_fwd over the same tokens (up to fp32 summation order).
  */
 OSDN_API osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
-                        const float* r, float eta, float scale, float* S, float* d, void* o,
-                        void* k_tilde, float* rho, int32_t N, int32_t H, int32_t Dk, int32_t Dv,
-                        osdn_dtype_t io, void* stream);
+                        const float* r, const float* alpha, int32_t alpha_per_channel, float eta,
+                        float scale, float* S, float* d, void* o, void* k_tilde, float* rho,
+                        int32_t N, int32_t H, int32_t Dk, int32_t Dv, osdn_dtype_t io,
+                        void* stream);
 
 OSDN_API osdn_status_t osdn_get_device_status(void* stream);
 

@@ -44,7 +44,7 @@ def test_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert L.osdn_abi_version() == 2
+    assert L.osdn_abi_version() == 3
     for s in range(7):
         assert osdn.status_string(s)
     assert osdn.status_string(99) == "unknown status"
@@ -128,14 +128,14 @@ def test_parity_metric_allows_exactly_the_output_rounding():
 
 
 def step_call(**kw):
-    args = dict(q=fake(1), k=fake(2), v=fake(3), beta=fake(4), r=None, eta=0.1, scale=1.0,
-                S=fake(5), d=fake(6), o=fake(7), kt=None, rho=None, N=4, H=2, Dk=128, Dv=128,
-                io=osdn.OSDN_BF16)
+    args = dict(q=fake(1), k=fake(2), v=fake(3), beta=fake(4), r=None, alpha=None, apc=0, eta=0.1,
+                scale=1.0, S=fake(5), d=fake(6), o=fake(7), kt=None, rho=None, N=4, H=2, Dk=128,
+                Dv=128, io=osdn.OSDN_BF16)
     args.update(kw)
-    return L.osdn_step(args["q"], args["k"], args["v"], args["beta"], args["r"], args["eta"],
-                       args["scale"], args["S"], args["d"], args["o"], args["kt"], args["rho"],
-                       args["N"],
-                       args["H"], args["Dk"], args["Dv"], args["io"], None)
+    return L.osdn_step(args["q"], args["k"], args["v"], args["beta"], args["r"], args["alpha"],
+                       args["apc"], args["eta"], args["scale"], args["S"], args["d"], args["o"],
+                       args["kt"], args["rho"], args["N"], args["H"], args["Dk"], args["Dv"],
+                       args["io"], None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -151,6 +151,9 @@ def step_call(**kw):
     (dict(d=ctypes.c_void_p(A + 5 * 0x1000000 + 4096)), osdn.OSDN_ERR_INVALID_ARG),  # d in S
     (dict(kt=fake(2)), osdn.OSDN_ERR_INVALID_ARG),                                # k~ aliases k
     (dict(rho=fake(4)), osdn.OSDN_ERR_INVALID_ARG),                               # rho = beta
+    (dict(alpha=fake(8), apc=2), osdn.OSDN_ERR_INVALID_ARG),                     # flag not 0 / 1
+    (dict(alpha=ctypes.c_void_p(A + 8 * 0x1000000 + 4)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(alpha=ctypes.c_void_p(A + 5 * 0x1000000 + 64), apc=1), osdn.OSDN_ERR_INVALID_ARG),  # in S
     (dict(N=0), osdn.OSDN_OK),                                                    # nothing to do
 ])
 def test_step_rejects(kw, status):

@@ -15,20 +15,22 @@ def _batch(io, N, T, H, Dk, Dv, seed, apf=True):
                               seed=seed, init_state=True))
 
 
-def _steps(inp, ts):
-    """Run osdn_step over tokens ts of every sequence; returns numpy (o[N, len(ts), H, Dv],
-    k_tilde[N, len(ts), H, Dk], S, d)."""
+def _steps(inp, ts, alpha=None):
+    """Run osdn_step over tokens ts of every sequence (alpha: optional decay, numpy [N, T, H] or
+    [N, T, H, Dk]); returns numpy (o[N, len(ts), H, Dv], k_tilde[N, len(ts), H, Dk], S, d)."""
     from delta_rule_recurrent_osdn_b200 import osdn
     t = W.to_torch(inp)
     S = t["S0"].clone()
     d = t["d0"].clone()
+    a = None if alpha is None else torch.from_numpy(alpha.astype(np.float32)).cuda()
     os_, kts = [], []
     for i in ts:
         kt = torch.empty_like(t["k"][:, i])
         o = osdn.osdn_step(t["q"][:, i].contiguous(), t["k"][:, i].contiguous(),
                            t["v"][:, i].contiguous(), t["beta"][:, i].contiguous(), S, d,
                            None if t["r"] is None else t["r"][:, i].contiguous(), t["eta"],
-                           t["scale"], k_tilde=kt)
+                           t["scale"], k_tilde=kt,
+                           alpha=None if a is None else a[:, i].contiguous())
         os_.append(o)
         kts.append(kt)
     torch.cuda.synchronize()
@@ -96,3 +98,30 @@ def test_many_heads():
     assert rel_err(o[pick], wo, "bf16") <= TOL["bf16"]
     assert rel_err(S[pick], wS) <= 1e-5
     assert rel_err(d[pick], wd) <= 1e-5
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+@pytest.mark.parametrize("per_channel", [False, True])
+def test_gated_steps_match_oracle(ref, io, per_channel):
+    """Decay of a gated backbone (Gated DeltaNet: per token and head; Kimi Delta Attention: per
+    key channel) before each write: 24 steps equal the oracle's gated token loop."""
+    inp = _batch(io, N=3, T=24, H=2, Dk=128, Dv=128, seed=26)
+    rng = np.random.default_rng(27)
+    shape = (3, 24, 2, 128) if per_channel else (3, 24, 2)
+    alpha = (1 / (1 + np.exp(-(2 + rng.standard_normal(shape))))).astype(np.float32)
+    o, kt, S, d = _steps(inp, range(24), alpha)
+    wo, wkt, wS, wd = ref.fwd_gated(inp.q, inp.k, inp.v, inp.beta, alpha.astype(np.float64),
+                                    r=inp.r, eta=inp.eta, d0=inp.d0, S0=inp.S0, scale=inp.scale)
+    assert rel_err(o, wo, io) <= TOL[io]
+    assert rel_err(kt, wkt, io) <= TOL[io]
+    assert rel_err(S, wS) <= 1e-4
+    assert rel_err(d, wd) <= 1e-4
+
+
+def test_unit_decay_equals_ungated_step():
+    """alpha == 1 gives the ungated step bit for bit."""
+    inp = _batch("f32", N=2, T=6, H=2, Dk=128, Dv=128, seed=28)
+    plain = _steps(inp, range(6))
+    ones = _steps(inp, range(6), np.ones((2, 6, 2), dtype=np.float32))
+    for a, b in zip(plain, ones):
+        np.testing.assert_array_equal(a, b)
