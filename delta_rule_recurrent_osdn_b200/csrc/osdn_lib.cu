@@ -232,8 +232,9 @@ bool make_tp_map(CUtensorMap* m, const void* o, int Dv, int H, int64_t rows) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Phase 2, bf16 with d_k = 128: the WY factors of all chunks (persistent pre-kernel, written
-// into o), then one CTA per (sequence, head, 64 value channels) for the state chain.
+// Phase 2, bf16 with d_k = d_v = 128: the WY factors of all chunks (persistent pre-kernel,
+// written into o as bf16 hi / lo operand rows), then one CTA per (sequence, head, 64 value
+// channels) for the state chain, the head's two CTAs as a cluster.
 template <int DV>
 osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, const void* v,
                               const float* beta, float scale, const float* S0, void* o,
