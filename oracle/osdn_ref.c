@@ -272,12 +272,15 @@ void osdn_ref_fwd_gated(const double* q, const double* k, const double* v, const
  *   s = <d, a>, w = d (.) k, u = v - S k, S' = S + beta u w^T, o = scale S' q,
  *   g = eta beta (1 - beta s) / n (0 when n == 0), d' = r d + g a.
  * ------------------------------------------------------------------------------- */
-void osdn_ref_bwd(const double* q, const double* k, const double* v, const double* beta,
-                  const double* r, double eta, const double* d0, const double* S0, double scale,
-                  const double* dO, const double* dST, const double* ddT, double* dq, double* dk,
-                  double* dv, double* dbeta, double* dr, double* deta, double* dS0, double* dd0,
-                  const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T, int32_t H,
-                  int32_t Dk, int32_t Dv) {
+/* The reverse sweep of osdn_ref_bwd; with alpha (NULL: no decay) it differentiates the gated
+ * loop of osdn_ref_fwd_gated and writes dL/dalpha into dalpha. */
+static void bwd_impl(const double* q, const double* k, const double* v, const double* beta,
+                     const double* r, double eta, const double* d0, const double* S0, double scale,
+                     const double* alpha, int32_t apc, const double* dO, const double* dST,
+                     const double* ddT, double* dq, double* dk, double* dv, double* dbeta,
+                     double* dr, double* deta, double* dalpha, double* dS0, double* dd0,
+                     const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                     int32_t Dk, int32_t Dv) {
     const int32_t N = cu_seqlens ? num_seqs : B;
     const int64_t SZ = (int64_t)Dv * Dk;
     double eta_total = 0.0;
@@ -300,6 +303,7 @@ void osdn_ref_bwd(const double* q, const double* k, const double* v, const doubl
             double* gk = (double*)malloc(sizeof(double) * Dk);
             double* gw = (double*)malloc(sizeof(double) * Dk);
             double* gu = (double*)malloc(sizeof(double) * Dv);
+            double* Sb = (double*)malloc(sizeof(double) * SZ);  /* the decayed state S Diag(alpha) */
             for (int64_t e = 0; e < SZ; ++e) Sall[e] = S0 ? S0[sbase + e] : 0.0;
             for (int32_t i = 0; i < Dk; ++i) dall[i] = d0 ? d0[dbase + i] : 1.0;
             /* forward sweep (the same steps as osdn_ref_fwd) */
@@ -308,7 +312,15 @@ void osdn_ref_bwd(const double* q, const double* k, const double* v, const doubl
                 const double* kt = k + th * Dk;
                 const double* vt = v + th * Dv;
                 const double bt = beta[th], rt = r ? r[th] : 1.0;
-                const double* S = Sall + c * SZ;
+                const double* Sp = Sall + c * SZ;  /* before the token */
+                const double* S = Sp;                /* after the decay: the state the write sees */
+                if (alpha) {
+                    for (int32_t j = 0; j < Dv; ++j)
+                        for (int32_t i = 0; i < Dk; ++i)
+                            Sb[(int64_t)j * Dk + i] =
+                                Sp[(int64_t)j * Dk + i] * (apc ? alpha[th * Dk + i] : alpha[th]);
+                    S = Sb;
+                }
                 const double* d = dall + c * Dk;
                 double* Sn = Sall + (c + 1) * SZ;
                 double* dn = dall + (c + 1) * Dk;
@@ -339,7 +351,15 @@ void osdn_ref_bwd(const double* q, const double* k, const double* v, const doubl
                 const double* vt = v + th * Dv;
                 const double* gOt = dO + th * Dv;
                 const double bt = beta[th], rt = r ? r[th] : 1.0;
-                const double* S = Sall + c * SZ;
+                const double* Sp = Sall + c * SZ;  /* before the token */
+                const double* S = Sp;                /* after the decay: the state the write sees */
+                if (alpha) {
+                    for (int32_t j = 0; j < Dv; ++j)
+                        for (int32_t i = 0; i < Dk; ++i)
+                            Sb[(int64_t)j * Dk + i] =
+                                Sp[(int64_t)j * Dk + i] * (apc ? alpha[th * Dk + i] : alpha[th]);
+                    S = Sb;
+                }
                 const double* d = dall + c * Dk;
                 const double* Sn = Sall + (c + 1) * SZ;
                 double knorm2 = 0.0, s = 0.0;
@@ -413,9 +433,27 @@ void osdn_ref_bwd(const double* q, const double* k, const double* v, const doubl
                     gd[i] = gdp[i];
                 }
                 dbeta[th] = gbeta;
+                if (alpha) {  /* S = Sp Diag(alpha): dalpha from Sp, then the adjoint of Sp */
+                    if (apc) {
+                        for (int32_t i = 0; i < Dk; ++i) {
+                            double acc = 0.0;
+                            for (int32_t j = 0; j < Dv; ++j)
+                                acc += gS[(int64_t)j * Dk + i] * Sp[(int64_t)j * Dk + i];
+                            dalpha[th * Dk + i] = acc;
+                        }
+                        for (int32_t j = 0; j < Dv; ++j)
+                            for (int32_t i = 0; i < Dk; ++i) gS[(int64_t)j * Dk + i] *= alpha[th * Dk + i];
+                    } else {
+                        double acc = 0.0;
+                        for (int64_t e = 0; e < SZ; ++e) acc += gS[e] * Sp[e];
+                        dalpha[th] = acc;
+                        for (int64_t e = 0; e < SZ; ++e) gS[e] *= alpha[th];
+                    }
+                }
             }
             for (int64_t e = 0; e < SZ; ++e) dS0[sbase + e] = gS[e];
             for (int32_t i = 0; i < Dk; ++i) dd0[dbase + i] = gd[i];
+            free(Sb);
             free(gu);
             free(gw);
             free(gk);
@@ -430,4 +468,28 @@ void osdn_ref_bwd(const double* q, const double* k, const double* v, const doubl
         }
     }
     if (deta) *deta = eta_total;
+}
+
+void osdn_ref_bwd(const double* q, const double* k, const double* v, const double* beta,
+                  const double* r, double eta, const double* d0, const double* S0, double scale,
+                  const double* dO, const double* dST, const double* ddT, double* dq, double* dk,
+                  double* dv, double* dbeta, double* dr, double* deta, double* dS0, double* dd0,
+                  const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                  int32_t Dk, int32_t Dv) {
+    bwd_impl(q, k, v, beta, r, eta, d0, S0, scale, NULL, 0, dO, dST, ddT, dq, dk, dv, dbeta, dr,
+             deta, NULL, dS0, dd0, cu_seqlens, num_seqs, B, T, H, Dk, Dv);
+}
+
+/* The gradient of osdn_ref_fwd_gated (same arguments as osdn_ref_bwd plus alpha as in
+ * osdn_ref_fwd_gated); dalpha has alpha's shape. */
+void osdn_ref_bwd_gated(const double* q, const double* k, const double* v, const double* beta,
+                        const double* r, double eta, const double* d0, const double* S0,
+                        double scale, const double* alpha, int32_t alpha_per_channel,
+                        const double* dO, const double* dST, const double* ddT, double* dq,
+                        double* dk, double* dv, double* dbeta, double* dr, double* deta,
+                        double* dalpha, double* dS0, double* dd0, const int32_t* cu_seqlens,
+                        int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk,
+                        int32_t Dv) {
+    bwd_impl(q, k, v, beta, r, eta, d0, S0, scale, alpha, alpha_per_channel, dO, dST, ddT, dq, dk,
+             dv, dbeta, dr, deta, dalpha, dS0, dd0, cu_seqlens, num_seqs, B, T, H, Dk, Dv);
 }

@@ -105,6 +105,10 @@ class Oracle:
             _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _D, _D, _D, _D, _D,
             _D, _D, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32, _i32]
         lib.osdn_ref_bwd.restype = None
+        lib.osdn_ref_bwd_gated.argtypes = [
+            _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _i32, _D, _D, _D, _D,
+            _D, _D, _D, _D, _D, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32, _i32]
+        lib.osdn_ref_bwd_gated.restype = None
         self.lib = lib
 
     def set_threads(self, n: int = 0) -> int:
@@ -184,11 +188,13 @@ class Oracle:
         return o, k_tilde, ST, dT
 
     def bwd(self, q, k, v, beta, dO, r=None, eta=0.0, d0=None, S0=None, scale=1.0, dST=None,
-            ddT=None, cu_seqlens=None):
-        """Gradient of L = <dO, o> + <dST, S_T> + <ddT, d_T> for the forward pass ``fwd`` with
-        the same arguments, by reverse-mode differentiation of its token loop.  Returns a dict
-        with dq, dk, dv, dbeta, dr (None without r), deta (float), dS0, dd0."""
-        q, k, v, beta, r, d0, S0, dO, dST, ddT = map(_f64, (q, k, v, beta, r, d0, S0, dO, dST, ddT))
+            ddT=None, cu_seqlens=None, alpha=None):
+        """Gradient of L = <dO, o> + <dST, S_T> + <ddT, d_T> for the forward pass ``fwd`` (or
+        ``fwd_gated`` when alpha is given) with the same arguments, by reverse-mode
+        differentiation of its token loop.  Returns a dict with dq, dk, dv, dbeta, dr (None
+        without r), deta (float), dS0, dd0, and dalpha (alpha's shape) when alpha is given."""
+        q, k, v, beta, r, d0, S0, dO, dST, ddT, alpha = map(
+            _f64, (q, k, v, beta, r, d0, S0, dO, dST, ddT, alpha))
         cu, cup = _cu(cu_seqlens)
         B, T, H, Dk, N = _dims(k, cu)
         Dv = v.shape[-1]
@@ -202,10 +208,21 @@ class Oracle:
              "dbeta": np.zeros_like(beta), "dr": None if r is None else np.zeros_like(r),
              "dS0": np.zeros((N, H, Dv, Dk)), "dd0": np.zeros((N, H, Dk))}
         deta = np.zeros(1)
-        self.lib.osdn_ref_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), float(eta), _ptr(d0),
-                              _ptr(S0), float(scale), _ptr(dO), _ptr(dST), _ptr(ddT), _ptr(g["dq"]),
-                              _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]), _ptr(g["dr"]),
-                              _ptr(deta), _ptr(g["dS0"]), _ptr(g["dd0"]), cup, N, B, T, H, Dk, Dv)
+        if alpha is None:
+            self.lib.osdn_ref_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), float(eta),
+                                  _ptr(d0), _ptr(S0), float(scale), _ptr(dO), _ptr(dST), _ptr(ddT),
+                                  _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]),
+                                  _ptr(g["dr"]), _ptr(deta), _ptr(g["dS0"]), _ptr(g["dd0"]), cup, N,
+                                  B, T, H, Dk, Dv)
+        else:
+            assert alpha.shape in ((B, T, H), (B, T, H, Dk))
+            g["dalpha"] = np.zeros_like(alpha)
+            self.lib.osdn_ref_bwd_gated(
+                _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(r), float(eta), _ptr(d0), _ptr(S0),
+                float(scale), _ptr(alpha), 1 if alpha.ndim == 4 else 0, _ptr(dO), _ptr(dST),
+                _ptr(ddT), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dbeta"]),
+                _ptr(g["dr"]), _ptr(deta), _ptr(g["dalpha"]), _ptr(g["dS0"]), _ptr(g["dd0"]), cup,
+                N, B, T, H, Dk, Dv)
         g["deta"] = float(deta[0])
         return g
 

@@ -35,6 +35,10 @@ def _problem(case, seed=0):
         "S0": 0.1 * rng.standard_normal((N, H, Dv, Dk)),
     }
     kw = {"eta": 0.3, "scale": 0.7, "cu_seqlens": cu}
+    p["alpha"] = None
+    if case in ("gated_gdn", "gated_kda"):  # decay of a gated backbone (the oracle's fwd_gated)
+        shape = (B, T, H, Dk) if case == "gated_kda" else (B, T, H)
+        p["alpha"] = 1.0 / (1.0 + np.exp(-(1.0 + rng.standard_normal(shape))))
     if case == "no_apf":
         p["r"] = None
     if case == "zero_key":  # the ||k||^2 == 0 branch (gradient of the surrogate taken as 0)
@@ -52,15 +56,19 @@ def _problem(case, seed=0):
 
 
 def _loss(ref, p, kw, up):
-    o, _, ST, dT = ref.fwd(p["q"], p["k"], p["v"], p["beta"], r=p["r"], eta=kw["eta"],
-                           d0=p["d0"], S0=p["S0"], scale=kw["scale"], cu_seqlens=kw["cu_seqlens"])
+    args = dict(r=p["r"], eta=kw["eta"], d0=p["d0"], S0=p["S0"], scale=kw["scale"],
+                cu_seqlens=kw["cu_seqlens"])
+    if p["alpha"] is None:
+        o, _, ST, dT = ref.fwd(p["q"], p["k"], p["v"], p["beta"], **args)
+    else:
+        o, _, ST, dT = ref.fwd_gated(p["q"], p["k"], p["v"], p["beta"], p["alpha"], **args)
     return (o * up["dO"]).sum() + (ST * up["dST"]).sum() + (dT * up["ddT"]).sum()
 
 
 def _grads(ref, p, kw, up):
     return ref.bwd(p["q"], p["k"], p["v"], p["beta"], up["dO"], r=p["r"], eta=kw["eta"],
                    d0=p["d0"], S0=p["S0"], scale=kw["scale"], dST=up["dST"], ddT=up["ddT"],
-                   cu_seqlens=kw["cu_seqlens"])
+                   cu_seqlens=kw["cu_seqlens"], alpha=p["alpha"])
 
 
 def _check(ref, case, seed=0):
@@ -69,7 +77,7 @@ def _check(ref, case, seed=0):
     g = _grads(ref, p, kw, up)
     rng = np.random.default_rng(100 + seed)
     worst = 0.0
-    names = [n for n in ("q", "k", "v", "beta", "r", "d0", "S0") if p[n] is not None]
+    names = [n for n in ("q", "k", "v", "beta", "r", "d0", "S0", "alpha") if p[n] is not None]
     for name in names + ["eta"]:
         for _ in range(2):
             if name == "eta":
@@ -90,7 +98,7 @@ def _check(ref, case, seed=0):
     return worst
 
 
-@pytest.mark.parametrize("case", ["apf", "no_apf", "packed", "zero_key"])
+@pytest.mark.parametrize("case", ["apf", "no_apf", "packed", "zero_key", "gated_gdn", "gated_kda"])
 def test_gradient_matches_central_differences(case):
     ref = osdn_ref._oracle()
     assert _check(ref, case) <= RTOL
@@ -135,3 +143,23 @@ def test_planted_mistake_in_backward_is_caught(tmp_path, name):
     path.write_text(src.replace(old, new))
     mutant = osdn_ref.Oracle(osdn_ref.compile_source(str(path), str(tmp_path / f"libbwd_{name}.so")))
     assert max(_check(mutant, case) for case in ("apf", "packed")) > 1e-4
+
+
+# mistakes in the decay's part of the reverse sweep (Gated DeltaNet decay, one factor per token)
+GATED_MUTATIONS = {
+    "decay_adjoint_dropped": ("for (int64_t e = 0; e < SZ; ++e) gS[e] *= alpha[th];", "(void)0;"),
+    "dalpha_from_decayed_state": ("for (int64_t e = 0; e < SZ; ++e) acc += gS[e] * Sp[e];",
+                                  "for (int64_t e = 0; e < SZ; ++e) acc += gS[e] * S[e];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(GATED_MUTATIONS))
+def test_planted_mistake_in_gated_backward_is_caught(tmp_path, name):
+    old, new = GATED_MUTATIONS[name]
+    src = open(osdn_ref.SOURCE).read()
+    assert old in src, f"mutation anchor for {name} not found"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    mutant = osdn_ref.Oracle(osdn_ref.compile_source(str(path), str(tmp_path / f"libgbwd_{name}.so")))
+    assert _check(mutant, "gated_gdn") > 1e-4
+    assert _check(osdn_ref._oracle(), "gated_gdn") <= RTOL
