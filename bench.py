@@ -1,18 +1,22 @@
 """Benchmark of the OSDN forward pass (phase 1 scan + phase 2 chunked delta rule) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 1p3b|340m|long|varlen|decode]
 
-One step is the whole hot path over one batch of the 1.3B-layer workload (B=4, T=4096, H=16,
-d_k=d_v=128, bf16 I/O, APF on, eta=0.05), seeded synthetic inputs resident in HBM.  Each
-timed step is bracketed by CUDA events on the launching stream, and a 256 MiB write between
-steps flushes the 126 MB L2 (outside the events).  Prints one JSON line on rank 0.
+One step is one ``osdn_fwd`` call -- the whole hot path: both phases, four kernels -- over one
+batch of seeded synthetic inputs resident in HBM.  The default workload is the 1.3B-layer shape
+(B=4, T=4096, H=16, d_k=d_v=128, bf16 I/O, APF on, eta=0.05); ``340m`` (B=8, T=2048, H=8, no
+APF), ``long`` (B=1, T=65536, H=16, S_0 and d_0 passed in) and ``varlen`` (32 packed sequences
+of U[128, 8192] tokens, H=16) are the other forward shapes; ``decode`` times ``osdn_step``.
+Each timed step is bracketed by CUDA events on the launching stream, and a 256 MiB write
+between steps flushes the 126 MB L2 (outside the events).  Prints one JSON line on rank 0.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own batch (independent
 sequences: weak scaling, no data-path collective); the elapsed device time is the max over
 ranks and ``value`` counts the tokens of all ranks.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead (rank 0 only), on a
-bounded prefix of the same batch per step.
+bounded sample of the same workload per step.
 """
 from __future__ import annotations
 
@@ -32,14 +36,30 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "OSDN fwd tokens/s (scan+chunk) at 1.3B-layer shape; % of HBM/TC roofline"
-WORKLOAD = "1p3b_apf"
 FLUSH_BYTES = 256 << 20
-# Algorithmic HBM bytes per token-head (bf16 I/O, d_k = d_v = 128), by kernel:
-#   scan : k in (256) + beta (4) + r (4) + k~ out (256)
-#   chunk: q, k, k~, v in (1024) + beta (4) + o out (256)
-#   fused forward (both phases in one kernel): q, k, v in (768) + beta, r (8) + o out (256)
-ALGO_BYTES = {"scan": 520, "chunk": 1284, "fwd": 1032}
+# forward workloads: bench name -> (inputs.CONFIGS name, shape label, description)
+FORWARD = {
+    "1p3b": ("1p3b_apf", "1.3B-layer",
+             "1.3B-layer OSDN token mixer (B=4, T=4096, H=16, d_k=d_v=128, APF)"),
+    "340m": ("340m", "340M-layer",
+             "340M-layer OSDN token mixer (B=8, T=2048, H=8, d_k=d_v=128, no APF)"),
+    "long": ("long_ctx", "long-context",
+             "long-context OSDN token mixer (B=1, T=65536, H=16, d_k=d_v=128, APF, S_0 and d_0 "
+             "passed in)"),
+    "varlen": ("varlen", "varlen",
+               "packed variable-length OSDN token mixer (32 sequences of U[128, 8192] tokens, "
+               "H=16, d_k=d_v=128, APF)"),
+}
+METRIC = "OSDN fwd tokens/s (scan+chunk) at 1.3B-layer shape; % of HBM/TC roofline"
+# the kernels one bf16 osdn_fwd call with d_k = d_v = 128 launches, in order
+FWD_KERNELS = ["precond_prep_kernel", "precond_chain_kernel", "wy_prep_kernel",
+               "chunk_fwd_tc_kernel"]
+FWD_SOURCES = ["osdn_lib.cu", "common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
+               "chunk_walk.cuh", "scan_tc.cuh", "chunk_prep.cuh", "chunk_tc.cuh"]
+
+
+def metric_name(label):
+    return f"OSDN fwd tokens/s (scan+chunk) at {label} shape; % of HBM/TC roofline"
 
 
 def read_peaks():
@@ -57,25 +77,33 @@ def kernel_source_sha(names):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"scan": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
-                           "chunk_walk.cuh", "scan_tc.cuh"],
-                  "chunk": ["common.cuh", "watchdog.cuh", "tc_ptx.cuh", "tril_inverse.cuh",
-                            "chunk_walk.cuh", "chunk_prep.cuh", "chunk_tc.cuh"],
-                  "step": ["common.cuh", "step.cuh"]}
-
-
-def profiled_traffic(kernel, workload=WORKLOAD):
-    """DRAM bytes per launch from the committed ncu summary of this kernel, if it was taken on
-    the current source (its recorded source hash matches); else None."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+def profile_record(name):
+    """Key: value lines of a committed ncu summary (profiles/<name>.md), or None when the file
+    is missing or was taken on other kernel sources (its recorded source hash differs)."""
+    path = os.path.join(ROOT, "profiles", f"{name}.md")
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", text)
-    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.e+]+)", text)
-    if not (m_sha and m_tr) or m_sha.group(1) != kernel_source_sha(KERNEL_SOURCES[kernel]):
+    rec = dict(re.findall(r"^(\w+):\s*(\S+)\s*$", open(path).read(), re.M))
+    if rec.get("source_sha") != kernel_source_sha(FWD_SOURCES if name.startswith("fwd_")
+                                                  else STEP_SOURCES):
         return None
-    return float(m_tr.group(1))
+    return rec
+
+
+def fwd_algorithmic_bytes(inp, es=2):
+    """Bytes the forward pass must move: q, k, v in and o out in the io
+    dtype, beta (and r with APF) in fp32 per token-head; per (sequence, head) the final state
+    S_T and d_T out in fp32, and S_0, d_0 in when given.  k~ is an intermediate, not counted."""
+    th = inp.B * inp.T * inp.H
+    per_th = (2 * inp.Dk + 2 * inp.Dv) * es + 4 + (4 if inp.r is not None else 0)
+    per_nh = (inp.Dv * inp.Dk + inp.Dk) * 4 * (2 if inp.S0 is not None else 1)
+    return th * per_th + inp.N * inp.H * per_nh
+
+
+def fwd_flops(inp):
+    """Chunk-form MMA FLOPs: 5 * 2 * C * d + 3 * 2 * d_k * d_v per
+    token-head."""
+    return inp.B * inp.T * inp.H * (5 * 2 * inp.chunk * inp.Dk + 3 * 2 * inp.Dk * inp.Dv)
 
 
 class ClockSampler:
@@ -168,78 +196,97 @@ def barrier(world, device=None):
             dist.barrier()
 
 
-def oracle_rate(inp, seconds_target, max_tokens=None):
-    """Oracle throughput (tokens/s over all heads) on a prefix of the batch sized to about
-    `seconds_target` of CPU time; returns (rate, threads, sample description, seconds)."""
-    from delta_rule_recurrent_osdn_b200 import inputs as W  # noqa: F401
+def oracle_sample(inp, m_tokens):
+    """The first sequences (packed input: whole sequences; fixed length: the first m_tokens
+    tokens of every sequence) of a batch, as the bounded sample the oracle is timed on."""
+    from delta_rule_recurrent_osdn_b200 import inputs as W
+    if inp.cu_seqlens is not None:
+        cu = inp.cu_seqlens
+        m = int(np.searchsorted(cu[1:], min(m_tokens, cu[-1]), side="left")) + 1
+        sub = W.select(inp, seqs=list(range(min(m, inp.N))))
+        return sub, int(sub.cu_seqlens[-1]), f"first {min(m, inp.N)} of {inp.N} packed sequences"
+    tp = int(max(1, min(inp.T, m_tokens)))
+    sub = W.select(inp)
+    sub.q, sub.k, sub.v, sub.beta = inp.q[:, :tp], inp.k[:, :tp], inp.v[:, :tp], inp.beta[:, :tp]
+    sub.r = None if inp.r is None else inp.r[:, :tp]
+    return sub, inp.B * tp, f"first {tp} of {inp.T} tokens of all {inp.B} sequences"
+
+
+def oracle_run(sub):
+    from oracle import osdn_ref
+    t0 = time.perf_counter()
+    osdn_ref.fwd(sub.q, sub.k, sub.v, sub.beta, sub.r, sub.eta, sub.d0, sub.S0, sub.scale,
+                 sub.cu_seqlens)
+    return time.perf_counter() - t0
+
+
+def oracle_rate(inp, seconds_target):
+    """Oracle throughput (tokens/s over all heads) on a bounded sample of the batch sized to
+    about `seconds_target` of CPU time; returns (rate, threads, sample description)."""
     from oracle import osdn_ref
     threads = osdn_ref.set_threads(0)
-
-    def run(tp):
-        q, k, v = inp.q[:, :tp], inp.k[:, :tp], inp.v[:, :tp]
-        beta = inp.beta[:, :tp]
-        r = None if inp.r is None else inp.r[:, :tp]
-        t0 = time.perf_counter()
-        osdn_ref.fwd(q, k, v, beta, r, inp.eta, inp.d0, inp.S0, inp.scale)
-        return time.perf_counter() - t0
-
-    probe = min(32, inp.T)
-    dt = run(probe)
-    tp = int(min(inp.T, max(probe, probe * seconds_target / max(dt, 1e-6))))
-    if max_tokens:
-        tp = min(tp, max_tokens)
-    dt = run(tp)
+    probe, ptok, _ = oracle_sample(inp, 32)
+    dt = oracle_run(probe)
+    per_token = dt / max(ptok, 1)
+    sub, tokens, desc = oracle_sample(inp, int(seconds_target / max(per_token, 1e-9) /
+                                              (inp.B if inp.cu_seqlens is None else 1)))
+    dt = oracle_run(sub)
     reps = 1
-    if tp == inp.T and dt < seconds_target / 2:  # whole batch is quick: repeat it
+    if dt < seconds_target / 2:  # the whole batch is quick: repeat it
         reps = max(1, int(seconds_target / max(dt, 1e-6)))
-        dt = sum(run(tp) for _ in range(reps))
-    tokens = inp.B * tp * reps
-    sample = (f"first {tp} of {inp.T} tokens of all {inp.B} sequences x {inp.H} heads "
-              f"({inp.B * tp * inp.H} token-heads, fp64), {reps} run(s), {dt:.1f} s")
-    return tokens / dt, threads, sample, dt, tp
+        dt = sum(oracle_run(sub) for _ in range(reps))
+    sample = (f"{desc} x {inp.H} heads ({tokens * inp.H} token-heads, fp64), {reps} run(s), "
+              f"{dt:.1f} s")
+    return tokens * reps / dt, threads, sample
+
+
+def forward_inputs(args, seed=None):
+    from delta_rule_recurrent_osdn_b200 import inputs as W
+    name, label, desc = FORWARD[args.workload]
+    return W.make_inputs(name, seed=seed), label, desc
+
+
+def config_dict(inp, desc):
+    cfg = {"workload": desc, "B": inp.B, "T": inp.T, "H": inp.H, "d_k": inp.Dk, "d_v": inp.Dv,
+           "chunk": inp.chunk, "apf": inp.r is not None, "eta": inp.eta, "io": inp.io,
+           "l2": "flushed between timed steps (256 MiB write)"}
+    if inp.cu_seqlens is not None:
+        cfg.update(num_seqs=inp.N, total_tokens=int(inp.cu_seqlens[-1]))
+    if inp.S0 is not None:
+        cfg["initial_state"] = "S_0 ~ N(0, 0.1^2), d_0 ~ U(0.5, 1.5)"
+    return cfg
 
 
 def bench_reference(args):
+    """The oracle as the reference arm: rank 0 only, a bounded sample of the workload per
+    step, timed on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from delta_rule_recurrent_osdn_b200 import inputs as W
-    inp = W.make_inputs(WORKLOAD)
-    rate, threads, sample, dt, tp = oracle_rate(inp, seconds_target=3.0)
-    from oracle import osdn_ref
-
-    def step():
-        q, k, v = inp.q[:, :tp], inp.k[:, :tp], inp.v[:, :tp]
-        r = None if inp.r is None else inp.r[:, :tp]
-        osdn_ref.fwd(q, k, v, inp.beta[:, :tp], r, inp.eta, inp.d0, inp.S0, inp.scale)
-
+    if args.workload == "decode":
+        return bench_reference_decode(args)
+    inp, label, desc = forward_inputs(args)
+    rate, threads, sample = oracle_rate(inp, seconds_target=3.0)
+    sub, tokens, sdesc = oracle_sample(inp, int(rate * 3.0 / (inp.B if inp.cu_seqlens is None
+                                                              else 1)))
     for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    el = time.perf_counter() - t0
-    value = inp.B * tp * args.steps / el
+        oracle_run(sub)
+    el = sum(oracle_run(sub) for _ in range(args.steps))
+    value = tokens * args.steps / el
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": metric_name(label), "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(inp),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
-                         "kind": "oracle", "sample": sample + " per step"},
+        "config": config_dict(inp, desc),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{sdesc} x {inp.H} heads ({tokens * inp.H} token-heads, "
+                                   f"fp64) per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     return 0
-
-
-def config_dict(inp):
-    return {"workload": "1.3B-layer OSDN token mixer (B=4, T=4096, H=16, d_k=d_v=128, APF)",
-            "B": inp.B, "T": inp.T, "H": inp.H, "d_k": inp.Dk, "d_v": inp.Dv,
-            "chunk": inp.chunk, "apf": inp.r is not None, "eta": inp.eta, "io": inp.io,
-            "l2": "flushed between timed steps (256 MiB write)"}
 
 
 def bench_ours(args):
@@ -250,103 +297,111 @@ def bench_ours(args):
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    inp = W.make_inputs(WORKLOAD, seed=None if rank == 0 else 1000 + rank)
+    inp, label, desc = forward_inputs(args, seed=None if rank == 0 else 1000 + rank)
     d = W.to_torch(inp, dev)
     stream = torch.cuda.current_stream(dev)
-    kt = torch.empty_like(d["k"])
     o = torch.empty_like(d["v"])
     N, H, Dk, Dv = inp.N, inp.H, inp.Dk, inp.Dv
     ST = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
     dT = torch.empty((N, H, Dk), dtype=torch.float32, device=dev)
+    ws = torch.empty(osdn.osdn_fwd_workspace_bytes(inp.B, inp.T, H, Dk), dtype=torch.uint8,
+                     device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    launches_per_step = 4  # per phase: a per-chunk pre-kernel and the sequential chain
+    launches_per_step = len(FWD_KERNELS)  # bf16, d_k = d_v = 128: both phases' two kernels
 
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        osdn.osdn_precond_scan(d["k"], d["beta"], d["r"], d["eta"], d["d0"], k_tilde=kt, dT=dT)
-        if ev:
-            ev[1].record(stream)
-        osdn.osdn_chunk_fwd(d["q"], d["k"], kt, d["v"], d["beta"], d["scale"], d["S0"],
-                            d["chunk"], o=o, ST=ST)
-        if ev:
-            ev[2].record(stream)
+    def step():
+        osdn.osdn_fwd(d["q"], d["k"], d["v"], d["beta"], d["r"], inp.eta, d["d0"], d["S0"],
+                      inp.scale, inp.chunk, d["cu_seqlens"], o=o, ST=ST, dT=dT, workspace=ws)
 
     for _ in range(args.warmup):
         flush.fill_(1)
         step()
     torch.cuda.synchronize(dev)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            step(events[i])
+            events[i][0].record(stream)
+            step()
+            events[i][1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(world, dev)
     if osdn.osdn_get_device_status() != osdn.OSDN_OK:
         raise RuntimeError("device status not OK after the timed region")
-    scan_ms = [e[0].elapsed_time(e[1]) for e in events]
-    chunk_ms = [e[1].elapsed_time(e[2]) for e in events]
-    step_ms = [e[0].elapsed_time(e[2]) for e in events]
+    step_ms = [e[0].elapsed_time(e[1]) for e in events]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     tokens = inp.B * inp.T
     value = world * tokens * args.steps / (total_ms / 1e3)
 
-    # ---- end to end through the public API with host buffers (pinned), copies timed
-    host = {k_: d[k_].cpu().pin_memory() for k_ in ("q", "k", "v", "beta", "r")}
+    # ---- end to end through the public API with host buffers (pinned): every step copies its
+    #      inputs host -> device and o back inside the events; the L2 flush stays outside them
+    names = [k_ for k_ in ("q", "k", "v", "beta", "r", "d0", "S0", "cu_seqlens")
+             if d[k_] is not None]
+    host = {k_: d[k_].cpu().pin_memory() for k_ in names}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     dev_in = {k_: torch.empty_like(d[k_]) for k_ in host}
-    ws = torch.empty(osdn.osdn_fwd_workspace_bytes(inp.B, inp.T, H, Dk), dtype=torch.uint8,
-                     device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = o_host.numel() * o_host.element_size()
 
     def e2e_step():
         for k_, t in host.items():
             dev_in[k_].copy_(t, non_blocking=True)
-        osdn.osdn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["r"],
-                      inp.eta, None, None, inp.scale, inp.chunk, o=o, ST=ST, dT=dT, workspace=ws)
+        osdn.osdn_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in.get("r"),
+                      inp.eta, dev_in.get("d0"), dev_in.get("S0"), inp.scale, inp.chunk,
+                      dev_in.get("cu_seqlens"), o=o, ST=ST, dT=dT, workspace=ws)
         o_host.copy_(o, non_blocking=True)
 
-    for _ in range(max(3, args.warmup // 2)):
+    for _ in range(3):
         e2e_step()
     torch.cuda.synchronize(dev)
     barrier(world, dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for i in range(args.steps):
         flush.fill_(3)
+        e2e_ev[i][0].record(stream)
         e2e_step()
-    e1.record(stream)
+        e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev)
     e2e_value = world * tokens * args.steps / (e2e_ms / 1e3)
 
     if rank == 0:
         hbm, tc, kind = read_peaks()
-        avg = {"scan": statistics.mean(scan_ms), "chunk": statistics.mean(chunk_ms)}
-        dom = max(avg, key=avg.get)
-        token_heads = tokens * H
-        achieved = ALGO_BYTES[dom] * token_heads / (avg[dom] / 1e3) / 1e9
-        traffic = profiled_traffic(dom)
-        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
-                "peak_kind": f"{kind} hbm_gbs", "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": traffic,
-                "algorithmic_bytes_per_launch": ALGO_BYTES[dom] * token_heads,
-                "kernel_ms": avg, "whole_step_hbm_frac":
-                    ALGO_BYTES["fwd"] * token_heads / (statistics.mean(step_ms) / 1e3) / 1e9 / hbm}
+        mean_ms = statistics.mean(step_ms)
+        byts = fwd_algorithmic_bytes(inp)
+        flops = fwd_flops(inp)
+        achieved = byts / (mean_ms / 1e3) / 1e9
+        t_hbm_us, t_tc_us = byts / (hbm * 1e9) * 1e6, flops / (tc * 1e12) * 1e6
+        rec = profile_record(f"fwd_{FORWARD[args.workload][0]}")
+        traffic = float(rec["dram_bytes_per_step"]) if rec and "dram_bytes_per_step" in rec \
+            else None
+        roof = {"bound": "hbm", "scope": "whole forward pass (one osdn_fwd call, 4 kernels)",
+                "achieved": achieved, "peak": hbm, "peak_kind": f"{kind} hbm_gbs", "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic,
+                "traffic_over_algorithmic": None if traffic is None else traffic / byts,
+                "algorithmic_bytes_per_launch": byts,
+                "hbm_floor_us": t_hbm_us, "tensor_floor_us": t_tc_us,
+                "tensor_flops_per_launch": flops, "tensor_peak": tc,
+                "tensor_peak_kind": f"{kind} bf16_tflops"}
+        if rec and "kernel_shares" in rec:
+            shares = {k_: float(v_) for k_, v_ in
+                      (x.split("=") for x in rec["kernel_shares"].split(";"))}
+            dom = max(shares, key=shares.get)
+            roof["dominant_kernel"] = {"name": dom, "ncu_share": shares[dom],
+                                       "ms_est": shares[dom] * mean_ms,
+                                       "shares": shares}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            rate, threads, sample, _, _ = oracle_rate(inp, seconds_target=args.cpu_seconds)
+            rate, threads, sample = oracle_rate(inp, seconds_target=args.cpu_seconds)
             cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                    "sample": sample}
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "metric": metric_name(label), "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_dict(inp), "roofline": roof,
+            "data": "synthetic", "config": config_dict(inp, desc), "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
@@ -360,6 +415,7 @@ def bench_ours(args):
     return 0
 
 
+STEP_SOURCES = ["common.cuh", "step.cuh"]
 DECODE_METRIC = ("OSDN decode tokens/s (one recurrent step per sequence, 256 sequences x 16 heads, "
                  "d_k=d_v=128); % of HBM roofline")
 DECODE = dict(B=256, T=8, H=16, Dk=128, Dv=128, io="bf16", apf=True, eta=0.05, chunk=64, seed=7,
@@ -438,14 +494,14 @@ def bench_decode(args):
         e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.fill_(3)
+        flush.fill_(3)  # outside the events
+        e2e_ev[i][0].record(stream)
         e2e_step(i)
-    e1.record(stream)
+        e2e_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, dev)
     e2e_value = world * N * args.steps / (e2e_ms / 1e3)
 
     if rank == 0:
@@ -455,7 +511,8 @@ def bench_decode(args):
         achieved = byts / (avg / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": "step", "achieved": achieved, "peak": hbm,
                 "peak_kind": f"{kind} hbm_gbs", "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": profiled_traffic("step", "decode"),
+                "traffic": (lambda r: None if not r or "dram_bytes_per_launch" not in r else
+                            float(r["dram_bytes_per_launch"]))(profile_record("step_decode")),
                 "algorithmic_bytes_per_launch": byts, "kernel_ms": {"step": avg}}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -494,6 +551,43 @@ def bench_decode(args):
     return 0
 
 
+def bench_reference_decode(args):
+    """The oracle as the reference arm of the decode workload: one token of every sequence per
+    step (the oracle's token loop over a one-token batch), on the host cores."""
+    from delta_rule_recurrent_osdn_b200 import inputs as W
+    from oracle import osdn_ref as R
+    inp = W.make_inputs(dict(DECODE))
+    threads = R.set_threads(0)
+
+    def step(i):
+        t = i % inp.T
+        R.fwd(inp.q[:, t:t + 1], inp.k[:, t:t + 1], inp.v[:, t:t + 1], inp.beta[:, t:t + 1],
+              inp.r[:, t:t + 1], inp.eta, inp.d0, inp.S0, inp.scale)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = inp.N * args.steps / el
+    line = {
+        "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"OSDN decode step, {inp.N} sequences x {inp.H} heads, "
+                               f"d_k=d_v={inp.Dk}, bf16 I/O, fp32 state, APF"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"one step of all {inp.N} sequences x {inp.H} heads (fp64) "
+                                   "per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -502,8 +596,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["forward", "decode"], default="forward",
-                    help="forward: the 1.3B-layer forward pass (default); decode: osdn_step")
+    ap.add_argument("--workload", choices=list(FORWARD) + ["decode"], default="1p3b",
+                    help="a forward-pass shape (default: the 1.3B layer) or decode (osdn_step)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

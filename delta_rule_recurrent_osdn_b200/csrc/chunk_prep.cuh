@@ -5,9 +5,9 @@
 // tokens with rows K, K~ and gates beta,
 //   T = (I + strict_tril(diag(beta) K K~^T))^-1,
 // which does not depend on the state.  wy_prep_kernel computes it for every chunk in parallel:
-// K K~^T by one bf16 MMA (both operands are exact bf16, so the fp32 accumulation is the only
-// rounding), the inverse by tril_inverse_64_g128.  The sequential kernel (chunk_tc.cuh) then
-// only reads T.
+// K K~^T by bf16 MMAs (both operands are exact bf16 -- K~ as one term, or as the hi + lo terms
+// phase 1 hands over inside osdn_fwd -- so the fp32 accumulation is the only rounding), the
+// inverse by tril_inverse_64_g128.  The sequential kernel (chunk_tc.cuh) then only reads T.
 //
 // Hand-off through the output buffer o, which the sequential kernel writes only after reading
 // T: each 128-value (256-byte) row of o for a head holds two 128-byte slices, and row t of a
@@ -29,20 +29,22 @@ namespace osdn {
 
 struct WyPrepSmem {
     static constexpr uint32_t K = 0;            // bf16 K tile: 2 K-blocks x (64 rows x 128 B)
-    static constexpr uint32_t KT = 16384;       // bf16 K~ tile, same layout
-    static constexpr uint32_t SL = 32768;       // fp32 L, then T in place (tsw)
-    static constexpr uint32_t BETA = 49152;     // 64 floats
+    static constexpr uint32_t KT = 16384;       // bf16 K~ tile (hi term), same layout
+    static constexpr uint32_t KTLO = 32768;     // bf16 K~ lo term (when handed over), same layout
+    static constexpr uint32_t SL = 49152;       // fp32 L, then T in place (tsw)
+    static constexpr uint32_t BETA = 65536;     // 64 floats
     static constexpr uint32_t BAR = BETA + 256;
     static constexpr uint32_t TMEM_SLOT = BAR + 16;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
-constexpr int WY_PREP_CTAS_PER_SM = 4;
+constexpr int WY_PREP_CTAS_PER_SM = 3;
 
 // Persistent grid of 128-thread CTAs walking the batch's chunks (ChunkWalk).  o_f32 is the
 // output buffer [rows, H, Dv] (bf16) seen as floats; Dv = 128.
 __global__ void __launch_bounds__(128, WY_PREP_CTAS_PER_SM)
 wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kt,
+               const __grid_constant__ CUtensorMap tm_ktlo, int has_lo,
                const float* __restrict__ beta, float* __restrict__ o_f32, int Dv,
                const int32_t* __restrict__ cu, int N, int T, int H, int64_t rows,
                long long limit_ns) {
@@ -59,6 +61,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
     uint8_t* sK = smem + L::K;
     uint8_t* sKT = smem + L::KT;
+    uint8_t* sKTLO = smem + L::KTLO;
     float* sL = reinterpret_cast<float*>(smem + L::SL);
     float* sBeta = reinterpret_cast<float*>(smem + L::BETA);
 
@@ -72,6 +75,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tm_k);
         tc::prefetch_tmap(&tm_kt);
+        if (has_lo) tc::prefetch_tmap(&tm_ktlo);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -80,11 +84,15 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
     const uint32_t tlane = static_cast<uint32_t>(warp * 32) << 16;
 
     auto issue_load = [&](int64_t row, int hh) {
-        tc::mbar_expect_tx(tma_bar, 32768);
+        tc::mbar_expect_tx(tma_bar, has_lo ? 49152 : 32768);
         tc::tma_load_3d(sK, &tm_k, 0, hh, (int)row, tma_bar);
         tc::tma_load_3d(sK + 8192, &tm_k, 64, hh, (int)row, tma_bar);
         tc::tma_load_3d(sKT, &tm_kt, 0, hh, (int)row, tma_bar);
         tc::tma_load_3d(sKT + 8192, &tm_kt, 64, hh, (int)row, tma_bar);
+        if (has_lo) {
+            tc::tma_load_3d(sKTLO, &tm_ktlo, 0, hh, (int)row, tma_bar);
+            tc::tma_load_3d(sKTLO + 8192, &tm_ktlo, 64, hh, (int)row, tma_bar);
+        }
     };
     auto load_beta = [&](int64_t row, int Lc, int hh) {
         return tid < Lc ? __ldg(beta + (row + tid) * H + hh) : 0.f;
@@ -112,12 +120,20 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         tma_pend = false;
         if (tid == 0) {
             tc::fence_after_sync();
-            const uint32_t aK = smem_u32(sK), aKT = smem_u32(sKT);
+            const uint32_t aK = smem_u32(sK), aKT = smem_u32(sKT), aKTLO = smem_u32(sKTLO);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const uint32_t o = (s >> 2) * 8192u + (s & 3) * 32u;
                 tc::mma_bf16(tmem, tc::sw128_desc(aK + o, 16, 1024), tc::sw128_desc(aKT + o, 16, 1024),
                              ID_G, s > 0);
+            }
+            if (has_lo) {  // K K~^T = K K~_hi^T + K K~_lo^T
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint32_t o = (s >> 2) * 8192u + (s & 3) * 32u;
+                    tc::mma_bf16(tmem, tc::sw128_desc(aK + o, 16, 1024),
+                                 tc::sw128_desc(aKTLO + o, 16, 1024), ID_G, 1);
+                }
             }
             tc::mma_commit(mma_bar);
             mma_pend = true;

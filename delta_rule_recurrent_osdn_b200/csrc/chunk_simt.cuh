@@ -55,7 +55,8 @@ __device__ __forceinline__ float dot_row(const float* __restrict__ a, const floa
 template <int DK, int DV, int BV, int C, typename IO>
 __global__ void __launch_bounds__(256)
 chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
-                      const IO* __restrict__ kt, const IO* __restrict__ v,
+                      const IO* __restrict__ kt, const IO* __restrict__ kt_lo,
+                      const IO* __restrict__ v,
                       const float* __restrict__ beta, float scale, const float* __restrict__ S0,
                       IO* __restrict__ o, float* __restrict__ ST, const int32_t* __restrict__ cu,
                       int N, int T, int H) {
@@ -104,6 +105,13 @@ chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                 xq = load4<IO>(q + off);
                 xk = load4<IO>(k + off);
                 xt = load4<IO>(kt + off);
+                if (kt_lo) {  // k~ handed over as io-dtype hi + lo terms
+                    const float4 xl = load4<IO>(kt_lo + off);
+                    xt.x += xl.x;
+                    xt.y += xl.y;
+                    xt.z += xl.z;
+                    xt.w += xl.w;
+                }
             }
             *reinterpret_cast<float4*>(sQ + t * KS + i) = xq;
             *reinterpret_cast<float4*>(sK + t * KS + i) = xk;

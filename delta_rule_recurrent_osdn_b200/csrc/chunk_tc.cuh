@@ -34,12 +34,12 @@
 // Warp roles (one CTA per (sequence, head, 64 value channels), 288 threads):
 //   chain    warps 0-3: R, W = T R, the [X; P] W product and the output rows (thread t owns
 //            tensor-memory lane t); its leader issues only the two MMA groups the chain waits on;
-//   prep     warps 4-7: the state's split, the [X; P] tiles from the Gram, identity rows in the
-//            T tiles of a short last chunk (the pre-kernel leaves T split into bf16 hi / lo operand
+//   prep     warps 4-7: the state's split, the [X; P] operand from the Gram (split in place in
+//            tensor memory), identity rows in the T tiles of a short last chunk (the pre-kernel leaves T split into bf16 hi / lo operand
 //            rows in the chunk's o rows; they reach the ring stage by TMA);
 //   producer warp 8: TMA loads into a 2-stage ring (no multicast) and the MMAs off the critical
 //            path (Gram, S += K~^T W, the next [K; Q] S^T).  Ring stage i holds [K_i; Q_{i-1}],
-//            K~_{i-1}, V_i and the T_i tiles, for i = 0 .. n (n chunks).
+//            K~_{i-1} (one bf16 term, or hi and lo), V_i and the T_i tiles, for i = 0 .. n (n chunks).
 // The head's two value-tile CTAs run as a 2-CTA cluster: each loads T hi and lo from both
 // 128-byte slices of the o rows, and each overwrites its own slice with outputs, so a CTA stores
 // O_c only after its sibling has loaded stage c (a counter in its shared memory that the
@@ -58,15 +58,14 @@
 namespace osdn {
 
 struct TcSmem {
-    // ring stage: [K;Q] 32K | K~ 16K | V 8K | T hi 8K | T lo 8K.  W = T R reads A as the 64 rows
-    // before each T tile followed by the tile ([V; T hi] and [T hi; T lo]), so W lands in
-    // accumulator lanes 64..127 and the rows in front, which stay unchanged while that MMA runs,
-    // reach only lanes 0..63, which nobody reads
-    static constexpr uint32_t STAGE = 73728;
-    static constexpr uint32_t KQ = 0, KT = 32768, V = 49152, THI = 57344, TLO = 65536;
-    static constexpr uint32_t XHI = 2 * STAGE;        // bf16 [X; P] hi / lo, K-major, 128 x 128 B
-    static constexpr uint32_t XLO = XHI + 16384;
-    static constexpr uint32_t SHI = XLO + 16384;      // bf16 S^T hi / lo, MN-major, 128 x 128 B
+    // ring stage: [K;Q] 32K | K~ hi 16K | K~ lo 16K | V 8K | T hi 8K | T lo 8K.  W = T R reads A
+    // as the 64 rows before each T tile followed by the tile ([V; T hi] and [T hi; T lo]), so W
+    // lands in accumulator lanes 64..127 and the rows in front, which stay unchanged while that
+    // MMA runs, reach only lanes 0..63, which nobody reads.  The K~ lo tile is loaded only when
+    // phase 1 hands K~ over as two bf16 terms.
+    static constexpr uint32_t STAGE = 90112;
+    static constexpr uint32_t KQ = 0, KT = 32768, KTLO = 49152, V = 65536, THI = 73728, TLO = 81920;
+    static constexpr uint32_t SHI = 2 * STAGE;        // bf16 S^T hi / lo, MN-major, 128 x 128 B
     static constexpr uint32_t SLO = SHI + 16384;
     static constexpr uint32_t RHI = SLO + 16384;      // bf16 R (then W) hi / lo, 64 x 128 B
     static constexpr uint32_t RLO = RHI + 8192;
@@ -79,7 +78,10 @@ static_assert(TcSmem::BYTES <= 232448, "shared memory");
 
 // Tensor-memory columns: S; D1 (two buffers: chunk c+1's product is assembled while chunk c is
 // read), D2 and the prep's Gram.  D1 and D2 are 128 columns wide: their MMAs take the hi and lo
-// terms of the right-hand operand side by side (N = 128), and a reader sums the two halves.
+// terms of the right-hand operand side by side (N = 128), and a reader sums the two halves.  The
+// Gram's 64 fp32 columns are read by the prep role and then overwritten with the [X; P] operand
+// of the chain's last MMA, as packed bf16 pairs: the hi term in columns G..G+31, the lo term in
+// G+32..G+63 (the next Gram is issued only after that MMA has completed).
 constexpr uint32_t TC_COL_S = 0, TC_COL_D1 = 64, TC_COL_D2 = 320, TC_COL_G = 448;
 constexpr uint32_t TC_TMEM_COLS = 512;
 constexpr int TC_THREADS = 288;
@@ -130,6 +132,19 @@ __device__ __forceinline__ void mma_split3(uint32_t d_tmem, const uint32_t* z, u
     }
 }
 
+// The same product with Z = [X; P] read from tensor memory: z_tmem holds Z_hi in its first 32
+// columns and Z_lo in the next 32 (two bf16 per column, K = 16 tokens per 8 columns).
+__device__ __forceinline__ void mma_split3_ts(uint32_t d_tmem, uint32_t z_tmem, uint32_t x_hi,
+                                              bool accumulate) {
+    constexpr uint32_t ID_W = tc::idesc(1, 0, 1, 128, 128), ID_N = tc::idesc(1, 0, 1, 128, 64);
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+        const int s = i & 3, lo = i >> 2;
+        tc::mma_bf16_ts(d_tmem, z_tmem + 32 * lo + 8 * s, tc::sw128_desc(x_hi + s * 2048, 8192, 1024),
+                        lo ? ID_N : ID_W, (accumulate || i > 0) ? 1u : 0u);
+    }
+}
+
 // D = A [S_hi | S_lo]^T over K = 128 key channels (N = 128, the halves of D sum to A S^T): A = a
 // ring stage's K-major [K; Q] tile (two 64-channel blocks 16 KB apart), B = the MN-major S^T
 // tiles with the lo term 16 KB after the hi term.
@@ -162,8 +177,8 @@ template <int DV>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_tp,
-                    const float* __restrict__ beta, float scale, const float* __restrict__ S0,
+                    const __grid_constant__ CUtensorMap tm_tp, const __grid_constant__ CUtensorMap tm_ktlo,
+                    int has_lo, const float* __restrict__ beta, float scale, const float* __restrict__ S0,
                     __nv_bfloat16* __restrict__ o, float* __restrict__ ST,
                     const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
     constexpr int DK = 128, BV = 64, C = 64, NVT = DV / BV;
@@ -253,6 +268,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::prefetch_tmap(&tm_kt);
             tc::prefetch_tmap(&tm_v);
             tc::prefetch_tmap(&tm_tp);
+            if (has_lo) tc::prefetch_tmap(&tm_ktlo);
             int pend[2] = {-1, -1};
             uint64_t* last_bar = nullptr;  // this thread's most recent MMA commit
             uint32_t last_par = 0;
@@ -262,13 +278,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int s = i & 1;
                 uint8_t* st = stage(i);
                 const int row = (int)(first + (int64_t)i * C), prow = row - C;
-                tc::mbar_expect_tx(&tma_full[s], L::STAGE);
+                tc::mbar_expect_tx(&tma_full[s], has_lo ? L::STAGE : L::STAGE - 16384u);
                 tc::tma_load_3d(st + L::KQ + 0, &tm_k, 0, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::KQ + 8192, &tm_q, 0, h, prow, &tma_full[s]);
                 tc::tma_load_3d(st + L::KQ + 16384, &tm_k, 64, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::KQ + 24576, &tm_q, 64, h, prow, &tma_full[s]);
                 tc::tma_load_3d(st + L::KT + 0, &tm_kt, 0, h, prow, &tma_full[s]);
                 tc::tma_load_3d(st + L::KT + 8192, &tm_kt, 64, h, prow, &tma_full[s]);
+                if (has_lo) {
+                    tc::tma_load_3d(st + L::KTLO + 0, &tm_ktlo, 0, h, prow, &tma_full[s]);
+                    tc::tma_load_3d(st + L::KTLO + 8192, &tm_ktlo, 64, h, prow, &tma_full[s]);
+                }
                 tc::tma_load_3d(st + L::V, &tm_v, c0, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::THI, &tm_tp, 0, h, row, &tma_full[s]);
                 tc::tma_load_3d(st + L::TLO, &tm_tp, 32, h, row, &tma_full[s]);
@@ -282,6 +302,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int k = 0; k < 4; ++k)
                         tc::mma_bf16(tmem + TC_COL_S, tc::sw128_desc(aKT + k * 2048, 8192, 1024),
                                      tc::sw128_desc(aR[p] + k * 2048, 8192, 1024), ID_3, 1);
+                if (has_lo) {  // + K~_lo^T W_hi
+                    const uint32_t aKL = smem_u32(stage(jj + 1) + L::KTLO);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(tmem + TC_COL_S, tc::sw128_desc(aKL + k * 2048, 8192, 1024),
+                                     tc::sw128_desc(aR[0] + k * 2048, 8192, 1024), ID_3, 1);
+                }
                 tc::mma_commit(mma_s);
                 last_bar = mma_s;
                 last_par = (uint32_t)jj & 1u;
@@ -303,10 +330,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::st_cluster_release(peer_ctr, (uint32_t)i + 1u);
                 {
                     const uint32_t aKQ = smem_u32(stage(i) + L::KQ), aKT = smem_u32(stage(i) + L::KT);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        tc::mma_bf16(tmem + TC_COL_G, tc::sw128_desc(aKQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                                     tc::sw128_desc(aKT + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), ID_G, k > 0);
+                    const int nk = has_lo ? 16 : 8;  // K~ = hi (+ lo): the lo term accumulates
+#pragma unroll 1
+                    for (int k = 0; k < nk; ++k)
+                        tc::mma_bf16(tmem + TC_COL_G, tc::sw128_desc(aKQ + ((k >> 2) & 1) * 16384 + (k & 3) * 32, 16, 1024),
+                                     tc::sw128_desc(aKT + (k >> 3) * (L::KTLO - L::KT) + ((k >> 2) & 1) * 8192 + (k & 3) * 32, 16, 1024),
+                                     ID_G, k > 0);
                     tc::mma_commit(mma_p);
                     last_bar = mma_p;
                     last_par = (uint32_t)j & 1u;
@@ -383,13 +412,25 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::fence_after_sync();
                 float x[64];
                 tc::tmem_ld64(tmem + lane + (job ? TC_COL_G : TC_COL_S), x);
-                if (job && t >= 64) {
-                    const int r = t - 64;
+                if (job) {  // [X; P] split into the Gram's own columns (the chain's MMA reads it there)
+                    if (t >= 64) {
+                        const int r = t - 64;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) x[c] = c <= r ? x[c] : 0.f;
+                        for (int c = 0; c < 64; ++c) x[c] = c <= r ? x[c] : 0.f;
+                    }
+                    uint32_t hw[32], lw[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) split2_bf16(x[2 * c], x[2 * c + 1], hw[c], lw[c]);
+                    const uint32_t tg = tmem + lane + TC_COL_G;
+                    tc::tmem_st16(tg + 0, reinterpret_cast<const float*>(hw));
+                    tc::tmem_st16(tg + 16, reinterpret_cast<const float*>(hw + 16));
+                    tc::tmem_st16(tg + 32, reinterpret_cast<const float*>(lw));
+                    tc::tmem_st16(tg + 48, reinterpret_cast<const float*>(lw + 16));
+                    tc::tmem_st_wait();
+                } else {
+                    st_row_split_bf16(smem + L::SHI, smem + L::SLO, t, x);
+                    tc::fence_async_smem();
                 }
-                st_row_split_bf16(smem + (job ? L::XHI : L::SHI), smem + (job ? L::XLO : L::SLO), t, x);
-                tc::fence_async_smem();
                 tc::fence_before_sync();
                 group_bar(2, 128);
                 if (leader) mbar_arrive(job ? zxp_full : s_ready);
@@ -413,7 +454,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool lower = t < 64, leader = t == 0 || t == 64;
         const int gbar = lower ? 1 : 3;  // each half's own named barrier
         const uint32_t t_S = tmem + lane + TC_COL_S, t_D2 = tmem + lane + TC_COL_D2;
-        const uint32_t aXP[2] = {smem_u32(smem + L::XHI), smem_u32(smem + L::XLO)};
         bool ok = true;
         uint64_t* last_bar = nullptr;  // the lower leader's most recent commit
         uint32_t last_par = 0;
@@ -508,7 +548,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (leader) {
                     tc::fence_after_sync();
-                    mma_split3(tmem + TC_COL_D1 + 128 * ((j + 1) & 1), aXP, aR[0], true);
+                    mma_split3_ts(tmem + TC_COL_D1 + 128 * ((j + 1) & 1), tmem + TC_COL_G, aR[0], true);
                     tc::mma_commit(mma_crit);
                     last_bar = mma_crit;
                     last_par = (uint32_t)j & 1u;

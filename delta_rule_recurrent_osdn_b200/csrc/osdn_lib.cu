@@ -19,6 +19,7 @@
 #include "chunk_prep.cuh"
 #include "step.cuh"
 #include "scan_tc.cuh"
+#include "rho_geomean.cuh"
 
 namespace osdn {
 namespace {
@@ -67,27 +68,27 @@ inline bool set_smem(KernelT kernel, size_t bytes) {
 // ---------------------------------------------------------------- phase 1 dispatch
 template <typename IO>
 osdn_status_t launch_scan_warp(const void* k, const float* beta, const float* r, float eta,
-                               const float* d0, void* k_tilde, float* dT, float* rho, const int32_t* cu,
-                               const Dims& d, cudaStream_t stream) {
+                               const float* d0, void* k_tilde, void* kt_lo, float* dT, float* rho,
+                               const int32_t* cu, const Dims& d, cudaStream_t stream) {
     const int units = d.N * d.H;
     if (units == 0) return OSDN_OK;
     const dim3 block(128), grid((units + 3) / 4);
     if (d.Dk == 128)
         precond_scan_warp_kernel<128, IO><<<grid, block, 0, stream>>>(
-            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, rho, cu, d.N,
-            d.T, d.H);
+            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde),
+            static_cast<IO*>(kt_lo), dT, rho, cu, d.N, d.T, d.H);
     else
         precond_scan_warp_kernel<64, IO><<<grid, block, 0, stream>>>(
-            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde), dT, rho, cu, d.N,
-            d.T, d.H);
+            static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde),
+            static_cast<IO*>(kt_lo), dT, rho, cu, d.N, d.T, d.H);
     return launch_status();
 }
 
 // ---------------------------------------------------------------- phase 2 dispatch
 template <int DK, int DV, int C, typename IO>
-osdn_status_t launch_chunk_simt(const void* q, const void* k, const void* kt, const void* v,
-                                const float* beta, float scale, const float* S0, void* o,
-                                float* ST, const int32_t* cu, const Dims& d,
+osdn_status_t launch_chunk_simt(const void* q, const void* k, const void* kt, const void* kt_lo,
+                                const void* v, const float* beta, float scale, const float* S0,
+                                void* o, float* ST, const int32_t* cu, const Dims& d,
                                 cudaStream_t stream) {
     constexpr int BV = 32;
     const int64_t ctas = (int64_t)d.N * d.H * (DV / BV);
@@ -98,25 +99,26 @@ osdn_status_t launch_chunk_simt(const void* q, const void* k, const void* kt, co
     if (!set_smem(kernel, smem)) return OSDN_ERR_CUDA;
     kernel<<<dim3((unsigned)ctas), dim3(256), smem, stream>>>(
         static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(kt),
-        static_cast<const IO*>(v), beta, scale, S0, static_cast<IO*>(o), ST, cu, d.N, d.T, d.H);
+        static_cast<const IO*>(kt_lo), static_cast<const IO*>(v), beta, scale, S0,
+        static_cast<IO*>(o), ST, cu, d.N, d.T, d.H);
     return launch_status();
 }
 
 template <int DK, int DV, typename IO>
 osdn_status_t launch_chunk_c(int chunk, const void* q, const void* k, const void* kt,
-                             const void* v, const float* beta, float scale, const float* S0,
-                             void* o, float* ST, const int32_t* cu, const Dims& d,
-                             cudaStream_t stream) {
+                             const void* kt_lo, const void* v, const float* beta, float scale,
+                             const float* S0, void* o, float* ST, const int32_t* cu,
+                             const Dims& d, cudaStream_t stream) {
     switch (chunk) {
         case 16:
-            return launch_chunk_simt<DK, DV, 16, IO>(q, k, kt, v, beta, scale, S0, o, ST, cu, d,
-                                                     stream);
+            return launch_chunk_simt<DK, DV, 16, IO>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
+                                                     d, stream);
         case 32:
-            return launch_chunk_simt<DK, DV, 32, IO>(q, k, kt, v, beta, scale, S0, o, ST, cu, d,
-                                                     stream);
+            return launch_chunk_simt<DK, DV, 32, IO>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
+                                                     d, stream);
         case 64:
-            return launch_chunk_simt<DK, DV, 64, IO>(q, k, kt, v, beta, scale, S0, o, ST, cu, d,
-                                                     stream);
+            return launch_chunk_simt<DK, DV, 64, IO>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
+                                                     d, stream);
         default:
             return OSDN_ERR_UNSUPPORTED;
     }
@@ -177,8 +179,8 @@ int sm_count() {
 // Phase 1, bf16 with 128 key channels: T_d of every chunk (prep kernel, written into the k~
 // buffer), then the chain across chunks (one CTA per (sequence, head)).
 osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, float eta,
-                             const float* d0, void* k_tilde, float* dT, float* rho, const int32_t* cu,
-                             const Dims& d, cudaStream_t stream) {
+                             const float* d0, void* k_tilde, void* kt_lo, float* dT, float* rho,
+                             const int32_t* cu, const Dims& d, cudaStream_t stream) {
     const int64_t nh = (int64_t)d.N * d.H;
     if (nh == 0) return OSDN_OK;
     if (nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
@@ -200,22 +202,23 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     auto chain = precond_chain_kernel;
     if (!set_smem(chain, ScanChainSmem::BYTES)) return OSDN_ERR_CUDA;
     chain<<<dim3((unsigned)nh), dim3(SCAN_CHAIN_THREADS), ScanChainSmem::BYTES, stream>>>(
-        mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde), dT, rho, cu, d.N, d.T, d.H,
-        (long long)kWaitLimitNs);
+        mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde),
+        static_cast<__nv_bfloat16*>(kt_lo), dT, rho, cu, d.N, d.T, d.H, (long long)kWaitLimitNs);
     return launch_status();
 }
 
 // Phase 1: bf16 keys with 128 channels use the chunk-parallel kernel; fp32 I/O, 64 channels
-// and token-free calls use the warp-per-(sequence, head) scan.
+// and token-free calls use the warp-per-(sequence, head) scan.  kt_lo (bf16 only; may be null):
+// also write the residual bf16(k~ - k~_hi) of each key's rounding.
 template <typename IO>
 osdn_status_t launch_scan(const void* k, const float* beta, const float* r, float eta,
-                          const float* d0, void* k_tilde, float* dT, float* rho, const int32_t* cu,
-                          const Dims& d, cudaStream_t stream) {
+                          const float* d0, void* k_tilde, void* kt_lo, float* dT, float* rho,
+                          const int32_t* cu, const Dims& d, cudaStream_t stream) {
     if constexpr (sizeof(IO) == 2) {
         if (d.Dk == 128 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
-            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, dT, rho, cu, d, stream);
+            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, kt_lo, dT, rho, cu, d, stream);
     }
-    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, dT, rho, cu, d, stream);
+    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, kt_lo, dT, rho, cu, d, stream);
 }
 
 // 3-D fp32 view [rows][H][Dv / 2] of the bf16 output buffer; boxes of 32 values (one 128-byte
@@ -236,17 +239,20 @@ bool make_tp_map(CUtensorMap* m, const void* o, int Dv, int H, int64_t rows) {
 // written into o as bf16 hi / lo operand rows), then one CTA per (sequence, head, 64 value
 // channels) for the state chain, the head's two CTAs as a cluster.
 template <int DV>
-osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, const void* v,
-                              const float* beta, float scale, const float* S0, void* o,
-                              float* ST, const int32_t* cu, const Dims& d, cudaStream_t stream) {
+osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, const void* kt_lo,
+                              const void* v, const float* beta, float scale, const float* S0,
+                              void* o, float* ST, const int32_t* cu, const Dims& d,
+                              cudaStream_t stream) {
     const int64_t ctas = (int64_t)d.N * d.H * (DV / 64);
     if (ctas == 0) return OSDN_OK;
     if (ctas > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
-    CUtensorMap mq, mk, mkt, mv, mtp;
+    CUtensorMap mq, mk, mkt, mktlo, mv, mtp;
     const int64_t rows = d.rows();  // > 0 on this path
+    const int has_lo = kt_lo != nullptr;
     if (!make_tile_map(&mq, q, 128, d.H, rows) || !make_tile_map(&mk, k, 128, d.H, rows) ||
         !make_tile_map(&mkt, kt, 128, d.H, rows) || !make_tile_map(&mv, v, DV, d.H, rows) ||
-        !make_tp_map(&mtp, o, DV, d.H, rows))
+        !make_tp_map(&mtp, o, DV, d.H, rows) ||
+        !make_tile_map(&mktlo, has_lo ? kt_lo : kt, 128, d.H, rows))
         return OSDN_ERR_CUDA;
     const int64_t items = ((rows + 63) / 64) * d.H;
     int64_t grid = (int64_t)WY_PREP_CTAS_PER_SM * sm_count();
@@ -254,7 +260,8 @@ osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, cons
     auto prep = wy_prep_kernel;
     if (!set_smem(prep, WyPrepSmem::BYTES)) return OSDN_ERR_CUDA;
     prep<<<dim3((unsigned)grid), dim3(128), WyPrepSmem::BYTES, stream>>>(
-        mk, mkt, beta, static_cast<float*>(o), DV, cu, d.N, d.T, d.H, rows, (long long)kWaitLimitNs);
+        mk, mkt, mktlo, has_lo, beta, static_cast<float*>(o), DV, cu, d.N, d.T, d.H, rows,
+        (long long)kWaitLimitNs);
     const osdn_status_t st = launch_status();
     if (st != OSDN_OK) return st;
     auto kernel = chunk_fwd_tc_kernel<DV>;
@@ -272,34 +279,36 @@ osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, cons
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, mq, mk, mkt, mv, mtp, beta, scale, S0,
+    if (cudaLaunchKernelEx(&cfg, kernel, mq, mk, mkt, mv, mtp, mktlo, has_lo, beta, scale, S0,
                            static_cast<__nv_bfloat16*>(o), ST, cu, d.N, d.T, d.H,
                            (long long)kWaitLimitNs) != cudaSuccess)
         return OSDN_ERR_CUDA;
     return launch_status();
 }
 
+// kt_lo (may be null): the lo term of K~ handed over as bf16 hi + lo (k~ = kt + kt_lo).
 template <typename IO>
 osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* kt,
-                           const void* v, const float* beta, float scale, const float* S0,
-                           void* o, float* ST, const int32_t* cu, const Dims& d,
+                           const void* kt_lo, const void* v, const float* beta, float scale,
+                           const float* S0, void* o, float* ST, const int32_t* cu, const Dims& d,
                            cudaStream_t stream) {
     // bf16 I/O with 128 key and 128 value channels runs on the tensor cores; fp32 I/O, 64-channel
     // heads and token-free calls (states pass through) run the fp32 SIMT kernel.
     if constexpr (sizeof(IO) == 2) {
         if (d.Dk == 128 && d.Dv == 128 && chunk == 64 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
-            return launch_chunk_tc<128>(q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
+            return launch_chunk_tc<128>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d, stream);
     }
     if (d.Dk == 128 && d.Dv == 128)
-        return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
-                                            stream);
+        return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
+                                            d, stream);
     if (d.Dk == 128 && d.Dv == 64)
-        return launch_chunk_c<128, 64, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+        return launch_chunk_c<128, 64, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d,
                                            stream);
     if (d.Dk == 64 && d.Dv == 128)
-        return launch_chunk_c<64, 128, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d,
+        return launch_chunk_c<64, 128, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d,
                                            stream);
-    return launch_chunk_c<64, 64, IO>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu, d, stream);
+    return launch_chunk_c<64, 64, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d,
+                                      stream);
 }
 
 osdn_status_t validate_scan(const void* k, const float* beta, const float* r, const float* d0,
@@ -404,8 +413,9 @@ osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r
     if (st != OSDN_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16)
-        return launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, k_tilde, dT, rho, cu_seqlens, d, s);
-    return launch_scan<float>(k, beta, r, eta, d0, k_tilde, dT, rho, cu_seqlens, d, s);
+        return launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, k_tilde, nullptr, dT, rho, cu_seqlens,
+                                          d, s);
+    return launch_scan<float>(k, beta, r, eta, d0, k_tilde, nullptr, dT, rho, cu_seqlens, d, s);
 }
 
 osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, const void* v,
@@ -421,16 +431,22 @@ osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, 
     if (st != OSDN_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16)
-        return launch_chunk<__nv_bfloat16>(chunk, q, k, k_tilde, v, beta, scale, S0, o, ST,
+        return launch_chunk<__nv_bfloat16>(chunk, q, k, k_tilde, nullptr, v, beta, scale, S0, o, ST,
                                            cu_seqlens, d, s);
-    return launch_chunk<float>(chunk, q, k, k_tilde, v, beta, scale, S0, o, ST, cu_seqlens, d, s);
+    return launch_chunk<float>(chunk, q, k, k_tilde, nullptr, v, beta, scale, S0, o, ST, cu_seqlens,
+                               d, s);
+}
+
+// Workspace of osdn_fwd: k~ (used when the caller passes no k_tilde_out), then, for bf16, the
+// residual of k~'s rounding to bf16, each part rounded up to 256 bytes.
+static size_t kt_part_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io) {
+    return (((size_t)B * T * H * Dk * io_size(io)) + 255) & ~(size_t)255;
 }
 
 size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io) {
     if (B < 0 || T < 0 || H < 1 || (Dk != 64 && Dk != 128) || (io != OSDN_BF16 && io != OSDN_F32))
         return 0;
-    const size_t raw = (size_t)B * T * H * Dk * io_size(io);
-    return (raw + 255) & ~(size_t)255;
+    return kt_part_bytes(B, T, H, Dk, io) * (io == OSDN_BF16 ? 2 : 1);
 }
 
 osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
@@ -443,13 +459,18 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
     osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
     if (st != OSDN_OK) return st;
     d.Dv = Dv;
-    // where the preconditioned keys go: the caller's buffer, else the workspace
-    void* kt = k_tilde_out;
+    // where the preconditioned keys go: the caller's buffer, else the workspace's first part; for
+    // bf16 the residual of their rounding goes to the workspace's second part, so phase 2 uses k~
+    // to about 2^-17 of its size rather than to bf16's 2^-9
     const size_t need = osdn_fwd_workspace_bytes(B, T, H, Dk, io);
-    if (!kt && need > 0) {
+    void* kt = k_tilde_out;
+    void* kt_lo = nullptr;
+    if (need > 0) {
         if (!workspace || workspace_bytes < need) return OSDN_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(workspace) & 255u) return OSDN_ERR_ALIGNMENT;
-        kt = workspace;
+        const size_t part = kt_part_bytes(B, T, H, Dk, io);
+        if (!kt) kt = workspace;
+        if (io == OSDN_BF16) kt_lo = static_cast<uint8_t*>(workspace) + part;
     }
     st = validate_scan(k, beta, r, d0, kt, dT, rho, d, io);
     if (st != OSDN_OK) return st;
@@ -459,6 +480,12 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
     const size_t kb = (size_t)d.rows() * d.H * d.Dk * es, vb = (size_t)d.rows() * d.H * d.Dv * es;
     const size_t db = (size_t)d.N * d.H * d.Dk * 4;
     const size_t gb = (size_t)d.rows() * d.H * 4;
+    // the lo part is written by phase 1 like k~ itself and read by phase 2 like k~
+    if (kt_lo && (validate_scan(k, beta, r, d0, kt_lo, dT, rho, d, io) != OSDN_OK ||
+                  validate_chunk(q, k, kt_lo, v, beta, S0, o, ST, d, chunk, io) != OSDN_OK ||
+                  overlaps(kt_lo, kb, kt, kb) || overlaps(kt_lo, kb, q, kb) ||
+                  overlaps(kt_lo, kb, v, vb)))
+        return OSDN_ERR_INVALID_ARG;
     if (overlaps(kt, kb, q, kb) || overlaps(kt, kb, v, vb) || overlaps(o, vb, dT, db) ||
         overlaps(o, vb, rho, gb) || overlaps(rho, gb, q, kb) || overlaps(rho, gb, v, vb) ||
         overlaps(rho, gb, S0, (size_t)d.N * d.H * d.Dv * d.Dk * 4) ||
@@ -466,14 +493,15 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
         return OSDN_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16) {
-        st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, dT, rho, cu_seqlens, d, s);
+        st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, kt_lo, dT, rho, cu_seqlens, d, s);
         if (st != OSDN_OK) return st;
-        return launch_chunk<__nv_bfloat16>(chunk, q, k, kt, v, beta, scale, S0, o, ST,
+        return launch_chunk<__nv_bfloat16>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST,
                                            cu_seqlens, d, s);
     }
-    st = launch_scan<float>(k, beta, r, eta, d0, kt, dT, rho, cu_seqlens, d, s);
+    st = launch_scan<float>(k, beta, r, eta, d0, kt, nullptr, dT, rho, cu_seqlens, d, s);
     if (st != OSDN_OK) return st;
-    return launch_chunk<float>(chunk, q, k, kt, v, beta, scale, S0, o, ST, cu_seqlens, d, s);
+    return launch_chunk<float>(chunk, q, k, kt, nullptr, v, beta, scale, S0, o, ST, cu_seqlens, d,
+                               s);
 }
 
 osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
@@ -507,6 +535,23 @@ osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float
                                                    scale, S, d, o, k_tilde, rho, nh, Dk, Dv, s);
     return osdn::launch_step_io<float>(q, k, v, beta, r, alpha, alpha_per_channel, eta, scale, S, d,
                                        o, k_tilde, rho, nh, Dk, Dv, s);
+}
+
+osdn_status_t osdn_rho_geomean(const float* rho, const int32_t* cu_seqlens, int32_t num_seqs,
+                               int32_t B, int32_t T, int32_t H, float* q_geo, void* stream) {
+    if (B < 0 || T < 0 || H < 1 || num_seqs < 0) return OSDN_ERR_INVALID_ARG;
+    if (cu_seqlens && B != 1) return OSDN_ERR_INVALID_ARG;
+    const int64_t N = cu_seqlens ? num_seqs : B;
+    const int64_t units = N * H;
+    if (units == 0) return OSDN_OK;
+    if (units > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    if (!q_geo || ((int64_t)B * T > 0 && !rho)) return OSDN_ERR_INVALID_ARG;
+    if ((rho && !aligned16(rho)) || !aligned16(q_geo) || (cu_seqlens && !aligned16(cu_seqlens)))
+        return OSDN_ERR_ALIGNMENT;
+    if (overlaps(rho, (size_t)B * T * H * 4, q_geo, (size_t)units * 4)) return OSDN_ERR_INVALID_ARG;
+    rho_geomean_kernel<<<dim3((unsigned)units), dim3(GEOMEAN_THREADS), 0,
+                         static_cast<cudaStream_t>(stream)>>>(rho, cu_seqlens, (int)N, T, H, q_geo);
+    return launch_status();
 }
 
 osdn_status_t osdn_get_device_status(void* stream) {
@@ -548,19 +593,41 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratch
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
+void* g_noalloc_ctx[kMaxDevices] = {};  // the CUDA context the cached address belongs to
+
+// cuCtxGetCurrent from the driver, looked up once through the runtime.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(p);
+    }();
+    return fn;
+}
 
 // Device address of the array on the current device.  In host code the array's name is only a
-// host-side stand-in, so the address is looked up once per device (with that device current)
-// and cached.
+// host-side stand-in, so the address is looked up with that device current and cached, together
+// with the context it was found in; a new context (after cudaDeviceReset, say) looks it up anew
+// instead of reusing an address that no longer exists.
 osdn_status_t noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OSDN_ERR_CUDA;
+    CtxGetCurrentFn get_ctx = ctx_get_current();
+    CUcontext ctx = nullptr;  // null until the runtime has made a context current on this thread
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return OSDN_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
+    if (ctx == nullptr || g_noalloc_ptr[dev] == nullptr ||
+        g_noalloc_ctx[dev] != static_cast<void*>(ctx)) {
+        void* p = nullptr;  // the lookup also sets up the device's context when there is none yet
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
             return OSDN_ERR_CUDA;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return OSDN_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
+        g_noalloc_ctx[dev] = static_cast<void*>(ctx);
     }
     *out = g_noalloc_ptr[dev];
     return OSDN_OK;
@@ -581,7 +648,7 @@ extern "C" osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const vo
         return OSDN_ERR_INVALID_ARG;
     if (Dk != 64 && Dk != 128) return OSDN_ERR_UNSUPPORTED;
     const size_t need = osdn_fwd_workspace_bytes(B, T, H, Dk, io);
-    if (need > kNoallocScratchBytes) return OSDN_ERR_UNSUPPORTED;  // keys do not fit the array
+    if (need > kNoallocScratchBytes) return OSDN_ERR_UNSUPPORTED;  // the hand-off does not fit
     void* scratch = nullptr;
     if (need > 0) {
         const osdn_status_t st = noalloc_scratch(&scratch);

@@ -327,17 +327,21 @@ struct ScanChainSmem {
     static constexpr uint32_t X = D + 3 * 512;        // 3 x x [64]
     static constexpr uint32_t GX = X + 3 * 256;       // g (.) x [64]
     static constexpr uint32_t BV = GX + 256;          // b [64]
-    static constexpr uint32_t BAR = BV + 256;         // 15 mbarriers
+    static constexpr uint32_t LO = BV + 256;          // bf16 k~ lo staging tile (16 KB, SW128)
+    static constexpr uint32_t BAR = LO + 16384;       // 15 mbarriers
     static constexpr uint32_t TOTAL = BAR + 15 * 8;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
 constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output, 8 loads and gates
 
 // One CTA per (sequence, head).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
+// k_tilde receives k~ rounded to bf16 (hi); k_tilde_lo, when not null, receives the rounding
+// residual bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.
 __global__ void __launch_bounds__(SCAN_CHAIN_THREADS, 1)
 precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_td,
                      const float* __restrict__ beta, const float* __restrict__ r, float eta,
                      const float* __restrict__ d0, __nv_bfloat16* __restrict__ k_tilde,
+                     __nv_bfloat16* __restrict__ k_tilde_lo,
                      float* __restrict__ dT, float* __restrict__ rho,
                      const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
     constexpr int C = SCAN_C, DK = 128;
@@ -563,6 +567,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             // scattered 2-byte stores would cost about three times the whole token pass
             uint8_t* stage = smem + L::TD + s * 16384;
             uint8_t* ocol = stage + blk * 8192u + ce * 2;
+            uint8_t* lcol = smem + L::LO + blk * 8192u + ce * 2;
 #pragma unroll 1
             for (int t0 = 0; t0 < Lc; t0 += 16) {
                 float kv[16], xt[16], rt[16];
@@ -575,24 +580,34 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 }
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    *reinterpret_cast<__nv_bfloat16*>(ocol + tc::sw128_off(t0 + u, cj)) =
-                        __float2bfloat16_rn(dd * kv[u]);
+                    const float kt = dd * kv[u];
+                    const __nv_bfloat16 hb = __float2bfloat16_rn(kt);
+                    *reinterpret_cast<__nv_bfloat16*>(ocol + tc::sw128_off(t0 + u, cj)) = hb;
+                    if (k_tilde_lo)
+                        *reinterpret_cast<__nv_bfloat16*>(lcol + tc::sw128_off(t0 + u, cj)) =
+                            __float2bfloat16_rn(kt - __bfloat162float(hb));
                     dd = fmaf(rt[u], dd, xt[u] * kv[u] * kv[u]);
                 }
             }
             group_bar(2, 128);
             {
                 const int piece = i & 15, blk16 = piece >> 3, j16 = piece & 7;
-                __nv_bfloat16* orow = k_tilde + ((first + (int64_t)c * C) * H + h) * DK + 8 * piece;
+                const int64_t off = ((first + (int64_t)c * C) * H + h) * DK + 8 * piece;
                 const int64_t rs = (int64_t)H * DK;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int row = (i >> 4) + 8 * q;
-                    if (row < Lc)
-                        *reinterpret_cast<uint4*>(orow + row * rs) = *reinterpret_cast<const uint4*>(
-                            stage + blk16 * 8192u + tc::sw128_off(row, j16));
+                    if (row < Lc) {
+                        const uint32_t so = blk16 * 8192u + tc::sw128_off(row, j16);
+                        *reinterpret_cast<uint4*>(k_tilde + off + row * rs) =
+                            *reinterpret_cast<const uint4*>(stage + so);
+                        if (k_tilde_lo)
+                            *reinterpret_cast<uint4*>(k_tilde_lo + off + row * rs) =
+                                *reinterpret_cast<const uint4*>(smem + L::LO + so);
+                    }
                 }
             }
+            if (k_tilde_lo) group_bar(2, 128);  // the single lo staging tile is read out
             mbar_arrive(&kempty[s]);
             mbar_arrive(&outdone[c % 3]);
         }

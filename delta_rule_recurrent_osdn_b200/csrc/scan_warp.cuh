@@ -21,7 +21,8 @@ template <int DK, typename IO>
 __global__ void __launch_bounds__(128)
 precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
                          const float* __restrict__ r, float eta, const float* __restrict__ d0,
-                         IO* __restrict__ k_tilde, float* __restrict__ dT, float* __restrict__ rho,
+                         IO* __restrict__ k_tilde, IO* __restrict__ k_tilde_lo,
+                         float* __restrict__ dT, float* __restrict__ rho,
                          const int32_t* __restrict__ cu, int N, int T, int H) {
     static_assert(DK == 64 || DK == 128, "DK");
     constexpr int E = DK / 32;  // consecutive channels per lane
@@ -41,6 +42,7 @@ precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ bet
     const int64_t rs = (int64_t)H * DK;  // row stride between tokens
     const IO* kp = k + (first * H + h) * DK + lane * E;
     IO* ktp = k_tilde + (first * H + h) * DK + lane * E;
+    IO* klp = k_tilde_lo ? k_tilde_lo + (first * H + h) * DK + lane * E : nullptr;
     const float* bp = beta + first * H + h;
     const float* rp = r ? r + first * H + h : nullptr;
 
@@ -89,6 +91,16 @@ precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ bet
                     store4<IO>(ktp + t * rs, make_float4(kt[0], kt[1], kt[2], kt[3]));
                 else
                     store2<IO>(ktp + t * rs, make_float2(kt[0], kt[1]));
+                if (klp) {  // the io rounding's residual: k~ = hi + lo to about 2^-17 in bf16
+                    float lo[E];
+#pragma unroll
+                    for (int e = 0; e < E; ++e)
+                        lo[e] = kt[e] - io_traits<IO>::to_f32(io_traits<IO>::from_f32(kt[e]));
+                    if constexpr (E == 4)
+                        store4<IO>(klp + t * rs, make_float4(lo[0], lo[1], lo[2], lo[3]));
+                    else
+                        store2<IO>(klp + t * rs, make_float2(lo[0], lo[1]));
+                }
                 if (rho && lane == 0) rho[(first + t) * H + h] = (1.f - bt * s) * (1.f - bt * s);
                 const float coef = nk > 0.f ? eta * bt * (1.0f - bt * s) / nk : 0.f;
 #pragma unroll

@@ -105,6 +105,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "l"(adesc), "l"(bdesc), "r"(id), "r"(accumulate)
         : "memory");
 }
+// The same MMA with the A operand read from tensor memory: M = 128 rows in lanes 0..127 of
+// `a_tmem`'s columns, K-major, two consecutive bf16 elements of a row per 32-bit column (the
+// lower half holding the even element), so K = 16 spans 8 columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t id, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(id), "r"(accumulate)
+        : "memory");
+}
 __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t id, uint32_t accumulate) {
     asm volatile(

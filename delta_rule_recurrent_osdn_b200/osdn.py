@@ -65,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _vp, _vp, _vp,
                               _vp, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_step.restype = ctypes.c_int
+    lib.osdn_rho_geomean.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
+    lib.osdn_rho_geomean.restype = ctypes.c_int
     lib.osdn_get_device_status.argtypes = [_vp]
     lib.osdn_get_device_status.restype = ctypes.c_int
     lib.osdn_debug_watchdog_selftest.argtypes = [ctypes.c_int64, _vp]
@@ -190,8 +192,9 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
              workspace=None, return_states: bool = True, rho=None, stream=None):
     """Both phases: returns ``(o, ST, dT)`` (states None when ``return_states`` is False).
 
-    When neither ``k_tilde`` nor ``workspace`` is given, a workspace of
-    ``osdn_fwd_workspace_bytes`` bytes is allocated with torch (device memory plumbing).
+    The call needs a device workspace of ``osdn_fwd_workspace_bytes`` bytes (for bf16 it holds
+    the residual of k~'s rounding, and k~ itself when ``k_tilde`` is not given); when
+    ``workspace`` is None it is allocated with torch (device memory plumbing).
     """
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
@@ -217,17 +220,16 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
     _req(dT, "dT", torch.float32, (N, H, Dk))
     _req(rho, "rho", torch.float32, (B, T, H))
     ws_bytes = 0
-    if k_tilde is None:
-        need = int(LIB.osdn_fwd_workspace_bytes(B, T, H, Dk, io))
-        if workspace is None and need > 0:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-        if workspace is not None:
-            _req(workspace, "workspace")
-            ws_bytes = workspace.numel() * workspace.element_size()
+    need = int(LIB.osdn_fwd_workspace_bytes(B, T, H, Dk, io))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _req(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
     _check(LIB.osdn_fwd(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), _p(d0), _p(S0),
                         float(scale), _p(o), _p(ST), _p(dT), _p(rho), _p(k_tilde), _p(cu_seqlens),
-                        num_seqs, B, T, H, Dk, Dv, int(chunk), io,
-                        _p(workspace) if k_tilde is None else None, ws_bytes, _stream(stream)),
+                        num_seqs, B, T, H, Dk, Dv, int(chunk), io, _p(workspace), ws_bytes,
+                        _stream(stream)),
            "osdn_fwd")
     return o, ST, dT
 
@@ -260,6 +262,20 @@ def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0,
                          Dk, Dv, io, _stream(stream)),
            "osdn_step")
     return o
+
+
+def osdn_rho_geomean(rho, cu_seqlens=None, q_geo=None, stream=None):
+    """q_geo [N, H] float32: exp(mean_t log rho_t) per (sequence, head), from a residual-ratio
+    tensor rho [B, T, H] (the ``rho`` output of the scan or the forward pass)."""
+    B, T, H = rho.shape
+    _req(rho, "rho", torch.float32)
+    num_seqs, N = _seqs(cu_seqlens, B)
+    if q_geo is None:
+        q_geo = torch.empty((N, H), dtype=torch.float32, device=rho.device)
+    _req(q_geo, "q_geo", torch.float32, (N, H))
+    _check(LIB.osdn_rho_geomean(_p(rho), _p(cu_seqlens), num_seqs, B, T, H, _p(q_geo),
+                                _stream(stream)), "osdn_rho_geomean")
+    return q_geo
 
 
 def osdn_get_device_status(stream=None) -> int:

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define OSDN_ABI_VERSION 3
+#define OSDN_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define OSDN_API __attribute__((visibility("default")))
@@ -124,16 +124,24 @@ OSDN_API osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* 
                              int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                              void* stream);
 
-/* Bytes of device workspace osdn_fwd needs for these sizes (0 when none). */
+/* Bytes of device workspace osdn_fwd needs for these sizes: for bf16, two parts of
+ * B*T*H*Dk*2 bytes each (k~ itself, used when k_tilde_out is NULL, and the residual of k~'s
+ * rounding to bf16), each rounded up to 256 bytes; for fp32, one part of B*T*H*Dk*4 bytes
+ * (rounded up likewise).  0 for unsupported sizes. */
 OSDN_API size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osdn_dtype_t io);
 
 /*
  * Both phases (section 2.2's two-phase forward pass) on one stream.  Arguments are those of
  * osdn_precond_scan and osdn_chunk_fwd; in addition:
  *   k_tilde_out  [B,T,H,Dk] io dtype, or NULL.  When given, the preconditioned keys are
- *                written there and the workspace is not used.
+ *                written there (rounded to the io dtype) instead of to the workspace.
  *   workspace    device scratch of at least osdn_fwd_workspace_bytes(...) bytes, 256-byte
- *                aligned, used when k_tilde_out is NULL; NULL only if that size is 0.
+ *                aligned; NULL only if that size is 0.  In bf16 mode phase 1 hands k~ to
+ *                phase 2 as two bf16 terms, k~ = hi + lo with hi = bf16(k~) and
+ *                lo = bf16(k~ - hi) (about 2^-17 of |k~| left out), and every phase-2 product
+ *                with K~ takes both terms, so phase 2 sees k~ essentially unrounded; the lo
+ *                term lives in the workspace.  (The two-call path osdn_precond_scan ->
+ *                osdn_chunk_fwd hands over hi only.)
  * The buffer rules of both phases apply; o must not overlap dT either.
  */
 OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
@@ -150,14 +158,18 @@ OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, con
  * synchronize the device and fragments a fixed memory budget).  The original paper has no
  * counterpart: this is an interface convenience, not part of the method.
  *
- * Arguments are those of osdn_fwd minus k_tilde_out / workspace.  The preconditioned keys that
- * phase 1 hands to phase 2 go to a fixed device array built into the library,
+ * Arguments are those of osdn_fwd minus k_tilde_out / workspace.  What osdn_fwd keeps in the
+ * caller's workspace (the preconditioned keys phase 1 hands to phase 2, as bf16 hi and lo
+ * terms in bf16 mode) goes to a fixed device array built into the library instead,
  * OSDN_NOALLOC_SCRATCH_BYTES (32 MiB) long, which every GPU that loads the library reserves
  * until the process exits.
- *   - Limit: B * T * H * Dk * sizeof(io element) must not exceed OSDN_NOALLOC_SCRATCH_BYTES;
- *     larger calls return OSDN_ERR_UNSUPPORTED before anything is enqueued.
+ *   - Limit: osdn_fwd_workspace_bytes(B, T, H, Dk, io) must not exceed
+ *     OSDN_NOALLOC_SCRATCH_BYTES (bf16: 2 * B * T * H * Dk * 2 bytes, each half rounded up to
+ *     256 bytes); larger calls return OSDN_ERR_UNSUPPORTED before anything is enqueued.
  *   - The first call on each device (with that device current) looks up the array's device
- *     address and caches it; make that first call before any stream capture.
+ *     address in the device's current CUDA context and caches it; a later call looks it up
+ *     again only if that context has changed (after cudaDeviceReset, for instance).  Make the
+ *     first call on a device before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents.  Phase 1 rewrites
  *     every key before phase 2 reads it, so nothing needs clearing; but calls that overlap on
  *     the GPU (other streams, other host threads) race on it and must be serialized.
@@ -173,11 +185,20 @@ OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void
                                         void* stream);
 
 /*
- * Synchronizes `stream`, then returns and clears the device status word of the current
- * device: OSDN_OK, OSDN_ERR_DEVICE_TIMEOUT or OSDN_ERR_DEVICE_BOUNDS (the first error any
- * kernel recorded since the last call; the word is shared by all streams of the device).
- * Returns OSDN_ERR_CUDA if the synchronization itself fails.
+ * q_geo, the residual-contraction diagnostic of section 3 (Theorem 5.2 bounds the product of
+ * the token-local ratios rho_t = f_t(S_t) / f_t(S_{t-1}); the experiments of section 4.3
+ * report their geometric mean): for every (sequence n, head h),
+ *   q_geo[n][h] = exp( mean over the sequence's tokens of log rho[t][h] ).
+ *   rho     [B,T,H] float32, read: the rho output of osdn_precond_scan or osdn_fwd (any
+ *           non-negative ratios).  A ratio of 0 gives q_geo = 0.
+ *   q_geo   [N,H] float32, written.  A sequence without tokens gets 1 (the empty product).
+ * cu_seqlens, num_seqs, B and T as for the other calls.  Logs are taken in fp32 and summed in
+ * fp64.  Pointers 16-byte aligned; q_geo must not overlap rho (OSDN_ERR_INVALID_ARG).
  */
+OSDN_API osdn_status_t osdn_rho_geomean(const float* rho, const int32_t* cu_seqlens,
+                                        int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                                        float* q_geo, void* stream);
+
 /*
  * One recurrent step per (sequence, head) -- the decode path (sections 2.1-2.3 applied to a
  * single token, the state carried in memory).  For each of the N*H (sequence, head) pairs, with
@@ -206,6 +227,12 @@ OSDN_API osdn_status_t osdn_step(const void* q, const void* k, const void* v, co
                         int32_t N, int32_t H, int32_t Dk, int32_t Dv, osdn_dtype_t io,
                         void* stream);
 
+/*
+ * Synchronizes `stream`, then returns and clears the device status word of the current
+ * device: OSDN_OK, OSDN_ERR_DEVICE_TIMEOUT or OSDN_ERR_DEVICE_BOUNDS (the first error any
+ * kernel recorded since the last call; the word is shared by all streams of the device).
+ * Returns OSDN_ERR_CUDA if the synchronization itself fails.
+ */
 OSDN_API osdn_status_t osdn_get_device_status(void* stream);
 
 /*

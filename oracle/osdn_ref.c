@@ -38,6 +38,7 @@
  *   Packed: B == 1, T = total tokens, N = num_seqs and sequence n is rows
  *   cu_seqlens[n] .. cu_seqlens[n+1]-1 (cu_seqlens is a HOST array of N+1 entries).
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -64,6 +65,27 @@ int osdn_ref_set_threads(int n) {
     (void)n;
     return 1;
 #endif
+}
+
+/* ---------------------------------------------------------------------------------
+ * Residual contraction (section 3, Theorem 5.2; the experiments' q_geo): the geometric mean
+ * of the token-local residual ratios rho_t = f_t(S_t) / f_t(S_{t-1}) of one (sequence, head),
+ *   q_geo = (prod_t rho_t)^(1 / T_n) = exp(mean_t log rho_t),
+ * given rho [B, T, H]; q_geo [N, H].  A ratio of 0 makes q_geo 0; a sequence with no tokens
+ * gets 1 (the empty product).
+ * ------------------------------------------------------------------------------- */
+void osdn_ref_rho_geomean(const double* rho, double* q_geo, const int32_t* cu_seqlens,
+                          int32_t num_seqs, int32_t B, int32_t T, int32_t H) {
+    const int32_t N = cu_seqlens ? num_seqs : B;
+    for (int32_t n = 0; n < N; ++n) {
+        int64_t first, count;
+        seq_bounds(n, cu_seqlens, T, &first, &count);
+        for (int32_t h = 0; h < H; ++h) {
+            double sum_log = 0.0;
+            for (int64_t t = 0; t < count; ++t) sum_log += log(rho[(first + t) * H + h]);
+            q_geo[(int64_t)n * H + h] = count > 0 ? exp(sum_log / (double)count) : 1.0;
+        }
+    }
 }
 
 /* ---------------------------------------------------------------------------------

@@ -109,6 +109,8 @@ class Oracle:
             _D, _D, _D, _D, _D, ctypes.c_double, _D, _D, ctypes.c_double, _D, _i32, _D, _D, _D, _D,
             _D, _D, _D, _D, _D, _D, _D, _D, _I, _i32, _i32, _i32, _i32, _i32, _i32]
         lib.osdn_ref_bwd_gated.restype = None
+        lib.osdn_ref_rho_geomean.argtypes = [_D, _D, _I, _i32, _i32, _i32, _i32]
+        lib.osdn_ref_rho_geomean.restype = None
         self.lib = lib
 
     def set_threads(self, n: int = 0) -> int:
@@ -130,6 +132,22 @@ class Oracle:
         self.lib.osdn_ref_precond_scan(_ptr(k), _ptr(beta), _ptr(r), float(eta), _ptr(d0),
                                        _ptr(k_tilde), _ptr(dT), _ptr(rho), cup, N, B, T, H, Dk)
         return (k_tilde, dT, rho) if with_rho else (k_tilde, dT)
+
+    def rho_geomean(self, rho, cu_seqlens=None, N=None):
+        """q_geo [N, H]: the geometric mean over each sequence's tokens of the residual ratios
+        rho [B, T, H] (section 3; the experiments' q_geo); 0 if a ratio is 0, 1 for a sequence
+        without tokens."""
+        rho = _f64(rho)
+        cu, cup = _cu(cu_seqlens)
+        B, T, H = rho.shape
+        if cu is not None:
+            assert B == 1 and cu[0] == 0 and cu[-1] == T and np.all(np.diff(cu) >= 0)
+            N = len(cu) - 1
+        else:
+            N = B
+        q_geo = np.zeros((N, H))
+        self.lib.osdn_ref_rho_geomean(_ptr(rho), _ptr(q_geo), cup, N, B, T, H)
+        return q_geo
 
     def delta_fwd(self, q, k, k_tilde, v, beta, scale=1.0, S0=None, cu_seqlens=None):
         """Phase 2 (section 2.1): delta rule with write key k_tilde. Returns (o, ST)."""
@@ -259,3 +277,7 @@ def bwd(*args, **kwargs):
 
 def fwd_gated(*args, **kwargs):
     return _oracle().fwd_gated(*args, **kwargs)
+
+
+def rho_geomean(*args, **kwargs):
+    return _oracle().rho_geomean(*args, **kwargs)

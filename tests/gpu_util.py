@@ -1,5 +1,18 @@
 """Shared helpers for the GPU tests: run the library through its binding, run the oracle on the
-same seeded inputs, and measure max|delta| / rms(reference)."""
+same seeded inputs, and measure max|delta| / rms(reference).
+
+Parity bound (written here, not derived from the GPU): max|gpu - oracle| / rms(oracle) <= 1e-2
+for bf16 I/O and <= 1e-4 for fp32 I/O, for o, k~, S_T and d_T.  The one allowance is the
+rounding of each stored result to its own dtype: an element's error first loses half an ulp of
+the exact value in the dtype it is stored in (bf16 for o and k~ in bf16 mode, fp32 for the
+states).  Rounding the exact fp64 o of the 340M and 1.3B workloads to bf16 alone already moves
+it by 1.2% and 1.6% of rms(o), so no bf16 output can meet the bound without it.
+
+The reference of the one-call forward pass (osdn_fwd) is the plain fp64 oracle: nothing is
+rounded between its phases.  Only the two-call path (osdn_precond_scan, then osdn_chunk_fwd),
+whose interface hands k~ over as an io-dtype tensor, is compared with the oracle's phase 2 fed
+that rounded k~.
+"""
 import numpy as np
 import torch
 
@@ -38,20 +51,22 @@ def host(t):
     return None if t is None else t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def gpu_fwd(inp, chunk=None, split=False):
-    """Run the library on one batch; returns numpy (o, k_tilde, ST, dT)."""
+def gpu_fwd(inp, chunk=None, split=False, scale=None):
+    """Run the library on one batch; returns numpy (o, k_tilde, ST, dT).  split=True runs the
+    two phases as two calls (k~ crosses between them as an io-dtype tensor)."""
     from delta_rule_recurrent_osdn_b200 import osdn
     d = W.to_torch(inp)
     chunk = chunk or d["chunk"]
+    sc = d["scale"] if scale is None else scale
     if split:
         kt, dT = osdn.osdn_precond_scan(d["k"], d["beta"], d["r"], d["eta"], d["d0"],
                                         d["cu_seqlens"])
-        o, ST = osdn.osdn_chunk_fwd(d["q"], d["k"], kt, d["v"], d["beta"], d["scale"], d["S0"],
+        o, ST = osdn.osdn_chunk_fwd(d["q"], d["k"], kt, d["v"], d["beta"], sc, d["S0"],
                                     chunk, d["cu_seqlens"])
     else:
         kt = torch.empty_like(d["k"])
         o, ST, dT = osdn.osdn_fwd(d["q"], d["k"], d["v"], d["beta"], d["r"], d["eta"], d["d0"],
-                                  d["S0"], d["scale"], chunk, d["cu_seqlens"], k_tilde=kt)
+                                  d["S0"], sc, chunk, d["cu_seqlens"], k_tilde=kt)
     torch.cuda.synchronize()
     assert osdn.osdn_get_device_status() == osdn.OSDN_OK
     return host(o), host(kt), host(ST), host(dT)
@@ -63,24 +78,22 @@ def round_io(x, io):
     return (W.bf16_round(x) if io == "bf16" else x).astype(np.float64)
 
 
-def oracle_fwd(ref, inp):
-    """Expected (o, k_tilde, ST, dT) for the two-phase forward pass.
-
-    Phase 1 is the oracle's scan.  Phase 2 is the oracle's token loop fed k~ rounded to the io
-    dtype: the two-phase interface hands k~ from the scan to the chunked pass as an io-dtype
-    tensor, so that rounding is part of what the library is asked to compute.  Everything else
-    is fp64.
-    """
-    kt, dT = ref.precond_scan(inp.k, inp.beta, inp.r, inp.eta, inp.d0, inp.cu_seqlens)
-    o, ST = ref.delta_fwd(inp.q, inp.k, round_io(kt, inp.io), inp.v, inp.beta, inp.scale,
-                          inp.S0, inp.cu_seqlens)
+def oracle_fwd(ref, inp, scale=None):
+    """Expected (o, k_tilde, ST, dT) of the forward pass: the fp64 oracle, both phases in one
+    token loop, nothing rounded between them."""
+    o, kt, ST, dT = ref.fwd(inp.q, inp.k, inp.v, inp.beta, inp.r, inp.eta, inp.d0, inp.S0,
+                            inp.scale if scale is None else scale, inp.cu_seqlens)
     return o, kt, ST, dT
 
 
-def oracle_fwd_unrounded(ref, inp):
-    """The fp64 oracle with no io rounding of k~ between the phases (for reporting)."""
-    return ref.fwd(inp.q, inp.k, inp.v, inp.beta, inp.r, inp.eta, inp.d0, inp.S0, inp.scale,
-                   inp.cu_seqlens)
+def oracle_fwd_split(ref, inp, scale=None):
+    """Expected (o, k_tilde, ST, dT) of the two-call path: phase 1 is the oracle's scan; phase 2
+    is the oracle's token loop fed k~ rounded to the io dtype, which is what osdn_chunk_fwd is
+    handed by that interface.  Everything else is fp64."""
+    kt, dT = ref.precond_scan(inp.k, inp.beta, inp.r, inp.eta, inp.d0, inp.cu_seqlens)
+    o, ST = ref.delta_fwd(inp.q, inp.k, round_io(kt, inp.io), inp.v, inp.beta,
+                          inp.scale if scale is None else scale, inp.S0, inp.cu_seqlens)
+    return o, kt, ST, dT
 
 
 # o and k~ are stored in the io dtype, S_T and d_T in float32
@@ -89,7 +102,8 @@ STORED = {"o": None, "k_tilde": None, "ST": "f32", "dT": "f32"}
 
 def check_all(got, want, io, names=("o", "k_tilde", "ST", "dT")):
     """Parity of every output: max|gpu - oracle| / rms(oracle) <= TOL[io], after removing from
-    each element the half-ulp rounding of the exact value to the dtype it is stored in."""
+    each element the half-ulp rounding of the exact value to the dtype it is stored in.
+    Returns both figures per output (the adjusted one is asserted)."""
     errs = {n: rel_err(g, w, STORED[n] or io) for n, g, w in zip(names, got, want)}
     raw = {n: rel_err(g, w) for n, g, w in zip(names, got, want)}
     bad = {n: e for n, e in errs.items() if not e <= TOL[io]}

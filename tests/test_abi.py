@@ -44,14 +44,16 @@ def test_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert L.osdn_abi_version() == 3
+    assert L.osdn_abi_version() == 4
     for s in range(7):
         assert osdn.status_string(s)
     assert osdn.status_string(99) == "unknown status"
 
 
 def test_workspace_size():
-    assert L.osdn_fwd_workspace_bytes(4, 4096, 16, 128, osdn.OSDN_BF16) == 4 * 4096 * 16 * 128 * 2
+    # bf16: k~ and the residual of its rounding, each part rounded up to 256 bytes
+    assert L.osdn_fwd_workspace_bytes(4, 4096, 16, 128, osdn.OSDN_BF16) == 2 * 4 * 4096 * 16 * 128 * 2
+    assert L.osdn_fwd_workspace_bytes(1, 3, 1, 64, osdn.OSDN_BF16) == 2 * 512
     assert L.osdn_fwd_workspace_bytes(1, 3, 1, 64, osdn.OSDN_F32) == 768
     assert L.osdn_fwd_workspace_bytes(1, 1, 1, 96, osdn.OSDN_BF16) == 0
 
@@ -98,6 +100,31 @@ def test_chunk_fwd_rejects(kw, status):
 ])
 def test_precond_scan_rejects(kw, status):
     assert scan_call(**kw) == status
+
+
+def test_fwd_needs_workspace_even_with_k_tilde_out():
+    """In bf16 mode the workspace holds the lo term of k~ even when k~ goes to k_tilde_out."""
+    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
+                    None, None, fake(8), None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16, None, 0,
+                    None)
+    assert st == osdn.OSDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(H=0), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(cu=fake(9), num_seqs=2, B=2), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(rho=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(out=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(out=ctypes.c_void_p(A + 2 * 0x1000000 + 4)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(out=ctypes.c_void_p(A + 1 * 0x1000000 + 16)), osdn.OSDN_ERR_INVALID_ARG),  # in rho
+    (dict(B=0), osdn.OSDN_OK),  # no sequences: nothing to do
+])
+def test_rho_geomean_rejects(kw, status):
+    args = dict(rho=fake(1), cu=None, num_seqs=0, B=2, T=64, H=4, out=fake(2))
+    args.update(kw)
+    assert L.osdn_rho_geomean(args["rho"], args["cu"], args["num_seqs"], args["B"], args["T"],
+                              args["H"], args["out"], None) == status
 
 
 def test_fwd_rejects_small_workspace():

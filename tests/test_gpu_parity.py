@@ -3,21 +3,27 @@
 Tolerance (written here, not derived from the GPU): max|gpu - oracle| / rms(oracle) <= 1e-2
 for bf16 I/O and <= 1e-4 for fp32 I/O, for o, k~ (phase 1 output), S_T and d_T, where each
 element's error first loses half an ulp of the exact value in the dtype the output is stored
-in (bf16 for o and k~ in bf16 mode), and where the oracle's phase 2 consumes k~ rounded to the
-io dtype, as the two-phase interface hands it over.  Without these two io roundings in the
-reference the bound is out of reach of any bf16-I/O implementation: rounding the exact fp64 o
-of the 340M and 1.3B workloads to bf16 already gives 1.2% and 1.6% of rms(o), and rounding
-only k~ to bf16 moves S_T by 1.0-1.9% of rms(S_T) on the bf16 workloads.  The error against
-the fully unrounded oracle is printed for every workload.
+in (bf16 for o and k~ in bf16 mode): rounding the exact fp64 o of the 340M and 1.3B workloads
+to bf16 already gives 1.2% and 1.6% of rms(o).
+
+osdn_fwd, the one-call forward pass, is compared with the plain fp64 oracle: nothing is rounded
+between its phases (phase 1 hands k~ to phase 2 as two bf16 terms).  The two-call path
+(osdn_precond_scan, then osdn_chunk_fwd) hands k~ over as one io-dtype tensor; it is compared
+with the oracle's phase 2 fed that rounded k~.  Each test prints a "PARITY" line with the error
+of every output against both references.
 """
+import json
+
 import numpy as np
 import pytest
 import torch
 
 from delta_rule_recurrent_osdn_b200 import inputs as W
-from tests.gpu_util import TOL, check_all, gpu_fwd, oracle_fwd, rel_err
+from tests.gpu_util import (TOL, check_all, gpu_fwd, oracle_fwd, oracle_fwd_split, rel_err)
 
 pytestmark = pytest.mark.gpu
+
+NAMES = ("o", "k_tilde", "ST", "dT")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -26,17 +32,22 @@ def _cuda():
     torch.cuda.set_device(0)
 
 
+def _report(case, path, got, want, want_split, io):
+    """Asserts parity against `want`; prints both references' errors on one line."""
+    res = check_all(got, want, io)
+    other = {n: rel_err(g, w, None) for n, g, w in zip(NAMES, got, want_split)}
+    print("PARITY " + json.dumps({"case": case, "path": path, "io": io, "vs_oracle": res["err"],
+                                  "vs_oracle_raw": res["raw"],
+                                  "vs_oracle_kt_rounded_raw": other}))
+    return res
+
+
 @pytest.mark.parametrize("name", ["tiny_fp32", "340m", "1p3b_apf"])
 def test_workload_full_parity(ref, name):
-    """Every output of every (sequence, head) against the oracle."""
-    from tests.gpu_util import oracle_fwd_unrounded
+    """Every output of every (sequence, head) against the plain fp64 oracle."""
     inp = W.make_inputs(name)
     got = gpu_fwd(inp)
-    want = oracle_fwd(ref, inp)
-    print(name, check_all(got, want, inp.io))
-    pure = oracle_fwd_unrounded(ref, inp)
-    print(name, "vs unrounded oracle:",
-          {n: rel_err(g, w) for n, g, w in zip(("o", "k_tilde", "ST", "dT"), got, pure)})
+    _report(name, "osdn_fwd", got, oracle_fwd(ref, inp), oracle_fwd_split(ref, inp), inp.io)
 
 
 def test_long_context_sampled_heads(ref):
@@ -45,26 +56,36 @@ def test_long_context_sampled_heads(ref):
     got = gpu_fwd(inp)
     heads = [0, 7, 15]
     sub = W.select(inp, heads=heads)
-    want = oracle_fwd(ref, sub)
     sel = (got[0][:, :, heads], got[1][:, :, heads], got[2][:, heads], got[3][:, heads])
-    print(check_all(sel, want, inp.io))
+    _report("long_ctx[heads 0,7,15]", "osdn_fwd", sel, oracle_fwd(ref, sub),
+            oracle_fwd_split(ref, sub), inp.io)
 
 
 def test_varlen_sampled_sequences(ref):
     """32 packed sequences: the full GPU run, checked on the shortest, the longest and two
-    others, every head."""
+    others, for three heads."""
     inp = W.make_inputs("varlen")
     got = gpu_fwd(inp)
     lens = np.diff(inp.cu_seqlens)
     seqs = sorted({int(np.argmin(lens)), int(np.argmax(lens)), 3, 17})
     heads = [0, 5, 11]
     sub = W.select(inp, seqs=seqs, heads=heads)
-    want = oracle_fwd(ref, sub)
     cu = inp.cu_seqlens
     rows = np.concatenate([np.arange(cu[n], cu[n + 1]) for n in seqs])
     sel = (got[0][:, rows][:, :, heads], got[1][:, rows][:, :, heads],
            got[2][seqs][:, heads], got[3][seqs][:, heads])
-    print(check_all(sel, want, inp.io))
+    _report(f"varlen[seqs {seqs}, heads {heads}]", "osdn_fwd", sel, oracle_fwd(ref, sub),
+            oracle_fwd_split(ref, sub), inp.io)
+
+
+@pytest.mark.parametrize("name", ["340m", "1p3b_apf"])
+def test_two_call_path_parity(ref, name):
+    """osdn_precond_scan then osdn_chunk_fwd: k~ crosses as a bf16 tensor, so phase 2's
+    reference is the oracle's phase 2 on that rounded k~."""
+    inp = W.make_inputs(name)
+    got = gpu_fwd(inp, split=True)
+    _report(name, "osdn_precond_scan+osdn_chunk_fwd", got, oracle_fwd_split(ref, inp),
+            oracle_fwd(ref, inp), inp.io)
 
 
 @pytest.mark.parametrize("name", ["tiny_fp32", "1p3b_apf"])

@@ -62,3 +62,50 @@ def test_step_rho_matches_oracle(ref):
     torch.cuda.synchronize()
     _, _, want = ref.precond_scan(inp.k, inp.beta, inp.r, inp.eta, inp.d0, with_rho=True)
     assert rel_err(host(rho), want[:, 0]) <= 1e-5
+
+
+@pytest.mark.parametrize("case", [
+    dict(lengths=[300, 0, 1, 700, 64], H=3, Dk=128, Dv=128, io="bf16", apf=True, eta=0.05,
+         seed=38, init_state=True),
+    dict(B=2, T=500, H=2, Dk=128, Dv=128, io="bf16", apf=False, eta=0.05, seed=39),
+    dict(B=2, T=150, H=2, Dk=64, Dv=64, io="f32", apf=True, eta=0.1, seed=40),
+])
+def test_q_geo_of_the_forward_pass(ref, case):
+    """q_geo = exp(mean_t log rho_t) per (sequence, head) from the forward pass's rho output,
+    against the oracle's q_geo of the oracle's rho; and against the fp64 host reduction of the
+    GPU's own rho (which isolates the reduction kernel)."""
+    from delta_rule_recurrent_osdn_b200 import osdn
+    inp = W.make_inputs(dict(chunk=64, **case))
+    d = W.to_torch(inp)
+    rho = torch.empty(d["beta"].shape, dtype=torch.float32, device="cuda")
+    osdn.osdn_fwd(d["q"], d["k"], d["v"], d["beta"], d["r"], d["eta"], d["d0"], d["S0"],
+                  d["scale"], 64, d["cu_seqlens"], rho=rho)
+    q_geo = osdn.osdn_rho_geomean(rho, d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert osdn.osdn_get_device_status() == osdn.OSDN_OK
+    got = host(q_geo)
+    own = ref.rho_geomean(host(rho), inp.cu_seqlens)
+    np.testing.assert_allclose(got, own, rtol=1e-5, atol=0)
+    _, _, rho_ref = ref.precond_scan(inp.k, inp.beta, inp.r, inp.eta, inp.d0, inp.cu_seqlens,
+                                     with_rho=True)
+    want = ref.rho_geomean(rho_ref, inp.cu_seqlens)
+    np.testing.assert_allclose(got, want, rtol=1e-3, atol=0)
+    print("q_geo", got.ravel()[:8], "oracle", want.ravel()[:8])
+
+
+def test_q_geo_zero_ratio_and_empty_sequence(ref):
+    """A sequence holding a ratio of exactly 0 has q_geo 0; a sequence without tokens has 1."""
+    from delta_rule_recurrent_osdn_b200 import osdn
+    rng = np.random.default_rng(41)
+    lengths = [5, 0, 1000, 1, 33]
+    T = sum(lengths)
+    rho = rng.uniform(0.05, 1.0, (1, T, 4)).astype(np.float32)
+    rho[0, 7, 2] = 0.0       # sequence 2 (rows 5..1004), head 2
+    rho[0, 1005, 0] = 0.0    # sequence 3 (its only row), head 0
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    out = host(osdn.osdn_rho_geomean(torch.from_numpy(rho).cuda(),
+                                     torch.from_numpy(cu).cuda()))
+    want = ref.rho_geomean(rho.astype(np.float64), cu)
+    assert out[2, 2] == 0.0 and out[3, 0] == 0.0
+    assert np.all(out[1] == 1.0)
+    np.testing.assert_allclose(out, want, rtol=1e-5, atol=0)

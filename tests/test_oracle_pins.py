@@ -272,6 +272,41 @@ def test_rho_output_is_the_residual_ratio(ref):
             S_prev = St[0, h]
 
 
+def test_q_geo_is_the_geometric_mean_of_explicit_loss_ratios(ref):
+    """q_geo of a (sequence, head) is the T_n-th root of the product of the token-local ratios
+    f_t(S_t) / f_t(S_{t-1}) (section 3, Theorem 5.2's product; the experiments report its
+    geometric mean), with the ratios built from the oracle's explicit states and the section-1
+    loss, two packed sequences and two heads."""
+    rng = np.random.default_rng(28)
+    q, k, v, beta = rand_case(rng, T=11, H=2, Dk=5, Dv=3)
+    r = rng.uniform(0.7, 1.0, beta.shape)
+    cu = np.array([0, 4, 11], dtype=np.int32)
+    _, _, rho = ref.precond_scan(k, beta, r, 0.3, cu_seqlens=cu, with_rho=True)
+    q_geo = ref.rho_geomean(rho, cu)
+    for n in range(2):
+        sl = slice(cu[n], cu[n + 1])
+        for h in range(2):
+            S_prev = np.zeros((3, 5))
+            prod, T_n = 1.0, int(cu[n + 1] - cu[n])
+            for t in range(T_n):
+                a = sl.start
+                _, _, St, _ = ref.fwd(q[:, a:a + t + 1], k[:, a:a + t + 1], v[:, a:a + t + 1],
+                                      beta[:, a:a + t + 1], r[:, a:a + t + 1], 0.3)
+                kk, vv = k[0, a + t, h], v[0, a + t, h]
+                prod *= loss(St[0, h], kk, vv) / loss(S_prev, kk, vv)
+                S_prev = St[0, h]
+            assert abs(q_geo[n, h] - prod ** (1.0 / T_n)) < 1e-12
+
+
+def test_q_geo_closed_forms(ref):
+    """Constant ratios give that constant; 1/4, 1, 4 give 1; a zero ratio gives 0; a sequence
+    without tokens gives 1 (the empty product)."""
+    rho = np.array([0.3, 0.3, 0.3, 0.25, 1.0, 4.0, 0.5, 0.0, 0.9]).reshape(1, 9, 1)
+    cu = np.array([0, 3, 6, 6, 9], dtype=np.int32)
+    np.testing.assert_allclose(ref.rho_geomean(rho, cu)[:, 0], [0.3, 1.0, 1.0, 0.0],
+                               rtol=1e-14, atol=0)
+
+
 # ------------------------------------------------------------------------------------ P8
 def test_phase1_independent_of_q_v_state(ref):
     """P8 (section 2.2): the surrogate depends only on k, beta (and d), so k~ and d_T do not
