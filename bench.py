@@ -588,6 +588,94 @@ def bench_reference_decode(args):
     return 0
 
 
+BWD_METRIC = "OSDN bwd tokens/s (dq, dk, dv, dbeta, dr, deta, dS0, dd0) at 1.3B-layer shape"
+
+
+def bench_bwd(args):
+    """The backward pass (osdn_bwd) over the 1.3B-layer batch, given dL/do and dL/dS_T, dL/dd_T."""
+    import torch
+    from delta_rule_recurrent_osdn_b200 import inputs as W
+    from delta_rule_recurrent_osdn_b200 import osdn
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = W.make_inputs("1p3b_apf", seed=None if rank == 0 else 1000 + rank)
+    d = W.to_torch(inp, dev)
+    rng = np.random.default_rng(123 + rank)
+    dO = torch.from_numpy(rng.standard_normal(inp.v.shape).astype(np.float32)).to(dev, torch.bfloat16)
+    N, H, Dk, Dv = inp.N, inp.H, inp.Dk, inp.Dv
+    dST = torch.from_numpy((0.3 * rng.standard_normal((N, H, Dv, Dk))).astype(np.float32)).to(dev)
+    ddT = torch.from_numpy(rng.standard_normal((N, H, Dk)).astype(np.float32)).to(dev)
+    ws = torch.empty(osdn.LIB.osdn_bwd_workspace_bytes(0, inp.B, inp.T, H, Dk, Dv, osdn.OSDN_BF16),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        return osdn.osdn_bwd(d["q"], d["k"], d["v"], d["beta"], dO, d["r"], inp.eta, d["d0"],
+                             d["S0"], inp.scale, dST, ddT, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(world, dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            events[i][0].record(stream)
+            step()
+            events[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    if osdn.osdn_get_device_status() != osdn.OSDN_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    step_ms = [a.elapsed_time(b) for a, b in events]
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    tokens = inp.B * inp.T
+    value = world * tokens * args.steps / (total_ms / 1e3)
+    if rank == 0:
+        hbm, tc, kind = read_peaks()
+        th = tokens * H
+        # q, k, v, dO in (bf16), beta, r in; dq, dk, dv, dbeta, dr out (fp32); per (sequence,
+        # head): dS_T, dd_T in and dS_0, dd_0 out (fp32)
+        byts = th * ((2 * Dk + 2 * Dv) * 2 + 8 + (2 * Dk + Dv) * 4 + 8) + N * H * 2 * (Dv * Dk + Dk) * 4
+        mean_ms = statistics.mean(step_ms)
+        achieved = byts / (mean_ms / 1e3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            from oracle import osdn_ref as R
+            threads = R.set_threads(0)
+            sub, ntok, desc = oracle_sample(inp, 256)
+            dO_np = dO.float().cpu().numpy()[:, :sub.T]
+            t0 = time.perf_counter()
+            R.bwd(sub.q, sub.k, sub.v, sub.beta, dO_np, sub.r, sub.eta, sub.d0, sub.S0, sub.scale)
+            dt = time.perf_counter() - t0
+            cpu = {"value": ntok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                   "sample": f"{desc} x {H} heads (fp64 gradient), {dt:.1f} s"}
+        line = {
+            "metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": dict(config_dict(inp, "backward of the " + FORWARD["1p3b"][2]),
+                           gradients="fp32"),
+            "roofline": {"bound": "hbm", "scope": "whole backward pass (one osdn_bwd call)",
+                         "achieved": achieved, "peak": hbm, "peak_kind": f"{kind} hbm_gbs",
+                         "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "algorithmic_bytes_per_launch": byts},
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": 5 * args.steps,
+            "clocks": clk.summary(), "gpu": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -596,8 +684,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=list(FORWARD) + ["decode"], default="1p3b",
-                    help="a forward-pass shape (default: the 1.3B layer) or decode (osdn_step)")
+    ap.add_argument("--workload", choices=list(FORWARD) + ["decode", "bwd"], default="1p3b",
+                    help="a forward-pass shape (default: the 1.3B layer), decode (osdn_step) or "
+                         "bwd (osdn_bwd at the 1.3B-layer shape)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -605,6 +694,8 @@ def main(argv=None):
         return bench_reference(args)
     if args.workload == "decode":
         return bench_decode(args)
+    if args.workload == "bwd":
+        return bench_bwd(args)
     return bench_ours(args)
 
 

@@ -13,7 +13,21 @@
 //
 // One CTA per (sequence, head, block of BV value channels): rows of S are independent, so
 // the value split is exact.  Everything lives in shared memory in fp32; this path serves the
-// fp32-I/O mode (every product in fp32 FMA) and any chunk size in {16, 32, 64}.
+// fp32-I/O mode (every product in fp32 FMA), any chunk size in {16, 32, 64}, and gated backbones.
+//
+// Gated backbones (decay alpha_t of the state's key channels before each write: Gated DeltaNet,
+// one factor per token, or Kimi Delta Attention, one per key channel; the gated delta rule of the
+// Gated DeltaNet-2 page, section 1, with OSDN's write key):
+//   S_t = S_{t-1} D_t + beta_t (v_t - S_{t-1} D_t k_t) k~_t^T,   D_t = Diag(alpha_t).
+// With lambda_t = sum of log alpha over the chunk's tokens up to t and Gamma_t = exp(lambda_t),
+// the rescaled state S_t Gamma_t^-1 obeys the ungated recurrence with read key Gamma_t k_t,
+// write key Gamma_t^-1 k~_t and query Gamma_t q_t, and S_end = S~_L Gamma_L.  Only decay ratios
+// between two tokens (<= 1) enter the Gram matrices: Gram[t][j] = sum_i k_ti k~_ji
+// exp(lambda_ti - lambda_ji).  They are evaluated as products of per-token factors scaled to a
+// reference token in the chunk's middle when every factor stays inside fp32's range (|lambda -
+// lambda_ref| < 80 over the chunk), else with one exponential per term.  After the Grams, K, Q
+// and K~ are rescaled in place to Gamma K, Gamma Q and (Gamma_L / Gamma) K~ (all factors <= 1),
+// and the ungated steps follow, with S decayed by Gamma_L before its update.
 #pragma once
 
 #include "common.cuh"
@@ -34,7 +48,9 @@ struct SimtSmem {
     static constexpr int oA = oQS + C * BV;
     static constexpr int oP = oA + C * AS;
     static constexpr int oB = oP + C * AS;
-    static constexpr int floats = oB + C;
+    static constexpr int oLam = oB + C;     // gated only: lambda [C][DK] (prefix of log alpha)
+    static constexpr int oRef = oLam + C * DK;  // lambda at the reference token [DK], flag
+    static constexpr int floats = oRef + DK + 4;
     static constexpr size_t bytes = sizeof(float) * floats;
 };
 
@@ -57,7 +73,8 @@ __global__ void __launch_bounds__(256)
 chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                       const IO* __restrict__ kt, const IO* __restrict__ kt_lo,
                       const IO* __restrict__ v,
-                      const float* __restrict__ beta, float scale, const float* __restrict__ S0,
+                      const float* __restrict__ beta, const float* __restrict__ alpha,
+                      int alpha_per_channel, float scale, const float* __restrict__ S0,
                       IO* __restrict__ o, float* __restrict__ ST, const int32_t* __restrict__ cu,
                       int N, int T, int H) {
     using L = SimtSmem<DK, BV, C>;
@@ -76,6 +93,8 @@ chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
     float* sA = sm + L::oA;
     float* sP = sm + L::oP;
     float* sB = sm + L::oB;
+    float* sLam = sm + L::oLam;
+    float* sRef = sm + L::oRef;
 
     const int tid = threadIdx.x;
     constexpr int NVT = DV / BV;
@@ -124,16 +143,79 @@ chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
             *reinterpret_cast<float2*>(sV + t * BV + c) = xv;
         }
         for (int t = tid; t < C; t += NT) sB[t] = t < Lc ? __ldg(beta + (first + cs + t) * H + h) : 0.f;
+        if (alpha) {  // lambda = prefix of log alpha per key channel (alpha = 1 past the end)
+            for (int i = tid; i < DK; i += NT) {
+                float lam = 0.f;
+                for (int t = 0; t < C; ++t) {
+                    float a = 1.f;
+                    if (t < Lc) {
+                        const int64_t th = (first + cs + t) * H + h;
+                        a = __ldg(alpha + (alpha_per_channel ? th * DK + i : th));
+                    }
+                    lam += __logf(a);
+                    sLam[t * DK + i] = lam;
+                }
+                sRef[i] = sLam[(C / 2) * DK + i];
+            }
+        }
         __syncthreads();
+        bool factored = false;  // gated: Gram ratios as products of reference-scaled factors
+        if (alpha) {
+            bool far = false;
+            for (int idx = tid; idx < C * DK; idx += NT) {
+                const int i = idx % DK;
+                far |= fabsf(sLam[idx] - sRef[i]) >= 80.f;
+            }
+            factored = !__syncthreads_or(far);
+            if (factored) {
+                for (int idx = tid; idx < C * DK; idx += NT) {
+                    const int t = idx / DK, i = idx - t * DK;
+                    const float dl = sLam[idx] - sRef[i];
+                    const float up = __expf(dl), dn = __expf(-dl);
+                    sK[t * KS + i] *= up;
+                    sQ[t * KS + i] *= up;
+                    sKt[t * KS + i] *= dn;
+                }
+                __syncthreads();
+            }
+        }
 
         // ---- Gram (strictly lower, beta-scaled rows) and intra-chunk scores (lower incl.)
         for (int idx = tid; idx < C * C; idx += NT) {
             const int t = idx / C, j = idx - t * C;
             float a = 0.f, p = 0.f;
-            if (j < t) a = sB[t] * dot_row(sK + t * KS, sKt + j * KS, DK);
-            if (j <= t) p = dot_row(sQ + t * KS, sKt + j * KS, DK);
+            if (alpha && !factored) {  // one exponential per term: sum_i x_ti k~_ji e^(lam_ti - lam_ji)
+                if (j <= t) {
+                    const float* lt = sLam + t * DK;
+                    const float* lj = sLam + j * DK;
+                    for (int i = 0; i < DK; ++i) {
+                        const float e = __expf(lt[i] - lj[i]) * sKt[j * KS + i];
+                        a = fmaf(sK[t * KS + i], e, a);
+                        p = fmaf(sQ[t * KS + i], e, p);
+                    }
+                    a = j < t ? sB[t] * a : 0.f;
+                }
+            } else {
+                if (j < t) a = sB[t] * dot_row(sK + t * KS, sKt + j * KS, DK);
+                if (j <= t) p = dot_row(sQ + t * KS, sKt + j * KS, DK);
+            }
             sA[t * AS + j] = a;
             sP[t * AS + j] = p;
+        }
+        if (alpha) {  // K -> Gamma K, Q -> Gamma Q, K~ -> (Gamma_L / Gamma) K~; S -> S Gamma_L below
+            __syncthreads();
+            const float* lamL = sLam + (C - 1) * DK;
+            for (int idx = tid; idx < C * DK; idx += NT) {
+                const int t = idx / DK, i = idx - t * DK;
+                const float lam = sLam[idx];
+                // factored: K and Q already carry exp(lam - ref), K~ carries exp(ref - lam)
+                const float gk = factored ? __expf(sRef[i]) : __expf(lam);
+                const float gt = factored ? __expf(lamL[i] - sRef[i]) : __expf(lamL[i] - lam);
+                sK[t * KS + i] *= gk;
+                sQ[t * KS + i] *= gk;
+                sKt[t * KS + i] *= gt;
+            }
+            __syncthreads();
         }
         // ---- right-hand side beta (V - K S0^T) and the readout Q S0^T
         for (int idx = tid; idx < C * BV; idx += NT) {
@@ -180,6 +262,7 @@ chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
             const int c = idx / DK, i = idx - c * DK;
             float acc = 0.f;
             for (int t = 0; t < Lc; ++t) acc = fmaf(sW[t * BV + c], sKt[t * KS + i], acc);
+            if (alpha) sS[c * KS + i] *= __expf(sLam[(C - 1) * DK + i]);  // S Gamma_L
             sS[c * KS + i] += acc;
         }
     }

@@ -20,6 +20,7 @@
 #include "step.cuh"
 #include "scan_tc.cuh"
 #include "rho_geomean.cuh"
+#include "bwd.cuh"
 
 namespace osdn {
 namespace {
@@ -68,28 +69,29 @@ inline bool set_smem(KernelT kernel, size_t bytes) {
 // ---------------------------------------------------------------- phase 1 dispatch
 template <typename IO>
 osdn_status_t launch_scan_warp(const void* k, const float* beta, const float* r, float eta,
-                               const float* d0, void* k_tilde, void* kt_lo, float* dT, float* rho,
-                               const int32_t* cu, const Dims& d, cudaStream_t stream) {
+                               const float* d0, void* k_tilde, void* kt_lo, float* d_all,
+                               float* dT, float* rho, const int32_t* cu, const Dims& d,
+                               cudaStream_t stream) {
     const int units = d.N * d.H;
     if (units == 0) return OSDN_OK;
     const dim3 block(128), grid((units + 3) / 4);
     if (d.Dk == 128)
         precond_scan_warp_kernel<128, IO><<<grid, block, 0, stream>>>(
             static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde),
-            static_cast<IO*>(kt_lo), dT, rho, cu, d.N, d.T, d.H);
+            static_cast<IO*>(kt_lo), d_all, dT, rho, cu, d.N, d.T, d.H);
     else
         precond_scan_warp_kernel<64, IO><<<grid, block, 0, stream>>>(
             static_cast<const IO*>(k), beta, r, eta, d0, static_cast<IO*>(k_tilde),
-            static_cast<IO*>(kt_lo), dT, rho, cu, d.N, d.T, d.H);
+            static_cast<IO*>(kt_lo), d_all, dT, rho, cu, d.N, d.T, d.H);
     return launch_status();
 }
 
 // ---------------------------------------------------------------- phase 2 dispatch
 template <int DK, int DV, int C, typename IO>
 osdn_status_t launch_chunk_simt(const void* q, const void* k, const void* kt, const void* kt_lo,
-                                const void* v, const float* beta, float scale, const float* S0,
-                                void* o, float* ST, const int32_t* cu, const Dims& d,
-                                cudaStream_t stream) {
+                                const void* v, const float* beta, const float* alpha, int apc,
+                                float scale, const float* S0, void* o, float* ST,
+                                const int32_t* cu, const Dims& d, cudaStream_t stream) {
     constexpr int BV = 32;
     const int64_t ctas = (int64_t)d.N * d.H * (DV / BV);
     if (ctas == 0) return OSDN_OK;
@@ -99,26 +101,26 @@ osdn_status_t launch_chunk_simt(const void* q, const void* k, const void* kt, co
     if (!set_smem(kernel, smem)) return OSDN_ERR_CUDA;
     kernel<<<dim3((unsigned)ctas), dim3(256), smem, stream>>>(
         static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(kt),
-        static_cast<const IO*>(kt_lo), static_cast<const IO*>(v), beta, scale, S0,
+        static_cast<const IO*>(kt_lo), static_cast<const IO*>(v), beta, alpha, apc, scale, S0,
         static_cast<IO*>(o), ST, cu, d.N, d.T, d.H);
     return launch_status();
 }
 
 template <int DK, int DV, typename IO>
 osdn_status_t launch_chunk_c(int chunk, const void* q, const void* k, const void* kt,
-                             const void* kt_lo, const void* v, const float* beta, float scale,
-                             const float* S0, void* o, float* ST, const int32_t* cu,
-                             const Dims& d, cudaStream_t stream) {
+                             const void* kt_lo, const void* v, const float* beta,
+                             const float* alpha, int apc, float scale, const float* S0, void* o,
+                             float* ST, const int32_t* cu, const Dims& d, cudaStream_t stream) {
     switch (chunk) {
         case 16:
-            return launch_chunk_simt<DK, DV, 16, IO>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
-                                                     d, stream);
+            return launch_chunk_simt<DK, DV, 16, IO>(q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0,
+                                                     o, ST, cu, d, stream);
         case 32:
-            return launch_chunk_simt<DK, DV, 32, IO>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
-                                                     d, stream);
+            return launch_chunk_simt<DK, DV, 32, IO>(q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0,
+                                                     o, ST, cu, d, stream);
         case 64:
-            return launch_chunk_simt<DK, DV, 64, IO>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
-                                                     d, stream);
+            return launch_chunk_simt<DK, DV, 64, IO>(q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0,
+                                                     o, ST, cu, d, stream);
         default:
             return OSDN_ERR_UNSUPPORTED;
     }
@@ -179,8 +181,8 @@ int sm_count() {
 // Phase 1, bf16 with 128 key channels: T_d of every chunk (prep kernel, written into the k~
 // buffer), then the chain across chunks (one CTA per (sequence, head)).
 osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, float eta,
-                             const float* d0, void* k_tilde, void* kt_lo, float* dT, float* rho,
-                             const int32_t* cu, const Dims& d, cudaStream_t stream) {
+                             const float* d0, void* k_tilde, void* kt_lo, float* d_all, float* dT,
+                             float* rho, const int32_t* cu, const Dims& d, cudaStream_t stream) {
     const int64_t nh = (int64_t)d.N * d.H;
     if (nh == 0) return OSDN_OK;
     if (nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
@@ -203,22 +205,27 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     if (!set_smem(chain, ScanChainSmem::BYTES)) return OSDN_ERR_CUDA;
     chain<<<dim3((unsigned)nh), dim3(SCAN_CHAIN_THREADS), ScanChainSmem::BYTES, stream>>>(
         mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde),
-        static_cast<__nv_bfloat16*>(kt_lo), dT, rho, cu, d.N, d.T, d.H, (long long)kWaitLimitNs);
+        static_cast<__nv_bfloat16*>(kt_lo), d_all, dT, rho, cu, d.N, d.T, d.H,
+        (long long)kWaitLimitNs);
     return launch_status();
 }
 
 // Phase 1: bf16 keys with 128 channels use the chunk-parallel kernel; fp32 I/O, 64 channels
 // and token-free calls use the warp-per-(sequence, head) scan.  kt_lo (bf16 only; may be null):
 // also write the residual bf16(k~ - k~_hi) of each key's rounding.
+// d_all (may be null): also write d_t, the preconditioner of every token, as fp32 [B,T,H,Dk].
 template <typename IO>
 osdn_status_t launch_scan(const void* k, const float* beta, const float* r, float eta,
                           const float* d0, void* k_tilde, void* kt_lo, float* dT, float* rho,
-                          const int32_t* cu, const Dims& d, cudaStream_t stream) {
+                          const int32_t* cu, const Dims& d, cudaStream_t stream,
+                          float* d_all = nullptr) {
     if constexpr (sizeof(IO) == 2) {
         if (d.Dk == 128 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
-            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, kt_lo, dT, rho, cu, d, stream);
+            return launch_scan_tc(k, beta, r, eta, d0, k_tilde, kt_lo, d_all, dT, rho, cu, d,
+                                  stream);
     }
-    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, kt_lo, dT, rho, cu, d, stream);
+    return launch_scan_warp<IO>(k, beta, r, eta, d0, k_tilde, kt_lo, d_all, dT, rho, cu, d,
+                                stream);
 }
 
 // 3-D fp32 view [rows][H][Dv / 2] of the bf16 output buffer; boxes of 32 values (one 128-byte
@@ -287,28 +294,42 @@ osdn_status_t launch_chunk_tc(const void* q, const void* k, const void* kt, cons
 }
 
 // kt_lo (may be null): the lo term of K~ handed over as bf16 hi + lo (k~ = kt + kt_lo).
+// alpha (may be null): the decay of a gated backbone, per token (apc = 0) or per key channel.
 template <typename IO>
 osdn_status_t launch_chunk(int chunk, const void* q, const void* k, const void* kt,
-                           const void* kt_lo, const void* v, const float* beta, float scale,
-                           const float* S0, void* o, float* ST, const int32_t* cu, const Dims& d,
-                           cudaStream_t stream) {
+                           const void* kt_lo, const void* v, const float* beta, const float* alpha,
+                           int apc, float scale, const float* S0, void* o, float* ST,
+                           const int32_t* cu, const Dims& d, cudaStream_t stream) {
     // bf16 I/O with 128 key and 128 value channels runs on the tensor cores; fp32 I/O, 64-channel
-    // heads and token-free calls (states pass through) run the fp32 SIMT kernel.
+    // heads, gated backbones and token-free calls (states pass through) run the fp32 SIMT kernel.
     if constexpr (sizeof(IO) == 2) {
-        if (d.Dk == 128 && d.Dv == 128 && chunk == 64 && d.rows() > 0 && d.rows() < (int64_t(1) << 31))
+        if (!alpha && d.Dk == 128 && d.Dv == 128 && chunk == 64 && d.rows() > 0 &&
+            d.rows() < (int64_t(1) << 31))
             return launch_chunk_tc<128>(q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d, stream);
     }
     if (d.Dk == 128 && d.Dv == 128)
-        return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu,
-                                            d, stream);
+        return launch_chunk_c<128, 128, IO>(chunk, q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0,
+                                            o, ST, cu, d, stream);
     if (d.Dk == 128 && d.Dv == 64)
-        return launch_chunk_c<128, 64, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d,
-                                           stream);
+        return launch_chunk_c<128, 64, IO>(chunk, q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0, o,
+                                           ST, cu, d, stream);
     if (d.Dk == 64 && d.Dv == 128)
-        return launch_chunk_c<64, 128, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d,
-                                           stream);
-    return launch_chunk_c<64, 64, IO>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST, cu, d,
-                                      stream);
+        return launch_chunk_c<64, 128, IO>(chunk, q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0, o,
+                                           ST, cu, d, stream);
+    return launch_chunk_c<64, 64, IO>(chunk, q, k, kt, kt_lo, v, beta, alpha, apc, scale, S0, o, ST,
+                                      cu, d, stream);
+}
+
+// alpha: a device pointer of [B,T,H] (apc = 0) or [B,T,H,Dk] (apc = 1) float32, or null.
+osdn_status_t validate_alpha(const float* alpha, int apc, const void* const* outs,
+                             const size_t* out_bytes, int n_outs, const Dims& d) {
+    if (apc != 0 && apc != 1) return OSDN_ERR_INVALID_ARG;
+    if (!alpha) return OSDN_OK;
+    if (!aligned16(alpha)) return OSDN_ERR_ALIGNMENT;
+    const size_t ab = (size_t)d.rows() * d.H * (apc ? d.Dk : 1) * 4;
+    for (int i = 0; i < n_outs; ++i)
+        if (overlaps(alpha, ab, outs[i], out_bytes[i])) return OSDN_ERR_INVALID_ARG;
+    return OSDN_OK;
 }
 
 osdn_status_t validate_scan(const void* k, const float* beta, const float* r, const float* d0,
@@ -419,7 +440,8 @@ osdn_status_t osdn_precond_scan(const void* k, const float* beta, const float* r
 }
 
 osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, const void* v,
-                             const float* beta, float scale, const float* S0, void* o, float* ST,
+                             const float* beta, const float* alpha, int32_t alpha_per_channel,
+                             float scale, const float* S0, void* o, float* ST,
                              const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                              int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                              void* stream) {
@@ -429,12 +451,19 @@ osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, 
     d.Dv = Dv;
     st = validate_chunk(q, k, k_tilde, v, beta, S0, o, ST, d, chunk, io);
     if (st != OSDN_OK) return st;
+    {
+        const void* outs[] = {o, ST};
+        const size_t ob[] = {(size_t)d.rows() * d.H * d.Dv * io_size(io),
+                             (size_t)d.N * d.H * d.Dv * d.Dk * 4};
+        st = validate_alpha(alpha, alpha_per_channel, outs, ob, 2, d);
+        if (st != OSDN_OK) return st;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16)
-        return launch_chunk<__nv_bfloat16>(chunk, q, k, k_tilde, nullptr, v, beta, scale, S0, o, ST,
-                                           cu_seqlens, d, s);
-    return launch_chunk<float>(chunk, q, k, k_tilde, nullptr, v, beta, scale, S0, o, ST, cu_seqlens,
-                               d, s);
+        return launch_chunk<__nv_bfloat16>(chunk, q, k, k_tilde, nullptr, v, beta, alpha,
+                                           alpha_per_channel, scale, S0, o, ST, cu_seqlens, d, s);
+    return launch_chunk<float>(chunk, q, k, k_tilde, nullptr, v, beta, alpha, alpha_per_channel,
+                               scale, S0, o, ST, cu_seqlens, d, s);
 }
 
 // Workspace of osdn_fwd: k~ (used when the caller passes no k_tilde_out), then, for bf16, the
@@ -450,11 +479,12 @@ size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_t Dk, osd
 }
 
 osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
-                       const float* r, float eta, const float* d0, const float* S0, float scale,
-                       void* o, float* ST, float* dT, float* rho, void* k_tilde_out,
-                       const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
-                       int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+                       const float* r, const float* alpha, int32_t alpha_per_channel, float eta,
+                       const float* d0, const float* S0, float scale, void* o, float* ST,
+                       float* dT, float* rho, void* k_tilde_out, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                       int32_t chunk, osdn_dtype_t io, void* workspace, size_t workspace_bytes,
+                       void* stream) {
     Dims d;
     osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
     if (st != OSDN_OK) return st;
@@ -491,17 +521,23 @@ osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float*
         overlaps(rho, gb, S0, (size_t)d.N * d.H * d.Dv * d.Dk * 4) ||
         overlaps(rho, gb, ST, (size_t)d.N * d.H * d.Dv * d.Dk * 4))
         return OSDN_ERR_INVALID_ARG;
+    {
+        const void* outs[] = {o, ST, dT, rho, kt, kt_lo};
+        const size_t ob[] = {vb, (size_t)d.N * d.H * d.Dv * d.Dk * 4, db, gb, kb, kb};
+        st = validate_alpha(alpha, alpha_per_channel, outs, ob, 6, d);
+        if (st != OSDN_OK) return st;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (io == OSDN_BF16) {
         st = launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, kt, kt_lo, dT, rho, cu_seqlens, d, s);
         if (st != OSDN_OK) return st;
-        return launch_chunk<__nv_bfloat16>(chunk, q, k, kt, kt_lo, v, beta, scale, S0, o, ST,
-                                           cu_seqlens, d, s);
+        return launch_chunk<__nv_bfloat16>(chunk, q, k, kt, kt_lo, v, beta, alpha,
+                                           alpha_per_channel, scale, S0, o, ST, cu_seqlens, d, s);
     }
     st = launch_scan<float>(k, beta, r, eta, d0, kt, nullptr, dT, rho, cu_seqlens, d, s);
     if (st != OSDN_OK) return st;
-    return launch_chunk<float>(chunk, q, k, kt, nullptr, v, beta, scale, S0, o, ST, cu_seqlens, d,
-                               s);
+    return launch_chunk<float>(chunk, q, k, kt, nullptr, v, beta, alpha, alpha_per_channel, scale,
+                               S0, o, ST, cu_seqlens, d, s);
 }
 
 osdn_status_t osdn_step(const void* q, const void* k, const void* v, const float* beta,
@@ -552,6 +588,172 @@ osdn_status_t osdn_rho_geomean(const float* rho, const int32_t* cu_seqlens, int3
     rho_geomean_kernel<<<dim3((unsigned)units), dim3(GEOMEAN_THREADS), 0,
                          static_cast<cudaStream_t>(stream)>>>(rho, cu_seqlens, (int)N, T, H, q_geo);
     return launch_status();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- backward pass
+namespace osdn {
+namespace {
+
+// Workspace of osdn_bwd, each part rounded up to 256 bytes: k~ (io dtype), d_t of every token,
+// the state checkpoints (every BWD_C tokens), the per-value-tile shares of dq, dk, dk~ and dbeta,
+// and deta per (sequence, head).
+struct BwdWorkspace {
+    size_t kt, dall, state, dq, dk, dkt, dbeta, deta, total;
+};
+
+inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+BwdWorkspace bwd_workspace(int64_t rows, int64_t N, int32_t H, int32_t Dk, int32_t Dv,
+                           osdn_dtype_t io) {
+    BwdWorkspace w;
+    const int64_t ntile = Dv / BWD_BV;
+    const int64_t th = rows * H;
+    size_t off = 0;
+    w.kt = off;
+    off += up256((size_t)th * Dk * io_size(io));
+    w.dall = off;
+    off += up256((size_t)th * Dk * 4);
+    w.state = off;
+    off += up256((size_t)((rows + BWD_C - 1) / BWD_C + N + 1) * H * Dv * Dk * 4);
+    w.dq = off;
+    off += up256((size_t)ntile * th * Dk * 4);
+    w.dk = off;
+    off += up256((size_t)ntile * th * Dk * 4);
+    w.dkt = off;
+    off += up256((size_t)ntile * th * Dk * 4);
+    w.dbeta = off;
+    off += up256((size_t)ntile * th * 4);
+    w.deta = off;
+    off += up256((size_t)N * H * 4);
+    w.total = off;
+    return w;
+}
+
+template <int DK, typename IO>
+osdn_status_t launch_bwd_kernels(const void* q, const void* k, const void* v, const float* beta,
+                                 const float* r, float eta, const float* S0, float scale,
+                                 const void* dO, const float* dST, const float* ddT, float* dq,
+                                 float* dk, float* dv, float* dbeta, float* dr, float* deta,
+                                 float* dS0, float* dd0, const int32_t* cu, const Dims& d,
+                                 uint8_t* ws, const BwdWorkspace& w, cudaStream_t stream) {
+    const int64_t rows = d.rows();
+    const int ntile = d.Dv / BWD_BV;
+    float* dall = reinterpret_cast<float*>(ws + w.dall);
+    float* dq_part = reinterpret_cast<float*>(ws + w.dq);
+    float* dk_part = reinterpret_cast<float*>(ws + w.dk);
+    float* dkt_part = reinterpret_cast<float*>(ws + w.dkt);
+    float* db_part = reinterpret_cast<float*>(ws + w.dbeta);
+    float* deta_part = reinterpret_cast<float*>(ws + w.deta);
+    const int64_t units = (int64_t)d.N * d.H;
+    {
+        auto kern = bwd_delta_kernel<DK, IO>;
+        if (!set_smem(kern, BwdSmem<DK>::bytes)) return OSDN_ERR_CUDA;
+        kern<<<dim3((unsigned)(units * ntile)), dim3(BWD_THREADS), BwdSmem<DK>::bytes, stream>>>(
+            static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), beta,
+            dall, S0, scale, static_cast<const IO*>(dO), dST, dv, dS0,
+            reinterpret_cast<float*>(ws + w.state), dq_part, dk_part, dkt_part, db_part, cu, d.N,
+            d.T, d.H, d.Dv, rows);
+        const osdn_status_t st = launch_status();
+        if (st != OSDN_OK) return st;
+    }
+    {
+        auto kern = bwd_precond_kernel<DK, IO>;
+        if (!set_smem(kern, BwdPrecondSmem<DK>::bytes)) return OSDN_ERR_CUDA;
+        kern<<<dim3((unsigned)units), dim3(128), BwdPrecondSmem<DK>::bytes, stream>>>(
+            static_cast<const IO*>(k), beta, r, eta, dall, ddT, dq_part, dk_part, dkt_part, db_part,
+            ntile, dq, dk, dbeta, dr, dd0, deta_part, cu, d.N, d.T, d.H, rows);
+        const osdn_status_t st = launch_status();
+        if (st != OSDN_OK) return st;
+    }
+    if (deta) {
+        bwd_sum_kernel<<<1, 256, 0, stream>>>(deta_part, units, deta);
+        return launch_status();
+    }
+    return OSDN_OK;
+}
+
+}  // namespace
+}  // namespace osdn
+
+extern "C" {
+
+size_t osdn_bwd_workspace_bytes(int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk,
+                                int32_t Dv, osdn_dtype_t io) {
+    if (B < 0 || T < 0 || H < 1 || num_seqs < 0 || (Dk != 64 && Dk != 128) ||
+        (Dv != 64 && Dv != 128) || (io != OSDN_BF16 && io != OSDN_F32))
+        return 0;
+    const int64_t N = num_seqs > 0 ? num_seqs : B;
+    return osdn::bwd_workspace((int64_t)B * T, N, H, Dk, Dv, io).total;
+}
+
+osdn_status_t osdn_bwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* r, float eta, const float* d0, const float* S0, float scale,
+                       const void* dO, const float* dST, const float* ddT, float* dq, float* dk,
+                       float* dv, float* dbeta, float* dr, float* deta, float* dS0, float* dd0,
+                       const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                       int32_t H, int32_t Dk, int32_t Dv, osdn_dtype_t io, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    Dims d;
+    osdn_status_t st = check_common(cu_seqlens, num_seqs, B, T, H, Dk, io, d);
+    if (st != OSDN_OK) return st;
+    if (Dv != 64 && Dv != 128) return OSDN_ERR_UNSUPPORTED;
+    d.Dv = Dv;
+    const int64_t th = d.rows() * d.H;
+    const bool tokens = th > 0;
+    if (tokens && (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta))
+        return OSDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, beta, r, d0, S0, dO, dST, ddT, dq, dk, dv, dbeta, dr, deta,
+                          dS0, dd0, cu_seqlens};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return OSDN_ERR_ALIGNMENT;
+    const osdn::BwdWorkspace w = osdn::bwd_workspace(d.rows(), d.N, H, Dk, Dv, io);
+    if (!workspace || workspace_bytes < w.total) return OSDN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return OSDN_ERR_ALIGNMENT;
+    // every output against every buffer (inputs, other outputs, the workspace)
+    const size_t es = osdn::io_size(io);
+    const size_t kb = (size_t)th * Dk * es, vb = (size_t)th * Dv * es, gb = (size_t)th * 4,
+                 sb = (size_t)d.N * H * Dv * Dk * 4, db = (size_t)d.N * H * Dk * 4;
+    const void* all[] = {q, k, v, beta, r, d0, S0, dO, dST, ddT, workspace,
+                         dq, dk, dv, dbeta, dr, deta, dS0, dd0};
+    const size_t allb[] = {kb, kb, vb, gb, gb, db, sb, vb, sb, db, w.total,
+                           (size_t)th * Dk * 4, (size_t)th * Dk * 4, (size_t)th * Dv * 4, gb, gb, 4,
+                           sb, db};
+    for (int a = 11; a < 19; ++a)
+        for (int b = 0; b < 19; ++b)
+            if (b != a && osdn::overlaps(all[a], allb[a], all[b], allb[b])) return OSDN_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t units = (int64_t)d.N * H;
+    if (units == 0) return OSDN_OK;
+    if (units * (Dv / osdn::BWD_BV) > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    // phase 1 forward: d_t of every token (k~ into the workspace, its own scratch)
+    if (io == OSDN_BF16)
+        st = osdn::launch_scan<__nv_bfloat16>(k, beta, r, eta, d0, ws + w.kt, nullptr, nullptr,
+                                              nullptr, cu_seqlens, d, s,
+                                              reinterpret_cast<float*>(ws + w.dall));
+    else
+        st = osdn::launch_scan<float>(k, beta, r, eta, d0, ws + w.kt, nullptr, nullptr, nullptr,
+                                      cu_seqlens, d, s, reinterpret_cast<float*>(ws + w.dall));
+    if (st != OSDN_OK) return st;
+    if (io == OSDN_BF16) {
+        if (Dk == 128)
+            return osdn::launch_bwd_kernels<128, __nv_bfloat16>(q, k, v, beta, r, eta, S0, scale, dO,
+                                                                dST, ddT, dq, dk, dv, dbeta, dr,
+                                                                deta, dS0, dd0, cu_seqlens, d, ws,
+                                                                w, s);
+        return osdn::launch_bwd_kernels<64, __nv_bfloat16>(q, k, v, beta, r, eta, S0, scale, dO,
+                                                           dST, ddT, dq, dk, dv, dbeta, dr, deta,
+                                                           dS0, dd0, cu_seqlens, d, ws, w, s);
+    }
+    if (Dk == 128)
+        return osdn::launch_bwd_kernels<128, float>(q, k, v, beta, r, eta, S0, scale, dO, dST, ddT,
+                                                    dq, dk, dv, dbeta, dr, deta, dS0, dd0,
+                                                    cu_seqlens, d, ws, w, s);
+    return osdn::launch_bwd_kernels<64, float>(q, k, v, beta, r, eta, S0, scale, dO, dST, ddT, dq,
+                                               dk, dv, dbeta, dr, deta, dS0, dd0, cu_seqlens, d,
+                                               ws, w, s);
 }
 
 osdn_status_t osdn_get_device_status(void* stream) {
@@ -637,7 +839,8 @@ osdn_status_t noalloc_scratch(void** out) {
 }  // namespace osdn
 
 extern "C" osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void* v,
-                                          const float* beta, const float* r, float eta,
+                                          const float* beta, const float* r, const float* alpha,
+                                          int32_t alpha_per_channel, float eta,
                                           const float* d0, const float* S0, float scale, void* o,
                                           float* ST, float* dT, float* rho,
                                           const int32_t* cu_seqlens,
@@ -654,7 +857,7 @@ extern "C" osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const vo
         const osdn_status_t st = noalloc_scratch(&scratch);
         if (st != OSDN_OK) return st;
     }
-    return osdn_fwd(q, k, v, beta, r, eta, d0, S0, scale, o, ST, dT, rho, nullptr, cu_seqlens,
-                    num_seqs, B, T, H, Dk, Dv, chunk, io, scratch, need > 0 ? kNoallocScratchBytes : 0,
-                    stream);
+    return osdn_fwd(q, k, v, beta, r, alpha, alpha_per_channel, eta, d0, S0, scale, o, ST, dT, rho,
+                    nullptr, cu_seqlens, num_seqs, B, T, H, Dk, Dv, chunk, io, scratch,
+                    need > 0 ? kNoallocScratchBytes : 0, stream);
 }

@@ -336,12 +336,13 @@ constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output, 8
 
 // One CTA per (sequence, head).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
 // k_tilde receives k~ rounded to bf16 (hi); k_tilde_lo, when not null, receives the rounding
-// residual bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.
+// residual bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.  d_all, when not
+// null ([B,T,H,Dk] fp32), receives d_t, the preconditioner each token writes with.
 __global__ void __launch_bounds__(SCAN_CHAIN_THREADS, 1)
 precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_td,
                      const float* __restrict__ beta, const float* __restrict__ r, float eta,
                      const float* __restrict__ d0, __nv_bfloat16* __restrict__ k_tilde,
-                     __nv_bfloat16* __restrict__ k_tilde_lo,
+                     __nv_bfloat16* __restrict__ k_tilde_lo, float* __restrict__ d_all,
                      float* __restrict__ dT, float* __restrict__ rho,
                      const int32_t* __restrict__ cu, int N, int T, int H, long long limit_ns) {
     constexpr int C = SCAN_C, DK = 128;
@@ -580,6 +581,8 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 }
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
+                    if (d_all && t0 + u < Lc)
+                        d_all[((first + (int64_t)c * C + t0 + u) * H + h) * DK + i] = dd;
                     const float kt = dd * kv[u];
                     const __nv_bfloat16 hb = __float2bfloat16_rn(kt);
                     *reinterpret_cast<__nv_bfloat16*>(ocol + tc::sw128_off(t0 + u, cj)) = hb;

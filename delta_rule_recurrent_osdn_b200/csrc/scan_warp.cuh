@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(128)
 precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
                          const float* __restrict__ r, float eta, const float* __restrict__ d0,
                          IO* __restrict__ k_tilde, IO* __restrict__ k_tilde_lo,
-                         float* __restrict__ dT, float* __restrict__ rho,
+                         float* __restrict__ d_all, float* __restrict__ dT, float* __restrict__ rho,
                          const int32_t* __restrict__ cu, int N, int T, int H) {
     static_assert(DK == 64 || DK == 128, "DK");
     constexpr int E = DK / 32;  // consecutive channels per lane
@@ -102,6 +102,11 @@ precond_scan_warp_kernel(const IO* __restrict__ k, const float* __restrict__ bet
                         store2<IO>(klp + t * rs, make_float2(lo[0], lo[1]));
                 }
                 if (rho && lane == 0) rho[(first + t) * H + h] = (1.f - bt * s) * (1.f - bt * s);
+                if (d_all) {  // the preconditioner this token wrote with
+                    float* dp = d_all + ((first + t) * H + h) * DK + lane * E;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) dp[e] = d[e];
+                }
                 const float coef = nk > 0.f ? eta * bt * (1.0f - bt * s) / nk : 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) d[e] = fmaf(rt, d[e], coef * a[e]);

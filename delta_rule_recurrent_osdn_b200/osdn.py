@@ -53,18 +53,24 @@ def _load() -> ctypes.CDLL:
     lib.osdn_precond_scan.argtypes = [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                       _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_precond_scan.restype = ctypes.c_int
-    lib.osdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _i32, _i32,
-                                   _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
+    lib.osdn_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _vp,
+                                   _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_chunk_fwd.restype = ctypes.c_int
     lib.osdn_fwd_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, ctypes.c_int]
     lib.osdn_fwd_workspace_bytes.restype = ctypes.c_size_t
-    lib.osdn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _f32, _vp, _vp, _vp, _vp,
-                             _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp,
-                             ctypes.c_size_t, _vp]
+    lib.osdn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _f32, _vp, _vp,
+                             _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                             ctypes.c_int, _vp, ctypes.c_size_t, _vp]
     lib.osdn_fwd.restype = ctypes.c_int
     lib.osdn_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _vp, _vp, _vp,
                               _vp, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
     lib.osdn_step.restype = ctypes.c_int
+    lib.osdn_bwd_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int]
+    lib.osdn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.osdn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _f32, _vp, _vp, _vp, _vp,
+                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                             _i32, ctypes.c_int, _vp, ctypes.c_size_t, _vp]
+    lib.osdn_bwd.restype = ctypes.c_int
     lib.osdn_rho_geomean.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
     lib.osdn_rho_geomean.restype = ctypes.c_int
     lib.osdn_get_device_status.argtypes = [_vp]
@@ -157,9 +163,21 @@ def osdn_precond_scan(k, beta, r=None, eta: float = 0.0, d0=None, cu_seqlens=Non
     return k_tilde, dT
 
 
+def _alpha(alpha, B, T, H, Dk):
+    """(pointer, per_channel flag) of a gated backbone's decay: [B, T, H] or [B, T, H, Dk]."""
+    if alpha is None:
+        return None, 0
+    per_channel = alpha.dim() == 4
+    _req(alpha, "alpha", torch.float32, (B, T, H, Dk) if per_channel else (B, T, H))
+    return _p(alpha), int(per_channel)
+
+
 def osdn_chunk_fwd(q, k, k_tilde, v, beta, scale: float = 1.0, S0=None, chunk: int = 64,
-                   cu_seqlens=None, o=None, ST=None, return_ST: bool = True, stream=None):
-    """Phase 2: returns ``(o, ST)`` (``ST`` is None when ``return_ST`` is False)."""
+                   cu_seqlens=None, o=None, ST=None, return_ST: bool = True, stream=None,
+                   alpha=None):
+    """Phase 2: returns ``(o, ST)`` (``ST`` is None when ``return_ST`` is False).  ``alpha``: the
+    decay of a gated backbone, [B, T, H] (Gated DeltaNet) or [B, T, H, Dk] (Kimi Delta Attention)
+    float32, or None."""
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
     io = _io(q)
@@ -175,7 +193,9 @@ def osdn_chunk_fwd(q, k, k_tilde, v, beta, scale: float = 1.0, S0=None, chunk: i
     if ST is None and return_ST:
         ST = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=q.device)
     _req(ST, "ST", torch.float32, (N, H, Dv, Dk))
-    _check(LIB.osdn_chunk_fwd(_p(q), _p(k), _p(k_tilde), _p(v), _p(beta), float(scale), _p(S0),
+    a_ptr, apc = _alpha(alpha, B, T, H, Dk)
+    _check(LIB.osdn_chunk_fwd(_p(q), _p(k), _p(k_tilde), _p(v), _p(beta), a_ptr, apc,
+                              float(scale), _p(S0),
                               _p(o), _p(ST), _p(cu_seqlens), num_seqs, B, T, H, Dk, Dv,
                               int(chunk), io, _stream(stream)),
            "osdn_chunk_fwd")
@@ -189,8 +209,9 @@ def osdn_fwd_workspace_bytes(B: int, T: int, H: int, Dk: int, dtype=torch.bfloat
 
 def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: float = 1.0,
              chunk: int = 64, cu_seqlens=None, o=None, ST=None, dT=None, k_tilde=None,
-             workspace=None, return_states: bool = True, rho=None, stream=None):
+             workspace=None, return_states: bool = True, rho=None, stream=None, alpha=None):
     """Both phases: returns ``(o, ST, dT)`` (states None when ``return_states`` is False).
+    ``alpha``: the decay of a gated backbone, as for :func:`osdn_chunk_fwd`.
 
     The call needs a device workspace of ``osdn_fwd_workspace_bytes`` bytes (for bf16 it holds
     the residual of k~'s rounding, and k~ itself when ``k_tilde`` is not given); when
@@ -226,7 +247,9 @@ def osdn_fwd(q, k, v, beta, r=None, eta: float = 0.0, d0=None, S0=None, scale: f
     if workspace is not None:
         _req(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(LIB.osdn_fwd(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), _p(d0), _p(S0),
+    a_ptr, apc = _alpha(alpha, B, T, H, Dk)
+    _check(LIB.osdn_fwd(_p(q), _p(k), _p(v), _p(beta), _p(r), a_ptr, apc, float(eta), _p(d0),
+                        _p(S0),
                         float(scale), _p(o), _p(ST), _p(dT), _p(rho), _p(k_tilde), _p(cu_seqlens),
                         num_seqs, B, T, H, Dk, Dv, int(chunk), io, _p(workspace), ws_bytes,
                         _stream(stream)),
@@ -262,6 +285,45 @@ def osdn_step(q, k, v, beta, S, d, r=None, eta: float = 0.0, scale: float = 1.0,
                          Dk, Dv, io, _stream(stream)),
            "osdn_step")
     return o
+
+
+def osdn_bwd(q, k, v, beta, dO, r=None, eta: float = 0.0, d0=None, S0=None, scale: float = 1.0,
+             dST=None, ddT=None, cu_seqlens=None, workspace=None, stream=None):
+    """Gradients of L (given dL/do = dO, and optionally dL/dS_T, dL/dd_T) with respect to every
+    input of :func:`osdn_fwd`.  Returns a dict of float32 tensors dq, dk, dv, dbeta, dr (None
+    without r), deta (one element), dS0, dd0.  A workspace of ``osdn_bwd_workspace_bytes``
+    bytes is allocated with torch when none is given (device memory plumbing)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    io = _io(q)
+    num_seqs, N = _seqs(cu_seqlens, B)
+    for name, t in (("q", q), ("k", k)):
+        _req(t, name, q.dtype, (B, T, H, Dk))
+    _req(v, "v", q.dtype, (B, T, H, Dv))
+    _req(dO, "dO", q.dtype, (B, T, H, Dv))
+    _req(beta, "beta", torch.float32, (B, T, H))
+    _req(r, "r", torch.float32, (B, T, H))
+    _req(d0, "d0", torch.float32, (N, H, Dk))
+    _req(S0, "S0", torch.float32, (N, H, Dv, Dk))
+    _req(dST, "dST", torch.float32, (N, H, Dv, Dk))
+    _req(ddT, "ddT", torch.float32, (N, H, Dk))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty((B, T, H, Dk), **f32), "dk": torch.empty((B, T, H, Dk), **f32),
+         "dv": torch.empty((B, T, H, Dv), **f32), "dbeta": torch.empty((B, T, H), **f32),
+         "dr": None if r is None else torch.empty((B, T, H), **f32),
+         "deta": torch.empty((1,), **f32), "dS0": torch.empty((N, H, Dv, Dk), **f32),
+         "dd0": torch.empty((N, H, Dk), **f32)}
+    need = int(LIB.osdn_bwd_workspace_bytes(num_seqs, B, T, H, Dk, Dv, io))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _req(workspace, "workspace")
+    _check(LIB.osdn_bwd(_p(q), _p(k), _p(v), _p(beta), _p(r), float(eta), _p(d0), _p(S0),
+                        float(scale), _p(dO), _p(dST), _p(ddT), _p(g["dq"]), _p(g["dk"]),
+                        _p(g["dv"]), _p(g["dbeta"]), _p(g["dr"]), _p(g["deta"]), _p(g["dS0"]),
+                        _p(g["dd0"]), _p(cu_seqlens), num_seqs, B, T, H, Dk, Dv, io,
+                        _p(workspace), workspace.numel(), _stream(stream)),
+           "osdn_bwd")
+    return g
 
 
 def osdn_rho_geomean(rho, cu_seqlens=None, q_geo=None, stream=None):

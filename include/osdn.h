@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define OSDN_ABI_VERSION 4
+#define OSDN_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define OSDN_API __attribute__((visibility("default")))
@@ -109,6 +109,14 @@ OSDN_API osdn_status_t osdn_precond_scan(const void* k, const float* beta, const
  *   q, k    [B,T,H,Dk] io dtype, read (k is the erase/read key of the residual).
  *   k_tilde [B,T,H,Dk] io dtype, read (the write key).
  *   v       [B,T,H,Dv] io dtype, read.   beta [B,T,H] float32, read.
+ *   alpha   decay of a gated backbone, or NULL for none: [B,T,H] float32 (Gated DeltaNet, one
+ *           factor per token and head; alpha_per_channel = 0) or [B,T,H,Dk] float32 (Kimi Delta
+ *           Attention, one per key channel; alpha_per_channel = 1).  The state's key channels
+ *           decay before each write, S_t = S_{t-1} D_t + beta_t (v_t - S_{t-1} D_t k_t) k~_t^T
+ *           with D_t = Diag(alpha_t) (the gated delta rule of the Gated DeltaNet-2 page,
+ *           section 1, with OSDN's write key; phase 1 is unchanged).  Gated calls run phase 2 in
+ *           fp32 FMA arithmetic (the SIMT kernel) in either io dtype.  alpha_per_channel must be
+ *           0 or 1; alpha must not overlap an output.
  *   scale   multiplies o only (1.0 for unit-norm q).
  *   S0      [N,H,Dv,Dk] initial state, or NULL for zeros.
  *   o       [B,T,H,Dv] io dtype, written: o_t = scale * S_t q_t (state after token t).  Must
@@ -119,7 +127,8 @@ OSDN_API osdn_status_t osdn_precond_scan(const void* k, const float* beta, const
  *           depend on it beyond rounding.
  */
 OSDN_API osdn_status_t osdn_chunk_fwd(const void* q, const void* k, const void* k_tilde, const void* v,
-                             const float* beta, float scale, const float* S0, void* o, float* ST,
+                             const float* beta, const float* alpha, int32_t alpha_per_channel,
+                             float scale, const float* S0, void* o, float* ST,
                              const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
                              int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                              void* stream);
@@ -145,11 +154,12 @@ OSDN_API size_t osdn_fwd_workspace_bytes(int32_t B, int32_t T, int32_t H, int32_
  * The buffer rules of both phases apply; o must not overlap dT either.
  */
 OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, const float* beta,
-                       const float* r, float eta, const float* d0, const float* S0, float scale,
-                       void* o, float* ST, float* dT, float* rho, void* k_tilde_out,
-                       const int32_t* cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
-                       int32_t H, int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
-                       void* workspace, size_t workspace_bytes, void* stream);
+                       const float* r, const float* alpha, int32_t alpha_per_channel, float eta,
+                       const float* d0, const float* S0, float scale, void* o, float* ST,
+                       float* dT, float* rho, void* k_tilde_out, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk, int32_t Dv,
+                       int32_t chunk, osdn_dtype_t io, void* workspace, size_t workspace_bytes,
+                       void* stream);
 
 /*
  * osdn_fwd without any workspace, for callers that cannot allocate device memory: code that
@@ -177,12 +187,42 @@ OSDN_API osdn_status_t osdn_fwd(const void* q, const void* k, const void* v, con
  */
 #define OSDN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void* v,
-                                        const float* beta, const float* r, float eta,
+                                        const float* beta, const float* r, const float* alpha,
+                                        int32_t alpha_per_channel, float eta,
                                         const float* d0, const float* S0, float scale, void* o,
                                         float* ST, float* dT, float* rho, const int32_t* cu_seqlens,
                                         int32_t num_seqs, int32_t B, int32_t T, int32_t H,
                                         int32_t Dk, int32_t Dv, int32_t chunk, osdn_dtype_t io,
                                         void* stream);
+
+/*
+ * Backward pass of osdn_fwd: the gradients of a loss L with respect to every input, given
+ * dL/do, dL/dS_T and dL/dd_T.  The pages give no backward; this is the chain rule applied to the
+ * forward recurrences (phase 1 and phase 2 as stated at the top of this header) in reverse order,
+ * in fp32 FMA arithmetic (the path matches osdn_fwd's fp64 reference gradient, not a rounded one).
+ *   q, k, v, beta, r, eta, d0, S0, scale   the forward pass's inputs (as for osdn_fwd).
+ *   dO      [B,T,H,Dv] io dtype, read: dL/do.
+ *   dST     [N,H,Dv,Dk] float32: dL/dS_T, or NULL for 0.   ddT [N,H,Dk] float32: dL/dd_T, or NULL.
+ *   dq, dk  [B,T,H,Dk] float32, written.        dv [B,T,H,Dv] float32, written.
+ *   dbeta   [B,T,H] float32, written.           dr [B,T,H] float32, written, or NULL to skip.
+ *   deta    one float32, written (dL/deta), or NULL to skip.
+ *   dS0     [N,H,Dv,Dk] float32, written, or NULL.   dd0 [N,H,Dk] float32, written, or NULL.
+ *   workspace  device scratch of at least osdn_bwd_workspace_bytes(...) bytes, 256-byte aligned
+ *           (about (4 + 3 Dv/64) x 4 B per key channel and token-head, plus one Dv x Dk fp32 state
+ *           per 32 tokens and head).
+ * cu_seqlens, num_seqs, B, T, H as for the forward pass; Dk, Dv in {64, 128}.  Outputs must not
+ * overlap one another, the inputs or the workspace (OSDN_ERR_INVALID_ARG).
+ */
+OSDN_API size_t osdn_bwd_workspace_bytes(int32_t num_seqs, int32_t B, int32_t T, int32_t H,
+                                         int32_t Dk, int32_t Dv, osdn_dtype_t io);
+OSDN_API osdn_status_t osdn_bwd(const void* q, const void* k, const void* v, const float* beta,
+                                const float* r, float eta, const float* d0, const float* S0,
+                                float scale, const void* dO, const float* dST, const float* ddT,
+                                float* dq, float* dk, float* dv, float* dbeta, float* dr,
+                                float* deta, float* dS0, float* dd0, const int32_t* cu_seqlens,
+                                int32_t num_seqs, int32_t B, int32_t T, int32_t H, int32_t Dk,
+                                int32_t Dv, osdn_dtype_t io, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /*
  * q_geo, the residual-contraction diagnostic of section 3 (Theorem 5.2 bounds the product of

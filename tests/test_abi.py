@@ -14,11 +14,12 @@ def fake(i):
 
 
 def chunk_call(**kw):
-    args = dict(q=fake(1), k=fake(2), kt=fake(3), v=fake(4), beta=fake(5), scale=1.0, S0=None,
-                o=fake(6), ST=None, cu=None, num_seqs=0, B=1, T=8, H=1, Dk=128, Dv=128, chunk=64,
-                io=osdn.OSDN_BF16)
+    args = dict(q=fake(1), k=fake(2), kt=fake(3), v=fake(4), beta=fake(5), alpha=None, apc=0,
+                scale=1.0, S0=None, o=fake(6), ST=None, cu=None, num_seqs=0, B=1, T=8, H=1, Dk=128,
+                Dv=128, chunk=64, io=osdn.OSDN_BF16)
     args.update(kw)
     return L.osdn_chunk_fwd(args["q"], args["k"], args["kt"], args["v"], args["beta"],
+                            args["alpha"], args["apc"],
                             args["scale"], args["S0"], args["o"], args["ST"], args["cu"],
                             args["num_seqs"], args["B"], args["T"], args["H"], args["Dk"],
                             args["Dv"], args["chunk"], args["io"], None)
@@ -44,7 +45,7 @@ def test_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert L.osdn_abi_version() == 4
+    assert L.osdn_abi_version() == 6
     for s in range(7):
         assert osdn.status_string(s)
     assert osdn.status_string(99) == "unknown status"
@@ -76,6 +77,9 @@ def test_workspace_size():
     (dict(beta=ctypes.c_void_p(A + 6 * 0x1000000 + 256)), osdn.OSDN_ERR_INVALID_ARG),  # in o
     (dict(S0=ctypes.c_void_p(A + 6 * 0x1000000)), osdn.OSDN_ERR_INVALID_ARG),
     (dict(ST=ctypes.c_void_p(A + 6 * 0x1000000 + 1024)), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(alpha=fake(8), apc=2), osdn.OSDN_ERR_INVALID_ARG),                    # flag not 0 / 1
+    (dict(alpha=ctypes.c_void_p(A + 8 * 0x1000000 + 4)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(alpha=ctypes.c_void_p(A + 6 * 0x1000000 + 32)), osdn.OSDN_ERR_INVALID_ARG),  # in o
 ])
 def test_chunk_fwd_rejects(kw, status):
     assert chunk_call(**kw) == status
@@ -104,9 +108,9 @@ def test_precond_scan_rejects(kw, status):
 
 def test_fwd_needs_workspace_even_with_k_tilde_out():
     """In bf16 mode the workspace holds the lo term of k~ even when k~ goes to k_tilde_out."""
-    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
-                    None, None, fake(8), None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16, None, 0,
-                    None)
+    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, None, 0, 0.1, None, None, 1.0,
+                    fake(6), None, None, None, fake(8), None, 0, 1, 64, 1, 128, 128, 64,
+                    osdn.OSDN_BF16, None, 0, None)
     assert st == osdn.OSDN_ERR_INVALID_ARG
 
 
@@ -128,13 +132,13 @@ def test_rho_geomean_rejects(kw, status):
 
 
 def test_fwd_rejects_small_workspace():
-    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
-                    None, None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16, fake(7), 100,
-                    None)
+    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, None, 0, 0.1, None, None, 1.0,
+                    fake(6), None, None, None, None, None, 0, 1, 64, 1, 128, 128, 64,
+                    osdn.OSDN_BF16, fake(7), 100, None)
     assert st == osdn.OSDN_ERR_INVALID_ARG
-    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, 0.1, None, None, 1.0, fake(6), None,
-                    None, None, None, None, 0, 1, 64, 1, 128, 128, 64, osdn.OSDN_BF16,
-                    ctypes.c_void_p(A + 0x7000010), 1 << 20, None)
+    st = L.osdn_fwd(fake(1), fake(2), fake(4), fake(5), None, None, 0, 0.1, None, None, 1.0,
+                    fake(6), None, None, None, None, None, 0, 1, 64, 1, 128, 128, 64,
+                    osdn.OSDN_BF16, ctypes.c_void_p(A + 0x7000010), 1 << 20, None)
     assert st == osdn.OSDN_ERR_ALIGNMENT  # workspace must be 256-byte aligned
 
 
@@ -185,3 +189,41 @@ def step_call(**kw):
 ])
 def test_step_rejects(kw, status):
     assert step_call(**kw) == status
+
+
+def bwd_call(**kw):
+    args = dict(q=fake(1), k=fake(2), v=fake(3), beta=fake(4), r=None, eta=0.1, d0=None, S0=None,
+                scale=1.0, dO=fake(5), dST=None, ddT=None, dq=fake(6), dk=fake(7), dv=fake(8),
+                dbeta=fake(9), dr=None, deta=None, dS0=None, dd0=None, cu=None, num_seqs=0, B=1,
+                T=64, H=2, Dk=128, Dv=128, io=osdn.OSDN_BF16, ws=fake(10), wsb=1 << 30)
+    args.update(kw)
+    a = args
+    return L.osdn_bwd(a["q"], a["k"], a["v"], a["beta"], a["r"], a["eta"], a["d0"], a["S0"],
+                      a["scale"], a["dO"], a["dST"], a["ddT"], a["dq"], a["dk"], a["dv"], a["dbeta"],
+                      a["dr"], a["deta"], a["dS0"], a["dd0"], a["cu"], a["num_seqs"], a["B"], a["T"],
+                      a["H"], a["Dk"], a["Dv"], a["io"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Dk=96), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(Dv=32), osdn.OSDN_ERR_UNSUPPORTED),
+    (dict(dq=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(dO=None), osdn.OSDN_ERR_INVALID_ARG),
+    (dict(wsb=1000), osdn.OSDN_ERR_INVALID_ARG),                     # workspace too small
+    (dict(ws=ctypes.c_void_p(A + 10 * 0x1000000 + 16)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(dk=fake(6)), osdn.OSDN_ERR_INVALID_ARG),                   # dk aliases dq
+    (dict(dv=fake(3)), osdn.OSDN_ERR_INVALID_ARG),                   # dv aliases v
+    (dict(dbeta=ctypes.c_void_p(A + 10 * 0x1000000 + 4096)), osdn.OSDN_ERR_INVALID_ARG),  # in ws
+    (dict(deta=ctypes.c_void_p(A + 9 * 0x1000000 + 4)), osdn.OSDN_ERR_ALIGNMENT),
+    (dict(B=-1), osdn.OSDN_ERR_INVALID_ARG),
+])
+def test_bwd_rejects(kw, status):
+    assert bwd_call(**kw) == status
+
+
+def test_bwd_workspace_size_grows_with_the_batch():
+    small = L.osdn_bwd_workspace_bytes(0, 1, 64, 2, 128, 128, osdn.OSDN_BF16)
+    big = L.osdn_bwd_workspace_bytes(0, 4, 4096, 16, 128, 128, osdn.OSDN_BF16)
+    assert 0 < small < big
+    assert big % 256 == 0
+    assert L.osdn_bwd_workspace_bytes(0, 1, 64, 2, 96, 128, osdn.OSDN_BF16) == 0

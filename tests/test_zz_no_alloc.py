@@ -27,8 +27,8 @@ def _lib():
     from delta_rule_recurrent_osdn_b200 import osdn
     lib = osdn.LIB
     f = lib.osdn_fwd_noalloc
-    f.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _i32,
-                  _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
+    f.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
+                  _i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_int, _vp]
     f.restype = ctypes.c_int
     return osdn, f
 
@@ -42,7 +42,8 @@ def _noalloc(f, d, inp, o, ST, dT, io):
     Dv = d["v"].shape[-1]
     cu = d["cu_seqlens"]
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    return f(_p(d["q"]), _p(d["k"]), _p(d["v"]), _p(d["beta"]), _p(d["r"]), d["eta"], _p(d["d0"]),
+    return f(_p(d["q"]), _p(d["k"]), _p(d["v"]), _p(d["beta"]), _p(d["r"]), None, 0, d["eta"],
+             _p(d["d0"]),
              _p(d["S0"]), d["scale"], _p(o), _p(ST), _p(dT), None, _p(cu),
              0 if cu is None else cu.numel() - 1, B, T, H, Dk, Dv, d["chunk"], io, stream)
 
@@ -81,7 +82,6 @@ def test_noalloc_rejects_keys_larger_than_its_array():
     the 32 MiB array: the call is refused before anything is enqueued."""
     osdn, f = _lib()
     fake = ctypes.c_void_p(0x10000000)
-    st = f(fake, fake, fake, fake, None, 0.05, None, None, 1.0, fake, None, None, None, None, 0, 4,
-           4096,
-           16, 128, 128, 64, osdn.OSDN_BF16, None)
+    st = f(fake, fake, fake, fake, None, None, 0, 0.05, None, None, 1.0, fake, None, None, None,
+           None, 0, 4, 4096, 16, 128, 128, 64, osdn.OSDN_BF16, None)
     assert st == osdn.OSDN_ERR_UNSUPPORTED
