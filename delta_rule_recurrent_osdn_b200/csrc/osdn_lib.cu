@@ -201,7 +201,8 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
         (long long)kWaitLimitNs);
     const osdn_status_t st = launch_status();
     if (st != OSDN_OK) return st;
-    auto chain = precond_chain_kernel;
+    auto chain = kt_lo ? (d_all ? precond_chain_kernel<true, true> : precond_chain_kernel<true, false>)
+                       : (d_all ? precond_chain_kernel<false, true> : precond_chain_kernel<false, false>);
     if (!set_smem(chain, ScanChainSmem::BYTES)) return OSDN_ERR_CUDA;
     chain<<<dim3((unsigned)nh), dim3(SCAN_CHAIN_THREADS), ScanChainSmem::BYTES, stream>>>(
         mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde),

@@ -327,17 +327,19 @@ struct ScanChainSmem {
     static constexpr uint32_t X = D + 3 * 512;        // 3 x x [64]
     static constexpr uint32_t GX = X + 3 * 256;       // g (.) x [64]
     static constexpr uint32_t BV = GX + 256;          // b [64]
-    static constexpr uint32_t LO = BV + 256;          // bf16 k~ lo staging tile (16 KB, SW128)
-    static constexpr uint32_t BAR = LO + 16384;       // 15 mbarriers
+    static constexpr uint32_t LO = BV + 256;          // 2 x bf16 k~ lo staging tile (16 KB, SW128)
+    static constexpr uint32_t BAR = LO + 2 * 16384;   // 15 mbarriers
     static constexpr uint32_t TOTAL = BAR + 15 * 8;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
-constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output, 8 loads and gates
+constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output (two groups), 8 loads and gates
 
 // One CTA per (sequence, head).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
-// k_tilde receives k~ rounded to bf16 (hi); k_tilde_lo, when not null, receives the rounding
-// residual bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.  d_all, when not
-// null ([B,T,H,Dk] fp32), receives d_t, the preconditioner each token writes with.
+// k_tilde receives k~ rounded to bf16 (hi); with kLo, k_tilde_lo receives the rounding residual
+// bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.  With kD, d_all
+// ([B,T,H,Dk] fp32) receives d_t, the preconditioner each token writes with.  (Compile-time
+// options: the token pass is issue-bound, and the forward pass needs neither check.)
+template <bool kLo, bool kD>
 __global__ void __launch_bounds__(SCAN_CHAIN_THREADS, 1)
 precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_td,
                      const float* __restrict__ beta, const float* __restrict__ r, float eta,
@@ -360,9 +362,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* full = bars;         // [3] TMA: k tile + T_d tile
     uint64_t* vready = bars + 3;   // [3] gate vectors (32 arrivals)
-    uint64_t* kempty = bars + 6;   // [3] output warps done with the slot (128)
+    uint64_t* kempty = bars + 6;   // [3] the chunk's writer group done with the slot (64)
     uint64_t* xready = bars + 9;   // [3] x and d of a chunk ready (128)
-    uint64_t* outdone = bars + 12; // [3] output warps done with x / d buffers (128)
+    uint64_t* outdone = bars + 12; // [3] the chunk's writer group done with x / d buffers (64)
     float* sD = reinterpret_cast<float*>(smem + L::D);
     float* sX = reinterpret_cast<float*>(smem + L::X);
     float* sGX = reinterpret_cast<float*>(smem + L::GX);
@@ -377,9 +379,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         for (int s = 0; s < 3; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&vready[s], 32);
-            mbar_init(&kempty[s], 128);
+            mbar_init(&kempty[s], 64);   // one writer group per chunk
             mbar_init(&xready[s], 128);
-            mbar_init(&outdone[s], 128);
+            mbar_init(&outdone[s], 64);
         }
         tc::fence_mbar_init();
     }
@@ -553,64 +555,75 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         if (ok && dT) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
     } else {
         // =============================================== k~ = d (.) k, token by token
-        const int i = tid - 128, blk = i >> 6, cj = (i & 63) >> 3, ce = i & 7;
-        for (int c = 0; c < nchunks; ++c) {
+        // Two groups of 64 threads take alternate chunks (group g: chunks c = g, g + 2, ...), so
+        // each has two chunk periods for its token pass; a thread carries the key-channel pair
+        // (2 jj, 2 jj + 1): packed bf16x2 conversions and 4-byte stores, two independent chains.
+        const int i = tid - 128, g = i >> 6, jj = i & 63;
+        const int blk = jj >> 5, cj = (jj & 31) >> 2, ce = 2 * (jj & 3);  // channel 2 jj in the tile
+        const int gbar = 2 + g;  // the group's named barrier
+        uint8_t* lo_stage = smem + L::LO + g * 16384;
+        for (int c = g; c < nchunks; c += 2) {
             const int s = c % 3;
-            if (group_any(2, 128, !mbar_wait_bounded(&xready[c % 3], (uint32_t)(c / 3) & 1u, limit_ns)))
+            if (group_any(gbar, 64, !mbar_wait_bounded(&xready[c % 3], (uint32_t)(c / 3) & 1u, limit_ns)))
                 break;
             const int Lc = chunk_len(c);
             const uint8_t* col = smem + L::KT + s * 16384 + blk * 8192u + ce * 2;
             const float* xv = sX + (c % 3) * 64;
             const float* rv = vecs(s) + 128;
-            float dd = sD[(c % 3) * 128 + i];
+            float2 dd = *reinterpret_cast<const float2*>(sD + (c % 3) * 128 + 2 * jj);
             // k~ goes to the chunk's T_d slot (consumed by step 2 before x was published) in the
             // key tile's swizzled layout, then to global memory as whole 16-byte row pieces:
             // scattered 2-byte stores would cost about three times the whole token pass
             uint8_t* stage = smem + L::TD + s * 16384;
             uint8_t* ocol = stage + blk * 8192u + ce * 2;
-            uint8_t* lcol = smem + L::LO + blk * 8192u + ce * 2;
+            uint8_t* lcol = lo_stage + blk * 8192u + ce * 2;
+            float* drow = kD ? d_all + ((first + (int64_t)c * C) * H + h) * DK + 2 * jj : nullptr;
 #pragma unroll 1
             for (int t0 = 0; t0 < Lc; t0 += 16) {
-                float kv[16], xt[16], rt[16];
+                float2 kv[16];
+                float xt[16], rt[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    kv[u] = __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16*>(col + tc::sw128_off(t0 + u, cj)));
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(col + tc::sw128_off(t0 + u, cj));
+                    kv[u] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
                     xt[u] = xv[t0 + u];
                     rt[u] = rv[t0 + u];
                 }
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    if (d_all && t0 + u < Lc)
-                        d_all[((first + (int64_t)c * C + t0 + u) * H + h) * DK + i] = dd;
-                    const float kt = dd * kv[u];
-                    const __nv_bfloat16 hb = __float2bfloat16_rn(kt);
-                    *reinterpret_cast<__nv_bfloat16*>(ocol + tc::sw128_off(t0 + u, cj)) = hb;
-                    if (k_tilde_lo)
-                        *reinterpret_cast<__nv_bfloat16*>(lcol + tc::sw128_off(t0 + u, cj)) =
-                            __float2bfloat16_rn(kt - __bfloat162float(hb));
-                    dd = fmaf(rt[u], dd, xt[u] * kv[u] * kv[u]);
+                    if (kD && t0 + u < Lc)
+                        *reinterpret_cast<float2*>(drow + (int64_t)(t0 + u) * H * DK) = dd;
+                    const float2 kt = __fmul2_rn(dd, kv[u]);
+                    const __nv_bfloat162 hb = __floats2bfloat162_rn(kt.x, kt.y);
+                    *reinterpret_cast<__nv_bfloat162*>(ocol + tc::sw128_off(t0 + u, cj)) = hb;
+                    if (kLo) {
+                        const float2 hf = __bfloat1622float2(hb);
+                        *reinterpret_cast<__nv_bfloat162*>(lcol + tc::sw128_off(t0 + u, cj)) =
+                            __floats2bfloat162_rn(kt.x - hf.x, kt.y - hf.y);
+                    }
+                    const float2 a = __fmul2_rn(kv[u], kv[u]);
+                    dd = __ffma2_rn(make_float2(rt[u], rt[u]), dd, __fmul2_rn(make_float2(xt[u], xt[u]), a));
                 }
             }
-            group_bar(2, 128);
-            {
-                const int piece = i & 15, blk16 = piece >> 3, j16 = piece & 7;
+            group_bar(gbar, 64);
+            {  // 64 rows x 16 pieces of 16 bytes per tile: piece jj & 15, rows (jj >> 4) + 4 q
+                const int piece = jj & 15, blk16 = piece >> 3, j16 = piece & 7;
                 const int64_t off = ((first + (int64_t)c * C) * H + h) * DK + 8 * piece;
                 const int64_t rs = (int64_t)H * DK;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int row = (i >> 4) + 8 * q;
+#pragma unroll 4
+                for (int q = 0; q < 16; ++q) {
+                    const int row = (jj >> 4) + 4 * q;
                     if (row < Lc) {
                         const uint32_t so = blk16 * 8192u + tc::sw128_off(row, j16);
                         *reinterpret_cast<uint4*>(k_tilde + off + row * rs) =
                             *reinterpret_cast<const uint4*>(stage + so);
-                        if (k_tilde_lo)
+                        if (kLo)
                             *reinterpret_cast<uint4*>(k_tilde_lo + off + row * rs) =
-                                *reinterpret_cast<const uint4*>(smem + L::LO + so);
+                                *reinterpret_cast<const uint4*>(lo_stage + so);
                     }
                 }
             }
-            if (k_tilde_lo) group_bar(2, 128);  // the single lo staging tile is read out
+            if (kLo) group_bar(gbar, 64);  // the group's lo staging tile is read out
             mbar_arrive(&kempty[s]);
             mbar_arrive(&outdone[c % 3]);
         }
