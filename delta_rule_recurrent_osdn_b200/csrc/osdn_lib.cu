@@ -204,10 +204,24 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     auto chain = kt_lo ? (d_all ? precond_chain_kernel<true, true> : precond_chain_kernel<true, false>)
                        : (d_all ? precond_chain_kernel<false, true> : precond_chain_kernel<false, false>);
     if (!set_smem(chain, ScanChainSmem::BYTES)) return OSDN_ERR_CUDA;
-    chain<<<dim3((unsigned)nh), dim3(SCAN_CHAIN_THREADS), ScanChainSmem::BYTES, stream>>>(
-        mk, mtd, beta, r, eta, d0, static_cast<__nv_bfloat16*>(k_tilde),
-        static_cast<__nv_bfloat16*>(kt_lo), d_all, dT, rho, cu, d.N, d.T, d.H,
-        (long long)kWaitLimitNs);
+    if (2 * nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
+    // one 2-CTA cluster per (sequence, head): the chain and the k~ token pass on separate SMs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * nh));
+    cfg.blockDim = dim3(SCAN_CHAIN_THREADS);
+    cfg.dynamicSmemBytes = ScanChainSmem::BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, chain, mk, mtd, beta, r, eta, d0,
+                           static_cast<__nv_bfloat16*>(k_tilde), static_cast<__nv_bfloat16*>(kt_lo),
+                           d_all, dT, rho, cu, d.N, d.T, d.H, (long long)kWaitLimitNs) != cudaSuccess)
+        return OSDN_ERR_CUDA;
     return launch_status();
 }
 

@@ -328,13 +328,21 @@ struct ScanChainSmem {
     static constexpr uint32_t GX = X + 3 * 256;       // g (.) x [64]
     static constexpr uint32_t BV = GX + 256;          // b [64]
     static constexpr uint32_t LO = BV + 256;          // 2 x bf16 k~ lo staging tile (16 KB, SW128)
-    static constexpr uint32_t BAR = LO + 2 * 16384;   // 15 mbarriers
-    static constexpr uint32_t TOTAL = BAR + 15 * 8;
+    static constexpr uint32_t XW = LO + 2 * 16384;    // 2 x the writer groups' copy of x [64]
+    static constexpr uint32_t BAR = XW + 2 * 256;     // 21 mbarriers
+    static constexpr uint32_t TOTAL = BAR + 21 * 8;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
 constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output (two groups), 8 loads and gates
 
-// One CTA per (sequence, head).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
+// One 2-CTA cluster per (sequence, head).  Rank 0 runs the chain (warps 0-3), its loads (warp 8:
+// k and T_d tiles, gate vectors) and a forwarder (warp 4); rank 1 runs the k~ token pass (warps
+// 4-7) and its own loads (warp 8: k tiles, r).  The token pass gets an SM of its own.  The chain
+// only arrives on local barriers; the forwarder copies x and the chunk-start d of each chunk into
+// rank 1's shared memory and arrives on rank 1's barrier (release / acquire at cluster scope), so
+// no chain thread waits for a cluster-scope release.  Rank 1's writers copy x out and arrive back
+// on rank 0 before their token pass.  The two CTAs of a cluster are co-scheduled, so these
+// cross-CTA waits are safe (and bounded like every other).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
 // k_tilde receives k~ rounded to bf16 (hi); with kLo, k_tilde_lo receives the rounding residual
 // bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.  With kD, d_all
 // ([B,T,H,Dk] fp32) receives d_t, the preconditioner each token writes with.  (Compile-time
@@ -352,19 +360,24 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = blockIdx.x / H, h = blockIdx.x - n * H;
-    if (n >= N) return;
+    const uint32_t rank = tc::cluster_rank();  // 0: the chain, 1: the k~ token pass
+    const int pair = blockIdx.x >> 1;
+    const int n = pair / H, h = pair - n * H;
+    if (n >= N) return;  // uniform over the cluster
     int64_t first, count;
-    if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the CTA
+    if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the cluster
     const int nchunks = (int)((count + C - 1) / C);
     const int64_t dbase = ((int64_t)n * H + h) * DK;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
-    uint64_t* full = bars;         // [3] TMA: k tile + T_d tile
+    uint64_t* full = bars;         // [3] TMA: k tile (+ T_d tile on rank 0)
     uint64_t* vready = bars + 3;   // [3] gate vectors (32 arrivals)
-    uint64_t* kempty = bars + 6;   // [3] the chunk's writer group done with the slot (64)
-    uint64_t* xready = bars + 9;   // [3] x and d of a chunk ready (128)
-    uint64_t* outdone = bars + 12; // [3] the chunk's writer group done with x / d buffers (64)
+    uint64_t* kempty = bars + 6;   // [3] slot released: rank 0 by the chain (128), rank 1 by the
+                                   //     chunk's writer group (64)
+    uint64_t* xready = bars + 9;   // [3] rank 1: x and d of a chunk, from rank 0's forwarder (32)
+    uint64_t* outdone = bars + 12; // [3] rank 0: rank 1's writer group has copied x / d (64)
+    uint64_t* fwdin = bars + 15;   // [3] rank 0: x and d of a chunk in local memory (128, chain)
+    uint64_t* fwdout = bars + 18;  // [3] rank 0: the forwarder has sent them (32)
     float* sD = reinterpret_cast<float*>(smem + L::D);
     float* sX = reinterpret_cast<float*>(smem + L::X);
     float* sGX = reinterpret_cast<float*>(smem + L::GX);
@@ -379,17 +392,54 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         for (int s = 0; s < 3; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&vready[s], 32);
-            mbar_init(&kempty[s], 64);   // one writer group per chunk
-            mbar_init(&xready[s], 128);
+            mbar_init(&kempty[s], rank == 0 ? 128 : 64);
+            mbar_init(&xready[s], 32);
             mbar_init(&outdone[s], 64);
+            mbar_init(&fwdin[s], 128);
+            mbar_init(&fwdout[s], 32);
         }
         tc::fence_mbar_init();
     }
     if (tid < DK) sD[tid] = d0 ? __ldg(d0 + dbase + tid) : 1.0f;
-    __syncthreads();
+    tc::fence_before_sync();
+    tc::cluster_sync();  // both CTAs initialised before either touches the other
+    // rank 0's view of rank 1's x / d buffers and barriers, and rank 1's of rank 0's
+    const uint32_t peer_x = tc::cluster_map(smem_u32(smem + L::X), 1u);
+    const uint32_t peer_d = tc::cluster_map(smem_u32(smem + L::D), 1u);
+    const uint32_t peer_xready = tc::cluster_map(smem_u32(xready), 1u);
+    const uint32_t peer_outdone = tc::cluster_map(smem_u32(outdone), 0u);
 
-    if (warp == 8) {
-        // =============================================== loads and gate vectors
+    if (warp == 8 && rank == 1) {
+        // =============================================== rank 1: k tiles and r for the token pass
+        if (lane == 0) tc::prefetch_tmap(&tm_k);
+        int last_issued = -1;
+        bool fail = false;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % 3;
+            if (c >= 3 && !mbar_wait_bounded(&kempty[s], (uint32_t)(c / 3 - 1) & 1u, limit_ns)) {
+                fail = true;
+                break;
+            }
+            const int64_t row0 = first + (int64_t)c * C;
+            if (lane == 0) {
+                uint8_t* kt = smem + L::KT + s * 16384;
+                tc::mbar_expect_tx(&full[s], 16384);
+                tc::tma_load_3d(kt, &tm_k, 0, h, (int)row0, &full[s]);
+                tc::tma_load_3d(kt + 8192, &tm_k, 64, h, (int)row0, &full[s]);
+            }
+            last_issued = c;
+            const int Lc = chunk_len(c), t0 = 2 * lane;
+            float* vv = vecs(s);
+            vv[128 + t0] = (r && t0 < Lc) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
+            vv[128 + t0 + 1] = (r && t0 + 1 < Lc) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
+            mbar_arrive(&vready[s]);
+        }
+        if (fail && lane == 0 && last_issued >= 0) {  // let the loads in flight land
+            for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
+                mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
+        }
+    } else if (warp == 8) {
+        // =============================================== rank 0: loads and gate vectors
         if (lane == 0) {
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_td);
@@ -443,7 +493,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
                 mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
         }
-    } else if (warp < 4) {
+    } else if (warp < 4 && rank == 0) {
         // =============================================== p = A d, x = T_d b, next d
         const int u = tid;
         const int t = 16 * warp + (lane & 15), half = lane >> 4;  // step 1/2 roles
@@ -455,8 +505,8 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             const uint32_t ph = (uint32_t)(c / 3) & 1u;
             bool got = mbar_wait_bounded(&full[s], ph, limit_ns) &&
                        mbar_wait_bounded(&vready[s], ph, limit_ns);
-            if (got && c >= 2)
-                got = mbar_wait_bounded(&outdone[(c - 2) % 3], (uint32_t)((c - 2) / 3) & 1u, limit_ns);
+            if (got && c >= 2)  // the forwarder has sent the x / d buffers this chunk overwrites
+                got = mbar_wait_bounded(&fwdout[(c - 2) % 3], (uint32_t)((c - 2) / 3) & 1u, limit_ns);
             if (group_any(1, 128, !got)) {
                 ok = false;
                 break;
@@ -545,15 +595,40 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 if (par == 0) {
                     const float rc = vv[256];
                     const float2 dv = *reinterpret_cast<const float2*>(d + 2 * cp);
-                    *reinterpret_cast<float2*>(sD + ((c + 1) % 3) * 128 + 2 * cp) =
-                        make_float2(fmaf(rc, dv.x, acc0), fmaf(rc, dv.y, acc1));
+                    const float2 dn = make_float2(fmaf(rc, dv.x, acc0), fmaf(rc, dv.y, acc1));
+                    *reinterpret_cast<float2*>(sD + ((c + 1) % 3) * 128 + 2 * cp) = dn;
                 }
             }
-            mbar_arrive(&xready[c % 3]);
+            mbar_arrive(&fwdin[c % 3]);  // x_c and d_c are in sX, sD: the forwarder sends them
+            mbar_arrive(&kempty[s]);     // the chain's last use of the slot
             group_bar(1, 128);
         }
         if (ok && dT) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
-    } else {
+    } else if (warp == 4 && rank == 0) {
+        // =============================================== forwarder: x_c, d_c to rank 1
+        // Chunk c's x and chunk-start d go into slot c % 3 of rank 1's buffers once rank 1's
+        // writer of chunk c - 3 has copied that slot out; the slot's local copies may then be
+        // overwritten by the chain (fwdout).
+        for (int c = 0; c < nchunks; ++c) {
+            const int k = c % 3;
+            bool got = mbar_wait_bounded(&fwdin[k], (uint32_t)(c / 3) & 1u, limit_ns);
+            if (got && c >= 3)
+                got = tc::mbar_wait_cluster(&outdone[k], (uint32_t)(c / 3 - 1) & 1u, limit_ns);
+            if (__any_sync(0xffffffffu, !got)) break;
+            {
+                const float2 xv = *reinterpret_cast<const float2*>(sX + k * 64 + 2 * lane);
+                tc::st_cluster_v2f32(peer_x + 4u * (uint32_t)(k * 64 + 2 * lane), xv.x, xv.y);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int e = 2 * lane + 64 * q;
+                    const float2 dv = *reinterpret_cast<const float2*>(sD + k * 128 + e);
+                    tc::st_cluster_v2f32(peer_d + 4u * (uint32_t)(k * 128 + e), dv.x, dv.y);
+                }
+            }
+            mbar_arrive(&fwdout[k]);                                // local copies are free
+            tc::mbar_arrive_cluster(peer_xready + 8u * (uint32_t)k);  // rank 1 may read them
+        }
+    } else if (warp >= 4 && warp < 8 && rank == 1) {
         // =============================================== k~ = d (.) k, token by token
         // Two groups of 64 threads take alternate chunks (group g: chunks c = g, g + 2, ...), so
         // each has two chunk periods for its token pass; a thread carries the key-channel pair
@@ -564,13 +639,20 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         uint8_t* lo_stage = smem + L::LO + g * 16384;
         for (int c = g; c < nchunks; c += 2) {
             const int s = c % 3;
-            if (group_any(gbar, 64, !mbar_wait_bounded(&xready[c % 3], (uint32_t)(c / 3) & 1u, limit_ns)))
-                break;
+            const uint32_t ph = (uint32_t)(c / 3) & 1u;
+            const bool got = mbar_wait_bounded(&full[s], ph, limit_ns) &&
+                             mbar_wait_bounded(&vready[s], ph, limit_ns) &&
+                             tc::mbar_wait_cluster(&xready[c % 3], ph, limit_ns);
+            if (group_any(gbar, 64, !got)) break;
             const int Lc = chunk_len(c);
             const uint8_t* col = smem + L::KT + s * 16384 + blk * 8192u + ce * 2;
-            const float* xv = sX + (c % 3) * 64;
-            const float* rv = vecs(s) + 128;
+            // copy x and this pair's d out of the slot rank 0's forwarder fills, and free it
+            float* xv = reinterpret_cast<float*>(smem + L::XW + g * 256);
+            xv[jj] = sX[(c % 3) * 64 + jj];
             float2 dd = *reinterpret_cast<const float2*>(sD + (c % 3) * 128 + 2 * jj);
+            group_bar(gbar, 64);
+            tc::mbar_arrive_cluster(peer_outdone + 8u * (uint32_t)(c % 3));
+            const float* rv = vecs(s) + 128;
             // k~ goes to the chunk's T_d slot (consumed by step 2 before x was published) in the
             // key tile's swizzled layout, then to global memory as whole 16-byte row pieces:
             // scattered 2-byte stores would cost about three times the whole token pass
@@ -623,12 +705,12 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     }
                 }
             }
-            if (kLo) group_bar(gbar, 64);  // the group's lo staging tile is read out
+            group_bar(gbar, 64);  // the group's staging tiles and x copy are read out
             mbar_arrive(&kempty[s]);
-            mbar_arrive(&outdone[c % 3]);
         }
     }
-    __syncthreads();
+    tc::fence_before_sync();
+    tc::cluster_sync();  // neither CTA leaves while the other may still write to it
 }
 
 }  // namespace osdn

@@ -157,6 +157,44 @@ __device__ __forceinline__ uint32_t ld_cluster_acquire(uint32_t local) {
     asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(local) : "memory");
     return v;
 }
+// Stores into another CTA's shared memory (a shared::cluster address from cluster_map).
+__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_v2f32(uint32_t cluster_addr, float a, float b) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(cluster_addr), "f"(a), "f"(b)
+                 : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster, ordering this thread's earlier writes
+// (to that CTA's shared memory included) before the arrival at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+// Bounded wait on a local mbarrier whose arrivals come from other CTAs of the cluster: acquire
+// at cluster scope, so their writes before arriving are visible after it.
+__device__ __forceinline__ bool mbar_try_parity_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int64_t limit_ns) {
+    if (mbar_try_parity_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_parity_cluster(bar, parity)) return true;
+        if (global_ns() - t0 > static_cast<uint64_t>(limit_ns)) break;
+    }
+    record_status(OSDN_ERR_DEVICE_TIMEOUT);
+    return false;
+}
+
 // Wait until the counter at `local` (written by another CTA of the cluster) reaches `target`,
 // for at most `limit_ns`; records OSDN_ERR_DEVICE_TIMEOUT and returns false otherwise.
 __device__ __forceinline__ bool wait_counter(uint32_t local, uint32_t target, int64_t limit_ns) {
