@@ -19,14 +19,21 @@
 // Kernels (one call of osdn_bwd):
 //   1. phase 1 forward (the forward pass's own kernels), which also writes d_t of every token;
 //   2. bwd_delta_kernel: one CTA per (sequence, head, 64 value rows).  Rows of S and of dS are
-//      independent, so each CTA carries its rows: a forward sweep over the sequence (states at
-//      every 32-token chunk start kept in a workspace, dq's share of these rows), then chunks in
-//      reverse: u_s of the chunk's tokens from the chunk-start state (S_{s-1} = S_c +
-//      sum_{j<s} beta_j u_j k~_j^T, a forward substitution with the chunk Gram K K~^T), and a
-//      reverse token sweep of dS.  dv is per row; dq, dk, dk~ and dbeta's phase-2 term are sums
-//      over all value rows, written as per-CTA shares;
-//   3. bwd_precond_kernel: one CTA per (sequence, head): adds the shares and runs the phase-1
-//      adjoint recurrence in reverse (one warp, a chunk of tokens staged in shared memory);
+//      independent, so each CTA carries its rows through the chunk-level algebra (32-token chunks,
+//      the state S_c at each chunk start, A = K K~^T, T = (I + strict_tril(diag(beta) A))^-1,
+//      E = V - K S_c^T, R = diag(beta) E, W = T R, P = tril(Q K~^T), S' = S_c + W^T K~): a forward
+//      sweep keeps S_c of every chunk in a workspace; then, chunks in reverse, with dS' the adjoint
+//      at the chunk's end,
+//        dW = K~ dS'^T + scale P^T dO,  dP = tril(scale dO W^T),  dR = T^T dW,
+//        dL = -strict_tril(T^T (dW R^T) T^T),  dv = diag(beta) dR,
+//        dq = scale dO S_c + dP K~,  dk~ = W dS' + dP^T Q + (diag(beta) dL)^T K,
+//        dk = diag(beta) dL K~ - diag(beta) dR S_c,  dbeta = rowsum(dL . A) + rowsum(dR . E),
+//        dS = dS' + scale dO^T Q - (diag(beta) dR)^T K.
+//      dv and dS are per row; dq, dk, dk~ and dbeta's phase-2 term sum over all value rows (dP and
+//      dL are linear in such sums), so each CTA writes its share;
+//   3. bwd_reduce_kernel: the shares added up, elementwise over the batch (dq final);
+//      bwd_precond_kernel: one CTA per (sequence, head) runs the phase-1 adjoint recurrence in
+//      reverse (one warp; 32-token chunks double-buffered in shared memory by asynchronous copies);
 //   4. bwd_sum_kernel: deta, summed over (sequence, head) in a fixed order.
 #pragma once
 
@@ -35,25 +42,36 @@
 namespace osdn {
 
 constexpr int BWD_BV = 64;      // value rows per bwd_delta_kernel CTA
-constexpr int BWD_C = 32;       // tokens per chunk (state checkpoints, staging)
+constexpr int BWD_C = 32;       // tokens per chunk (state checkpoints, chunk algebra)
 constexpr int BWD_THREADS = 256;
 
 template <int DK>
 struct BwdSmem {
-    static constexpr int KS = DK + 4;  // row stride (floats): conflict-free row and column walks
-    static constexpr int S = 0;                              // [BV][KS] state rows (S_c)
-    static constexpr int DS = S + BWD_BV * KS;               // [BV][KS] adjoint rows
-    static constexpr int K = DS + BWD_BV * KS;               // [C][KS] keys of the chunk
-    static constexpr int KT = K + BWD_C * KS;                // [C][KS] k~ = d (.) k
-    static constexpr int Q = KT + BWD_C * KS;                // [C][KS] queries
-    static constexpr int U = Q + BWD_C * KS;                 // [C][BV] u_t (this CTA's rows)
-    static constexpr int V = U + BWD_C * BWD_BV;             // [C][BV] v_t, then v_t - S_c k_t
-    static constexpr int DO = V + BWD_C * BWD_BV;            // [C][BV] dL/do_t (rows)
-    static constexpr int A = DO + BWD_C * BWD_BV;            // [C][C + 1] k_s . k~_j
-    static constexpr int BETA = A + BWD_C * (BWD_C + 1);     // [C]
-    static constexpr int G = BETA + BWD_C;                   // [BV] g_t
-    static constexpr int SIG = G + BWD_BV;                   // [C] beta_s <u_s, g_t> (s < t)
-    static constexpr int floats = SIG + BWD_C + 4;
+    static constexpr int KS = DK + 4;          // row strides (floats), multiples of 4, = 4 mod 32
+    static constexpr int VS = BWD_BV + 4;
+    static constexpr int CS = BWD_C + 4;
+    static constexpr int S = 0;                                // [BV][KS] state rows S_c
+    static constexpr int DS = S + BWD_BV * KS;                 // [BV][KS] adjoint rows
+    static constexpr int K = DS + BWD_BV * KS;                 // [C][KS] keys of the chunk
+    static constexpr int KT = K + BWD_C * KS;                  // [C][KS] k~ = d (.) k
+    static constexpr int Q = KT + BWD_C * KS;                  // [C][KS] queries
+    static constexpr int O = Q + BWD_C * KS;                   // [C][KS] a gradient share, staged
+    static constexpr int V = O + BWD_C * KS;                   // [C][VS] v, then E = v - S_c k
+    static constexpr int G = V + BWD_C * VS;                   // [C][VS] dL/do
+    static constexpr int R = G + BWD_C * VS;                   // [C][VS] R = beta E
+    static constexpr int W = R + BWD_C * VS;                   // [C][VS] W = T R
+    static constexpr int DW = W + BWD_C * VS;                  // [C][VS] dW
+    static constexpr int DR = DW + BWD_C * VS;                 // [C][VS] dR = T^T dW
+    static constexpr int DRB = DR + BWD_C * VS;                // [C][VS] beta dR (= dv)
+    static constexpr int A = DRB + BWD_C * VS;                 // [C][CS] K K~^T
+    static constexpr int P = A + BWD_C * CS;           // [C][CS] tril(Q K~^T)
+    static constexpr int TT = P + BWD_C * CS;          // [C][CS] T = (I + L)^-1
+    static constexpr int DP = TT + BWD_C * CS;         // [C][CS] dP
+    static constexpr int M = DP + BWD_C * CS;          // [C][CS] dW R^T, then dL
+    static constexpr int X = M + BWD_C * CS;           // [C][CS] T^T M
+    static constexpr int DLB = X + BWD_C * CS;         // [C][CS] beta dL
+    static constexpr int BETA = DLB + BWD_C * CS;      // [C]
+    static constexpr int floats = BETA + BWD_C;
     static constexpr size_t bytes = sizeof(float) * floats;
 };
 
@@ -64,12 +82,87 @@ __device__ __forceinline__ int64_t bwd_slot(int64_t first, int ch, int n) {
     return first / BWD_C + ch + n;
 }
 
-// Row `it` (0 .. BV/NP - 1) of the column-walk part `hp` (0 .. NP - 1): 8-row blocks split into
-// NP runs of 8 / NP rows, so the lanes of a warp read distinct banks.
-template <int NP>
-__device__ __forceinline__ int bwd_row(int it, int hp) {
-    constexpr int SPAN = 8 / NP;
-    return 8 * (it / SPAN) + SPAN * hp + (it % SPAN);
+// Shared-memory matrix products of the chunk algebra, all 256 threads:
+//   C[m][n] (= or +=) alpha * rs[m] * sum_k A(m, k) B(k, n)   (rs optional; tri 1 keeps n <= m,
+//   tri 2 keeps n < m), with A(m, k) = A[m lda + k] (NN, NT) or A[k lda + m] (TN) and
+//   B(k, n) = B[k ldb + n] (NN, TN) or B[n ldb + k] (NT).  A thread owns TM rows x TN columns of C;
+//   NT walks k four at a time with 16-byte loads of both operands.  The columns of a thread are
+//   spread over the row (NT: n = tn + j N / TN; NN, TN: groups of four at 4 tn + j N / TN) so the
+//   lanes of a warp read consecutive 16-byte pieces.
+enum { GEMM_NN = 0, GEMM_TN = 1, GEMM_NT = 2 };
+
+template <int MODE, int TM, int TN>
+__device__ __forceinline__ void bwd_gemm(int Mr, int Nc, int Kd, const float* __restrict__ A, int lda,
+                                         const float* __restrict__ B, int ldb, float* Cm, int ldc,
+                                         float alpha, bool accum, int tri = 0,
+                                         const float* __restrict__ rs = nullptr) {
+    const int ntn = Nc / TN, ntm = Mr / TM;
+    for (int tile = threadIdx.x; tile < ntn * ntm; tile += BWD_THREADS) {
+        const int tn = tile % ntn, tm = tile / ntn;
+        float acc[TM][TN];
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+        if constexpr (MODE == GEMM_NT) {
+#pragma unroll 2
+            for (int k = 0; k < Kd; k += 4) {
+                float4 a[TM], b[TN];
+#pragma unroll
+                for (int i = 0; i < TM; ++i) a[i] = *reinterpret_cast<const float4*>(A + (tm * TM + i) * lda + k);
+#pragma unroll
+                for (int j = 0; j < TN; ++j) b[j] = *reinterpret_cast<const float4*>(B + (tn + ntn * j) * ldb + k);
+#pragma unroll
+                for (int i = 0; i < TM; ++i)
+#pragma unroll
+                    for (int j = 0; j < TN; ++j) {
+                        acc[i][j] = fmaf(a[i].x, b[j].x, acc[i][j]);
+                        acc[i][j] = fmaf(a[i].y, b[j].y, acc[i][j]);
+                        acc[i][j] = fmaf(a[i].z, b[j].z, acc[i][j]);
+                        acc[i][j] = fmaf(a[i].w, b[j].w, acc[i][j]);
+                    }
+            }
+        } else {
+#pragma unroll 4
+            for (int k = 0; k < Kd; ++k) {
+                float a[TM], b[TN];
+#pragma unroll
+                for (int i = 0; i < TM; ++i)
+                    a[i] = MODE == GEMM_NN ? A[(tm * TM + i) * lda + k] : A[k * lda + tm * TM + i];
+                if constexpr (TN % 4 == 0) {
+#pragma unroll
+                    for (int j = 0; j < TN; j += 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(B + k * ldb + 4 * tn + ntn * j);
+                        b[j] = v.x;
+                        b[j + 1] = v.y;
+                        b[j + 2] = v.z;
+                        b[j + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < TN; ++j) b[j] = B[k * ldb + tn * TN + j];
+                }
+#pragma unroll
+                for (int i = 0; i < TM; ++i)
+#pragma unroll
+                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < TM; ++i) {
+            const int m = tm * TM + i;
+            const float sc = alpha * (rs ? rs[m] : 1.f);
+#pragma unroll
+            for (int j = 0; j < TN; ++j) {
+                const int n = MODE == GEMM_NT ? tn + ntn * j
+                            : (TN % 4 == 0 ? 4 * tn + ntn * (j & ~3) + (j & 3) : tn * TN + j);
+                float v = sc * acc[i][j];
+                if ((tri == 1 && n > m) || (tri == 2 && n >= m)) v = 0.f;
+                float* c = Cm + m * ldc + n;
+                *c = accum ? *c + v : v;
+            }
+        }
+    }
 }
 
 template <int DK, typename IO>
@@ -84,10 +177,8 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
                  int H, int Dv, int64_t rows) {
     using L = BwdSmem<DK>;
     using tr = io_traits<IO>;
-    constexpr int BV = BWD_BV, C = BWD_C, NT = BWD_THREADS, KS = L::KS;
-    constexpr int NP = NT / DK;   // column walk: DK columns x NP row parts
-    constexpr int CP = DK / 4;    // row walk: BV rows x 4 column parts (columns 4 j + part)
-    static_assert(NT == 4 * BV && C * 8 == NT, "thread layouts");
+    constexpr int BV = BWD_BV, C = BWD_C, NT = BWD_THREADS, KS = L::KS, VS = L::VS, CS = L::CS;
+    constexpr int TNK = DK / 16;  // a thread's columns in the DK-wide products (16 x 16 tiles)
     extern __shared__ float4 bwd_smem4[];
     float* sm = reinterpret_cast<float*>(bwd_smem4);
     float* sS = sm + L::S;
@@ -95,13 +186,22 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
     float* sK = sm + L::K;
     float* sKt = sm + L::KT;
     float* sQ = sm + L::Q;
-    float* sU = sm + L::U;
+    float* sO = sm + L::O;
     float* sV = sm + L::V;
-    float* sDO = sm + L::DO;
-    float* sA = sm + L::A;
-    float* sB = sm + L::BETA;
     float* sG = sm + L::G;
-    float* sSig = sm + L::SIG;
+    float* sR = sm + L::R;
+    float* sW = sm + L::W;
+    float* sdW = sm + L::DW;
+    float* sdR = sm + L::DR;
+    float* sdRb = sm + L::DRB;
+    float* sA = sm + L::A;
+    float* sP = sm + L::P;
+    float* sT = sm + L::TT;
+    float* sdP = sm + L::DP;
+    float* sM = sm + L::M;
+    float* sX = sm + L::X;
+    float* sdLb = sm + L::DLB;
+    float* sB = sm + L::BETA;
 
     const int tid = threadIdx.x;
     const int ntile = Dv / BV, vt = blockIdx.x % ntile, nh = blockIdx.x / ntile;
@@ -111,298 +211,298 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
     if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the CTA
     const int c0 = vt * BV;
     const int nchunks = (int)((count + C - 1) / C);
-    const int r1 = tid >> 2, p1 = tid & 3;      // row walk
-    const int c2 = tid / NP, hp = tid % NP;     // column walk
     const int64_t sbase = (int64_t)nh * Dv * DK + (int64_t)c0 * DK;
 
-    auto load_chunk = [&](int ch) -> int {
+    // the chunk's tokens (rows past its end are zero, so they contribute nothing); loops unrolled
+    // and 4 elements wide so that a thread's loads are all in flight at once
+    auto load_chunk = [&](int ch, bool grads) -> int {
         const int64_t row0 = first + (int64_t)ch * C;
         const int Lc = count - (int64_t)ch * C < C ? (int)(count - (int64_t)ch * C) : C;
-        for (int idx = tid; idx < C * DK; idx += NT) {
-            const int t = idx / DK, c = idx - t * DK;
-            float kk = 0.f, dd = 0.f, qq = 0.f;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int it = 0; it < C * DK / 4 / NT; ++it) {
+            const int idx = tid + it * NT, t = idx / (DK / 4), c = 4 * (idx - t * (DK / 4));
+            float4 kk = z, dd = z, qq = z;
             if (t < Lc) {
                 const int64_t o = ((row0 + t) * H + h) * DK + c;
-                kk = tr::to_f32(k[o]);
-                dd = dall[o];
-                qq = tr::to_f32(q[o]);
+                kk = load4<IO>(k + o);
+                dd = __ldg(reinterpret_cast<const float4*>(dall + o));
+                if (grads) qq = load4<IO>(q + o);
             }
-            sK[t * KS + c] = kk;
-            sKt[t * KS + c] = dd * kk;
-            sQ[t * KS + c] = qq;
+            *reinterpret_cast<float4*>(sK + t * KS + c) = kk;
+            *reinterpret_cast<float4*>(sKt + t * KS + c) =
+                make_float4(dd.x * kk.x, dd.y * kk.y, dd.z * kk.z, dd.w * kk.w);
+            *reinterpret_cast<float4*>(sQ + t * KS + c) = qq;
         }
-        for (int idx = tid; idx < C * BV; idx += NT) {
-            const int t = idx / BV, r = idx - t * BV;
-            float vv = 0.f, gg = 0.f;
+#pragma unroll
+        for (int it = 0; it < C * BV / 4 / NT; ++it) {
+            const int idx = tid + it * NT, t = idx / (BV / 4), r = 4 * (idx - t * (BV / 4));
+            float4 vv = z, gg = z;
             if (t < Lc) {
                 const int64_t o = ((row0 + t) * H + h) * Dv + c0 + r;
-                vv = tr::to_f32(v[o]);
-                gg = tr::to_f32(dO[o]);
+                vv = load4<IO>(v + o);
+                if (grads) gg = load4<IO>(dO + o);
             }
-            sV[t * BV + r] = vv;
-            sDO[t * BV + r] = gg;
+            *reinterpret_cast<float4*>(sV + t * VS + r) = vv;
+            *reinterpret_cast<float4*>(sG + t * VS + r) = gg;
         }
         if (tid < C) sB[tid] = tid < Lc ? __ldg(beta + (row0 + tid) * H + h) : 0.f;
         return Lc;
     };
-
-    // =========================================================== forward sweep
-    for (int idx = tid; idx < BV * DK; idx += NT) {
-        const int r = idx / DK, c = idx - r * DK;
-        sS[r * KS + c] = S0 ? __ldg(S0 + sbase + idx) : 0.f;
-    }
-    for (int ch = 0; ch < nchunks; ++ch) {
-        __syncthreads();  // the state rows are settled; the chunk buffers are free
-        {
-            float* dst = ws_state + (bwd_slot(first, ch, n) * H + h) * (int64_t)Dv * DK +
-                         (int64_t)c0 * DK;
-            for (int idx = tid; idx < BV * DK; idx += NT) {
-                const int r = idx / DK, c = idx - r * DK;
-                dst[idx] = sS[r * KS + c];
-            }
-        }
-        const int Lc = load_chunk(ch);
-        __syncthreads();
-        for (int t = 0; t < Lc; ++t) {
-            {  // u_t = v_t - S_{t-1} k_t on row r1, then S += beta_t u_t k~_t^T (own columns)
-                float acc = 0.f;
-#pragma unroll 8
-                for (int j = 0; j < CP; ++j) acc = fmaf(sS[r1 * KS + 4 * j + p1], sK[t * KS + 4 * j + p1], acc);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                const float bu = sB[t] * (sV[t * BV + r1] - acc);
-#pragma unroll 8
-                for (int j = 0; j < CP; ++j)
-                    sS[r1 * KS + 4 * j + p1] = fmaf(bu, sKt[t * KS + 4 * j + p1], sS[r1 * KS + 4 * j + p1]);
-            }
-            __syncthreads();
-            {  // this CTA's share of dq_t = scale S_t^T do_t
-                float acc = 0.f;
-#pragma unroll 8
-                for (int it = 0; it < BV / NP; ++it) {
-                    const int r = bwd_row<NP>(it, hp);
-                    acc = fmaf(sS[r * KS + c2], sDO[t * BV + r], acc);
-                }
+    // a BV x DK state tile between global memory (row stride DK) and shared memory (row stride KS)
+    auto tile_in = [&](float* dst, const float* src) {
 #pragma unroll
-                for (int off = 1; off < NP; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (hp == 0)
-                    dq_part[(((int64_t)vt * rows + first + (int64_t)ch * C + t) * H + h) * DK + c2] =
-                        scale * acc;
-            }
-            __syncthreads();
+        for (int it = 0; it < BV * DK / 4 / NT; ++it) {
+            const int idx = tid + it * NT, rr = idx / (DK / 4), c = 4 * (idx - rr * (DK / 4));
+            *reinterpret_cast<float4*>(dst + rr * KS + c) =
+                src ? __ldg(reinterpret_cast<const float4*>(src + rr * DK + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-    }
-
-    // =========================================================== reverse sweep
-    for (int idx = tid; idx < BV * DK; idx += NT) {
-        const int r = idx / DK, c = idx - r * DK;
-        sdS[r * KS + c] = dST ? __ldg(dST + sbase + idx) : 0.f;
-    }
-    for (int ch = nchunks - 1; ch >= 0; --ch) {
-        __syncthreads();
-        {
-            const float* src = ws_state + (bwd_slot(first, ch, n) * H + h) * (int64_t)Dv * DK +
-                               (int64_t)c0 * DK;
-            for (int idx = tid; idx < BV * DK; idx += NT) {
-                const int r = idx / DK, c = idx - r * DK;
-                sS[r * KS + c] = src[idx];
-            }
+    };
+    auto tile_out = [&](float* dst, const float* src) {
+#pragma unroll
+        for (int it = 0; it < BV * DK / 4 / NT; ++it) {
+            const int idx = tid + it * NT, rr = idx / (DK / 4), c = 4 * (idx - rr * (DK / 4));
+            *reinterpret_cast<float4*>(dst + rr * DK + c) = *reinterpret_cast<const float4*>(src + rr * KS + c);
         }
-        const int Lc = load_chunk(ch);
-        __syncthreads();
-        // chunk Gram A[s][j] = k_s . k~_j (j < s) and V' = V - S_c K^T
-        for (int idx = tid; idx < C * C; idx += NT) {
-            const int s = idx / C, j = idx - s * C;
-            float a = 0.f;
-            if (j < s && s < Lc) {
-#pragma unroll 8
-                for (int c = 0; c < DK; ++c) a = fmaf(sK[s * KS + c], sKt[j * KS + c], a);
+    };
+    // T = (I + strict_tril(diag(beta) A))^-1 by columns (thread j < C), then R = beta E, W = T R
+    auto wy = [&]() {
+        if (tid < C) {
+            const int j = tid;
+            float x[C];
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] = 0.f;
+#pragma unroll
+            for (int i = 0; i < C; ++i) {
+                if (i < j) continue;
+                float acc = i == j ? 1.f : 0.f;
+                const float bi = sB[i];
+#pragma unroll
+                for (int s2 = 0; s2 < i; ++s2) acc = fmaf(-bi * sA[i * CS + s2], x[s2], acc);
+                x[i] = acc;
             }
-            sA[s * (C + 1) + j] = a;
+#pragma unroll
+            for (int i = 0; i < C; ++i) sT[i * CS + j] = x[i];
         }
         for (int idx = tid; idx < C * BV; idx += NT) {
-            const int s = idx / BV, r = idx - s * BV;
-            if (s < Lc) {
-                float a = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < DK; ++c) a = fmaf(sS[r * KS + c], sK[s * KS + c], a);
-                sV[s * BV + r] -= a;
-            }
+            const int t = idx / BV, r = idx - t * BV;
+            sR[t * VS + r] = sB[t] * sV[t * VS + r];
         }
         __syncthreads();
-        // u_s = V'[s] - sum_{j<s} beta_j u_j A[s][j], row by row (the row's 4 lanes share a warp)
-        for (int s = 0; s < Lc; ++s) {
+        bwd_gemm<GEMM_NN, 2, 4>(C, BV, C, sT, CS, sR, VS, sW, VS, 1.f, false);
+    };
+    auto store_share = [&](float* dst, int ch, int Lc) {  // sO rows t < Lc -> a [rows, H, DK] share
+        const int64_t row0 = first + (int64_t)ch * C;
+#pragma unroll
+        for (int it = 0; it < C * DK / 4 / NT; ++it) {
+            const int idx = tid + it * NT, t = idx / (DK / 4), c = 4 * (idx - t * (DK / 4));
+            if (t < Lc)
+                *reinterpret_cast<float4*>(dst + (((int64_t)vt * rows + row0 + t) * H + h) * DK + c) =
+                    *reinterpret_cast<const float4*>(sO + t * KS + c);
+        }
+    };
+
+    // =========================================================== forward: state at chunk starts
+    tile_in(sS, S0 ? S0 + sbase : nullptr);
+    for (int ch = 0; ch < nchunks; ++ch) {
+        __syncthreads();  // the state rows are settled; the chunk buffers are free
+        tile_out(ws_state + (bwd_slot(first, ch, n) * H + h) * (int64_t)Dv * DK + (int64_t)c0 * DK, sS);
+        load_chunk(ch, false);
+        __syncthreads();
+        bwd_gemm<GEMM_NT, 2, 2>(C, C, DK, sK, KS, sKt, KS, sA, CS, 1.f, false);       // A = K K~^T
+        bwd_gemm<GEMM_NT, 2, 4>(C, BV, DK, sK, KS, sS, KS, sV, VS, -1.f, true);       // E = V - K S^T
+        __syncthreads();
+        wy();
+        __syncthreads();
+        bwd_gemm<GEMM_TN, 4, TNK>(BV, DK, C, sW, VS, sKt, KS, sS, KS, 1.f, true);     // S += W^T K~
+    }
+
+    // =========================================================== reverse over chunks
+    tile_in(sdS, dST ? dST + sbase : nullptr);
+    for (int ch = nchunks - 1; ch >= 0; --ch) {
+        __syncthreads();
+        tile_in(sS, ws_state + (bwd_slot(first, ch, n) * H + h) * (int64_t)Dv * DK + (int64_t)c0 * DK);
+        const int Lc = load_chunk(ch, true);
+        const int64_t row0 = first + (int64_t)ch * C;
+        __syncthreads();
+        bwd_gemm<GEMM_NT, 2, 2>(C, C, DK, sK, KS, sKt, KS, sA, CS, 1.f, false);       // A = K K~^T
+        bwd_gemm<GEMM_NT, 2, 2>(C, C, DK, sQ, KS, sKt, KS, sP, CS, 1.f, false, 1);    // P = tril(Q K~^T)
+        bwd_gemm<GEMM_NT, 2, 4>(C, BV, DK, sK, KS, sS, KS, sV, VS, -1.f, true);       // E = V - K S_c^T
+        bwd_gemm<GEMM_NT, 2, 4>(C, BV, DK, sKt, KS, sdS, KS, sdW, VS, 1.f, false);    // dW = K~ dS'^T
+        __syncthreads();
+        wy();                                                                         // T, R, W
+        __syncthreads();
+        bwd_gemm<GEMM_TN, 2, 4>(C, BV, C, sP, CS, sG, VS, sdW, VS, scale, true);      // dW += s P^T dO
+        bwd_gemm<GEMM_NT, 2, 2>(C, C, BV, sG, VS, sW, VS, sdP, CS, scale, false, 1);  // dP = tril(s dO W^T)
+        __syncthreads();
+        bwd_gemm<GEMM_TN, 2, 4>(C, BV, C, sT, CS, sdW, VS, sdR, VS, 1.f, false);      // dR = T^T dW
+        bwd_gemm<GEMM_NT, 2, 2>(C, C, BV, sdW, VS, sR, VS, sM, CS, 1.f, false);       // M = dW R^T
+        bwd_gemm<GEMM_NN, 2, TNK>(C, DK, BV, sG, VS, sS, KS, sO, KS, scale, false);   // dQ = s dO S_c
+        __syncthreads();
+        bwd_gemm<GEMM_NN, 2, TNK>(C, DK, C, sdP, CS, sKt, KS, sO, KS, 1.f, true);     //   + dP K~
+        bwd_gemm<GEMM_TN, 2, 2>(C, C, C, sT, CS, sM, CS, sX, CS, 1.f, false);         // X = T^T M
+        for (int idx = tid; idx < C * BV; idx += NT) {                                // beta dR = dv
+            const int t = idx / BV, r = idx - t * BV;
+            const float x = sB[t] * sdR[t * VS + r];
+            sdRb[t * VS + r] = x;
+            if (t < Lc) dv[((row0 + t) * H + h) * Dv + c0 + r] = x;
+        }
+        __syncthreads();
+        store_share(dq_part, ch, Lc);
+        bwd_gemm<GEMM_NT, 2, 2>(C, C, C, sX, CS, sT, CS, sM, CS, -1.f, false, 2);     // dL = -stril(X T^T)
+        __syncthreads();
+        if (tid < C) {  // this share of dbeta: rowsum(dL . A) + rowsum(dR . E)
+            const int t = tid;
             float acc = 0.f;
-            for (int j = p1; j < s; j += 4) acc = fmaf(sB[j] * sU[j * BV + r1], sA[s * (C + 1) + j], acc);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (p1 == 0) sU[s * BV + r1] = sV[s * BV + r1] - acc;
-            __syncwarp();
+            for (int j = 0; j < t; ++j) acc = fmaf(sM[t * CS + j], sA[t * CS + j], acc);
+            for (int r = 0; r < BV; ++r) acc = fmaf(sdR[t * VS + r], sV[t * VS + r], acc);
+            if (t < Lc) dbeta_part[((int64_t)vt * rows + row0 + t) * H + h] = acc;
         }
+        for (int idx = tid; idx < C * C; idx += NT) {                                 // beta dL
+            const int t = idx / C, j = idx - t * C;
+            sdLb[t * CS + j] = sB[t] * sM[t * CS + j];
+        }
+        bwd_gemm<GEMM_NN, 2, TNK>(C, DK, BV, sW, VS, sdS, KS, sO, KS, 1.f, false);    // dK~ = W dS'
         __syncthreads();
-        float g_prev = 0.f, b_prev = 0.f;  // token t+1's pending update dS -= beta g k^T (row r1)
-        for (int t = Lc - 1; t >= 0; --t) {
-            const int64_t row = first + (int64_t)ch * C + t;
-            {  // dS_t = dS_{t+1} - beta_{t+1} g_{t+1} k_{t+1}^T + scale do_t q_t^T;  g_t = dS_t k~_t
-                const float dor = scale * sDO[t * BV + r1];
-                const float bg = (t + 1 < Lc) ? b_prev * g_prev : 0.f;
-                const int tn = (t + 1 < Lc) ? t + 1 : t;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int j = 0; j < CP; ++j) {
-                    const int c = 4 * j + p1;
-                    float x = sdS[r1 * KS + c];
-                    x = fmaf(-bg, sK[tn * KS + c], x);
-                    x = fmaf(dor, sQ[t * KS + c], x);
-                    sdS[r1 * KS + c] = x;
-                    acc = fmaf(x, sKt[t * KS + c], acc);
-                }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                g_prev = acc;
-                b_prev = sB[t];
-                if (p1 == 0) {
-                    sG[r1] = acc;
-                    dv[(row * H + h) * Dv + c0 + r1] = b_prev * acc;
-                }
-            }
-            __syncthreads();
-            float a1 = 0.f, a2 = 0.f;  // column walk: sum_r dS[r][c] u_t[r], sum_r S_c[r][c] g[r]
-#pragma unroll 8
-            for (int it = 0; it < BV / NP; ++it) {
-                const int r = bwd_row<NP>(it, hp);
-                a1 = fmaf(sdS[r * KS + c2], sU[t * BV + r], a1);
-                a2 = fmaf(sS[r * KS + c2], sG[r], a2);
-            }
-#pragma unroll
-            for (int off = 1; off < NP; off <<= 1) {
-                a1 += __shfl_xor_sync(0xffffffffu, a1, off);
-                a2 += __shfl_xor_sync(0xffffffffu, a2, off);
-            }
-            {  // <u_s, g_t> over this CTA's rows for s <= t (thread: s = tid / 8, rows q8 + 8 i)
-                const int s = tid >> 3, q8 = tid & 7;
-                float x = 0.f;
-                if (s <= t) {
-#pragma unroll
-                    for (int i = 0; i < BV / 8; ++i) x = fmaf(sU[s * BV + q8 + 8 * i], sG[q8 + 8 * i], x);
-                }
-                x += __shfl_xor_sync(0xffffffffu, x, 1);
-                x += __shfl_xor_sync(0xffffffffu, x, 2);
-                x += __shfl_xor_sync(0xffffffffu, x, 4);
-                if (q8 == 0) sSig[s] = s < t ? sB[s] * x : (s == t ? x : 0.f);
-            }
-            __syncthreads();
-            if (hp == 0) {  // S_{t-1}^T g_t = S_c^T g_t + sum_{s<t} k~_s beta_s <u_s, g_t>
-                float sk = 0.f;
-                for (int s = 0; s < t; ++s) sk = fmaf(sKt[s * KS + c2], sSig[s], sk);
-                const int64_t o = (((int64_t)vt * rows + row) * H + h) * DK + c2;
-                dkt_part[o] = sB[t] * a1;
-                dk_part[o] = -sB[t] * (a2 + sk);
-            }
-            if (tid == 0) dbeta_part[((int64_t)vt * rows + row) * H + h] = sSig[t];
-        }
-        if (Lc > 0) {  // token 0's pending update
-#pragma unroll 8
-            for (int j = 0; j < CP; ++j) {
-                const int c = 4 * j + p1;
-                sdS[r1 * KS + c] = fmaf(-b_prev * g_prev, sK[c], sdS[r1 * KS + c]);
-            }
-        }
+        bwd_gemm<GEMM_TN, 2, TNK>(C, DK, C, sdP, CS, sQ, KS, sO, KS, 1.f, true);      //   + dP^T Q
+        __syncthreads();
+        bwd_gemm<GEMM_TN, 2, TNK>(C, DK, C, sdLb, CS, sK, KS, sO, KS, 1.f, true);     //   + (beta dL)^T K
+        __syncthreads();
+        store_share(dkt_part, ch, Lc);
+        __syncthreads();
+        bwd_gemm<GEMM_NN, 2, TNK>(C, DK, C, sdLb, CS, sKt, KS, sO, KS, 1.f, false);   // dK = beta dL K~
+        __syncthreads();
+        bwd_gemm<GEMM_NN, 2, TNK>(C, DK, BV, sdRb, VS, sS, KS, sO, KS, -1.f, true);   //   - beta dR S_c
+        __syncthreads();
+        store_share(dk_part, ch, Lc);
+        bwd_gemm<GEMM_TN, 4, TNK>(BV, DK, C, sG, VS, sQ, KS, sdS, KS, scale, true);   // dS += s dO^T Q
+        __syncthreads();
+        bwd_gemm<GEMM_TN, 4, TNK>(BV, DK, C, sdRb, VS, sK, KS, sdS, KS, -1.f, true);  //    - (beta dR)^T K
     }
     __syncthreads();
-    if (dS0) {
-        for (int idx = tid; idx < BV * DK; idx += NT) {
-            const int r = idx / DK, c = idx - r * DK;
-            dS0[sbase + idx] = sdS[r * KS + c];
+    if (dS0) tile_out(dS0 + sbase, sdS);
+}
+
+// The value-row shares of bwd_delta_kernel added up, elementwise over the whole batch: dq (the
+// final gradient), and dk~, dk's phase-2 term and dbeta's phase-2 term summed into share 0.
+__global__ void __launch_bounds__(256)
+bwd_reduce_kernel(const float4* __restrict__ dq_part, float4* __restrict__ dk_part,
+                  float4* __restrict__ dkt_part, float* __restrict__ dbeta_part, int ntile,
+                  int64_t n4, int64_t nb, float4* __restrict__ dq) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+        float4 a = dq_part[i], b = dk_part[i], c = dkt_part[i];
+        for (int p = 1; p < ntile; ++p) {
+            const float4 x = dq_part[p * n4 + i], y = dk_part[p * n4 + i], z = dkt_part[p * n4 + i];
+            a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+            b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+            c.x += z.x; c.y += z.y; c.z += z.z; c.w += z.w;
         }
+        dq[i] = a;
+        dk_part[i] = b;
+        dkt_part[i] = c;
+    }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += stride) {
+        float v = dbeta_part[i];
+        for (int p = 1; p < ntile; ++p) v += dbeta_part[p * nb + i];
+        dbeta_part[i] = v;
     }
 }
 
-// Phase 1 in reverse, with the shares of bwd_delta_kernel added up.  One CTA of 128 threads per
-// (sequence, head): all threads stage a chunk of BWD_C tokens (and write dq), warp 0 runs the
-// adjoint recurrence over it.
-template <int DK>
+// Phase 1 in reverse.  One CTA of 128 threads per (sequence, head): warp 0 runs the adjoint
+// recurrence over a 32-token chunk staged in shared memory while warps 1-3 fetch the next chunk
+// (in reverse order) into the other buffer with asynchronous copies.
+template <int DK, typename IO>
 struct BwdPrecondSmem {
-    static constexpr int DKT = 0;                    // [C][DK] dk~ (summed)
-    static constexpr int DK2 = DKT + BWD_C * DK;     // [C][DK] dk, phase-2 term (summed)
-    static constexpr int D = DK2 + BWD_C * DK;       // [C][DK] d_t
-    static constexpr int K = D + BWD_C * DK;         // [C][DK] k_t
-    static constexpr int VEC = K + BWD_C * DK;       // [C] beta, r, dbeta phase-2 term
-    static constexpr int floats = VEC + 3 * BWD_C;
+    static constexpr int KB = DK * (int)sizeof(IO) / 4;  // a token's key row, in 4-byte words
+    static constexpr int DKT = 0;                        // [C][DK] dk~
+    static constexpr int DK2 = DKT + BWD_C * DK;         // [C][DK] dk, phase-2 term
+    static constexpr int D = DK2 + BWD_C * DK;           // [C][DK] d_t
+    static constexpr int K = D + BWD_C * DK;             // [C][KB] k_t in the io dtype
+    static constexpr int VEC = K + BWD_C * KB;           // [C] beta, r, dbeta phase-2 term
+    static constexpr int BUF = VEC + 3 * BWD_C;          // one buffer
+    static constexpr int floats = 2 * BUF;
     static constexpr size_t bytes = sizeof(float) * floats;
 };
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(gsrc))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 
 template <int DK, typename IO>
 __global__ void __launch_bounds__(128)
 bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
                    const float* __restrict__ r, float eta, const float* __restrict__ dall,
-                   const float* __restrict__ ddT, const float* __restrict__ dq_part,
-                   const float* __restrict__ dk_part, const float* __restrict__ dkt_part,
-                   const float* __restrict__ dbeta_part, int ntile, float* __restrict__ dq,
+                   const float* __restrict__ ddT, const float* __restrict__ dk_sum,
+                   const float* __restrict__ dkt_sum, const float* __restrict__ dbeta_sum,
                    float* __restrict__ dk, float* __restrict__ dbeta, float* __restrict__ dr,
                    float* __restrict__ dd0, float* __restrict__ deta_part,
-                   const int32_t* __restrict__ cu, int N, int T, int H, int64_t rows) {
-    using L = BwdPrecondSmem<DK>;
+                   const int32_t* __restrict__ cu, int N, int T, int H) {
+    using L = BwdPrecondSmem<DK, IO>;
     using tr = io_traits<IO>;
     constexpr int C = BWD_C, E = DK / 32;
     extern __shared__ float4 bwdp_smem4[];
     float* sm = reinterpret_cast<float*>(bwdp_smem4);
-    float* sDkt = sm + L::DKT;
-    float* sDk2 = sm + L::DK2;
-    float* sD = sm + L::D;
-    float* sK = sm + L::K;
-    float* sBeta = sm + L::VEC;
-    float* sR = sBeta + C;
-    float* sDb = sR + C;
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nh = blockIdx.x, n = nh / H, h = nh - n * H;
     if (n >= N) return;
     int64_t first, count;
     if (!seq_range(cu, n, N, T, first, count)) return;
     const int nchunks = (int)((count + C - 1) / C);
-    const int64_t part_stride = rows * H * DK;
+    auto chunk_len = [&](int ch) -> int {
+        const int64_t rem = count - (int64_t)ch * C;
+        return rem < C ? (int)rem : C;
+    };
+    // warps 1-3: chunk ch into buffer b (tokens past the chunk's end are not read)
+    auto fetch = [&](int b, int ch) {
+        float* buf = sm + b * L::BUF;
+        const int64_t row0 = first + (int64_t)ch * C;
+        const int Lc = chunk_len(ch), i = tid - 32;
+        constexpr int P4 = DK / 4, PK = L::KB / 4;  // 16-byte pieces per token row
+        for (int idx = i; idx < Lc * (3 * P4 + PK); idx += 96) {
+            const int t = idx / (3 * P4 + PK), q = idx - t * (3 * P4 + PK);
+            const int64_t o = ((row0 + t) * H + h) * DK;
+            if (q < P4) cp_async16(buf + L::DKT + t * DK + 4 * q, dkt_sum + o + 4 * q);
+            else if (q < 2 * P4) cp_async16(buf + L::DK2 + t * DK + 4 * (q - P4), dk_sum + o + 4 * (q - P4));
+            else if (q < 3 * P4) cp_async16(buf + L::D + t * DK + 4 * (q - 2 * P4), dall + o + 4 * (q - 2 * P4));
+            else cp_async16(buf + L::K + t * L::KB + 4 * (q - 3 * P4),
+                            reinterpret_cast<const float*>(k + o) + 4 * (q - 3 * P4));
+        }
+        for (int t = i; t < Lc; t += 96) {
+            const int64_t th = (row0 + t) * H + h;
+            buf[L::VEC + t] = __ldg(beta + th);
+            buf[L::VEC + C + t] = r ? __ldg(r + th) : 1.f;
+            buf[L::VEC + 2 * C + t] = dbeta_sum[th];
+        }
+        cp_async_wait_all();
+    };
 
     float dd[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) dd[e] = ddT ? __ldg(ddT + (int64_t)nh * DK + lane * E + e) : 0.f;
     float deta = 0.f;
-
+    if (warp > 0 && nchunks > 0) fetch(0, nchunks - 1);
+    __syncthreads();
     for (int ch = nchunks - 1; ch >= 0; --ch) {
-        const int64_t row0 = first + (int64_t)ch * C;
-        const int Lc = count - (int64_t)ch * C < C ? (int)(count - (int64_t)ch * C) : C;
-        __syncthreads();  // warp 0 is done with the previous chunk's tiles
-        for (int idx = tid; idx < Lc * DK; idx += 128) {
-            const int t = idx / DK, c = idx - t * DK;
-            const int64_t o = ((row0 + t) * H + h) * DK + c;
-            float skt = 0.f, sk2 = 0.f, sq = 0.f;
-            for (int p = 0; p < ntile; ++p) {
-                skt += dkt_part[p * part_stride + o];
-                sk2 += dk_part[p * part_stride + o];
-                sq += dq_part[p * part_stride + o];
-            }
-            dq[o] = sq;
-            sDkt[idx] = skt;
-            sDk2[idx] = sk2;
-            sD[idx] = dall[o];
-            sK[idx] = tr::to_f32(k[o]);
-        }
-        for (int t = tid; t < Lc; t += 128) {
-            const int64_t th = (row0 + t) * H + h;
-            sBeta[t] = __ldg(beta + th);
-            sR[t] = r ? __ldg(r + th) : 1.f;
-            float sb = 0.f;
-            for (int p = 0; p < ntile; ++p) sb += dbeta_part[(int64_t)p * rows * H + th];
-            sDb[t] = sb;
-        }
-        __syncthreads();
-        if (tid < 32) {
-            for (int t = Lc - 1; t >= 0; --t) {
+        const int b = (nchunks - 1 - ch) & 1;
+        if (warp > 0) {
+            if (ch > 0) fetch(b ^ 1, ch - 1);
+        } else {
+            const float* buf = sm + b * L::BUF;
+            const int64_t row0 = first + (int64_t)ch * C;
+            for (int t = chunk_len(ch) - 1; t >= 0; --t) {
                 float kk[E], dv_[E], a[E];
                 float nk = 0.f, s = 0.f, y = 0.f, rd = 0.f;
+                const IO* krow = reinterpret_cast<const IO*>(buf + L::K + t * L::KB);
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
-                    kk[e] = sK[t * DK + lane * E + e];
-                    dv_[e] = sD[t * DK + lane * E + e];
+                    kk[e] = tr::to_f32(krow[lane * E + e]);
+                    dv_[e] = buf[L::D + t * DK + lane * E + e];
                     a[e] = kk[e] * kk[e];
                     nk += a[e];
                     s = fmaf(dv_[e], a[e], s);
@@ -416,28 +516,29 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
                     y += __shfl_xor_sync(0xffffffffu, y, off);
                     rd += __shfl_xor_sync(0xffffffffu, rd, off);
                 }
-                const float bt = sBeta[t], rt = sR[t];
+                const float bt = buf[L::VEC + t], rt = buf[L::VEC + C + t];
                 const bool ok = nk > 0.f;
                 const float inv = ok ? 1.f / nk : 0.f;
                 const float xt = ok ? bt * (1.f - bt * s) * inv : 0.f;
                 const int64_t th = (row0 + t) * H + h;
                 if (lane == 0) {
-                    dbeta[th] = sDb[t] + (ok ? eta * y * (1.f - 2.f * bt * s) * inv : 0.f);
+                    dbeta[th] = buf[L::VEC + 2 * C + t] + (ok ? eta * y * (1.f - 2.f * bt * s) * inv : 0.f);
                     if (dr) dr[th] = rd;
                 }
                 deta = fmaf(xt, y, deta);
                 const float cy = ok ? eta * bt * bt * inv * y : 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
-                    const float dkt = sDkt[t * DK + lane * E + e];
+                    const float dkt = buf[L::DKT + t * DK + lane * E + e];
                     const float da = ok ? eta * xt * dd[e] - eta * y * (bt * bt * dv_[e] + xt) * inv : 0.f;
-                    dk[th * DK + lane * E + e] = sDk2[t * DK + lane * E + e] + dkt * dv_[e] + 2.f * kk[e] * da;
+                    dk[th * DK + lane * E + e] = buf[L::DK2 + t * DK + lane * E + e] + dkt * dv_[e] + 2.f * kk[e] * da;
                     dd[e] = fmaf(rt, dd[e], fmaf(-cy, a[e], dkt * kk[e]));
                 }
             }
         }
+        __syncthreads();  // chunk ch is consumed and chunk ch - 1 has landed
     }
-    if (tid < 32) {
+    if (warp == 0) {
         if (dd0) {
 #pragma unroll
             for (int e = 0; e < E; ++e) dd0[(int64_t)nh * DK + lane * E + e] = dd[e];

@@ -673,12 +673,24 @@ osdn_status_t launch_bwd_kernels(const void* q, const void* k, const void* v, co
         const osdn_status_t st = launch_status();
         if (st != OSDN_OK) return st;
     }
+    if (rows > 0) {
+        const int64_t n4 = rows * d.H * DK / 4, nb = rows * d.H;
+        int64_t grid = (n4 + 255) / 256;
+        const int64_t cap = 8LL * sm_count();
+        grid = grid < cap ? grid : cap;
+        bwd_reduce_kernel<<<dim3((unsigned)grid), dim3(256), 0, stream>>>(
+            reinterpret_cast<const float4*>(dq_part), reinterpret_cast<float4*>(dk_part),
+            reinterpret_cast<float4*>(dkt_part), db_part, ntile, n4, nb,
+            reinterpret_cast<float4*>(dq));
+        const osdn_status_t st = launch_status();
+        if (st != OSDN_OK) return st;
+    }
     {
         auto kern = bwd_precond_kernel<DK, IO>;
-        if (!set_smem(kern, BwdPrecondSmem<DK>::bytes)) return OSDN_ERR_CUDA;
-        kern<<<dim3((unsigned)units), dim3(128), BwdPrecondSmem<DK>::bytes, stream>>>(
-            static_cast<const IO*>(k), beta, r, eta, dall, ddT, dq_part, dk_part, dkt_part, db_part,
-            ntile, dq, dk, dbeta, dr, dd0, deta_part, cu, d.N, d.T, d.H, rows);
+        if (!set_smem(kern, BwdPrecondSmem<DK, IO>::bytes)) return OSDN_ERR_CUDA;
+        kern<<<dim3((unsigned)units), dim3(128), BwdPrecondSmem<DK, IO>::bytes, stream>>>(
+            static_cast<const IO*>(k), beta, r, eta, dall, ddT, dk_part, dkt_part, db_part, dk, dbeta,
+            dr, dd0, deta_part, cu, d.N, d.T, d.H);
         const osdn_status_t st = launch_status();
         if (st != OSDN_OK) return st;
     }
