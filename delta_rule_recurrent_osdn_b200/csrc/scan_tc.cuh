@@ -333,10 +333,12 @@ struct ScanChainSmem {
     static constexpr uint32_t TOTAL = BAR + 21 * 8;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
-constexpr int SCAN_CHAIN_THREADS = 288;  // warps 0-3 products, 4-7 k~ output (two groups), 8 loads and gates
+// rank 0: warps 0-7 the chain's products, 8 loads and gates, 9 the forwarder; rank 1: warps 4-7
+// the k~ output (two groups), 8 loads
+constexpr int SCAN_CHAIN_THREADS = 320;
 
-// One 2-CTA cluster per (sequence, head).  Rank 0 runs the chain (warps 0-3), its loads (warp 8:
-// k and T_d tiles, gate vectors) and a forwarder (warp 4); rank 1 runs the k~ token pass (warps
+// One 2-CTA cluster per (sequence, head).  Rank 0 runs the chain (warps 0-7), its loads (warp 8:
+// k and T_d tiles, gate vectors) and a forwarder (warp 9); rank 1 runs the k~ token pass (warps
 // 4-7) and its own loads (warp 8: k tiles, r).  The token pass gets an SM of its own.  The chain
 // only arrives on local barriers; the forwarder copies x and the chunk-start d of each chunk into
 // rank 1's shared memory and arrives on rank 1's barrier (release / acquire at cluster scope), so
@@ -372,11 +374,11 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* full = bars;         // [3] TMA: k tile (+ T_d tile on rank 0)
     uint64_t* vready = bars + 3;   // [3] gate vectors (32 arrivals)
-    uint64_t* kempty = bars + 6;   // [3] slot released: rank 0 by the chain (128), rank 1 by the
+    uint64_t* kempty = bars + 6;   // [3] slot released: rank 0 by the chain (256), rank 1 by the
                                    //     chunk's writer group (64)
     uint64_t* xready = bars + 9;   // [3] rank 1: x and d of a chunk, from rank 0's forwarder (32)
     uint64_t* outdone = bars + 12; // [3] rank 0: rank 1's writer group has copied x / d (64)
-    uint64_t* fwdin = bars + 15;   // [3] rank 0: x and d of a chunk in local memory (128, chain)
+    uint64_t* fwdin = bars + 15;   // [3] rank 0: x and d of a chunk in local memory (256, chain)
     uint64_t* fwdout = bars + 18;  // [3] rank 0: the forwarder has sent them (32)
     float* sD = reinterpret_cast<float*>(smem + L::D);
     float* sX = reinterpret_cast<float*>(smem + L::X);
@@ -392,10 +394,10 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         for (int s = 0; s < 3; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&vready[s], 32);
-            mbar_init(&kempty[s], rank == 0 ? 128 : 64);
+            mbar_init(&kempty[s], rank == 0 ? 256 : 64);
             mbar_init(&xready[s], 32);
             mbar_init(&outdone[s], 64);
-            mbar_init(&fwdin[s], 128);
+            mbar_init(&fwdin[s], 256);
             mbar_init(&fwdout[s], 32);
         }
         tc::fence_mbar_init();
@@ -493,11 +495,11 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
                 mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
         }
-    } else if (warp < 4 && rank == 0) {
+    } else if (warp < 8 && rank == 0) {
         // =============================================== p = A d, x = T_d b, next d
         const int u = tid;
-        const int t = 16 * warp + (lane & 15), half = lane >> 4;  // step 1/2 roles
-        const int cp = u >> 1, par = u & 1;  // step 3 role: channel pair, token half
+        const int t = 8 * warp + (lane & 7), qd = lane >> 3;  // step 1/2 roles: token, channel quarter
+        const int cp = u >> 2, par = u & 3;  // step 3 role: channel pair, token quarter
         const int cblk = cp >> 5, cj = (cp & 31) >> 2, cpe = 2 * (cp & 3);
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
@@ -507,7 +509,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                        mbar_wait_bounded(&vready[s], ph, limit_ns);
             if (got && c >= 2)  // the forwarder has sent the x / d buffers this chunk overwrites
                 got = mbar_wait_bounded(&fwdout[(c - 2) % 3], (uint32_t)((c - 2) / 3) & 1u, limit_ns);
-            if (group_any(1, 128, !got)) {
+            if (group_any(1, 256, !got)) {
                 ok = false;
                 break;
             }
@@ -521,11 +523,12 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             {
                 float2 p2 = make_float2(0.f, 0.f), nk2 = make_float2(0.f, 0.f);  // channel pairs
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(kt + half * 8192u + tc::sw128_off(t, j));
+                for (int j = 0; j < 4; ++j) {  // channels 32 qd + 8 j .. + 7
+                    const int ch16 = 4 * (qd & 1) + j;
+                    const uint4 raw = *reinterpret_cast<const uint4*>(kt + (qd >> 1) * 8192u + tc::sw128_off(t, ch16));
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                    const float4 da = *reinterpret_cast<const float4*>(d + 64 * half + 8 * j);
-                    const float4 db = *reinterpret_cast<const float4*>(d + 64 * half + 8 * j + 4);
+                    const float4 da = *reinterpret_cast<const float4*>(d + 32 * qd + 8 * j);
+                    const float4 db = *reinterpret_cast<const float4*>(d + 32 * qd + 8 * j + 4);
                     const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w),
                                           make_float2(db.x, db.y), make_float2(db.z, db.w)};
 #pragma unroll
@@ -537,22 +540,24 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     }
                 }
                 float p = p2.x + p2.y, nk = nk2.x + nk2.y;
+                p += __shfl_xor_sync(0xffffffffu, p, 8);
+                nk += __shfl_xor_sync(0xffffffffu, nk, 8);
                 p += __shfl_xor_sync(0xffffffffu, p, 16);
                 nk += __shfl_xor_sync(0xffffffffu, nk, 16);
-                if (half == 0) {
+                if (qd == 0) {
                     const float bt = vv[192 + t];
                     e_t = (t < Lc && nk > 0.f) ? eta * bt / nk : 0.f;
                     sB[t] = e_t * (1.f - bt * vv[t] * p);
                     bRp = bt * vv[t] * p;
                 }
             }
-            group_bar(1, 128);
+            group_bar(1, 256);
             // ---- step 2: x_t = sum_{j <= t} T_d[t][j] b_j
             {
                 float acc = 0.f;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int g = 8 * half + q;
+                for (int q = 0; q < 4; ++q) {
+                    const int g = 4 * qd + q;
                     const float4 tv = tsw_ld4(td, t, g);
                     const float4 bv = *reinterpret_cast<const float4*>(sB + 4 * g);
                     const int j = 4 * g;
@@ -561,8 +566,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     acc = fmaf(j + 2 <= t ? tv.z : 0.f, bv.z, acc);
                     acc = fmaf(j + 3 <= t ? tv.w : 0.f, bv.w, acc);
                 }
+                acc += __shfl_xor_sync(0xffffffffu, acc, 8);
                 acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-                if (half == 0) {
+                if (qd == 0) {
                     const float x = t < Lc ? acc : 0.f;
                     sX[(c % 3) * 64 + t] = x;
                     sGX[t] = vv[64 + t] * x;
@@ -574,16 +580,16 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     }
                 }
             }
-            group_bar(1, 128);
+            group_bar(1, 256);
             // ---- step 3: d_C[i] = R_C d[i] + sum_j g_j x_j a_j[i]; thread: channels 2cp, 2cp + 1
-            //      over the tokens with bit 2 clear (par 0) or set (par 1) -- rows whose swizzle
-            //      phases differ, so the lane pair reads disjoint banks -- summed by a shuffle
+            //      over the tokens j = 8 m + 2 par + {0, 1} -- the four parts read rows of distinct
+            //      swizzle phases, so the lanes read disjoint banks -- summed by shuffles
             {
                 float2 acc = make_float2(0.f, 0.f);  // the two channels of the pair
                 const uint8_t* col = kt + cblk * 8192u + cpe * 2;
 #pragma unroll 8
-                for (int jj = 0; jj < C / 2; ++jj) {
-                    const int j = (jj & 3) + ((jj >> 2) << 3) + 4 * par;
+                for (int jj = 0; jj < C / 4; ++jj) {
+                    const int j = 8 * (jj >> 1) + 2 * par + (jj & 1);
                     const uint32_t w = *reinterpret_cast<const uint32_t*>(col + tc::sw128_off(j, cj));
                     const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
                     const float gx = sGX[j];
@@ -592,6 +598,8 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 float acc0 = acc.x, acc1 = acc.y;
                 acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
                 acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
                 if (par == 0) {
                     const float rc = vv[256];
                     const float2 dv = *reinterpret_cast<const float2*>(d + 2 * cp);
@@ -601,10 +609,10 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             }
             mbar_arrive(&fwdin[c % 3]);  // x_c and d_c are in sX, sD: the forwarder sends them
             mbar_arrive(&kempty[s]);     // the chain's last use of the slot
-            group_bar(1, 128);
+            group_bar(1, 256);
         }
-        if (ok && dT) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
-    } else if (warp == 4 && rank == 0) {
+        if (ok && dT && u < DK) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
+    } else if (warp == 9 && rank == 0) {
         // =============================================== forwarder: x_c, d_c to rank 1
         // Chunk c's x and chunk-start d go into slot c % 3 of rank 1's buffers once rank 1's
         // writer of chunk c - 3 has copied that slot out; the slot's local copies may then be
