@@ -187,8 +187,10 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     if (nh == 0) return OSDN_OK;
     if (nh > 0x7fffffff) return OSDN_ERR_UNSUPPORTED;
     const int64_t rows = d.rows();  // > 0: token-free calls take the warp scan
-    CUtensorMap mk, mtd;
-    if (!make_tile_map(&mk, k, 128, d.H, rows) || !make_td_map(&mtd, k_tilde, d.H, rows))
+    CUtensorMap mk, mtd, mkto, mktlo;
+    if (!make_tile_map(&mk, k, 128, d.H, rows) || !make_td_map(&mtd, k_tilde, d.H, rows) ||
+        !make_tile_map(&mkto, k_tilde, 128, d.H, rows) ||
+        !make_tile_map(&mktlo, kt_lo ? kt_lo : k_tilde, 128, d.H, rows))
         return OSDN_ERR_CUDA;
     // persistent prep grid over (64-row window, head) items
     const int64_t items = ((rows + 63) / 64) * d.H;
@@ -218,7 +220,7 @@ osdn_status_t launch_scan_tc(const void* k, const float* beta, const float* r, f
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, chain, mk, mtd, beta, r, eta, d0,
+    if (cudaLaunchKernelEx(&cfg, chain, mk, mtd, mkto, mktlo, beta, r, eta, d0,
                            static_cast<__nv_bfloat16*>(k_tilde), static_cast<__nv_bfloat16*>(kt_lo),
                            d_all, dT, rho, cu, d.N, d.T, d.H, (long long)kWaitLimitNs) != cudaSuccess)
         return OSDN_ERR_CUDA;

@@ -78,8 +78,8 @@ struct ScanPrepSmem {
     static constexpr uint32_t A = 16384;          // bf16 [a_hi; a_lo] per K-block, 2 x 16 KB
     static constexpr uint32_t SL = A;             // fp32 L_d, then T_d (tsw), over A after the Gram
     static constexpr uint32_t ST = A + 16384;     // fp32 scratch (tsw), over A
-    static constexpr uint32_t VEC = A + 32768;    // c, lr, lr1, sg, sg1, R, Rinv (7 x 64) + flag
-    static constexpr uint32_t BAR = VEC + 7 * 256 + 16;
+    static constexpr uint32_t VEC = A + 32768;    // c, lr, lr1, sg, sg1, R, Rinv, e (8 x 64) + flag
+    static constexpr uint32_t BAR = VEC + 8 * 256 + 16;
     static constexpr uint32_t TMEM_SLOT = BAR + 16;
     static constexpr uint32_t TOTAL = TMEM_SLOT + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
@@ -115,7 +115,8 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
     float* vsg1 = vc + 256;
     float* vR = vc + 320;     // sg e^lr
     float* vRi = vc + 384;    // sg1 e^-lr1
-    int* vsafe = reinterpret_cast<int*>(vc + 448);
+    float* ve = vc + 448;     // e = eta beta / ||k||^2 (0 for a zero key or past the end)
+    int* vsafe = reinterpret_cast<int*>(vc + 512);
 
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, 128);
@@ -186,6 +187,7 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
                 const float bt = valid ? __ldg(beta + (row0 + t) * H + h) : 0.f;
                 const float e = nk > 0.f ? eta * bt / nk : 0.f;
                 vc[t] = e * bt;
+                ve[t] = e;
             }
         }
         if (warp == 3) {  // prefix of log|r| over the chunk
@@ -295,6 +297,10 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
         }
         __syncthreads();
         tril_inverse_64_g128(sL, tid, 1);  // T_d over L_d
+        // e_t rides in the tile's upper-right block (rows 0-1, columns 32-63), which holds only
+        // scratch of the inverse: the chain kernel reads it there instead of recomputing ||k_t||
+        if (tid < 64) sL[tsw(tid >> 5, 32 + (tid & 31))] = ve[tid];
+        __syncthreads();
         // ---- rows t < Lc of T_d (tsw order kept) to the chunk's rows of the k~ buffer
         {
             const int t = tid >> 1, half = tid & 1;
@@ -321,30 +327,33 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
 struct ScanChainSmem {
     static constexpr uint32_t KT = 0;                 // 3 x bf16 k tiles (16 KB, SW128)
     static constexpr uint32_t TD = 3 * 16384;         // 3 x fp32 T_d tiles (16 KB, tsw rows)
-    static constexpr uint32_t VEC = 6 * 16384;        // 3 x {R, g, r, beta [64], R_C}
-    static constexpr uint32_t VECB = 1280;
+    static constexpr uint32_t LO = 6 * 16384;         // 2 x bf16 k~ lo staging tile (16 KB, SW128)
+    static constexpr uint32_t VEC = LO + 2 * 16384;   // 3 x {R, g, r, beta, R_C, e, beta R}
+    static constexpr uint32_t VECB = 2048;
     static constexpr uint32_t D = VEC + 3 * VECB;     // 3 x d at chunk start [128]
     static constexpr uint32_t X = D + 3 * 512;        // 3 x x [64]
     static constexpr uint32_t GX = X + 3 * 256;       // g (.) x [64]
     static constexpr uint32_t BV = GX + 256;          // b [64]
-    static constexpr uint32_t LO = BV + 256;          // 2 x bf16 k~ lo staging tile (16 KB, SW128)
-    static constexpr uint32_t XW = LO + 2 * 16384;    // 2 x the writer groups' copy of x [64]
+    static constexpr uint32_t XW = BV + 256;          // 2 x the writer groups' copy of x [64]
     static constexpr uint32_t BAR = XW + 2 * 256;     // 21 mbarriers
-    static constexpr uint32_t TOTAL = BAR + 21 * 8;
+    static constexpr uint32_t FAIL = BAR + 21 * 8;    // rank 0: the loader's failure flag
+    static constexpr uint32_t TOTAL = FAIL + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
-// rank 0: warps 0-7 the chain's products, 8 loads and gates, 9 the forwarder; rank 1: warps 4-7
-// the k~ output (two groups), 8 loads
+// rank 0: warps 0-7 the chain's products, 8 the chain's per-chunk inputs, 9 the forwarder and
+// refills; rank 1: warps 4-7 the k~ output (two groups), 8 loads
 constexpr int SCAN_CHAIN_THREADS = 320;
 
-// One 2-CTA cluster per (sequence, head).  Rank 0 runs the chain (warps 0-7), its loads (warp 8:
-// k and T_d tiles, gate vectors) and a forwarder (warp 9); rank 1 runs the k~ token pass (warps
-// 4-7) and its own loads (warp 8: k tiles, r).  The token pass gets an SM of its own.  The chain
-// only arrives on local barriers; the forwarder copies x and the chunk-start d of each chunk into
-// rank 1's shared memory and arrives on rank 1's barrier (release / acquire at cluster scope), so
-// no chain thread waits for a cluster-scope release.  Rank 1's writers copy x out and arrive back
-// on rank 0 before their token pass.  The two CTAs of a cluster are co-scheduled, so these
-// cross-CTA waits are safe (and bounded like every other).  td_in is the k~ buffer holding the prep kernel's T_d tiles.
+// One 2-CTA cluster per (sequence, head).  Rank 0 runs the chain (warps 0-7), a loader (warp 8:
+// waits for each chunk's k and T_d tiles, writes the gate vectors, e_t and beta_t R_t, then meets
+// the chain at a named barrier, so the chain threads never wait on an mbarrier) and a forwarder
+// (warp 9: refills the ring slot the chain has finished with, copies x and the chunk-start d of
+// each chunk into rank 1's shared memory and arrives on rank 1's barrier, release / acquire at
+// cluster scope); rank 1 runs the k~ token pass (warps 4-7) and its own loads (warp 8: k tiles,
+// r).  The token pass gets an SM of its own.  Rank 1's writers copy x out and arrive back on
+// rank 0 before their token pass.  The two CTAs of a cluster are co-scheduled, so these
+// cross-CTA waits are safe (and bounded like every other).  td_in is the k~ buffer holding the
+// prep kernel's T_d tiles.
 // k_tilde receives k~ rounded to bf16 (hi); with kLo, k_tilde_lo receives the rounding residual
 // bf16(k~ - hi), so that hi + lo carries k~ to about 2^-17 of its size.  With kD, d_all
 // ([B,T,H,Dk] fp32) receives d_t, the preconditioner each token writes with.  (Compile-time
@@ -352,6 +361,7 @@ constexpr int SCAN_CHAIN_THREADS = 320;
 template <bool kLo, bool kD>
 __global__ void __launch_bounds__(SCAN_CHAIN_THREADS, 1)
 precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_td,
+                     const __grid_constant__ CUtensorMap tm_kto, const __grid_constant__ CUtensorMap tm_ktlo,
                      const float* __restrict__ beta, const float* __restrict__ r, float eta,
                      const float* __restrict__ d0, __nv_bfloat16* __restrict__ k_tilde,
                      __nv_bfloat16* __restrict__ k_tilde_lo, float* __restrict__ d_all,
@@ -373,12 +383,12 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* full = bars;         // [3] TMA: k tile (+ T_d tile on rank 0)
-    uint64_t* vready = bars + 3;   // [3] gate vectors (32 arrivals)
-    uint64_t* kempty = bars + 6;   // [3] slot released: rank 0 by the chain (256), rank 1 by the
-                                   //     chunk's writer group (64)
+    uint64_t* vready = bars + 3;   // [3] rank 1: r of the chunk (32 arrivals)
+    uint64_t* kempty = bars + 6;   // [3] rank 1: slot released by the chunk's writer group (64)
     uint64_t* xready = bars + 9;   // [3] rank 1: x and d of a chunk, from rank 0's forwarder (32)
     uint64_t* outdone = bars + 12; // [3] rank 0: rank 1's writer group has copied x / d (64)
-    uint64_t* fwdin = bars + 15;   // [3] rank 0: x and d of a chunk in local memory (256, chain)
+    uint64_t* fwdin = bars + 15;   // [3] rank 0: x and d of a chunk in local memory, the chain
+                                   //     done with the slot (256)
     uint64_t* fwdout = bars + 18;  // [3] rank 0: the forwarder has sent them (32)
     float* sD = reinterpret_cast<float*>(smem + L::D);
     float* sX = reinterpret_cast<float*>(smem + L::X);
@@ -394,7 +404,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         for (int s = 0; s < 3; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&vready[s], 32);
-            mbar_init(&kempty[s], rank == 0 ? 256 : 64);
+            mbar_init(&kempty[s], 64);
             mbar_init(&xready[s], 32);
             mbar_init(&outdone[s], 64);
             mbar_init(&fwdin[s], 256);
@@ -403,6 +413,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         tc::fence_mbar_init();
     }
     if (tid < DK) sD[tid] = d0 ? __ldg(d0 + dbase + tid) : 1.0f;
+    if (tid == 0) *reinterpret_cast<int*>(smem + L::FAIL) = 0;
     tc::fence_before_sync();
     tc::cluster_sync();  // both CTAs initialised before either touches the other
     // rank 0's view of rank 1's x / d buffers and barriers, and rank 1's of rank 0's
@@ -441,14 +452,14 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
         }
     } else if (warp == 8) {
-        // =============================================== rank 0: loads and gate vectors
-        if (lane == 0) {
-            tc::prefetch_tmap(&tm_k);
-            tc::prefetch_tmap(&tm_td);
-        }
-        int last_issued = -1;
-        bool fail = false;
-        // gates of the next chunk are fetched one iteration early to hide their load latency
+        // =============================================== rank 0: the chain's per-chunk inputs
+        // For chunk c, once its tiles have landed and the forwarder has sent chunk c - 2 (whose
+        // d slot the chain overwrites in chunk c): the gate vectors, e_t = eta beta_t / ||k_t||^2
+        // (computed by the prep kernel, carried in the T_d tile) and beta_t R_t, then the
+        // chain's barrier.  Every wait of the chain's inputs happens
+        // here, one chunk ahead, so the chain threads never wait on an mbarrier; a wait that runs
+        // out sets the failure flag before the barrier, and the chain leaves at that chunk.
+        volatile int* fail_flag = reinterpret_cast<volatile int*>(smem + L::FAIL);
         float nr0 = 1.f, nr1 = 1.f, nb0 = 0.f, nb1 = 0.f;
         auto fetch_gates = [&](int c) {
             const int64_t row0 = first + (int64_t)c * C;
@@ -462,10 +473,174 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         if (nchunks > 0) fetch_gates(0);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % 3;
-            if (c >= 3 && !mbar_wait_bounded(&kempty[s], (uint32_t)(c / 3 - 1) & 1u, limit_ns)) {
-                fail = true;
+            bool got = mbar_wait_bounded(&full[s], (uint32_t)(c / 3) & 1u, limit_ns);
+            if (got && c >= 2)
+                got = mbar_wait_bounded(&fwdout[(c - 2) % 3], (uint32_t)((c - 2) / 3) & 1u, limit_ns);
+            if (__any_sync(0xffffffffu, !got)) {
+                if (lane == 0) *fail_flag = 1;
+                __threadfence_block();
+                group_bar(1, 288);  // the chain reads the flag and leaves
                 break;
             }
+            const int Lc = chunk_len(c), t0 = 2 * lane;
+            const float r0 = nr0, r1 = nr1, b0 = nb0, b1 = nb1;
+            if (c + 1 < nchunks) fetch_gates(c + 1);
+            const GatePrefix g = gate_prefix(r0, r1, lane);
+            float* vv = vecs(s);  // R | g | r | beta | R_C | e | beta R
+            const float R0 = g.sg0 * __expf(g.lr0), R1 = g.sg_1 * __expf(g.lr_1);
+            vv[t0] = R0;
+            vv[t0 + 1] = R1;
+            vv[64 + t0] = g.sgC * g.sg1_0 * __expf(g.lrC - g.lr1_0);
+            vv[64 + t0 + 1] = g.sgC * g.sg1_1 * __expf(g.lrC - g.lr1_1);
+            vv[128 + t0] = r0;
+            vv[128 + t0 + 1] = r1;
+            vv[192 + t0] = b0;
+            vv[192 + t0 + 1] = b1;
+            if (lane == 0) vv[256] = g.sgC * __expf(g.lrC);
+            {  // e_t from the T_d tile's spare block (written there by the prep kernel)
+                const float* td = reinterpret_cast<const float*>(smem + L::TD + s * 16384);
+                vv[320 + t0] = t0 < Lc ? td[tsw(t0 >> 5, 32 + (t0 & 31))] : 0.f;
+                vv[320 + t0 + 1] = t0 + 1 < Lc ? td[tsw((t0 + 1) >> 5, 32 + ((t0 + 1) & 31))] : 0.f;
+                vv[384 + t0] = b0 * R0;
+                vv[384 + t0 + 1] = b1 * R1;
+            }
+            __threadfence_block();
+            group_bar(1, 288);  // chunk c's inputs are in place; the chain starts it
+        }
+    } else if (warp < 8 && rank == 0) {
+        // =============================================== p = A d, x = T_d b, next d
+        // Per chunk: the loader's barrier (its inputs are in place), then three steps separated
+        // by the chain's own barrier; every operand that does not depend on the chain's values
+        // (the key and T_d tiles, the gate vectors) is read before the first step.
+        const volatile int* fail_flag = reinterpret_cast<const volatile int*>(smem + L::FAIL);
+        const int u = tid;
+        const int t = 8 * warp + (lane & 7), qd = lane >> 3;  // step 1/2 roles: token, channel quarter
+        const int cp = u >> 2, par = u & 3;  // step 3 role: channel pair, token quarter
+        const int cblk = cp >> 5, cj = (cp & 31) >> 2, cpe = 2 * (cp & 3);
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            group_bar(1, 288);
+            if (*fail_flag) {
+                ok = false;
+                break;
+            }
+            const int s = c % 3;
+            const int Lc = chunk_len(c);
+            const uint8_t* kt = smem + L::KT + s * 16384;
+            const float* td = reinterpret_cast<const float*>(smem + L::TD + s * 16384);
+            const float* vv = vecs(s);
+            const float* d = sD + (c % 3) * 128;
+            uint4 k1[4];   // step 1: token t, channels 32 qd .. 32 qd + 31
+            float4 tv[4];  // step 2: T_d[t][16 qd .. 16 qd + 15]
+            uint32_t k3[C / 4];  // step 3: channels 2 cp, 2 cp + 1 of the tokens 8 m + 2 par + {0, 1}
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                k1[j] = *reinterpret_cast<const uint4*>(kt + (qd >> 1) * 8192u + tc::sw128_off(t, 4 * (qd & 1) + j));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tv[q] = tsw_ld4(td, t, 4 * qd + q);
+            {
+                const uint8_t* col = kt + cblk * 8192u + cpe * 2;
+#pragma unroll
+                for (int jj = 0; jj < C / 4; ++jj) {
+                    const int j = 8 * (jj >> 1) + 2 * par + (jj & 1);
+                    k3[jj] = *reinterpret_cast<const uint32_t*>(col + tc::sw128_off(j, cj));
+                }
+            }
+            const float e_t = vv[320 + t], hR_t = vv[384 + t], g_t = vv[64 + t], rc = vv[256];
+            // ---- step 1: p_t = <a_t, d>, b_t = e_t (1 - beta_t R_t p_t)
+            float bRp = 0.f;  // kept for the residual ratio of step 2
+            {
+                float2 pa = make_float2(0.f, 0.f), pb = make_float2(0.f, 0.f);  // channel pairs
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {  // channels 32 qd + 8 j .. + 7
+                    const uint32_t w4[4] = {k1[j].x, k1[j].y, k1[j].z, k1[j].w};
+                    const float4 da = *reinterpret_cast<const float4*>(d + 32 * qd + 8 * j);
+                    const float4 db = *reinterpret_cast<const float4*>(d + 32 * qd + 8 * j + 4);
+                    const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w),
+                                          make_float2(db.x, db.y), make_float2(db.z, db.w)};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                        if (e & 1) pb = __ffma2_rn(__fmul2_rn(kk, kk), dv[e], pb);
+                        else pa = __ffma2_rn(__fmul2_rn(kk, kk), dv[e], pa);
+                    }
+                }
+                float p = (pa.x + pb.x) + (pa.y + pb.y);
+                p += __shfl_xor_sync(0xffffffffu, p, 8);
+                p += __shfl_xor_sync(0xffffffffu, p, 16);
+                if (qd == 0) {
+                    bRp = hR_t * p;
+                    sB[t] = e_t * (1.f - bRp);
+                }
+            }
+            group_bar(5, 256);
+            // ---- step 2: x_t = sum_{j <= t} T_d[t][j] b_j
+            {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int g = 4 * qd + q;
+                    const float4 bv = *reinterpret_cast<const float4*>(sB + 4 * g);
+                    const int j = 4 * g;
+                    acc[q] = fmaf(j <= t ? tv[q].x : 0.f, bv.x, acc[q]);
+                    acc[q] = fmaf(j + 1 <= t ? tv[q].y : 0.f, bv.y, acc[q]);
+                    acc[q] = fmaf(j + 2 <= t ? tv[q].z : 0.f, bv.z, acc[q]);
+                    acc[q] = fmaf(j + 3 <= t ? tv[q].w : 0.f, bv.w, acc[q]);
+                }
+                float xs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                xs += __shfl_xor_sync(0xffffffffu, xs, 8);
+                xs += __shfl_xor_sync(0xffffffffu, xs, 16);
+                if (qd == 0) {
+                    const float x = t < Lc ? xs : 0.f;
+                    sX[(c % 3) * 64 + t] = x;
+                    sGX[t] = g_t * x;
+                    // residual-contraction ratio (1 - beta s)^2: x = e (1 - beta s) when e != 0;
+                    // else d_t = R_t d_0 on this token's row, so beta s = beta R p
+                    if (rho && t < Lc) {
+                        const float gr = e_t != 0.f ? x / e_t : 1.f - bRp;
+                        rho[(first + (int64_t)c * C + t) * H + h] = gr * gr;
+                    }
+                }
+            }
+            group_bar(5, 256);
+            // ---- step 3: d_C[i] = R_C d[i] + sum_j g_j x_j a_j[i]; thread: channels 2cp, 2cp + 1
+            //      over the tokens j = 8 m + 2 par + {0, 1} -- the four parts read rows of distinct
+            //      swizzle phases, so the lanes read disjoint banks -- summed by shuffles
+            {
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // the channel pair
+#pragma unroll
+                for (int jj = 0; jj < C / 4; ++jj) {
+                    const int j = 8 * (jj >> 1) + 2 * par + (jj & 1);
+                    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k3[jj]));
+                    const float gx = sGX[j];
+                    acc[jj & 1] = __ffma2_rn(make_float2(gx, gx), __fmul2_rn(kv, kv), acc[jj & 1]);
+                }
+                float acc0 = acc[0].x + acc[1].x, acc1 = acc[0].y + acc[1].y;
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+                if (par == 0) {
+                    const float2 dv = *reinterpret_cast<const float2*>(d + 2 * cp);
+                    const float2 dn = make_float2(fmaf(rc, dv.x, acc0), fmaf(rc, dv.y, acc1));
+                    *reinterpret_cast<float2*>(sD + ((c + 1) % 3) * 128 + 2 * cp) = dn;
+                }
+            }
+            // x_c and d_c are in sX, sD and this thread is done with the slot: the forwarder sends
+            // them and refills the slot
+            mbar_arrive(&fwdin[c % 3]);
+        }
+        group_bar(5, 256);  // the last chunk's d is complete
+        if (ok && dT && u < DK) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
+    } else if (warp == 9 && rank == 0) {
+        // =============================================== forwarder: x_c, d_c to rank 1; refills
+        // Once the chain is done with chunk c (fwdin): the refill of its ring slot with chunk
+        // c + 3; then chunk c's x and chunk-start d go into slot c % 3 of rank 1's buffers once
+        // rank 1's writer of chunk c - 3 has copied that slot out; the slot's local copies may
+        // then be overwritten by the chain (fwdout).
+        int last_issued = -1;
+        auto issue = [&](int c) {
+            const int s = c % 3;
             const int64_t row0 = first + (int64_t)c * C;
             if (lane == 0) {
                 uint8_t* kt = smem + L::KT + s * 16384;
@@ -475,153 +650,18 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 tc::tma_load_3d(smem + L::TD + s * 16384, &tm_td, 0, h, (int)row0, &full[s]);
             }
             last_issued = c;
-            const int t0 = 2 * lane;
-            const float r0 = nr0, r1 = nr1, b0 = nb0, b1 = nb1;
-            if (c + 1 < nchunks) fetch_gates(c + 1);
-            const GatePrefix g = gate_prefix(r0, r1, lane);
-            float* vv = vecs(s);  // R | g | r | beta | R_C
-            vv[t0] = g.sg0 * __expf(g.lr0);
-            vv[t0 + 1] = g.sg_1 * __expf(g.lr_1);
-            vv[64 + t0] = g.sgC * g.sg1_0 * __expf(g.lrC - g.lr1_0);
-            vv[64 + t0 + 1] = g.sgC * g.sg1_1 * __expf(g.lrC - g.lr1_1);
-            vv[128 + t0] = r0;
-            vv[128 + t0 + 1] = r1;
-            vv[192 + t0] = b0;
-            vv[192 + t0 + 1] = b1;
-            if (lane == 0) vv[256] = g.sgC * __expf(g.lrC);
-            mbar_arrive(&vready[s]);
+        };
+        if (lane == 0) {
+            tc::prefetch_tmap(&tm_k);
+            tc::prefetch_tmap(&tm_td);
         }
-        if (fail && lane == 0 && last_issued >= 0) {  // let the loads in flight land
-            for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
-                mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
-        }
-    } else if (warp < 8 && rank == 0) {
-        // =============================================== p = A d, x = T_d b, next d
-        const int u = tid;
-        const int t = 8 * warp + (lane & 7), qd = lane >> 3;  // step 1/2 roles: token, channel quarter
-        const int cp = u >> 2, par = u & 3;  // step 3 role: channel pair, token quarter
-        const int cblk = cp >> 5, cj = (cp & 31) >> 2, cpe = 2 * (cp & 3);
-        bool ok = true;
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % 3;
-            const uint32_t ph = (uint32_t)(c / 3) & 1u;
-            bool got = mbar_wait_bounded(&full[s], ph, limit_ns) &&
-                       mbar_wait_bounded(&vready[s], ph, limit_ns);
-            if (got && c >= 2)  // the forwarder has sent the x / d buffers this chunk overwrites
-                got = mbar_wait_bounded(&fwdout[(c - 2) % 3], (uint32_t)((c - 2) / 3) & 1u, limit_ns);
-            if (group_any(1, 256, !got)) {
-                ok = false;
-                break;
-            }
-            const int Lc = chunk_len(c);
-            const uint8_t* kt = smem + L::KT + s * 16384;
-            const float* td = reinterpret_cast<const float*>(smem + L::TD + s * 16384);
-            const float* vv = vecs(s);
-            const float* d = sD + (c % 3) * 128;
-            // ---- step 1: p_t = <a_t, d>, ||k_t||^2, b_t
-            float e_t = 0.f, bRp = 0.f;  // kept for the residual ratio of step 2
-            {
-                float2 p2 = make_float2(0.f, 0.f), nk2 = make_float2(0.f, 0.f);  // channel pairs
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {  // channels 32 qd + 8 j .. + 7
-                    const int ch16 = 4 * (qd & 1) + j;
-                    const uint4 raw = *reinterpret_cast<const uint4*>(kt + (qd >> 1) * 8192u + tc::sw128_off(t, ch16));
-                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                    const float4 da = *reinterpret_cast<const float4*>(d + 32 * qd + 8 * j);
-                    const float4 db = *reinterpret_cast<const float4*>(d + 32 * qd + 8 * j + 4);
-                    const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w),
-                                          make_float2(db.x, db.y), make_float2(db.z, db.w)};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-                        const float2 a = __fmul2_rn(kk, kk);
-                        nk2 = __fadd2_rn(nk2, a);
-                        p2 = __ffma2_rn(a, dv[e], p2);
-                    }
-                }
-                float p = p2.x + p2.y, nk = nk2.x + nk2.y;
-                p += __shfl_xor_sync(0xffffffffu, p, 8);
-                nk += __shfl_xor_sync(0xffffffffu, nk, 8);
-                p += __shfl_xor_sync(0xffffffffu, p, 16);
-                nk += __shfl_xor_sync(0xffffffffu, nk, 16);
-                if (qd == 0) {
-                    const float bt = vv[192 + t];
-                    e_t = (t < Lc && nk > 0.f) ? eta * bt / nk : 0.f;
-                    sB[t] = e_t * (1.f - bt * vv[t] * p);
-                    bRp = bt * vv[t] * p;
-                }
-            }
-            group_bar(1, 256);
-            // ---- step 2: x_t = sum_{j <= t} T_d[t][j] b_j
-            {
-                float acc = 0.f;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int g = 4 * qd + q;
-                    const float4 tv = tsw_ld4(td, t, g);
-                    const float4 bv = *reinterpret_cast<const float4*>(sB + 4 * g);
-                    const int j = 4 * g;
-                    acc = fmaf(j <= t ? tv.x : 0.f, bv.x, acc);
-                    acc = fmaf(j + 1 <= t ? tv.y : 0.f, bv.y, acc);
-                    acc = fmaf(j + 2 <= t ? tv.z : 0.f, bv.z, acc);
-                    acc = fmaf(j + 3 <= t ? tv.w : 0.f, bv.w, acc);
-                }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-                if (qd == 0) {
-                    const float x = t < Lc ? acc : 0.f;
-                    sX[(c % 3) * 64 + t] = x;
-                    sGX[t] = vv[64 + t] * x;
-                    // residual-contraction ratio (1 - beta s)^2: x = e (1 - beta s) when e != 0;
-                    // else d_t = R_t d_0 on this token's row, so beta s = beta R p
-                    if (rho && t < Lc) {
-                        const float g = e_t != 0.f ? x / e_t : 1.f - bRp;
-                        rho[(first + (int64_t)c * C + t) * H + h] = g * g;
-                    }
-                }
-            }
-            group_bar(1, 256);
-            // ---- step 3: d_C[i] = R_C d[i] + sum_j g_j x_j a_j[i]; thread: channels 2cp, 2cp + 1
-            //      over the tokens j = 8 m + 2 par + {0, 1} -- the four parts read rows of distinct
-            //      swizzle phases, so the lanes read disjoint banks -- summed by shuffles
-            {
-                float2 acc = make_float2(0.f, 0.f);  // the two channels of the pair
-                const uint8_t* col = kt + cblk * 8192u + cpe * 2;
-#pragma unroll 8
-                for (int jj = 0; jj < C / 4; ++jj) {
-                    const int j = 8 * (jj >> 1) + 2 * par + (jj & 1);
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(col + tc::sw128_off(j, cj));
-                    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-                    const float gx = sGX[j];
-                    acc = __ffma2_rn(make_float2(gx, gx), __fmul2_rn(kv, kv), acc);
-                }
-                float acc0 = acc.x, acc1 = acc.y;
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-                if (par == 0) {
-                    const float rc = vv[256];
-                    const float2 dv = *reinterpret_cast<const float2*>(d + 2 * cp);
-                    const float2 dn = make_float2(fmaf(rc, dv.x, acc0), fmaf(rc, dv.y, acc1));
-                    *reinterpret_cast<float2*>(sD + ((c + 1) % 3) * 128 + 2 * cp) = dn;
-                }
-            }
-            mbar_arrive(&fwdin[c % 3]);  // x_c and d_c are in sX, sD: the forwarder sends them
-            mbar_arrive(&kempty[s]);     // the chain's last use of the slot
-            group_bar(1, 256);
-        }
-        if (ok && dT && u < DK) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
-    } else if (warp == 9 && rank == 0) {
-        // =============================================== forwarder: x_c, d_c to rank 1
-        // Chunk c's x and chunk-start d go into slot c % 3 of rank 1's buffers once rank 1's
-        // writer of chunk c - 3 has copied that slot out; the slot's local copies may then be
-        // overwritten by the chain (fwdout).
+        for (int c = 0; c < 3 && c < nchunks; ++c) issue(c);
         for (int c = 0; c < nchunks; ++c) {
             const int k = c % 3;
             bool got = mbar_wait_bounded(&fwdin[k], (uint32_t)(c / 3) & 1u, limit_ns);
-            if (got && c >= 3)
-                got = tc::mbar_wait_cluster(&outdone[k], (uint32_t)(c / 3 - 1) & 1u, limit_ns);
+            if (__any_sync(0xffffffffu, !got)) break;
+            if (c + 3 < nchunks) issue(c + 3);
+            if (c >= 3) got = tc::mbar_wait_cluster(&outdone[k], (uint32_t)(c / 3 - 1) & 1u, limit_ns);
             if (__any_sync(0xffffffffu, !got)) break;
             {
                 const float2 xv = *reinterpret_cast<const float2*>(sX + k * 64 + 2 * lane);
@@ -635,6 +675,12 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             }
             mbar_arrive(&fwdout[k]);                                // local copies are free
             tc::mbar_arrive_cluster(peer_xready + 8u * (uint32_t)k);  // rank 1 may read them
+        }
+        // let the copies in flight land (the last one issued into each slot): on the normal
+        // path the loader has waited for all of them already
+        if (lane == 0 && last_issued >= 0) {
+            for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
+                mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
         }
     } else if (warp >= 4 && warp < 8 && rank == 1) {
         // =============================================== k~ = d (.) k, token by token
@@ -695,8 +741,24 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     dd = __ffma2_rn(make_float2(rt[u], rt[u]), dd, __fmul2_rn(make_float2(xt[u], xt[u]), a));
                 }
             }
+            // a whole chunk leaves by TMA stores (64 rows x 64 channels per box); a short one, whose
+            // box would reach the next sequence's rows, by 16-byte row pieces
+            const bool bulk = Lc == C;
+            if (bulk) tc::fence_async_smem();
             group_bar(gbar, 64);
-            {  // 64 rows x 16 pieces of 16 bytes per tile: piece jj & 15, rows (jj >> 4) + 4 q
+            if (bulk) {
+                if (jj == 0) {
+                    const int row0 = (int)(first + (int64_t)c * C);
+                    tc::tma_store_3d(&tm_kto, stage, 0, h, row0);
+                    tc::tma_store_3d(&tm_kto, stage + 8192, 64, h, row0);
+                    if (kLo) {
+                        tc::tma_store_3d(&tm_ktlo, lo_stage, 0, h, row0);
+                        tc::tma_store_3d(&tm_ktlo, lo_stage + 8192, 64, h, row0);
+                    }
+                    tc::bulk_commit();
+                    tc::bulk_wait_read_all();  // the staging tiles may be reused
+                }
+            } else {  // 64 rows x 16 pieces of 16 bytes per tile: piece jj & 15, rows (jj >> 4) + 4 q
                 const int piece = jj & 15, blk16 = piece >> 3, j16 = piece & 7;
                 const int64_t off = ((first + (int64_t)c * C) * H + h) * DK + 8 * piece;
                 const int64_t rs = (int64_t)H * DK;
@@ -716,6 +778,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             group_bar(gbar, 64);  // the group's staging tiles and x copy are read out
             mbar_arrive(&kempty[s]);
         }
+        if (jj == 0) tc::bulk_wait_all();  // this thread's stores are complete
     }
     tc::fence_before_sync();
     tc::cluster_sync();  // neither CTA leaves while the other may still write to it
