@@ -182,11 +182,15 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
 #pragma unroll
                 for (int g = g0; g < g0 + 4; ++g) {
                     uint32_t hw[4], lw[4];
+                    // columns 8 g .. 8 g + 7 as two 16-byte loads (the lanes of a warp, on
+                    // consecutive rows, meet each bank at most four times: the minimum for 512 B)
+                    const float4 va = tsw_ld4(sL, r, 2 * g), vb = tsw_ld4(sL, r, 2 * g + 1);
+                    const float tv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c = 8 * g + 2 * e;
-                        const float a = c < r ? sL[tsw(r, c)] : (c == r ? 1.f : 0.f);
-                        const float b = c + 1 < r ? sL[tsw(r, c + 1)] : (c + 1 == r ? 1.f : 0.f);
+                        const float a = c < r ? tv[2 * e] : (c == r ? 1.f : 0.f);
+                        const float b = c + 1 < r ? tv[2 * e + 1] : (c + 1 == r ? 1.f : 0.f);
                         const __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
                         const float2 hf = __bfloat1622float2(hb);
                         const __nv_bfloat162 lb = __floats2bfloat162_rn(a - hf.x, b - hf.y);

@@ -301,15 +301,14 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
         // scratch of the inverse: the chain kernel reads it there instead of recomputing ||k_t||
         if (tid < 64) sL[tsw(tid >> 5, 32 + (tid & 31))] = ve[tid];
         __syncthreads();
-        // ---- rows t < Lc of T_d (tsw order kept) to the chunk's rows of the k~ buffer
-        {
-            const int t = tid >> 1, half = tid & 1;
-            if (t < Lc) {
-                const float4* src = reinterpret_cast<const float4*>(sL + t * 64) + 8 * half;
-                float4* dst = reinterpret_cast<float4*>(td_out + ((row0 + t) * H + h) * 64) + 8 * half;
+        // ---- rows t < Lc of T_d (tsw order kept) to the chunk's rows of the k~ buffer; 16 lanes
+        //      per row, so a warp reads two whole rows (no bank conflicts) and writes them whole
 #pragma unroll
-                for (int q = 0; q < 8; ++q) dst[q] = src[q];
-            }
+        for (int it = 0; it < 8; ++it) {
+            const int idx = it * 128 + tid, t = idx >> 4, piece = idx & 15;
+            if (t < Lc)
+                reinterpret_cast<float4*>(td_out + ((row0 + t) * H + h) * 64)[piece] =
+                    reinterpret_cast<const float4*>(sL + t * 64)[piece];
         }
         __syncthreads();  // sT and sL lie over the next chunk's a tiles
     }
