@@ -409,9 +409,16 @@ bwd_reduce_kernel(const float4* __restrict__ dq_part, float4* __restrict__ dk_pa
     }
 }
 
-// Phase 1 in reverse.  One CTA of 128 threads per (sequence, head): warp 0 runs the adjoint
-// recurrence over a 32-token chunk staged in shared memory while warps 1-3 fetch the next chunk
-// (in reverse order) into the other buffer with asynchronous copies.
+// Phase 1 in reverse.  One CTA of 128 threads per (sequence, head), 32-token chunks in reverse
+// order, three chunk buffers in turn (two when three do not fit in shared memory):
+//   warp 0 runs the adjoint recurrence dd_t = r_t dd_{t+1} - c_t y_t a_t + dk~_t (.) k_t over chunk
+//     ch, where y_t = <a_t, dd_{t+1}> is its only reduction, and keeps dd_{t+1} and y_t of every
+//     token (c_t = eta beta_t^2 / ||k_t||^2, 0 for a zero key);
+//   warps 1-3 meanwhile start fetching chunk ch - 1 (asynchronous copies), turn chunk ch + 1's
+//     kept values into dk, dr, dbeta and deta, and then compute chunk ch - 1's per-token
+//     scalars, none of which depends on dd: ||k_t||^2, s_t = <d_t, a_t>, x_t, c_t and the dbeta
+//     factor.  Every value they read is staged in shared memory, so their per-token loops do not
+//     wait on global loads.
 template <int DK, typename IO>
 struct BwdPrecondSmem {
     static constexpr int KB = DK * (int)sizeof(IO) / 4;  // a token's key row, in 4-byte words
@@ -419,9 +426,14 @@ struct BwdPrecondSmem {
     static constexpr int DK2 = DKT + BWD_C * DK;         // [C][DK] dk, phase-2 term
     static constexpr int D = DK2 + BWD_C * DK;           // [C][DK] d_t
     static constexpr int K = D + BWD_C * DK;             // [C][KB] k_t in the io dtype
-    static constexpr int VEC = K + BWD_C * KB;           // [C] beta, r, dbeta phase-2 term
-    static constexpr int BUF = VEC + 3 * BWD_C;          // one buffer
-    static constexpr int floats = 2 * BUF;
+    static constexpr int SC = K + BWD_C * KB;            // [7][C] beta, r, dbeta phase-2 term,
+                                                         //   1/||k||^2, x, c, dbeta factor
+    static constexpr int BUF = SC + 7 * BWD_C;           // one chunk buffer
+    static constexpr int NB = 3 * BUF + 2 * BWD_C * DK + 2 * BWD_C + 4 <= 232448 / 4 - 256 ? 3 : 2;
+    static constexpr int DD = NB * BUF;                  // [2][C][DK] dd_{t+1}, kept by warp 0
+    static constexpr int Y = DD + 2 * BWD_C * DK;        // [2][C] y_t
+    static constexpr int ETA = Y + 2 * BWD_C;            // [4] deta shares of warps 1-3
+    static constexpr int floats = ETA + 4;
     static constexpr size_t bytes = sizeof(float) * floats;
 };
 
@@ -458,9 +470,13 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
         const int64_t rem = count - (int64_t)ch * C;
         return rem < C ? (int)rem : C;
     };
-    // warps 1-3: chunk ch into buffer b (tokens past the chunk's end are not read)
-    auto fetch = [&](int b, int ch) {
-        float* buf = sm + b * L::BUF;
+    auto buf_of = [&](int ch) { return sm + (ch % L::NB) * L::BUF; };
+
+    // warps 1-3: chunk ch into its buffer (tokens past the chunk's end are not read): copies
+    // issued here, the gates held in registers until fetch_finish stores them
+    float gb = 0.f, gr = 1.f, gd = 0.f;  // beta, r and the dbeta phase-2 term of token tid - 32
+    auto fetch_issue = [&](int ch) {
+        float* buf = buf_of(ch);
         const int64_t row0 = first + (int64_t)ch * C;
         const int Lc = chunk_len(ch), i = tid - 32;
         constexpr int P4 = DK / 4, PK = L::KB / 4;  // 16-byte pieces per token row
@@ -473,77 +489,145 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
             else cp_async16(buf + L::K + t * L::KB + 4 * (q - 3 * P4),
                             reinterpret_cast<const float*>(k + o) + 4 * (q - 3 * P4));
         }
-        for (int t = i; t < Lc; t += 96) {
-            const int64_t th = (row0 + t) * H + h;
-            buf[L::VEC + t] = __ldg(beta + th);
-            buf[L::VEC + C + t] = r ? __ldg(r + th) : 1.f;
-            buf[L::VEC + 2 * C + t] = dbeta_sum[th];
+        if (i < Lc) {
+            const int64_t th = (row0 + i) * H + h;
+            gb = __ldg(beta + th);
+            gr = r ? __ldg(r + th) : 1.f;
+            gd = dbeta_sum[th];
+        }
+    };
+    // ... then, once the copies have landed, the per-token scalars (one warp per token)
+    auto fetch_finish = [&](int ch) {
+        float* buf = buf_of(ch);
+        const int Lc = chunk_len(ch), i = tid - 32;
+        if (i < Lc) {
+            buf[L::SC + i] = gb;
+            buf[L::SC + C + i] = gr;
+            buf[L::SC + 2 * C + i] = gd;
         }
         cp_async_wait_all();
+        asm volatile("bar.sync 1, 96;" ::: "memory");  // the chunk is in place for warps 1-3
+#pragma unroll 2
+        for (int t = warp - 1; t < Lc; t += 3) {
+            const IO* krow = reinterpret_cast<const IO*>(buf + L::K + t * L::KB);
+            float nk = 0.f, sv = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float kk = tr::to_f32(krow[lane * E + e]), a = kk * kk;
+                nk += a;
+                sv = fmaf(buf[L::D + t * DK + lane * E + e], a, sv);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                nk += __shfl_xor_sync(0xffffffffu, nk, off);
+                sv += __shfl_xor_sync(0xffffffffu, sv, off);
+            }
+            if (lane == 0) {
+                const float bt = buf[L::SC + t];
+                const bool ok = nk > 0.f;
+                const float inv = ok ? 1.f / nk : 0.f;
+                buf[L::SC + 3 * C + t] = inv;
+                buf[L::SC + 4 * C + t] = ok ? bt * (1.f - bt * sv) * inv : 0.f;     // x_t
+                buf[L::SC + 5 * C + t] = ok ? eta * bt * bt * inv : 0.f;           // c_t
+                buf[L::SC + 6 * C + t] = ok ? eta * (1.f - 2.f * bt * sv) * inv : 0.f;
+            }
+        }
+    };
+    // warps 1-3: the gradients of chunk ch from dd_{t+1} and y_t (one warp per token)
+    float deta_acc = 0.f;
+    auto outputs = [&](int ch) {
+        const float* buf = buf_of(ch);
+        const float* sdd = sm + L::DD + (ch & 1) * C * DK;
+        const float* sy = sm + L::Y + (ch & 1) * C;
+        const int64_t row0 = first + (int64_t)ch * C;
+        const int Lc = chunk_len(ch);
+#pragma unroll 2
+        for (int t = warp - 1; t < Lc; t += 3) {
+            const IO* krow = reinterpret_cast<const IO*>(buf + L::K + t * L::KB);
+            const float y = sy[t], bt = buf[L::SC + t], inv = buf[L::SC + 3 * C + t];
+            const float xt = buf[L::SC + 4 * C + t];
+            const int64_t th = (row0 + t) * H + h;
+            float rd = 0.f, g[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int c = lane * E + e;
+                const float ddv = sdd[t * DK + c], dv = buf[L::D + t * DK + c];
+                const float kk = tr::to_f32(krow[c]);
+                rd = fmaf(ddv, dv, rd);
+                const float da = inv > 0.f ? eta * xt * ddv - eta * y * (bt * bt * dv + xt) * inv : 0.f;
+                g[e] = buf[L::DK2 + t * DK + c] + buf[L::DKT + t * DK + c] * dv + 2.f * kk * da;
+            }
+            if constexpr (E == 4) {
+                *reinterpret_cast<float4*>(dk + th * DK + lane * E) = make_float4(g[0], g[1], g[2], g[3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) dk[th * DK + lane * E + e] = g[e];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) rd += __shfl_xor_sync(0xffffffffu, rd, off);
+            if (lane == 0) {
+                dbeta[th] = buf[L::SC + 2 * C + t] + buf[L::SC + 6 * C + t] * y;
+                if (dr) dr[th] = rd;
+                deta_acc = fmaf(xt, y, deta_acc);
+            }
+        }
     };
 
     float dd[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) dd[e] = ddT ? __ldg(ddT + (int64_t)nh * DK + lane * E + e) : 0.f;
-    float deta = 0.f;
-    if (warp > 0 && nchunks > 0) fetch(0, nchunks - 1);
+    if (warp > 0 && nchunks > 0) {
+        fetch_issue(nchunks - 1);
+        fetch_finish(nchunks - 1);
+    }
     __syncthreads();
     for (int ch = nchunks - 1; ch >= 0; --ch) {
-        const int b = (nchunks - 1 - ch) & 1;
-        if (warp > 0) {
-            if (ch > 0) fetch(b ^ 1, ch - 1);
-        } else {
-            const float* buf = sm + b * L::BUF;
-            const int64_t row0 = first + (int64_t)ch * C;
+        if (warp == 0) {
+            const float* buf = buf_of(ch);
+            float* sdd = sm + L::DD + (ch & 1) * C * DK;
+            float* sy = sm + L::Y + (ch & 1) * C;
             for (int t = chunk_len(ch) - 1; t >= 0; --t) {
-                float kk[E], dv_[E], a[E];
-                float nk = 0.f, s = 0.f, y = 0.f, rd = 0.f;
                 const IO* krow = reinterpret_cast<const IO*>(buf + L::K + t * L::KB);
+                float a[E], kk[E], dkt[E];
+                float y = 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
                     kk[e] = tr::to_f32(krow[lane * E + e]);
-                    dv_[e] = buf[L::D + t * DK + lane * E + e];
+                    dkt[e] = buf[L::DKT + t * DK + lane * E + e];
                     a[e] = kk[e] * kk[e];
-                    nk += a[e];
-                    s = fmaf(dv_[e], a[e], s);
                     y = fmaf(a[e], dd[e], y);
-                    rd = fmaf(dd[e], dv_[e], rd);
+                    sdd[t * DK + lane * E + e] = dd[e];  // dd_{t+1}
                 }
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    nk += __shfl_xor_sync(0xffffffffu, nk, off);
-                    s += __shfl_xor_sync(0xffffffffu, s, off);
-                    y += __shfl_xor_sync(0xffffffffu, y, off);
-                    rd += __shfl_xor_sync(0xffffffffu, rd, off);
-                }
-                const float bt = buf[L::VEC + t], rt = buf[L::VEC + C + t];
-                const bool ok = nk > 0.f;
-                const float inv = ok ? 1.f / nk : 0.f;
-                const float xt = ok ? bt * (1.f - bt * s) * inv : 0.f;
-                const int64_t th = (row0 + t) * H + h;
-                if (lane == 0) {
-                    dbeta[th] = buf[L::VEC + 2 * C + t] + (ok ? eta * y * (1.f - 2.f * bt * s) * inv : 0.f);
-                    if (dr) dr[th] = rd;
-                }
-                deta = fmaf(xt, y, deta);
-                const float cy = ok ? eta * bt * bt * inv * y : 0.f;
+                for (int off = 16; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+                if (lane == 0) sy[t] = y;
+                const float cy = buf[L::SC + 5 * C + t] * y, rt = buf[L::SC + C + t];
 #pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float dkt = buf[L::DKT + t * DK + lane * E + e];
-                    const float da = ok ? eta * xt * dd[e] - eta * y * (bt * bt * dv_[e] + xt) * inv : 0.f;
-                    dk[th * DK + lane * E + e] = buf[L::DK2 + t * DK + lane * E + e] + dkt * dv_[e] + 2.f * kk[e] * da;
-                    dd[e] = fmaf(rt, dd[e], fmaf(-cy, a[e], dkt * kk[e]));
-                }
+                for (int e = 0; e < E; ++e) dd[e] = fmaf(rt, dd[e], fmaf(-cy, a[e], dkt[e] * kk[e]));
+            }
+        } else if constexpr (L::NB == 3) {  // chunk ch - 1's copies land under chunk ch + 1's outputs
+            if (ch > 0) fetch_issue(ch - 1);
+            if (ch + 1 < nchunks) outputs(ch + 1);
+            if (ch > 0) fetch_finish(ch - 1);
+        } else {  // chunks ch + 1 and ch - 1 share a buffer
+            if (ch + 1 < nchunks) outputs(ch + 1);
+            asm volatile("bar.sync 1, 96;" ::: "memory");
+            if (ch > 0) {
+                fetch_issue(ch - 1);
+                fetch_finish(ch - 1);
             }
         }
-        __syncthreads();  // chunk ch is consumed and chunk ch - 1 has landed
+        __syncthreads();  // chunk ch's dd and y are kept; chunk ch - 1 has landed
     }
+    if (warp > 0 && nchunks > 0) outputs(0);
+    if (warp > 0 && lane == 0) sm[L::ETA + warp] = deta_acc;
+    __syncthreads();
     if (warp == 0) {
         if (dd0) {
 #pragma unroll
             for (int e = 0; e < E; ++e) dd0[(int64_t)nh * DK + lane * E + e] = dd[e];
         }
-        if (lane == 0) deta_part[nh] = deta;
+        if (lane == 0) deta_part[nh] = (sm[L::ETA + 1] + sm[L::ETA + 2]) + sm[L::ETA + 3];  // fixed order
     }
 }
 
