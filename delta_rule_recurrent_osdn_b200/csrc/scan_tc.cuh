@@ -324,23 +324,34 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
 // ===================================================================== chain: d across chunks
 
 struct ScanChainSmem {
+    // rank 0 (the chain)
     static constexpr uint32_t KT = 0;                 // 3 x bf16 k tiles (16 KB, SW128)
     static constexpr uint32_t TD = 3 * 16384;         // 3 x fp32 T_d tiles (16 KB, tsw rows)
-    static constexpr uint32_t LO = 6 * 16384;         // 2 x bf16 k~ lo staging tile (16 KB, SW128)
-    static constexpr uint32_t VEC = LO + 2 * 16384;   // 3 x {R, g, r, beta, R_C, e, beta R}
+    // rank 1 (the k~ token pass): a deeper key ring, staging tiles per writer group
+    static constexpr int NS1 = 5;                     // key ring slots
+    static constexpr int NG = 4;                      // writer groups
+    static constexpr uint32_t KT1 = 0;                // NS1 x bf16 k tiles
+    static constexpr uint32_t HI = NS1 * 16384;       // NG x bf16 k~ hi staging tile (SW128)
+    static constexpr uint32_t LO = HI + NG * 16384;   // NG x bf16 k~ lo staging tile (SW128)
+    static constexpr uint32_t RV = LO + NG * 16384;   // NS1 x r of the chunk [64]
+    static constexpr uint32_t XR = RV + NS1 * 256;    // NG x x of a chunk [64], from rank 0
+    static constexpr uint32_t DR = XR + NG * 256;     // NG x chunk-start d [128], from rank 0
+    // rank 0
+    static constexpr uint32_t VEC = DR + NG * 512;    // 3 x {R, g, r, beta, R_C, e, beta R}
     static constexpr uint32_t VECB = 2048;
     static constexpr uint32_t D = VEC + 3 * VECB;     // 3 x d at chunk start [128]
     static constexpr uint32_t X = D + 3 * 512;        // 3 x x [64]
     static constexpr uint32_t GX = X + 3 * 256;       // g (.) x [64]
     static constexpr uint32_t BV = GX + 256;          // b [64]
-    static constexpr uint32_t XW = BV + 256;          // 2 x the writer groups' copy of x [64]
-    static constexpr uint32_t BAR = XW + 2 * 256;     // 21 mbarriers
-    static constexpr uint32_t FAIL = BAR + 21 * 8;    // rank 0: the loader's failure flag
+    static constexpr uint32_t XW = BV + 256;          // NG x the writer groups' copy of x [64]
+    static constexpr uint32_t BAR = XW + NG * 256;    // 29 mbarriers
+    static constexpr uint32_t FAIL = BAR + 29 * 8;    // rank 0: the loader's failure flag
     static constexpr uint32_t TOTAL = FAIL + 16;
     static constexpr size_t BYTES = TOTAL + 1024;
 };
+static_assert(ScanChainSmem::BYTES <= 232448, "shared memory");
 // rank 0: warps 0-7 the chain's products, 8 the chain's per-chunk inputs, 9 the forwarder and
-// refills; rank 1: warps 4-7 the k~ output (two groups), 8 loads
+// refills; rank 1: warps 0-7 the k~ output (four groups of two warps), 8 loads
 constexpr int SCAN_CHAIN_THREADS = 320;
 
 // One 2-CTA cluster per (sequence, head).  Rank 0 runs the chain (warps 0-7), a loader (warp 8:
@@ -348,7 +359,7 @@ constexpr int SCAN_CHAIN_THREADS = 320;
 // the chain at a named barrier, so the chain threads never wait on an mbarrier) and a forwarder
 // (warp 9: refills the ring slot the chain has finished with, copies x and the chunk-start d of
 // each chunk into rank 1's shared memory and arrives on rank 1's barrier, release / acquire at
-// cluster scope); rank 1 runs the k~ token pass (warps 4-7) and its own loads (warp 8: k tiles,
+// cluster scope); rank 1 runs the k~ token pass (warps 0-7) and its own loads (warp 8: k tiles,
 // r).  The token pass gets an SM of its own.  Rank 1's writers copy x out and arrive back on
 // rank 0 before their token pass.  The two CTAs of a cluster are co-scheduled, so these
 // cross-CTA waits are safe (and bounded like every other).  td_in is the k~ buffer holding the
@@ -381,14 +392,16 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     const int64_t dbase = ((int64_t)n * H + h) * DK;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
-    uint64_t* full = bars;         // [3] TMA: k tile (+ T_d tile on rank 0)
-    uint64_t* vready = bars + 3;   // [3] rank 1: r of the chunk (32 arrivals)
-    uint64_t* kempty = bars + 6;   // [3] rank 1: slot released by the chunk's writer group (64)
-    uint64_t* xready = bars + 9;   // [3] rank 1: x and d of a chunk, from rank 0's forwarder (32)
-    uint64_t* outdone = bars + 12; // [3] rank 0: rank 1's writer group has copied x / d (64)
-    uint64_t* fwdin = bars + 15;   // [3] rank 0: x and d of a chunk in local memory, the chain
+    uint64_t* full = bars;         // [5] TMA: k tile (+ T_d tile on rank 0, whose ring has 3 slots)
+    uint64_t* vready = bars + 5;   // [5] rank 1: r of the chunk (32 arrivals)
+    uint64_t* kempty = bars + 10;  // [5] rank 1: slot released by the chunk's writer group (64)
+    // x and d cross to rank 1 through NG receive slots: a writer group is at most NG chunks
+    // ahead of the forwarder, so a slot's barrier is never waited on two phases early
+    uint64_t* xready = bars + 15;  // [NG] rank 1: x and d of a chunk, from rank 0's forwarder (32)
+    uint64_t* outdone = bars + 19; // [NG] rank 0: rank 1's writer group has copied x / d (64)
+    uint64_t* fwdin = bars + 23;   // [3] rank 0: x and d of a chunk in local memory, the chain
                                    //     done with the slot (256)
-    uint64_t* fwdout = bars + 18;  // [3] rank 0: the forwarder has sent them (32)
+    uint64_t* fwdout = bars + 26;  // [3] rank 0: the forwarder has sent them (32)
     float* sD = reinterpret_cast<float*>(smem + L::D);
     float* sX = reinterpret_cast<float*>(smem + L::X);
     float* sGX = reinterpret_cast<float*>(smem + L::GX);
@@ -400,12 +413,16 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     };
 
     if (tid == 0) {
-        for (int s = 0; s < 3; ++s) {
+        for (int s = 0; s < L::NS1; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&vready[s], 32);
             mbar_init(&kempty[s], 64);
+        }
+        for (int s = 0; s < L::NG; ++s) {
             mbar_init(&xready[s], 32);
             mbar_init(&outdone[s], 64);
+        }
+        for (int s = 0; s < 3; ++s) {
             mbar_init(&fwdin[s], 256);
             mbar_init(&fwdout[s], 32);
         }
@@ -416,39 +433,40 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     tc::fence_before_sync();
     tc::cluster_sync();  // both CTAs initialised before either touches the other
     // rank 0's view of rank 1's x / d buffers and barriers, and rank 1's of rank 0's
-    const uint32_t peer_x = tc::cluster_map(smem_u32(smem + L::X), 1u);
-    const uint32_t peer_d = tc::cluster_map(smem_u32(smem + L::D), 1u);
+    const uint32_t peer_x = tc::cluster_map(smem_u32(smem + L::XR), 1u);
+    const uint32_t peer_d = tc::cluster_map(smem_u32(smem + L::DR), 1u);
     const uint32_t peer_xready = tc::cluster_map(smem_u32(xready), 1u);
     const uint32_t peer_outdone = tc::cluster_map(smem_u32(outdone), 0u);
 
     if (warp == 8 && rank == 1) {
         // =============================================== rank 1: k tiles and r for the token pass
         if (lane == 0) tc::prefetch_tmap(&tm_k);
+        constexpr int NS = L::NS1;
         int last_issued = -1;
         bool fail = false;
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c % 3;
-            if (c >= 3 && !mbar_wait_bounded(&kempty[s], (uint32_t)(c / 3 - 1) & 1u, limit_ns)) {
+            const int s = c % NS;
+            if (c >= NS && !mbar_wait_bounded(&kempty[s], (uint32_t)(c / NS - 1) & 1u, limit_ns)) {
                 fail = true;
                 break;
             }
             const int64_t row0 = first + (int64_t)c * C;
             if (lane == 0) {
-                uint8_t* kt = smem + L::KT + s * 16384;
+                uint8_t* kt = smem + L::KT1 + s * 16384;
                 tc::mbar_expect_tx(&full[s], 16384);
                 tc::tma_load_3d(kt, &tm_k, 0, h, (int)row0, &full[s]);
                 tc::tma_load_3d(kt + 8192, &tm_k, 64, h, (int)row0, &full[s]);
             }
             last_issued = c;
             const int Lc = chunk_len(c), t0 = 2 * lane;
-            float* vv = vecs(s);
-            vv[128 + t0] = (r && t0 < Lc) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
-            vv[128 + t0 + 1] = (r && t0 + 1 < Lc) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
+            float* rv = reinterpret_cast<float*>(smem + L::RV + s * 256);
+            rv[t0] = (r && t0 < Lc) ? __ldg(r + (row0 + t0) * H + h) : 1.f;
+            rv[t0 + 1] = (r && t0 + 1 < Lc) ? __ldg(r + (row0 + t0 + 1) * H + h) : 1.f;
             mbar_arrive(&vready[s]);
         }
         if (fail && lane == 0 && last_issued >= 0) {  // let the loads in flight land
-            for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
-                mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
+            for (int c = last_issued > NS - 1 ? last_issued - (NS - 1) : 0; c <= last_issued; ++c)
+                mbar_wait_bounded(&full[c % NS], (uint32_t)(c / NS) & 1u, limit_ns);
         }
     } else if (warp == 8) {
         // =============================================== rank 0: the chain's per-chunk inputs
@@ -634,9 +652,9 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     } else if (warp == 9 && rank == 0) {
         // =============================================== forwarder: x_c, d_c to rank 1; refills
         // Once the chain is done with chunk c (fwdin): the refill of its ring slot with chunk
-        // c + 3; then chunk c's x and chunk-start d go into slot c % 3 of rank 1's buffers once
-        // rank 1's writer of chunk c - 3 has copied that slot out; the slot's local copies may
-        // then be overwritten by the chain (fwdout).
+        // c + 3; then chunk c's x and chunk-start d go into receive slot c % NG of rank 1 once
+        // rank 1's writer of chunk c - NG has copied that slot out; the chain may then overwrite
+        // its local copies (fwdout).
         int last_issued = -1;
         auto issue = [&](int c) {
             const int s = c % 3;
@@ -660,20 +678,22 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             bool got = mbar_wait_bounded(&fwdin[k], (uint32_t)(c / 3) & 1u, limit_ns);
             if (__any_sync(0xffffffffu, !got)) break;
             if (c + 3 < nchunks) issue(c + 3);
-            if (c >= 3) got = tc::mbar_wait_cluster(&outdone[k], (uint32_t)(c / 3 - 1) & 1u, limit_ns);
+            const int m = c % L::NG;  // rank 1's receive slot
+            if (c >= L::NG)
+                got = tc::mbar_wait_cluster(&outdone[m], (uint32_t)(c / L::NG - 1) & 1u, limit_ns);
             if (__any_sync(0xffffffffu, !got)) break;
             {
                 const float2 xv = *reinterpret_cast<const float2*>(sX + k * 64 + 2 * lane);
-                tc::st_cluster_v2f32(peer_x + 4u * (uint32_t)(k * 64 + 2 * lane), xv.x, xv.y);
+                tc::st_cluster_v2f32(peer_x + 4u * (uint32_t)(m * 64 + 2 * lane), xv.x, xv.y);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int e = 2 * lane + 64 * q;
                     const float2 dv = *reinterpret_cast<const float2*>(sD + k * 128 + e);
-                    tc::st_cluster_v2f32(peer_d + 4u * (uint32_t)(k * 128 + e), dv.x, dv.y);
+                    tc::st_cluster_v2f32(peer_d + 4u * (uint32_t)(m * 128 + e), dv.x, dv.y);
                 }
             }
             mbar_arrive(&fwdout[k]);                                // local copies are free
-            tc::mbar_arrive_cluster(peer_xready + 8u * (uint32_t)k);  // rank 1 may read them
+            tc::mbar_arrive_cluster(peer_xready + 8u * (uint32_t)m);  // rank 1 may read them
         }
         // let the copies in flight land (the last one issued into each slot): on the normal
         // path the loader has waited for all of them already
@@ -681,35 +701,40 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             for (int c = last_issued > 2 ? last_issued - 2 : 0; c <= last_issued; ++c)
                 mbar_wait_bounded(&full[c % 3], (uint32_t)(c / 3) & 1u, limit_ns);
         }
-    } else if (warp >= 4 && warp < 8 && rank == 1) {
+    } else if (warp < 8 && rank == 1) {
         // =============================================== k~ = d (.) k, token by token
-        // Two groups of 64 threads take alternate chunks (group g: chunks c = g, g + 2, ...), so
-        // each has two chunk periods for its token pass; a thread carries the key-channel pair
-        // (2 jj, 2 jj + 1): packed bf16x2 conversions and 4-byte stores, two independent chains.
-        const int i = tid - 128, g = i >> 6, jj = i & 63;
+        // Four groups of 64 threads take every fourth chunk (group g: chunks c = g, g + 4, ...),
+        // so each has four chunk periods for its token pass and stores; a thread carries the
+        // key-channel pair (2 jj, 2 jj + 1): packed bf16x2 conversions and 4-byte stores.
+        constexpr int NS = L::NS1, NG = L::NG;
+        const int i = tid, g = i >> 6, jj = i & 63;
         const int blk = jj >> 5, cj = (jj & 31) >> 2, ce = 2 * (jj & 3);  // channel 2 jj in the tile
         const int gbar = 2 + g;  // the group's named barrier
         uint8_t* lo_stage = smem + L::LO + g * 16384;
-        for (int c = g; c < nchunks; c += 2) {
-            const int s = c % 3;
-            const uint32_t ph = (uint32_t)(c / 3) & 1u;
-            const bool got = mbar_wait_bounded(&full[s], ph, limit_ns) &&
+        for (int c = g; c < nchunks; c += NG) {
+            const int s = c % NS;
+            const uint32_t ph = (uint32_t)(c / NS) & 1u;
+            // the slot's previous chunk (another group's) released first: then its full and vready
+            // barriers are at most one phase behind this chunk, and the parity waits are exact
+            const bool got = (c < NS || mbar_wait_bounded(&kempty[s], (uint32_t)(c / NS - 1) & 1u, limit_ns)) &&
+                             mbar_wait_bounded(&full[s], ph, limit_ns) &&
                              mbar_wait_bounded(&vready[s], ph, limit_ns) &&
-                             tc::mbar_wait_cluster(&xready[c % 3], ph, limit_ns);
+                             tc::mbar_wait_cluster(&xready[c % NG], (uint32_t)(c / NG) & 1u, limit_ns);
             if (group_any(gbar, 64, !got)) break;
             const int Lc = chunk_len(c);
-            const uint8_t* col = smem + L::KT + s * 16384 + blk * 8192u + ce * 2;
+            const uint8_t* col = smem + L::KT1 + s * 16384 + blk * 8192u + ce * 2;
             // copy x and this pair's d out of the slot rank 0's forwarder fills, and free it
             float* xv = reinterpret_cast<float*>(smem + L::XW + g * 256);
-            xv[jj] = sX[(c % 3) * 64 + jj];
-            float2 dd = *reinterpret_cast<const float2*>(sD + (c % 3) * 128 + 2 * jj);
+            const int m = c % NG;  // the receive slot rank 0's forwarder filled
+            xv[jj] = reinterpret_cast<const float*>(smem + L::XR)[m * 64 + jj];
+            float2 dd = reinterpret_cast<const float2*>(smem + L::DR)[m * 64 + jj];
             group_bar(gbar, 64);
-            tc::mbar_arrive_cluster(peer_outdone + 8u * (uint32_t)(c % 3));
-            const float* rv = vecs(s) + 128;
-            // k~ goes to the chunk's T_d slot (consumed by step 2 before x was published) in the
-            // key tile's swizzled layout, then to global memory as whole 16-byte row pieces:
-            // scattered 2-byte stores would cost about three times the whole token pass
-            uint8_t* stage = smem + L::TD + s * 16384;
+            tc::mbar_arrive_cluster(peer_outdone + 8u * (uint32_t)m);
+            const float* rv = reinterpret_cast<const float*>(smem + L::RV + s * 256);
+            // k~ goes to the group's staging tiles in the key tile's swizzled layout, then to
+            // global memory as whole tiles or 16-byte row pieces: scattered 2-byte stores would
+            // cost about three times the whole token pass
+            uint8_t* stage = smem + L::HI + g * 16384;
             uint8_t* ocol = stage + blk * 8192u + ce * 2;
             uint8_t* lcol = lo_stage + blk * 8192u + ce * 2;
             float* drow = kD ? d_all + ((first + (int64_t)c * C) * H + h) * DK + 2 * jj : nullptr;
