@@ -446,6 +446,39 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// E consecutive values of a row (E = 4 or 2, starting at a multiple of E) as one 16- or 8-byte
+// shared-memory access: lane-strided scalar accesses would meet each bank E times.
+template <int E>
+__device__ __forceinline__ void row_ld(const float* p, float* x) {
+    if constexpr (E == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+        const float2 v = *reinterpret_cast<const float2*>(p);
+        x[0] = v.x; x[1] = v.y;
+    }
+}
+template <int E>
+__device__ __forceinline__ void row_st(float* p, const float* x) {
+    if constexpr (E == 4) *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    else *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+}
+template <int E, typename IO>
+__device__ __forceinline__ void row_ld_io(const IO* p, float* x) {
+    if constexpr (sizeof(IO) == 4) {
+        row_ld<E>(reinterpret_cast<const float*>(p), x);
+    } else if constexpr (E == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    } else {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+        x[0] = a.x; x[1] = a.y;
+    }
+}
+
 template <int DK, typename IO>
 __global__ void __launch_bounds__(128)
 bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
@@ -456,7 +489,6 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
                    float* __restrict__ dd0, float* __restrict__ deta_part,
                    const int32_t* __restrict__ cu, int N, int T, int H) {
     using L = BwdPrecondSmem<DK, IO>;
-    using tr = io_traits<IO>;
     constexpr int C = BWD_C, E = DK / 32;
     extern __shared__ float4 bwdp_smem4[];
     float* sm = reinterpret_cast<float*>(bwdp_smem4);
@@ -510,12 +542,15 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
 #pragma unroll 2
         for (int t = warp - 1; t < Lc; t += 3) {
             const IO* krow = reinterpret_cast<const IO*>(buf + L::K + t * L::KB);
+            float kk[E], dv[E];
+            row_ld_io<E>(krow + lane * E, kk);
+            row_ld<E>(buf + L::D + t * DK + lane * E, dv);
             float nk = 0.f, sv = 0.f;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const float kk = tr::to_f32(krow[lane * E + e]), a = kk * kk;
+                const float a = kk[e] * kk[e];
                 nk += a;
-                sv = fmaf(buf[L::D + t * DK + lane * E + e], a, sv);
+                sv = fmaf(dv[e], a, sv);
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
@@ -547,15 +582,17 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
             const float y = sy[t], bt = buf[L::SC + t], inv = buf[L::SC + 3 * C + t];
             const float xt = buf[L::SC + 4 * C + t];
             const int64_t th = (row0 + t) * H + h;
-            float rd = 0.f, g[E];
+            float rd = 0.f, g[E], ddv[E], dv[E], kk[E], dk2[E], dkt[E];
+            row_ld<E>(sdd + t * DK + lane * E, ddv);
+            row_ld<E>(buf + L::D + t * DK + lane * E, dv);
+            row_ld_io<E>(krow + lane * E, kk);
+            row_ld<E>(buf + L::DK2 + t * DK + lane * E, dk2);
+            row_ld<E>(buf + L::DKT + t * DK + lane * E, dkt);
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const int c = lane * E + e;
-                const float ddv = sdd[t * DK + c], dv = buf[L::D + t * DK + c];
-                const float kk = tr::to_f32(krow[c]);
-                rd = fmaf(ddv, dv, rd);
-                const float da = inv > 0.f ? eta * xt * ddv - eta * y * (bt * bt * dv + xt) * inv : 0.f;
-                g[e] = buf[L::DK2 + t * DK + c] + buf[L::DKT + t * DK + c] * dv + 2.f * kk * da;
+                rd = fmaf(ddv[e], dv[e], rd);
+                const float da = inv > 0.f ? eta * xt * ddv[e] - eta * y * (bt * bt * dv[e] + xt) * inv : 0.f;
+                g[e] = dk2[e] + dkt[e] * dv[e] + 2.f * kk[e] * da;
             }
             if constexpr (E == 4) {
                 *reinterpret_cast<float4*>(dk + th * DK + lane * E) = make_float4(g[0], g[1], g[2], g[3]);
@@ -589,14 +626,14 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
             for (int t = chunk_len(ch) - 1; t >= 0; --t) {
                 const IO* krow = reinterpret_cast<const IO*>(buf + L::K + t * L::KB);
                 float a[E], kk[E], dkt[E];
+                row_ld_io<E>(krow + lane * E, kk);
+                row_ld<E>(buf + L::DKT + t * DK + lane * E, dkt);
+                row_st<E>(sdd + t * DK + lane * E, dd);  // dd_{t+1}
                 float y = 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
-                    kk[e] = tr::to_f32(krow[lane * E + e]);
-                    dkt[e] = buf[L::DKT + t * DK + lane * E + e];
                     a[e] = kk[e] * kk[e];
                     y = fmaf(a[e], dd[e], y);
-                    sdd[t * DK + lane * E + e] = dd[e];  // dd_{t+1}
                 }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
