@@ -44,6 +44,9 @@ namespace osdn {
 constexpr int BWD_BV = 64;      // value rows per bwd_delta_kernel CTA
 constexpr int BWD_C = 32;       // tokens per chunk (state checkpoints, chunk algebra)
 constexpr int BWD_THREADS = 256;
+// Per chunk and value tile, the forward sweep keeps A = K K~^T, T, E = V - K S_c^T and W for the
+// reverse sweep: C x C + C x C + C x BV + C x BV floats.
+constexpr int BWD_FW = 2 * BWD_C * BWD_C + 2 * BWD_C * BWD_BV;
 
 template <int DK>
 struct BwdSmem {
@@ -171,7 +174,7 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
                  const float* __restrict__ beta, const float* __restrict__ dall,
                  const float* __restrict__ S0, float scale, const IO* __restrict__ dO,
                  const float* __restrict__ dST, float* __restrict__ dv, float* __restrict__ dS0,
-                 float* __restrict__ ws_state, float* __restrict__ dq_part,
+                 float* __restrict__ ws_state, float* __restrict__ ws_fw, float* __restrict__ dq_part,
                  float* __restrict__ dk_part, float* __restrict__ dkt_part,
                  float* __restrict__ dbeta_part, const int32_t* __restrict__ cu, int N, int T,
                  int H, int Dv, int64_t rows) {
@@ -291,6 +294,27 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         __syncthreads();
         bwd_gemm<GEMM_NN, 2, 4>(C, BV, C, sT, CS, sR, VS, sW, VS, 1.f, false);
     };
+    // the forward sweep's A, T, E, W of chunk ch <-> the workspace (dense rows)
+    auto fw_of = [&](int ch) {
+        return ws_fw + ((bwd_slot(first, ch, n) * H + h) * ntile + vt) * (int64_t)BWD_FW;
+    };
+    auto fw_move = [&](int ch, bool store) {
+        float* g = fw_of(ch);
+        float* const src[4] = {sA, sT, sV, sW};
+        const int ld[4] = {CS, CS, VS, VS}, w4[4] = {C / 4, C / 4, BV / 4, BV / 4};
+        int base = 0;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            for (int idx = tid; idx < C * w4[m]; idx += NT) {
+                const int t = idx / w4[m], c = 4 * (idx - t * w4[m]);
+                float4* gp = reinterpret_cast<float4*>(g + base + t * 4 * w4[m] + c);
+                float4* sp = reinterpret_cast<float4*>(src[m] + t * ld[m] + c);
+                if (store) *gp = *sp;
+                else *sp = *gp;
+            }
+            base += C * 4 * w4[m];
+        }
+    };
     auto store_share = [&](float* dst, int ch, int Lc) {  // sO rows t < Lc -> a [rows, H, DK] share
         const int64_t row0 = first + (int64_t)ch * C;
 #pragma unroll
@@ -314,6 +338,7 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         __syncthreads();
         wy();
         __syncthreads();
+        fw_move(ch, true);                                                            // keep A, T, E, W
         bwd_gemm<GEMM_TN, 4, TNK>(BV, DK, C, sW, VS, sKt, KS, sS, KS, 1.f, true);     // S += W^T K~
     }
 
@@ -325,12 +350,14 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         const int Lc = load_chunk(ch, true);
         const int64_t row0 = first + (int64_t)ch * C;
         __syncthreads();
-        bwd_gemm<GEMM_NT, 2, 2>(C, C, DK, sK, KS, sKt, KS, sA, CS, 1.f, false);       // A = K K~^T
+        fw_move(ch, false);                                    // A, T, E (over V), W from the forward sweep
         bwd_gemm<GEMM_NT, 2, 2>(C, C, DK, sQ, KS, sKt, KS, sP, CS, 1.f, false, 1);    // P = tril(Q K~^T)
-        bwd_gemm<GEMM_NT, 2, 4>(C, BV, DK, sK, KS, sS, KS, sV, VS, -1.f, true);       // E = V - K S_c^T
         bwd_gemm<GEMM_NT, 2, 4>(C, BV, DK, sKt, KS, sdS, KS, sdW, VS, 1.f, false);    // dW = K~ dS'^T
         __syncthreads();
-        wy();                                                                         // T, R, W
+        for (int idx = tid; idx < C * BV; idx += NT) {                                // R = beta E
+            const int t = idx / BV, r = idx - t * BV;
+            sR[t * VS + r] = sB[t] * sV[t * VS + r];
+        }
         __syncthreads();
         bwd_gemm<GEMM_TN, 2, 4>(C, BV, C, sP, CS, sG, VS, sdW, VS, scale, true);      // dW += s P^T dO
         bwd_gemm<GEMM_NT, 2, 2>(C, C, BV, sG, VS, sW, VS, sdP, CS, scale, false, 1);  // dP = tril(s dO W^T)

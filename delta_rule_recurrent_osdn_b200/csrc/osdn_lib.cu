@@ -617,7 +617,7 @@ namespace {
 // the state checkpoints (every BWD_C tokens), the per-value-tile shares of dq, dk, dk~ and dbeta,
 // and deta per (sequence, head).
 struct BwdWorkspace {
-    size_t kt, dall, state, dq, dk, dkt, dbeta, deta, total;
+    size_t kt, dall, state, fw, dq, dk, dkt, dbeta, deta, total;
 };
 
 inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -632,8 +632,11 @@ BwdWorkspace bwd_workspace(int64_t rows, int64_t N, int32_t H, int32_t Dk, int32
     off += up256((size_t)th * Dk * io_size(io));
     w.dall = off;
     off += up256((size_t)th * Dk * 4);
+    const size_t slots = (size_t)((rows + BWD_C - 1) / BWD_C + N + 1);
     w.state = off;
-    off += up256((size_t)((rows + BWD_C - 1) / BWD_C + N + 1) * H * Dv * Dk * 4);
+    off += up256(slots * H * Dv * Dk * 4);
+    w.fw = off;
+    off += up256(slots * H * ntile * BWD_FW * 4);
     w.dq = off;
     off += up256((size_t)ntile * th * Dk * 4);
     w.dk = off;
@@ -670,7 +673,8 @@ osdn_status_t launch_bwd_kernels(const void* q, const void* k, const void* v, co
         kern<<<dim3((unsigned)(units * ntile)), dim3(BWD_THREADS), BwdSmem<DK>::bytes, stream>>>(
             static_cast<const IO*>(q), static_cast<const IO*>(k), static_cast<const IO*>(v), beta,
             dall, S0, scale, static_cast<const IO*>(dO), dST, dv, dS0,
-            reinterpret_cast<float*>(ws + w.state), dq_part, dk_part, dkt_part, db_part, cu, d.N,
+            reinterpret_cast<float*>(ws + w.state), reinterpret_cast<float*>(ws + w.fw), dq_part,
+            dk_part, dkt_part, db_part, cu, d.N,
             d.T, d.H, d.Dv, rows);
         const osdn_status_t st = launch_status();
         if (st != OSDN_OK) return st;

@@ -208,8 +208,8 @@ OSDN_API osdn_status_t osdn_fwd_noalloc(const void* q, const void* k, const void
  *   deta    one float32, written (dL/deta), or NULL to skip.
  *   dS0     [N,H,Dv,Dk] float32, written, or NULL.   dd0 [N,H,Dk] float32, written, or NULL.
  *   workspace  device scratch of at least osdn_bwd_workspace_bytes(...) bytes, 256-byte aligned
- *           (about (4 + 3 Dv/64) x 4 B per key channel and token-head, plus one Dv x Dk fp32 state
- *           per 32 tokens and head).
+ *           (about (4 + 3 Dv/64) x 4 B per key channel and token-head, plus, per 32 tokens and
+ *           head, one Dv x Dk fp32 state and 24 KB per 64 value channels of chunk factors).
  * cu_seqlens, num_seqs, B, T, H as for the forward pass; Dk, Dv in {64, 128}.  Outputs must not
  * overlap one another, the inputs or the workspace (OSDN_ERR_INVALID_ARG).
  */
