@@ -91,7 +91,7 @@ def profile_record(name):
 
 
 def fwd_algorithmic_bytes(inp, es=2):
-    """Bytes the forward pass must move: q, k, v in and o out in the io
+    """Bytes the forward pass must move (the roofline's algorithmic bytes): q, k, v in and o out in the io
     dtype, beta (and r with APF) in fp32 per token-head; per (sequence, head) the final state
     S_T and d_T out in fp32, and S_0, d_0 in when given.  k~ is an intermediate, not counted."""
     th = inp.B * inp.T * inp.H
@@ -101,7 +101,7 @@ def fwd_algorithmic_bytes(inp, es=2):
 
 
 def fwd_flops(inp):
-    """Chunk-form MMA FLOPs: 5 * 2 * C * d + 3 * 2 * d_k * d_v per
+    """Chunk-form MMA FLOPs (the roofline's algorithmic tensor work): 5 * 2 * C * d + 3 * 2 * d_k * d_v per
     token-head."""
     return inp.B * inp.T * inp.H * (5 * 2 * inp.chunk * inp.Dk + 3 * 2 * inp.Dk * inp.Dv)
 

@@ -320,7 +320,7 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
 #pragma unroll
         for (int it = 0; it < C * DK / 4 / NT; ++it) {
             const int idx = tid + it * NT, t = idx / (DK / 4), c = 4 * (idx - t * (DK / 4));
-            if (t < Lc)
+            if (t < Lc && OSDN_IN_BOUNDS(row0 + t, rows))
                 *reinterpret_cast<float4*>(dst + (((int64_t)vt * rows + row0 + t) * H + h) * DK + c) =
                     *reinterpret_cast<const float4*>(sO + t * KS + c);
         }
@@ -330,7 +330,8 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
     tile_in(sS, S0 ? S0 + sbase : nullptr);
     for (int ch = 0; ch < nchunks; ++ch) {
         __syncthreads();  // the state rows are settled; the chunk buffers are free
-        tile_out(ws_state + (bwd_slot(first, ch, n) * H + h) * (int64_t)Dv * DK + (int64_t)c0 * DK, sS);
+        if (OSDN_IN_BOUNDS(bwd_slot(first, ch, n), (rows + C - 1) / C + N + 1))  // block-uniform
+            tile_out(ws_state + (bwd_slot(first, ch, n) * H + h) * (int64_t)Dv * DK + (int64_t)c0 * DK, sS);
         load_chunk(ch, false);
         __syncthreads();
         bwd_gemm<GEMM_NT, 2, 2>(C, C, DK, sK, KS, sKt, KS, sA, CS, 1.f, false);       // A = K K~^T
@@ -338,7 +339,8 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
         __syncthreads();
         wy();
         __syncthreads();
-        fw_move(ch, true);                                                            // keep A, T, E, W
+        if (OSDN_IN_BOUNDS(bwd_slot(first, ch, n), (rows + C - 1) / C + N + 1))
+            fw_move(ch, true);                                                        // keep A, T, E, W
         bwd_gemm<GEMM_TN, 4, TNK>(BV, DK, C, sW, VS, sKt, KS, sS, KS, 1.f, true);     // S += W^T K~
     }
 
@@ -372,7 +374,7 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
             const int t = idx / BV, r = idx - t * BV;
             const float x = sB[t] * sdR[t * VS + r];
             sdRb[t * VS + r] = x;
-            if (t < Lc) dv[((row0 + t) * H + h) * Dv + c0 + r] = x;
+            if (t < Lc && OSDN_IN_BOUNDS(row0 + t, rows)) dv[((row0 + t) * H + h) * Dv + c0 + r] = x;
         }
         __syncthreads();
         store_share(dq_part, ch, Lc);
@@ -383,7 +385,7 @@ bwd_delta_kernel(const IO* __restrict__ q, const IO* __restrict__ k, const IO* _
             float acc = 0.f;
             for (int j = 0; j < t; ++j) acc = fmaf(sM[t * CS + j], sA[t * CS + j], acc);
             for (int r = 0; r < BV; ++r) acc = fmaf(sdR[t * VS + r], sV[t * VS + r], acc);
-            if (t < Lc) dbeta_part[((int64_t)vt * rows + row0 + t) * H + h] = acc;
+            if (t < Lc && OSDN_IN_BOUNDS(row0 + t, rows)) dbeta_part[((int64_t)vt * rows + row0 + t) * H + h] = acc;
         }
         for (int idx = tid; idx < C * C; idx += NT) {                                 // beta dL
             const int t = idx / C, j = idx - t * C;
@@ -609,6 +611,7 @@ bwd_precond_kernel(const IO* __restrict__ k, const float* __restrict__ beta,
             const float y = sy[t], bt = buf[L::SC + t], inv = buf[L::SC + 3 * C + t];
             const float xt = buf[L::SC + 4 * C + t];
             const int64_t th = (row0 + t) * H + h;
+            if (!OSDN_IN_BOUNDS(row0 + t, cu ? (int64_t)T : (int64_t)N * T)) continue;  // warp-uniform
             float rd = 0.f, g[E], ddv[E], dv[E], kk[E], dk2[E], dkt[E];
             row_ld<E>(sdd + t * DK + lane * E, ddv);
             row_ld<E>(buf + L::D + t * DK + lane * E, dv);

@@ -177,7 +177,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
         //      its 16-byte groups), into the chunk's o rows
         {
             const int r = tid & 63, g0 = 4 * (tid >> 6);
-            if (r < Lc) {
+            if (r < Lc && OSDN_IN_BOUNDS(row0 + r, rows)) {
                 uint8_t* orow = reinterpret_cast<uint8_t*>(o_f32 + ((row0 + r) * H + h) * half_f);
 #pragma unroll
                 for (int g = g0; g < g0 + 4; ++g) {

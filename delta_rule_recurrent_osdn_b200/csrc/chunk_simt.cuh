@@ -254,8 +254,9 @@ chunk_fwd_simt_kernel(const IO* __restrict__ q, const IO* __restrict__ k,
                     a0 = fmaf(pj, sW[j * BV + c], a0);
                     a1 = fmaf(pj, sW[j * BV + c + 1], a1);
                 }
-                store2<IO>(o + ((first + cs + t) * H + h) * DV + c0 + c,
-                           make_float2(scale * a0, scale * a1));
+                if (OSDN_IN_BOUNDS(first + cs + t, cu ? (int64_t)T : (int64_t)N * T))
+                    store2<IO>(o + ((first + cs + t) * H + h) * DV + c0 + c,
+                               make_float2(scale * a0, scale * a1));
             }
         }
         for (int idx = tid; idx < BV * DK; idx += NT) {

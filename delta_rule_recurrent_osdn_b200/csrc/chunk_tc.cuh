@@ -196,6 +196,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int c0 = vt * BV;
     const int64_t sbase = ((int64_t)n * H + h) * DV * DK + (int64_t)c0 * DK;
     const int nchunks = (int)((count + C - 1) / C);
+    [[maybe_unused]] const int64_t rows_all = cu ? (int64_t)T : (int64_t)N * T;  // debug-bounds checks
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* tma_full = bars + 0;     // [2] ring stage landed
@@ -583,7 +584,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::fence_after_sync();
                 float x[64];
                 tmem_ld64_sum(tmem + lane + TC_COL_D1 + 128 * ((j + 1) & 1), x);
-                if (r < chunk_len(j)) {
+                if (r < chunk_len(j) && OSDN_IN_BOUNDS(first + (int64_t)j * C + r, rows_all)) {
                     __nv_bfloat16* orow = o + ((first + (int64_t)j * C + r) * H + h) * DV + c0;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
@@ -609,7 +610,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float s1[64];
             tc::tmem_ld64(t_S, s1);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) ST[sbase + (int64_t)c * DK + t] = s1[c];
+            for (int c = 0; c < 64; ++c)
+                if (OSDN_IN_BOUNDS(sbase + (int64_t)c * DK + t, (int64_t)N * H * DV * DK))
+                    ST[sbase + (int64_t)c * DK + t] = s1[c];
         }
         if (!ok && lower && leader && last_bar) mbar_wait_bounded(last_bar, last_par, limit_ns);
     }

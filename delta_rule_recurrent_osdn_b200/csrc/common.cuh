@@ -17,6 +17,21 @@ __device__ __forceinline__ void record_status(int code) {
     atomicCAS(&g_device_status, 0, code);
 }
 
+// Debug-bounds builds (compiled with -DOSDN_DEBUG_BOUNDS; `build.py --debug-bounds` writes
+// libosdn_debug.so): the kernels' computed global stores check their index against the extent
+// of the buffer they write; a violation records OSDN_ERR_DEVICE_BOUNDS and skips the store
+// instead of writing outside the buffer.  Release builds compile the checks out.
+#ifdef OSDN_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(int64_t i, int64_t n) {
+    if (i >= 0 && i < n) return true;
+    record_status(OSDN_ERR_DEVICE_BOUNDS);
+    return false;
+}
+#define OSDN_IN_BOUNDS(idx, extent) (::osdn::bounds_ok((int64_t)(idx), (int64_t)(extent)))
+#else
+#define OSDN_IN_BOUNDS(idx, extent) true
+#endif
+
 // Token range of sequence n: fixed length (cu == nullptr) or packed (device offsets).
 // Returns false, after recording OSDN_ERR_DEVICE_BOUNDS, when the offsets are unusable.
 __device__ __forceinline__ bool seq_range(const int32_t* __restrict__ cu, int n, int N, int T,

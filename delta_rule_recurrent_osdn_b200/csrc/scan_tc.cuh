@@ -306,7 +306,7 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
             const int idx = it * 128 + tid, t = idx >> 4, piece = idx & 15;
-            if (t < Lc)
+            if (t < Lc && OSDN_IN_BOUNDS(row0 + t, rows))
                 reinterpret_cast<float4*>(td_out + ((row0 + t) * H + h) * 64)[piece] =
                     reinterpret_cast<const float4*>(sL + t * 64)[piece];
         }
@@ -390,6 +390,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
     if (!seq_range(cu, n, N, T, first, count)) return;  // uniform over the cluster
     const int nchunks = (int)((count + C - 1) / C);
     const int64_t dbase = ((int64_t)n * H + h) * DK;
+    [[maybe_unused]] const int64_t rows_all = cu ? (int64_t)T : (int64_t)N * T;  // debug-bounds checks
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR);
     uint64_t* full = bars;         // [5] TMA: k tile (+ T_d tile on rank 0, whose ring has 3 slots)
@@ -613,7 +614,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                     sGX[t] = g_t * x;
                     // residual-contraction ratio (1 - beta s)^2: x = e (1 - beta s) when e != 0;
                     // else d_t = R_t d_0 on this token's row, so beta s = beta R p
-                    if (rho && t < Lc) {
+                    if (rho && t < Lc && OSDN_IN_BOUNDS(first + (int64_t)c * C + t, rows_all)) {
                         const float gr = e_t != 0.f ? x / e_t : 1.f - bRp;
                         rho[(first + (int64_t)c * C + t) * H + h] = gr * gr;
                     }
@@ -648,7 +649,8 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             mbar_arrive(&fwdin[c % 3]);
         }
         group_bar(5, 256);  // the last chunk's d is complete
-        if (ok && dT && u < DK) dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
+        if (ok && dT && u < DK && OSDN_IN_BOUNDS(dbase + u, (int64_t)N * H * DK))
+            dT[dbase + u] = sD[(nchunks % 3) * 128 + u];
     } else if (warp == 9 && rank == 0) {
         // =============================================== forwarder: x_c, d_c to rank 1; refills
         // Once the chain is done with chunk c (fwdin): the refill of its ring slot with chunk
@@ -751,7 +753,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
                 }
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    if (kD && t0 + u < Lc)
+                    if (kD && t0 + u < Lc && OSDN_IN_BOUNDS(first + (int64_t)c * C + t0 + u, rows_all))
                         *reinterpret_cast<float2*>(drow + (int64_t)(t0 + u) * H * DK) = dd;
                     const float2 kt = __fmul2_rn(dd, kv[u]);
                     const __nv_bfloat162 hb = __floats2bfloat162_rn(kt.x, kt.y);
@@ -771,7 +773,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
             if (bulk) tc::fence_async_smem();
             group_bar(gbar, 64);
             if (bulk) {
-                if (jj == 0) {
+                if (jj == 0 && OSDN_IN_BOUNDS(first + (int64_t)c * C + C - 1, rows_all)) {
                     const int row0 = (int)(first + (int64_t)c * C);
                     tc::tma_store_3d(&tm_kto, stage, 0, h, row0);
                     tc::tma_store_3d(&tm_kto, stage + 8192, 64, h, row0);
@@ -789,7 +791,7 @@ precond_chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
 #pragma unroll 4
                 for (int q = 0; q < 16; ++q) {
                     const int row = (jj >> 4) + 4 * q;
-                    if (row < Lc) {
+                    if (row < Lc && OSDN_IN_BOUNDS(first + (int64_t)c * C + row, rows_all)) {
                         const uint32_t so = blk16 * 8192u + tc::sw128_off(row, j16);
                         *reinterpret_cast<uint4*>(k_tilde + off + row * rs) =
                             *reinterpret_cast<const uint4*>(stage + so);

@@ -16,7 +16,8 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libosdn.so")
+# OSDN_LIBRARY selects another build of the library (the debug-bounds build, libosdn_debug.so)
+LIB_PATH = os.environ.get("OSDN_LIBRARY") or os.path.join(_PKG, "libosdn.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "osdn.h")
 
 OSDN_OK = 0

@@ -41,6 +41,10 @@
  *     may run concurrently as long as their output buffers do not overlap.
  *   - Argument errors are reported before anything is enqueued and leave outputs untouched.
  *     A failed kernel launch returns OSDN_ERR_CUDA.  No C++ exception crosses this ABI.
+ *   - A debug-bounds build of this library (compiled with -DOSDN_DEBUG_BOUNDS; same symbols,
+ *     same results) also checks every computed row or slot index of the kernels' global
+ *     stores against its buffer's extent; an index outside it skips that store and records
+ *     OSDN_ERR_DEVICE_BOUNDS.  The release build compiles these checks out.
  */
 #ifndef OSDN_H_
 #define OSDN_H_

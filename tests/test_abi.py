@@ -227,3 +227,23 @@ def test_bwd_workspace_size_grows_with_the_batch():
     assert 0 < small < big
     assert big % 256 == 0
     assert L.osdn_bwd_workspace_bytes(0, 1, 64, 2, 96, 128, osdn.OSDN_BF16) == 0
+
+
+def test_debug_bounds_build_exports_the_same_symbols_and_validates_alike():
+    """libosdn_debug.so (-DOSDN_DEBUG_BOUNDS) is the same ABI: it loads, exports every declared
+    symbol and rejects bad arguments on the host with the same status as the release build."""
+    from delta_rule_recurrent_osdn_b200 import build as B
+    lib = ctypes.CDLL(B.build(debug_bounds=True))
+    for n in osdn.header_symbols():
+        assert hasattr(lib, n), n
+    lib.osdn_abi_version.restype = ctypes.c_int
+    assert lib.osdn_abi_version() == L.osdn_abi_version()
+    lib.osdn_fwd_workspace_bytes.restype = ctypes.c_int64
+    lib.osdn_fwd_workspace_bytes.argtypes = L.osdn_fwd_workspace_bytes.argtypes
+    assert lib.osdn_fwd_workspace_bytes(4, 4096, 16, 128, osdn.OSDN_BF16) == \
+        L.osdn_fwd_workspace_bytes(4, 4096, 16, 128, osdn.OSDN_BF16)
+    f = lib.osdn_chunk_fwd
+    f.restype, f.argtypes = L.osdn_chunk_fwd.restype, L.osdn_chunk_fwd.argtypes
+    bad = f(fake(1), fake(2), fake(3), fake(4), fake(5), None, 0, 1.0, None, fake(6), None, None,
+            0, 1, 8, 1, 96, 128, 64, osdn.OSDN_BF16, None)
+    assert bad == osdn.OSDN_ERR_UNSUPPORTED == chunk_call(Dk=96)
