@@ -193,7 +193,8 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__
                         const float b = c + 1 < r ? tv[2 * e + 1] : (c + 1 == r ? 1.f : 0.f);
                         const __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
                         const float2 hf = __bfloat1622float2(hb);
-                        const __nv_bfloat162 lb = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+                        const float2 ld = __ffma2_rn(hf, make_float2(-1.f, -1.f), make_float2(a, b));
+                        const __nv_bfloat162 lb = __floats2bfloat162_rn(ld.x, ld.y);
                         hw[e] = *reinterpret_cast<const uint32_t*>(&hb);
                         lw[e] = *reinterpret_cast<const uint32_t*>(&lb);
                     }

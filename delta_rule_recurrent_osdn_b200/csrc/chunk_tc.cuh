@@ -169,7 +169,11 @@ __device__ __forceinline__ void tmem_ld64_sum(uint32_t taddr, float* x) {
         tc::tmem_ld16(taddr + 80 + 32 * h, t + 16);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[32 * h + c] += t[c];
+        for (int c = 0; c < 32; c += 2) {
+            const float2 s = __fadd2_rn(make_float2(x[32 * h + c], x[32 * h + c + 1]), make_float2(t[c], t[c + 1]));
+            x[32 * h + c] = s.x;
+            x[32 * h + c + 1] = s.y;
+        }
     }
 }
 
@@ -507,6 +511,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 float y[64];  // R = beta (V - K S^T), token row t
                 tmem_ld64_sum(tmem + lane + TC_COL_D1 + 128 * s, y);
                 const uint8_t* vtile = stage(j) + L::V;
+                const float2 bt2 = make_float2(bt, bt), m1 = make_float2(-1.f, -1.f);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const uint4 raw = *reinterpret_cast<const uint4*>(vtile + tc::sw128_off(t, q));
@@ -514,8 +519,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 vv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-                        y[8 * q + 2 * e] = bt * (vv.x - y[8 * q + 2 * e]);
-                        y[8 * q + 2 * e + 1] = bt * (vv.y - y[8 * q + 2 * e + 1]);
+                        // beta (v - y): the fma with -1 rounds v - y once, as a subtraction does
+                        const float2 d = __ffma2_rn(make_float2(y[8 * q + 2 * e], y[8 * q + 2 * e + 1]), m1, vv);
+                        const float2 yy = __fmul2_rn(bt2, d);
+                        y[8 * q + 2 * e] = yy.x;
+                        y[8 * q + 2 * e + 1] = yy.y;
                     }
                 }
                 // W_{j-1} (the R tiles' previous contents) has been read by the state update
@@ -591,8 +599,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         uint32_t pk[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale * x[8 * q + 2 * e],
-                                                                            scale * x[8 * q + 2 * e + 1]);
+                            const float2 sx = __fmul2_rn(make_float2(scale, scale),
+                                                         make_float2(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]));
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(sx.x, sx.y);
                             pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
                         }
                         *reinterpret_cast<uint4*>(orow + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);

@@ -164,17 +164,19 @@ precond_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const float* __res
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t off = blk * 8192u + tc::sw128_off(t, j);
-                const uint4 raw = *reinterpret_cast<const uint4*>(sK + off);
+                uint4 raw = *reinterpret_cast<const uint4*>(sK + off);
+                if (!valid) raw = make_uint4(0u, 0u, 0u, 0u);  // rows past the chunk's end: a = 0
                 const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
                 uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-                    const float a0 = valid ? kk.x * kk.x : 0.f, a1 = valid ? kk.y * kk.y : 0.f;
-                    nk += a0 + a1;
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+                    const float2 a = __fmul2_rn(kk, kk);
+                    nk += a.x + a.y;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(a.x, a.y);
                     const float2 hf = __bfloat1622float2(h2);
-                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+                    const float2 ld = __ffma2_rn(hf, make_float2(-1.f, -1.f), a);  // a - hi, exact
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(ld.x, ld.y);
                     hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
                     lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
                 }
