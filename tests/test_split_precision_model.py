@@ -1,0 +1,116 @@
+"""The precision design of the phase-2 tensor-core chain, emulated on the CPU in fp32.
+
+chunk_fwd_tc_kernel and wy_prep_kernel multiply only bf16 operands and accumulate in fp32.  Every
+operand that is computed on the way (T, R, W, the lookahead's X and P, the state S) is first split
+into two bf16 terms, x = hi + lo with |x - hi - lo| <= 2^-16 |x| (Veltkamp head, truncated
+residual); a product of an exact bf16 operand with a computed one takes both terms (2 MMAs), a
+product of two computed operands three (hi hi + hi lo + lo hi); k~ arrives as its own hi + lo
+terms.  This file runs that arithmetic (the lookahead form, fp32 accumulation of bf16-valued
+operands, an fp32 inverse for T) on the 1.3B-layer workload's first 1024 tokens of two heads and
+compares it with the fp64 oracle:
+  - with the splits, o and S_T stay within 2e-4 of rms, two orders of magnitude inside the 1e-2
+    bound, so the bound is left to the bf16 rounding of the inputs and the output;
+  - with single-term bf16 operands (and k~ rounded to bf16), the same arithmetic misses the bound.
+"""
+import numpy as np
+import pytest
+
+from delta_rule_recurrent_osdn_b200 import inputs as W
+from oracle import osdn_ref
+
+
+def bf16(x):
+    """Round to the nearest bf16 value (ties to even), returned as float32."""
+    b = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32)
+
+
+def split(x):
+    """Two bf16 terms: Veltkamp's 8-bit head and the upper half of the exact residual."""
+    x = np.asarray(x, np.float32)
+    t = np.float32(65537.0) * x
+    hi = t - (t - x)
+    lo = ((x - hi).view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    return hi, lo
+
+
+def single(x):
+    return bf16(x), np.zeros_like(np.asarray(x, np.float32))
+
+
+def mm(a, b):
+    """bf16-valued operands, fp32 accumulation."""
+    return a.astype(np.float32) @ b.astype(np.float32)
+
+
+def chain(q, k, kth, ktl, v, beta, scale, C, sp):
+    """One (sequence, head) through the lookahead form with the operand splits `sp`."""
+    T = k.shape[0]
+    nch = (T + C - 1) // C
+
+    def tile(a, c):
+        out = np.zeros((C,) + a.shape[1:], np.float32)
+        if c < nch:
+            part = a[c * C:min((c + 1) * C, T)]
+            out[:len(part)] = part
+        return out
+
+    S = np.zeros((v.shape[1], k.shape[1]), np.float32)
+    O = np.zeros(v.shape, np.float32)
+    Sh, Sl = sp(S)
+    K0 = tile(k, 0)
+    D1 = mm(K0, Sh.T) + mm(K0, Sl.T)
+    for c in range(nch):
+        K, Kh, Kl, Q, V, b = (tile(a, c) for a in (k, kth, ktl, q, v, beta))
+        Tm = np.linalg.inv(np.eye(C, dtype=np.float32) +
+                           np.tril(b[:, None] * (mm(K, Kh.T) + mm(K, Kl.T)), -1)).astype(np.float32)
+        Th, Tl = sp(Tm)
+        Rh, Rl = sp(b[:, None] * (V - D1))
+        Wm = mm(Th, Rh) + mm(Th, Rl) + mm(Tl, Rh)
+        Wh, Wl = sp(Wm)
+        Kn = tile(k, c + 1)
+        Xh, Xl = sp(mm(Kn, Kh.T) + mm(Kn, Kl.T))
+        Ph, Pl = sp(np.tril(mm(Q, Kh.T) + mm(Q, Kl.T)))
+        top = mm(Kn, Sh.T) + mm(Kn, Sl.T) + mm(Xh, Wh) + mm(Xh, Wl) + mm(Xl, Wh)
+        bottom = mm(Q, Sh.T) + mm(Q, Sl.T) + mm(Ph, Wh) + mm(Ph, Wl) + mm(Pl, Wh)
+        S = S + mm(Wh.T, Kh) + mm(Wl.T, Kh) + mm(Wh.T, Kl)
+        Sh, Sl = sp(S)
+        L = min(C, T - c * C)
+        O[c * C:c * C + L] = scale * bottom[:L]
+        D1 = top
+    return O, S
+
+
+@pytest.fixture(scope="module")
+def workload():
+    cfg = dict(W.CONFIGS["1p3b_apf"])
+    cfg.update(B=1, T=1024, H=2)
+    inp = W.make_inputs(cfg)
+    o, kt, ST, _ = osdn_ref.fwd(inp.q, inp.k, inp.v, inp.beta, inp.r, inp.eta, inp.d0, inp.S0,
+                                inp.scale)
+    return inp, o, kt, ST
+
+
+def errors(workload, sp, kt_terms):
+    inp, o_ex, kt, S_ex = workload
+    rms = lambda x: np.sqrt(np.mean(x * x))
+    eo, es = [], []
+    for h in range(inp.H):
+        q, k, v = (a[0, :, h].astype(np.float32) for a in (inp.q, inp.k, inp.v))
+        kth = bf16(kt[0, :, h])
+        ktl = bf16(kt[0, :, h] - kth) if kt_terms == 2 else np.zeros_like(kth)
+        O, S = chain(q, k, kth, ktl, v, inp.beta[0, :, h].astype(np.float32), inp.scale, 64, sp)
+        eo.append(np.max(np.abs(O - o_ex[0, :, h])) / rms(o_ex[0, :, h]))
+        es.append(np.max(np.abs(S - S_ex[0, h])) / rms(S_ex[0, h]))
+    return max(eo), max(es)
+
+
+def test_split_operands_keep_the_chain_at_the_fp32_level(workload):
+    eo, es = errors(workload, split, 2)
+    assert eo < 2e-4 and es < 2e-4, (eo, es)
+
+
+def test_single_term_bf16_operands_miss_the_bound(workload):
+    eo, es = errors(workload, single, 1)
+    assert eo > 1e-2 and es > 1e-2, (eo, es)
