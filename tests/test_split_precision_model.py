@@ -9,7 +9,8 @@ terms.  This file runs that arithmetic (the lookahead form, fp32 accumulation of
 operands, an fp32 inverse for T) on the 1.3B-layer workload's first 1024 tokens of two heads and
 compares it with the fp64 oracle:
   - with the splits, o and S_T stay within 2e-4 of rms, two orders of magnitude inside the 1e-2
-    bound, so the bound is left to the bf16 rounding of the inputs and the output;
+    bound, so the bound is left to the bf16 rounding of the inputs and the output; the same holds
+    for chunks of 128 tokens, a redesign that would halve the chain's serial steps;
   - with single-term bf16 operands (and k~ rounded to bf16), the same arithmetic misses the bound.
 """
 import numpy as np
@@ -92,7 +93,7 @@ def workload():
     return inp, o, kt, ST
 
 
-def errors(workload, sp, kt_terms):
+def errors(workload, sp, kt_terms, C=64):
     inp, o_ex, kt, S_ex = workload
     rms = lambda x: np.sqrt(np.mean(x * x))
     eo, es = [], []
@@ -100,14 +101,16 @@ def errors(workload, sp, kt_terms):
         q, k, v = (a[0, :, h].astype(np.float32) for a in (inp.q, inp.k, inp.v))
         kth = bf16(kt[0, :, h])
         ktl = bf16(kt[0, :, h] - kth) if kt_terms == 2 else np.zeros_like(kth)
-        O, S = chain(q, k, kth, ktl, v, inp.beta[0, :, h].astype(np.float32), inp.scale, 64, sp)
+        O, S = chain(q, k, kth, ktl, v, inp.beta[0, :, h].astype(np.float32), inp.scale, C, sp)
         eo.append(np.max(np.abs(O - o_ex[0, :, h])) / rms(o_ex[0, :, h]))
         es.append(np.max(np.abs(S - S_ex[0, h])) / rms(S_ex[0, h]))
     return max(eo), max(es)
 
 
-def test_split_operands_keep_the_chain_at_the_fp32_level(workload):
-    eo, es = errors(workload, split, 2)
+@pytest.mark.parametrize("C", [64, 128])
+def test_split_operands_keep_the_chain_at_the_fp32_level(workload, C):
+    """C = 64 is the built chunk; C = 128 (half the serial steps) keeps the same accuracy."""
+    eo, es = errors(workload, split, 2, C)
     assert eo < 2e-4 and es < 2e-4, (eo, es)
 
 
