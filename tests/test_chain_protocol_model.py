@@ -85,3 +85,130 @@ def test_two_groups_with_three_slots_are_exact():
     """The earlier two-group layout (3-slot ring, 3 receive slots) is exact as well."""
     for seed in range(40):
         assert simulate(64, seed, ns=3, ng=2, nx=3) == "ok"
+
+
+# ---------------------------------------------------------------------------------------------
+# All roles of both CTAs, on the shared executor (tests/protocol_model.py): every buffer that
+# crosses a role boundary is versioned by its chunk, so a wait that is missing or too weak shows
+# up as a read of the wrong chunk's data or a write under a pending read.  Per chunk c:
+#   rank 0  forwarder  TMA of k and T_d into ring slot c % 3 (chunks 0-2 up front, chunk c + 3
+#                      after fwdin(c)); after fwdin(c) and outdone(c - NG) it copies x_c and the
+#                      chunk-start d_c into rank 1's receive slot c % NG, then fwdout(c), xready
+#           loader     full(c), fwdout(c - 2); reads e_t from the T_d tile, writes the gate
+#                      vectors of slot c % 3, meets the chain at the named barrier
+#           chain      the named barrier; reads the tiles, the gate vectors and d_c (slot c % 3),
+#                      writes x_c (slot c % 3) and d_{c+1} (slot (c + 1) % 3), then fwdin(c)
+#   rank 1  loader     kempty(c - NS); TMA of k into key slot c % NS; r of the chunk, vready
+#           writer g   chunks c = g mod NG: kempty(c - NS), full, vready, xready; copies x_c and
+#                      d_c out of the receive slot, outdone; reads the key tile and r; kempty
+# The named barrier (bar.sync of the loader warp and the 256 chain threads) is modelled as a
+# two-party barrier with one phase per chunk.
+
+def chain_roles(N, ns=NS, ng=NG, nx=NX, mut=None):
+    def r0_forwarder():
+        last = {}
+
+        def issue(c):
+            last[c % 3] = c
+            return ("tma", [("r0ring", c % 3, "K"), ("r0ring", c % 3, "TD")], c,
+                    f"r0full{c % 3}", c // 3)
+
+        for c in range(min(3, N)):
+            yield issue(c)
+        for c in range(N):
+            k, m = c % 3, c % nx
+            yield ("wait", f"fwdin{k}", c // 3)
+            if c + 3 < N:
+                yield issue(c + 3)
+            if c >= nx:
+                yield ("wait", f"outdone{m}", c // nx - 1)
+            yield ("read", ("sX", k), c)
+            yield ("read", ("sD", k), c)
+            yield ("write", ("XR", m), c)
+            yield ("write", ("DR", m), c)
+            yield ("arrive", f"fwdout{k}", c // 3)
+            yield ("arrive", f"xready{m}", c // nx)
+        for s, c in last.items():  # the copies in flight land before the block leaves
+            yield ("wait", f"r0full{s}", c // 3)
+
+    def r0_loader():
+        for c in range(N):
+            s = c % 3
+            yield ("wait", f"r0full{s}", c // 3)
+            if c >= 2 and mut != "loader_skips_fwdout":
+                yield ("wait", f"fwdout{(c - 2) % 3}", (c - 2) // 3)
+            yield ("read", ("r0ring", s, "TD"), c)  # e_t rides in the T_d tile
+            yield ("write", ("vecs", s), c)
+            yield ("arrive", "bar1", c)
+            yield ("wait", "bar1", c)
+
+    def r0_chain():
+        yield ("write", ("sD", 0), 0)  # d_0, written by these threads before the cluster barrier
+        for c in range(N):
+            s = c % 3
+            yield ("arrive", "bar1", c)
+            yield ("wait", "bar1", c)
+            yield ("read", ("r0ring", s, "K"), c)
+            yield ("read", ("r0ring", s, "TD"), c)
+            yield ("read", ("vecs", s), c)
+            yield ("read", ("sD", s), c)
+            yield ("write", ("sX", s), c)
+            yield ("write", ("sD", (c + 1) % 3), c + 1)
+            yield ("arrive", f"fwdin{s}", c // 3)
+        yield ("read", ("sD", N % 3), N)  # d_T
+
+    def r1_loader():
+        for c in range(N):
+            s = c % ns
+            if c >= ns:
+                yield ("wait", f"kempty{s}", c // ns - 1)
+            yield ("tma", [("r1ring", s)], c, f"r1full{s}", c // ns)
+            yield ("write", ("rv", s), c)
+            yield ("arrive", f"vready{s}", c // ns)
+
+    def r1_writer(g):
+        for c in range(g, N, ng):
+            s, m = c % ns, c % nx
+            if c >= ns and mut != "writer_skips_kempty":
+                yield ("wait", f"kempty{s}", c // ns - 1)
+            yield ("wait", f"r1full{s}", c // ns)
+            yield ("wait", f"vready{s}", c // ns)
+            yield ("wait", f"xready{m}", c // nx)
+            yield ("read", ("XR", m), c)
+            yield ("read", ("DR", m), c)
+            yield ("arrive", f"outdone{m}", c // nx)
+            yield ("read", ("r1ring", s), c)
+            yield ("read", ("rv", s), c)
+            yield ("arrive", f"kempty{s}", c // ns)
+
+    barriers = {"bar1": 2}
+    for s in range(3):
+        barriers.update({f"r0full{s}": 1, f"fwdin{s}": 1, f"fwdout{s}": 1})
+    for s in range(ns):
+        barriers.update({f"r1full{s}": 1, f"vready{s}": 1, f"kempty{s}": 1})
+    for m in range(nx):
+        barriers.update({f"xready{m}": 1, f"outdone{m}": 1})
+    roles = {"r0_forwarder": r0_forwarder(), "r0_loader": r0_loader(), "r0_chain": r0_chain(),
+             "r1_loader": r1_loader()}
+    roles.update({f"r1_writer{g}": r1_writer(g) for g in range(ng)})
+    return barriers, roles
+
+
+def chain_model(N, seed, **kw):
+    from tests.protocol_model import Model
+    barriers, roles = chain_roles(N, **kw)
+    return Model(barriers, roles, seed)
+
+
+@pytest.mark.parametrize("N", [0, 1, 3, 4, 5, 6, 9, 13])
+def test_all_roles_exact_in_every_schedule(N):
+    for seed in range(200):
+        chain_model(N, seed).run()
+
+
+@pytest.mark.parametrize("kw", [dict(nx=3), dict(mut="writer_skips_kempty"),
+                                dict(mut="loader_skips_fwdout")],
+                         ids=["three_receive_slots", "writer_skips_kempty", "loader_skips_fwdout"])
+def test_all_roles_model_catches_planted_mistakes(kw):
+    from tests.protocol_model import count_caught
+    assert count_caught(lambda seed: chain_model(13, seed, **kw), range(200)) > 0

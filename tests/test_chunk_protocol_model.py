@@ -22,9 +22,9 @@ Planted mistakes in the protocol (a single T-tile barrier for both ring slots, a
 the release of the stage, a missing wait) must each be caught.  The peer CTA's counter and the
 cluster barriers are outside the model (they order the two CTAs of a head, not the roles).
 """
-import random
-
 import pytest
+
+from tests.protocol_model import Model, count_caught
 
 BARRIERS = {"tma_full0": 1, "tma_full1": 1, "stage_empty0": 2, "stage_empty1": 2,
             "zt_full0": 1, "zt_full1": 1, "mma_c": 1, "mma_p": 1, "mma_crit": 1, "mma_s": 1,
@@ -32,8 +32,9 @@ BARRIERS = {"tma_full0": 1, "tma_full1": 1, "stage_empty0": 2, "stage_empty1": 2
 STAGE_PARTS = ("KQ", "KT", "V", "T")
 
 
-class ProtocolError(AssertionError):
-    pass
+def load(i):
+    """TMA of ring stage i: every part of slot i & 1; lands on tma_full of the slot."""
+    return ("tma", [("stage", i & 1, p) for p in STAGE_PARTS], i, f"tma_full{i & 1}", i >> 1)
 
 
 # ------------------------------------------------------------------ the roles, as in the kernel
@@ -42,8 +43,8 @@ def producer(N, mut):
     if N == 0:
         return
     last = {}
-    yield ("tma", 0, 0)
-    yield ("tma", 1, 1)
+    yield load(0)
+    yield load(1)
     last[0], last[1] = 0, 1
     yield ("wait", "tma_full0", 0)
 
@@ -72,7 +73,7 @@ def producer(N, mut):
         if j + 2 <= N:
             if mut != "refill_without_release":
                 yield ("wait", f"stage_empty{j & 1}", j >> 1)
-            yield ("tma", (j + 2) & 1, j + 2)
+            yield load(j + 2)
             last[(j + 2) & 1] = j + 2
     yield ("wait", "mma_crit", N - 1)
     yield from state_update(N - 1)
@@ -179,200 +180,20 @@ def upper(N, mut):
 ROLES = {"P": producer, "Q": prep, "L": lower, "U": upper}
 
 
-# ------------------------------------------------------------------ the executor
-
-class Model:
-    def __init__(self, N, seed, mut=None):
-        self.rng = random.Random(seed)
-        self.bars = {b: {"count": c, "arr": 0, "n": 0} for b, c in BARRIERS.items()}
-        self.res = {}
-        self.agents = {}
-        for name, fn in ROLES.items():
-            self.agents[name] = {"gen": fn(N, mut), "op": None, "done": False, "wait": None}
-        self.tma = []                                  # in-flight copies
-        self.open = {"P": [], "L": []}                 # MMAs issued since the last commit
-        self.queue = {"P": [], "L": []}                # committed groups, in issue order
-        self.gid = 0
-
-    def r(self, key):
-        return self.res.setdefault(key, {"tag": None, "reads": [], "writes": []})
-
-    def fail(self, what):
-        raise ProtocolError(what)
-
-    # barriers
-    def arrive(self, bar, phase, who):
-        b = self.bars[bar]
-        if phase != b["n"]:
-            self.fail(f"{who}: arrival for phase {phase} on {bar} in phase {b['n']}")
-        b["arr"] += 1
-        if b["arr"] == b["count"]:
-            b["arr"] = 0
-            b["n"] += 1
-            m = b["n"] - 1  # the phase that just completed
-            for name, a in self.agents.items():
-                if a["wait"] and a["wait"][0] == bar and a["wait"][1] < m:
-                    self.fail(f"{name}: {bar} completed phase {m} while it still waited for "
-                              f"phase {a['wait'][1]}")
-
-    def wait_state(self, bar, k, who):
-        n = self.bars[bar]["n"]
-        if n < k:
-            self.fail(f"{who}: waits for phase {k} of {bar}, which has completed only {n}")
-        if n >= k + 2:
-            self.fail(f"{who}: waits for phase {k} of {bar}, which has completed {n}")
-        return n == k + 1
-
-    # resources
-    def sync_read(self, key, tag, who):
-        r = self.r(key)
-        if r["writes"]:
-            self.fail(f"{who}: reads {key} while an asynchronous write is in flight")
-        if r["tag"] != tag:
-            self.fail(f"{who}: reads {key} as {tag}, finds {r['tag']}")
-
-    def sync_write(self, key, tag, who):
-        r = self.r(key)
-        if r["reads"] or r["writes"]:
-            self.fail(f"{who}: writes {key} while an asynchronous access is in flight")
-        r["tag"] = tag
-
-    def issue_mma(self, who, reads, writes):
-        gid = self.gid
-        self.gid += 1
-        for key, tag in reads:
-            r = self.r(key)
-            mine = [w for w in r["writes"] if w[0] == who]
-            other = [w for w in r["writes"] if w[0] != who]
-            if other:
-                self.fail(f"{who}: MMA reads {key} while another thread's write is in flight")
-            have = mine[-1][2] if mine else r["tag"]
-            if have != tag:
-                self.fail(f"{who}: MMA reads {key} as {tag}, finds {have}")
-        for key, tag in writes:
-            r = self.r(key)
-            if any(x[0] != who for x in r["reads"]) or any(x[0] != who for x in r["writes"]):
-                self.fail(f"{who}: MMA writes {key} while another access is in flight")
-        for key, tag in reads:
-            self.r(key)["reads"].append((who, gid))
-        for key, tag in writes:
-            self.r(key)["writes"].append((who, gid, tag))
-        self.open[who].append(gid)
-
-    def complete_group(self, who):
-        g = self.queue[who].pop(0)
-        ids = set(g["ids"])
-        for key, r in self.res.items():
-            for w in [w for w in r["writes"] if w[0] == who and w[1] in ids]:
-                r["tag"] = w[2]
-            r["writes"] = [w for w in r["writes"] if not (w[0] == who and w[1] in ids)]
-            r["reads"] = [x for x in r["reads"] if not (x[0] == who and x[1] in ids)]
-        self.arrive(g["bar"], g["phase"], who)
-
-    def issue_tma(self, slot, stage):
-        for part in STAGE_PARTS:
-            r = self.r(("stage", slot, part))
-            if r["reads"] or r["writes"]:
-                self.fail(f"TMA of stage {stage} overwrites slot {slot} ({part}) under an "
-                          "asynchronous access")
-            r["writes"].append(("tma", stage, stage))
-        self.tma.append((slot, stage))
-
-    def complete_tma(self, idx):
-        slot, stage = self.tma.pop(idx)
-        for part in STAGE_PARTS:
-            r = self.r(("stage", slot, part))
-            r["writes"] = [w for w in r["writes"] if w[0] != "tma" or w[1] != stage]
-            r["tag"] = stage
-        self.arrive(f"tma_full{slot}", stage >> 1, "TMA")
-
-    # one agent step
-    def fetch(self, name):
-        a = self.agents[name]
-        try:
-            a["op"] = next(a["gen"])
-        except StopIteration:
-            a["done"], a["op"] = True, None
-            return
-        op = a["op"]
-        if op[0] == "wait":
-            a["wait"] = (op[1], op[2])
-            self.wait_state(op[1], op[2], name)
-
-    def runnable(self, name):
-        a = self.agents[name]
-        if a["done"]:
-            return False
-        if a["op"] is None:
-            return True
-        if a["op"][0] == "wait":
-            return self.wait_state(a["op"][1], a["op"][2], name)
-        return True
-
-    def step(self, name):
-        a = self.agents[name]
-        if a["op"] is None:
-            self.fetch(name)
-            return
-        op, a["op"] = a["op"], None
-        kind = op[0]
-        if kind == "wait":
-            a["wait"] = None
-        elif kind == "arrive":
-            self.arrive(op[1], op[2], name)
-        elif kind == "read":
-            self.sync_read(op[1], op[2], name)
-        elif kind == "write":
-            self.sync_write(op[1], op[2], name)
-        elif kind == "rmw":
-            self.sync_read(op[1], op[2], name)
-            self.sync_write(op[1], op[3], name)
-        elif kind == "tma":
-            self.issue_tma(op[1], op[2])
-        elif kind == "mma":
-            self.issue_mma(name, op[1], op[2])
-        elif kind == "commit":
-            self.queue[name].append({"ids": self.open[name], "bar": op[1], "phase": op[2]})
-            self.open[name] = []
-        else:
-            raise ValueError(kind)
-
-    def run(self, max_steps=200000):
-        for _ in range(max_steps):
-            cands = [("agent", n) for n in self.agents if self.runnable(n)]
-            cands += [("tma", i) for i in range(len(self.tma))]
-            cands += [("mma", w) for w in self.queue if self.queue[w]]
-            if not cands:
-                left = [n for n, a in self.agents.items() if not a["done"]]
-                if left:
-                    self.fail(f"deadlock: {[(n, self.agents[n]['op']) for n in left]}")
-                return
-            kind, x = self.rng.choice(cands)
-            if kind == "agent":
-                self.step(x)
-            elif kind == "tma":
-                self.complete_tma(x)
-            else:
-                self.complete_group(x)
-        raise AssertionError("schedule did not finish")
+def model(N, seed, mut=None):
+    return Model(BARRIERS, {name: fn(N, mut) for name, fn in ROLES.items()}, seed)
 
 
 @pytest.mark.parametrize("N", [0, 1, 2, 3, 4, 7])
 def test_protocol_is_exact_in_every_schedule(N):
     for seed in range(300):
-        Model(N, seed).run()
+        model(N, seed).run()
 
 
 @pytest.mark.parametrize("mut", ["single_zt_barrier", "refill_without_release",
                                  "lower_skips_mma_s", "lower_skips_w_done"])
 def test_planted_mistakes_are_caught(mut):
-    caught = 0
-    for seed in range(200):
-        try:
-            Model(5, seed, mut).run()
-        except ProtocolError:
-            caught += 1
-    assert caught > 0, mut
+    assert count_caught(lambda seed: model(5, seed, mut), range(200)) > 0, mut
 
 
 def test_o_free_is_implied_by_the_other_waits():
@@ -381,4 +202,4 @@ def test_o_free_is_implied_by_the_other_waits():
     W_{j-1}, which the producer's wait on mma_crit covers.  The model finds no schedule without
     it that breaks a check (the kernel keeps the wait)."""
     for seed in range(300):
-        Model(5, seed, "producer_skips_o_free").run()
+        model(5, seed, "producer_skips_o_free").run()
