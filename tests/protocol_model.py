@@ -24,7 +24,9 @@ Checks (ProtocolError on the first violation):
   - an arrival lands in the phase it is meant for;
   - a buffer is read in the expected version and not under an in-flight write; it is not written
     (synchronously, by a copy or by another role's MMA) while another access is in flight;
-  - nothing deadlocks and every role finishes.
+  - nothing deadlocks and every role finishes;
+  - when the last role finishes (the block's final cluster barrier, then the release of tensor
+    memory), no copy and no MMA group is still in flight.
 """
 import random
 
@@ -158,6 +160,9 @@ class Model:
                 a["op"] = next(a["gen"])
             except StopIteration:
                 a["done"] = True
+                if all(x["done"] for x in self.agents.values()) and (
+                        self.tma or any(self.queue.values()) or any(self.open.values())):
+                    self.fail("the block leaves with copies or MMAs in flight")
                 return
             if a["op"][0] == "wait":
                 a["wait"] = (a["op"][1], a["op"][2])
