@@ -2,11 +2,15 @@
 
 A model is a set of roles, each a generator of operations in program order, and a table of
 barriers with their arrival counts.  Operations:
-    ("wait", bar, k)                 parity wait for the completion of phase k of `bar`
+    ("wait", bar, k[, kind])         parity wait for the completion of phase k of `bar`; the
+                                     role receives True, or False when the wait timed out; kind
+                                     "drain" marks the waits of a role's exit path, "sync" a
+                                     named barrier (bar.sync), which has no timeout
     ("arrive", bar, k)               one arrival, meant for phase k
     ("read", key, tag)               synchronous read of a buffer, expecting version `tag`
     ("write", key, tag)              synchronous write of version `tag`
     ("rmw", key, tag_in, tag_out)    read then write
+    ("peek", key)                    the role receives the buffer's current version (a flag)
     ("tma", keys, tag, bar, k)       asynchronous copy writing version `tag` into every buffer in
                                      `keys`; on landing it arrives on `bar` for phase k
     ("mma", reads, writes)           asynchronous tensor-core work of this role: reads and writes
@@ -27,6 +31,11 @@ Checks (ProtocolError on the first violation):
   - nothing deadlocks and every role finishes;
   - when the last role finishes (the block's final cluster barrier, then the release of tensor
     memory), no copy and no MMA group is still in flight.
+With timeouts=True the schedule may also let any blocked wait run out (a drain wait, marked
+"drain", only with drain_timeouts=True).  From the first timeout on, the barriers behave as the
+hardware's do (a parity wait passes when the completed-phase count has the other parity; arrivals
+just count) and the buffer checks stop, since a timed-out kernel's outputs are void; what must
+still hold is the exit check: every role that gave up has waited for its own copies and MMAs.
 """
 import random
 
@@ -36,10 +45,14 @@ class ProtocolError(AssertionError):
 
 
 class Model:
-    def __init__(self, barriers, roles, seed):
+    def __init__(self, barriers, roles, seed, timeouts=False, drain_timeouts=False, init=None):
         self.rng = random.Random(seed)
+        self.timeouts, self.drain_timeouts = timeouts, drain_timeouts
+        self.failed = False  # a wait has timed out
         self.bars = {b: {"count": c, "arr": 0, "n": 0} for b, c in barriers.items()}
         self.res = {}
+        for key, tag in (init or {}).items():  # state set up before the roles start
+            self.r(key)["tag"] = tag
         self.agents = {name: {"gen": gen, "op": None, "done": False, "wait": None,
                               "speed": self.rng.choice((1.0, 1.0, 0.3, 0.05))}
                        for name, gen in roles.items()}
@@ -57,7 +70,7 @@ class Model:
     # ---- barriers
     def arrive(self, bar, phase, who):
         b = self.bars[bar]
-        if phase != b["n"]:
+        if phase != b["n"] and not self.failed:
             self.fail(f"{who}: arrival for phase {phase} on {bar} in phase {b['n']}")
         b["arr"] += 1
         if b["arr"] == b["count"]:
@@ -65,12 +78,16 @@ class Model:
             b["n"] += 1
             m = b["n"] - 1
             for name, a in self.agents.items():
+                if self.failed:
+                    break
                 if a["wait"] and a["wait"][0] == bar and a["wait"][1] < m:
                     self.fail(f"{name}: {bar} completed phase {m} while it still waited for "
                               f"phase {a['wait'][1]}")
 
     def passable(self, bar, k, who):
         n = self.bars[bar]["n"]
+        if self.failed:
+            return (n & 1) != (k & 1)
         if n < k:
             self.fail(f"{who}: waits for phase {k} of {bar}, which has completed only {n}")
         if n >= k + 2:
@@ -80,6 +97,8 @@ class Model:
     # ---- buffers
     def sync_read(self, key, tag, who):
         r = self.r(key)
+        if self.failed:
+            return
         if r["writes"]:
             self.fail(f"{who}: reads {key} while an asynchronous write is in flight")
         if r["tag"] != tag:
@@ -87,6 +106,9 @@ class Model:
 
     def sync_write(self, key, tag, who):
         r = self.r(key)
+        if self.failed:
+            r["tag"] = tag
+            return
         if r["reads"] or r["writes"]:
             self.fail(f"{who}: writes {key} while an asynchronous access is in flight")
         r["tag"] = tag
@@ -94,7 +116,7 @@ class Model:
     def issue_mma(self, who, reads, writes):
         gid = self.gid
         self.gid += 1
-        for key, tag in reads:
+        for key, tag in ([] if self.failed else reads):
             r = self.r(key)
             mine = [w for w in r["writes"] if w[0] == who]
             if any(w[0] != who for w in r["writes"]):
@@ -102,7 +124,7 @@ class Model:
             have = mine[-1][2] if mine else r["tag"]
             if have != tag:
                 self.fail(f"{who}: MMA reads {key} as {tag}, finds {have}")
-        for key, _ in writes:
+        for key, _ in ([] if self.failed else writes):
             r = self.r(key)
             if any(x[0] != who for x in r["reads"]) or any(x[0] != who for x in r["writes"]):
                 self.fail(f"{who}: MMA writes {key} while another access is in flight")
@@ -131,7 +153,7 @@ class Model:
         self.gid += 1
         for key in keys:
             r = self.r(key)
-            if r["reads"] or r["writes"]:
+            if (r["reads"] or r["writes"]) and not self.failed:
                 self.fail(f"{who}: copy of {tag} into {key} under an asynchronous access")
             r["writes"].append((cid, None, tag))
         self.tma.append((cid, keys, tag, bar, phase, self.latency()))
@@ -157,7 +179,7 @@ class Model:
         a = self.agents[name]
         if a["op"] is None:
             try:
-                a["op"] = next(a["gen"])
+                a["op"] = a["gen"].send(a.pop("send", None))
             except StopIteration:
                 a["done"] = True
                 if all(x["done"] for x in self.agents.values()) and (
@@ -172,12 +194,15 @@ class Model:
         kind = op[0]
         if kind == "wait":
             a["wait"] = None
+            a["send"] = True
         elif kind == "arrive":
             self.arrive(op[1], op[2], name)
         elif kind == "read":
             self.sync_read(op[1], op[2], name)
         elif kind == "write":
             self.sync_write(op[1], op[2], name)
+        elif kind == "peek":
+            a["send"] = self.r(op[1])["tag"]
         elif kind == "rmw":
             self.sync_read(op[1], op[2], name)
             self.sync_write(op[1], op[3], name)
@@ -197,7 +222,15 @@ class Model:
             cands = [("role", n) for n in self.agents if self.runnable(n)]
             cands += [("tma", i) for i in range(len(self.tma))]
             cands += [("mma", w) for w in self.queue if self.queue[w]]
-            weights = [self.agents[x]["speed"] if k == "role" else
+            if self.timeouts:
+                for n, a in self.agents.items():
+                    op = a["op"]
+                    if (not a["done"] and op is not None and op[0] == "wait" and
+                            (len(op) < 4 or (op[3] == "drain" and self.drain_timeouts)) and
+                            not self.passable(op[1], op[2], n)):
+                        cands.append(("timeout", n))
+            weights = [0.02 if k == "timeout" else
+                       self.agents[x]["speed"] if k == "role" else
                        self.tma[x][5] if k == "tma" else self.queue[x][0]["w"] for k, x in cands]
             if not cands:
                 left = [n for n, a in self.agents.items() if not a["done"]]
@@ -205,7 +238,11 @@ class Model:
                     self.fail(f"deadlock: {[(n, self.agents[n]['op']) for n in left]}")
                 return
             kind, x = self.rng.choices(cands, weights)[0]
-            if kind == "role":
+            if kind == "timeout":
+                self.failed = True
+                a = self.agents[x]
+                a["op"], a["wait"], a["send"] = None, None, False
+            elif kind == "role":
                 self.step(x)
             elif kind == "tma":
                 self.complete_tma(x)

@@ -14,6 +14,8 @@ import random
 
 import pytest
 
+from tests.protocol_model import Model, ProtocolError, count_caught
+
 NS, NG, NX = 5, 4, 4  # key ring slots, writer groups, receive slots (ScanChainSmem)
 
 
@@ -106,10 +108,10 @@ def test_two_groups_with_three_slots_are_exact():
 
 def chain_roles(N, ns=NS, ng=NG, nx=NX, mut=None):
     def r0_forwarder():
-        last = {}
+        last = []
 
         def issue(c):
-            last[c % 3] = c
+            last.append(c)
             return ("tma", [("r0ring", c % 3, "K"), ("r0ring", c % 3, "TD")], c,
                     f"r0full{c % 3}", c // 3)
 
@@ -117,37 +119,45 @@ def chain_roles(N, ns=NS, ng=NG, nx=NX, mut=None):
             yield issue(c)
         for c in range(N):
             k, m = c % 3, c % nx
-            yield ("wait", f"fwdin{k}", c // 3)
+            if not (yield ("wait", f"fwdin{k}", c // 3)):
+                break
             if c + 3 < N:
                 yield issue(c + 3)
-            if c >= nx:
-                yield ("wait", f"outdone{m}", c // nx - 1)
+            if c >= nx and not (yield ("wait", f"outdone{m}", c // nx - 1)):
+                break
             yield ("read", ("sX", k), c)
             yield ("read", ("sD", k), c)
             yield ("write", ("XR", m), c)
             yield ("write", ("DR", m), c)
             yield ("arrive", f"fwdout{k}", c // 3)
             yield ("arrive", f"xready{m}", c // nx)
-        for s, c in last.items():  # the copies in flight land before the block leaves
-            yield ("wait", f"r0full{s}", c // 3)
+        for c in last[-3:]:  # the copies in flight land before the block leaves
+            yield ("wait", f"r0full{c % 3}", c // 3, "drain")
 
     def r0_loader():
         for c in range(N):
             s = c % 3
-            yield ("wait", f"r0full{s}", c // 3)
-            if c >= 2 and mut != "loader_skips_fwdout":
-                yield ("wait", f"fwdout{(c - 2) % 3}", (c - 2) // 3)
+            got = yield ("wait", f"r0full{s}", c // 3)
+            if got and c >= 2 and mut != "loader_skips_fwdout":
+                got = yield ("wait", f"fwdout{(c - 2) % 3}", (c - 2) // 3)
+            if not got:  # the failure flag, then the barrier: the chain leaves at this chunk
+                yield ("write", "fail", c if mut == "fixed_exit_paths" else 1)
+                yield ("arrive", "bar1", c)
+                yield ("wait", "bar1", c, "sync")
+                return
             yield ("read", ("r0ring", s, "TD"), c)  # e_t rides in the T_d tile
             yield ("write", ("vecs", s), c)
             yield ("arrive", "bar1", c)
-            yield ("wait", "bar1", c)
+            yield ("wait", "bar1", c, "sync")
 
     def r0_chain():
-        yield ("write", ("sD", 0), 0)  # d_0, written by these threads before the cluster barrier
         for c in range(N):
             s = c % 3
             yield ("arrive", "bar1", c)
-            yield ("wait", "bar1", c)
+            yield ("wait", "bar1", c, "sync")
+            flag = yield ("peek", "fail")
+            if (flag <= c) if mut == "fixed_exit_paths" else flag:
+                return
             yield ("read", ("r0ring", s, "K"), c)
             yield ("read", ("r0ring", s, "TD"), c)
             yield ("read", ("vecs", s), c)
@@ -158,22 +168,32 @@ def chain_roles(N, ns=NS, ng=NG, nx=NX, mut=None):
         yield ("read", ("sD", N % 3), N)  # d_T
 
     def r1_loader():
+        issued = []
         for c in range(N):
             s = c % ns
-            if c >= ns:
-                yield ("wait", f"kempty{s}", c // ns - 1)
+            if c >= ns and not (yield ("wait", f"kempty{s}", c // ns - 1)):
+                for cc in issued[-ns:]:  # its own wait ran out: the loads in flight land
+                    yield ("wait", f"r1full{cc % ns}", cc // ns, "drain")
+                return
             yield ("tma", [("r1ring", s)], c, f"r1full{s}", c // ns)
+            issued.append(c)
             yield ("write", ("rv", s), c)
             yield ("arrive", f"vready{s}", c // ns)
+            if mut == "fixed_exit_paths" and c == N - 1:
+                for cc in issued[-ns:]:
+                    yield ("wait", f"r1full{cc % ns}", cc // ns, "drain")
 
     def r1_writer(g):
         for c in range(g, N, ng):
             s, m = c % ns, c % nx
+            got = True
             if c >= ns and mut != "writer_skips_kempty":
-                yield ("wait", f"kempty{s}", c // ns - 1)
-            yield ("wait", f"r1full{s}", c // ns)
-            yield ("wait", f"vready{s}", c // ns)
-            yield ("wait", f"xready{m}", c // nx)
+                got = yield ("wait", f"kempty{s}", c // ns - 1)
+            got = got and (yield ("wait", f"r1full{s}", c // ns))
+            got = got and (yield ("wait", f"vready{s}", c // ns))
+            got = got and (yield ("wait", f"xready{m}", c // nx))
+            if not got:
+                return
             yield ("read", ("XR", m), c)
             yield ("read", ("DR", m), c)
             yield ("arrive", f"outdone{m}", c // nx)
@@ -191,13 +211,15 @@ def chain_roles(N, ns=NS, ng=NG, nx=NX, mut=None):
     roles = {"r0_forwarder": r0_forwarder(), "r0_loader": r0_loader(), "r0_chain": r0_chain(),
              "r1_loader": r1_loader()}
     roles.update({f"r1_writer{g}": r1_writer(g) for g in range(ng)})
-    return barriers, roles
+    # set before the cluster barrier that starts the roles: d_0 and the failure flag
+    init = {("sD", 0): 0, "fail": N + 1 if mut == "fixed_exit_paths" else 0}
+    return barriers, roles, init
 
 
-def chain_model(N, seed, **kw):
-    from tests.protocol_model import Model
-    barriers, roles = chain_roles(N, **kw)
-    return Model(barriers, roles, seed)
+def chain_model(N, seed, timeouts=False, drain_timeouts=False, **kw):
+    barriers, roles, init = chain_roles(N, **kw)
+    return Model(barriers, roles, seed, timeouts=timeouts, drain_timeouts=drain_timeouts,
+                 init=init)
 
 
 @pytest.mark.parametrize("N", [0, 1, 3, 4, 5, 6, 9, 13])
@@ -210,5 +232,37 @@ def test_all_roles_exact_in_every_schedule(N):
                                 dict(mut="loader_skips_fwdout")],
                          ids=["three_receive_slots", "writer_skips_kempty", "loader_skips_fwdout"])
 def test_all_roles_model_catches_planted_mistakes(kw):
-    from tests.protocol_model import count_caught
     assert count_caught(lambda seed: chain_model(13, seed, **kw), range(200)) > 0
+
+
+# ---- exit paths when a bounded wait runs out (any wait may time out; drains do not)
+
+@pytest.mark.parametrize("N", [1, 3, 5, 9, 13])
+def test_exit_paths_with_the_two_fixes_are_complete(N):
+    """With rank 1's loader waiting for its own copies on every exit, and the failure flag
+    carrying the chunk at which the loader gave up (the chain leaves at that chunk's barrier),
+    every schedule ends with both CTAs done and nothing in flight."""
+    took = 0
+    for seed in range(300):
+        m = chain_model(N, seed, timeouts=True, mut="fixed_exit_paths")
+        m.run()
+        took += m.failed
+    assert took > 200
+
+
+def test_exit_paths_as_built_rely_on_the_long_bound():
+    """The kernel as built has two exit-path gaps that only a wait far shorter than its 2 s
+    bound can reach: rank 1's loader waits for its copies only when its own wait ran out (copies
+    may still land after the writers gave up), and the chain reads a yes/no failure flag after
+    the named barrier of chunk c, so a loader already failing at chunk c + 1 makes the chain leave
+    a chunk early and leaves the loader at a barrier without a timeout.  Under the 2 s bound a
+    key copy lands long before, and the flag is set 2 s after the chain's read."""
+    kinds = set()
+    for N in (3, 9):
+        for seed in range(300):
+            try:
+                chain_model(N, seed, timeouts=True).run()
+            except ProtocolError as e:
+                kinds.add("in flight" if "in flight" in str(e) else
+                          "barrier" if "deadlock" in str(e) and "bar1" in str(e) else str(e))
+    assert kinds == {"in flight", "barrier"}, kinds
